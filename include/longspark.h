@@ -1,0 +1,199 @@
+/*
+ * longspark.h — C ABI of the LongSpark fixed-cost drafting round on B200 (sm_100a).
+ *
+ * Method: "LongSpark: Efficient speculative decoding with a fixed-cost parallel
+ * drafter" (arXiv 2609.37029), as printed on the thelatestinai.com paper page:
+ *   - Figure 2 caption: one decoding round = (a) the target verifies the proposed
+ *     block, (b) three fixed-size context views are extracted from the target's
+ *     state — a boundary state, a recent KV window and a global context summary —
+ *     and (c) the drafter proposes the next block from those views at a cost that
+ *     does not depend on the prefix length.
+ *   - Figure 3 caption: the global summary is initialised over the whole prefix at
+ *     target prefill and afterwards updated only from the newly retained KV rows N,
+ *     with Delta = |N| <= B + 1.
+ *   - Figure 1 caption / abstract: O(1) drafting cost and a drafter state whose size
+ *     does not grow with the prefix ("fixed-size, multiscale views").
+ * The pages print no formula for the views; the definitions used here are:
+ *   accept scan   a = number of leading positions i < B with draft[i] == target[i];
+ *                 next token = target[a]; Delta = a + 1 retained rows (verify rows 0..a).
+ *   window        the last min(len, W) retained K/V rows; row p lives in ring slot p mod W.
+ *   summary       per tapped layer and KV head, for each scale s_k: segment j covers the
+ *                 absolute rows [j*s_k, (j+1)*s_k); the slots hold the K/V means of the
+ *                 `slots` most recent complete segments (segment j in slot j mod slots),
+ *                 plus the open partial segment (its sum; its mean is an attention slot),
+ *                 plus one running mean over all retained rows.
+ *   boundary      the tapped-layer hidden vectors at the last retained position.
+ *   attention     per (layer, query head qh), KV head g = qh / (Hq/Hkv): softmax(q k^T * scale)
+ *                 over [boundary, window rows, per scale: slots + partial mean, global mean],
+ *                 empty slots masked, no mask among the B block queries.
+ *
+ * Conventions for every entry point:
+ *   - Return value: LS_OK (0) or a negative LS_ERR_* code. Nothing traps or aborts.
+ *   - Every d_* pointer is DEVICE memory owned by the caller; h_* pointers are host
+ *     memory owned by the caller. The library never allocates device memory; the only
+ *     host allocation is the opaque ls_state handle (ls_init_state / ls_destroy_state).
+ *   - Device work is enqueued asynchronously on `stream`; no call synchronises except
+ *     ls_read_state and ls_get_error, which say so.
+ *   - Element types: `dtype` (LS_BF16 or LS_F32) is the type of K/V/hidden/q/out and of
+ *     the window and mirror rows in the arena. Summary sums and segment means are fp32.
+ *   - Kernels never trap. Conditions found on the device (bad prefix length, bounded
+ *     waits that ran out) set bits in the device error word; read it with ls_get_error.
+ */
+#ifndef LONGSPARK_H_
+#define LONGSPARK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------------ */
+#define LS_OK                   0
+#define LS_ERR_INVALID_ARG    (-1)  /* null pointer, negative size, bad enum           */
+#define LS_ERR_SHAPE          (-2)  /* sizes inconsistent with each other or the arena  */
+#define LS_ERR_UNSUPPORTED    (-3)  /* valid for the method, not for this GPU path      */
+#define LS_ERR_CUDA           (-4)  /* a CUDA runtime call failed                       */
+#define LS_ERR_DEVICE         (-5)  /* the device error word holds a non-zero code      */
+#define LS_ERR_DEVICE_TIMEOUT (-6)  /* a bounded device wait gave up                    */
+
+/* ---- device error word bits (ls_get_error) ----------------------------------- */
+#define LS_DEVERR_PREFIX_LEN   0x1  /* prefix_len[b] < 0 or beyond what the buffers hold */
+#define LS_DEVERR_WAIT_TIMEOUT 0x2  /* an mbarrier wait exceeded its iteration limit     */
+#define LS_DEVERR_ORDER        0x4  /* prefill chunk does not continue the state          */
+
+/* ---- dtypes and flags -------------------------------------------------------- */
+#define LS_F32  0
+#define LS_BF16 1
+#define LS_FLAG_FORCE_SIMT 0x1      /* run draft attention on CUDA cores even where the
+                                       tcgen05 tensor-core kernel applies              */
+
+#define LS_MAX_SCALES 4
+
+/* Shapes of one drafting state (one batch of sequences).
+ *   batch b, n_layers L (tapped layers), n_kv_heads Hkv, n_q_heads Hq (multiple of Hkv),
+ *   head_dim D (multiple of 8, <= 256), hidden (multiple of 8), block B (1..32),
+ *   window W (>= B+1, multiple of 8), n_scales (1..4), scales ascending, each >= B+1,
+ *   each dividing the next (so no segment of any scale straddles a larger one),
+ *   slots_per_scale >= 1, dtype LS_F32 | LS_BF16, flags LS_FLAG_*.              */
+typedef struct {
+  int32_t batch, n_layers, n_kv_heads, n_q_heads, head_dim, hidden;
+  int32_t block;
+  int32_t window;
+  int32_t n_scales;
+  int32_t scales[LS_MAX_SCALES];
+  int32_t slots_per_scale;
+  int32_t dtype;
+  int32_t flags;
+} ls_config;
+
+/* Byte offsets (from the arena base) and shapes of the regions of the state arena.
+ * All offsets are multiples of 256. e = element size of `dtype`.
+ *   counters  int64 [b][L][1 + n_scales]: retained length len, then for each scale the
+ *             number of segments finalised so far (floor(len / s_k)).
+ *   error     int32 [4]: word 0 is the device error word.
+ *   kv        e     [b][L][Hkv][2][kv_rows][D]: for K (index 0) and V (index 1) of each
+ *             (sequence, layer, KV head) tile, rows 0..W-1 are the ring window, then for
+ *             each scale k rows W + k*(slots+1) + i hold the mean of the segment in slot i
+ *             (i < slots) or the open partial's mean (i == slots), and the last row
+ *             (W + n_scales*(slots+1)) holds the global mean. kv_rows = that count + 1.
+ *             These mean rows are the attention's copy, rounded to `dtype`.
+ *   seg_mean  fp32  [b][L][Hkv][n_scales][slots][2][D]: segment means in full fp32.
+ *   part_sum  fp32  [b][L][Hkv][n_scales][2][D]: sums of the open partial segments.
+ *   glob_sum  fp32  [b][L][Hkv][2][D]: sum of all retained rows.
+ *   boundary  e     [b][L][hidden]: hidden vectors at the last retained position.     */
+typedef struct {
+  size_t total_bytes;
+  size_t off_counters, off_error, off_kv, off_seg_mean, off_part_sum, off_glob_sum,
+         off_boundary;
+  int32_t kv_rows;
+  int32_t elem_bytes;
+} ls_layout;
+
+typedef struct ls_state ls_state; /* opaque host handle */
+
+/* Bytes of the state arena for `cfg`. Depends on the shapes only, never on a prefix
+ * length (the views are fixed-size: Figure 1 caption, abstract). 0 if cfg is invalid. */
+size_t ls_state_bytes(const ls_config* cfg);
+
+/* Fills *out with the arena layout for `cfg` (host-only computation). */
+int ls_get_layout(const ls_config* cfg, ls_layout* out);
+
+/* Validates cfg, records d_arena (>= ls_state_bytes(cfg) bytes, 256-byte aligned,
+ * caller-owned), zeroes it on `stream` (len = 0, every view empty) and creates the
+ * host handle in *out. The arena must stay allocated until ls_destroy_state.        */
+int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_state** out,
+                  cudaStream_t stream);
+
+/* Workspace bytes that ls_prefill_summary needs for rows [row_begin, row_end). */
+size_t ls_prefill_workspace_bytes(const ls_config* cfg, int64_t row_begin, int64_t row_end);
+
+/* Summary initialisation over the prefix at target prefill (Figure 3 caption).
+ * Appends prefix rows p in [row_begin, min(row_end, prefix_len[b])) of every sequence.
+ *   d_k, d_v       element (b, l, p, h, d) at d_k[(b*L + l)*plane_stride
+ *                  + (p - row_begin)*row_stride + h*D + d]  (`dtype`); row_stride >= Hkv*D,
+ *                  both strides multiples of 8 elements, pointers 16-byte aligned.
+ *   d_prefix_len   int64 [b]: final prefix length P_b of each sequence (0 <= P_b).
+ *   row_begin/end  chunk of positions. Chunks must be passed in order starting at 0,
+ *                  row_begin a multiple of the largest scale, on a state that holds
+ *                  exactly min(row_begin, P_b) rows of each sequence. One call with
+ *                  [0, max P_b) prefills everything.
+ *   d_last_hidden  [b][L][hidden] hidden vectors at position P_b - 1 (becomes the
+ *                  boundary view) or NULL to leave the boundary untouched.
+ *   d_workspace    >= ls_prefill_workspace_bytes(...) bytes of caller scratch.
+ * After the call len = min(row_end, P_b), the window holds the last min(len, W) rows,
+ * the summary covers rows [0, len).                                                  */
+int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t plane_stride,
+                       int64_t row_stride, const int64_t* d_prefix_len, int64_t row_begin,
+                       int64_t row_end, const void* d_last_hidden, void* d_workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
+
+/* One round's view extraction from the target's verification pass (Figure 2 (a)-(b),
+ * Figure 3 caption). Verify row 0 is the previous round's bonus token, rows 1..B the
+ * B drafts; target_ids[i] is the target's greedy choice after verify row i.
+ *   d_draft_ids     int32 [b][B];   d_target_ids int32 [b][B+1]
+ *   d_verify_k/v    `dtype` [b][L][B+1][Hkv][D]
+ *   d_verify_hidden `dtype` [b][L][B+1][hidden]
+ *   d_accept_len    int32 [b] out: a;  d_next_token int32 [b] out: target_ids[a]
+ * Retains verify rows 0..a (Delta = a + 1 <= B + 1): ring window, summary sums,
+ * segment finalisation and mean rows, boundary = verify_hidden[a], len += Delta.   */
+int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
+                    const void* d_verify_k, const void* d_verify_v,
+                    const void* d_verify_hidden, int32_t* d_accept_len,
+                    int32_t* d_next_token, cudaStream_t stream);
+
+/* The drafter's block attention over the three views (Figure 2 (c)).
+ *   layers [layer_begin, layer_begin + layer_count)
+ *   d_q, d_out     `dtype` [b][layer_count][B][Hq][D]
+ *   d_boundary_k/v `dtype`, element (b, l, g, d) at [(b*L + l)*boundary_stride + g*D + d]
+ *                  with l the absolute layer; boundary_stride >= Hkv*D, multiple of 8.
+ *   softmax_scale  logit multiplier (1/sqrt(D) for the usual attention).
+ * Uses the tcgen05 tensor-core kernel when dtype is bf16, (Hq/Hkv)*B == 64, D == 128 and
+ * kv_rows <= 768 (unless LS_FLAG_FORCE_SIMT), otherwise a CUDA-core kernel.          */
+int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count,
+                    const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
+                    int64_t boundary_stride, float softmax_scale, void* d_out,
+                    cudaStream_t stream);
+
+/* 1 if ls_draft_attend takes the tcgen05 path for this state, 0 if the CUDA-core one. */
+int ls_attend_uses_tensor_cores(const ls_state* st);
+
+/* Copies the first `bytes` bytes of the arena to h_dst; synchronises `stream`. */
+int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStream_t stream);
+
+/* Reads the device error word into *h_code (synchronous). Returns LS_ERR_DEVICE or
+ * LS_ERR_DEVICE_TIMEOUT when it is non-zero, LS_OK otherwise.                      */
+int ls_get_error(const ls_state* st, int32_t* h_code);
+
+/* Frees the host handle only; the arena stays the caller's. */
+void ls_destroy_state(ls_state* st);
+
+/* Static description of a status code. */
+const char* ls_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LONGSPARK_H_ */

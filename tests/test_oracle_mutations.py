@@ -1,0 +1,115 @@
+"""Each plausible mistake planted in the oracle must make at least one pin fail.
+
+The mistakes are planted on the CPU, in the oracle only, through monkeypatching; the
+pins are the functions of test_oracle_pins.py.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.longspark_oracle as M
+import tests.test_oracle_pins as P
+
+
+def _patch(monkeypatch, name, fn):
+    monkeypatch.setattr(M, name, fn)
+    monkeypatch.setattr(oracle, name, fn)
+
+
+def _scan_off_by_one(draft, target):
+    a, _ = ORIG["accept_scan"](draft, target)
+    a = min(a + 1, len(draft))
+    return a, int(target[a])
+
+
+def _retain_wrong_slot(sh, v, k_row, v_row):
+    # finalised segment written one slot too far
+    p = v.length
+    v.ring_k[:, :, p % sh.window, :] = k_row
+    v.ring_v[:, :, p % sh.window, :] = v_row
+    for k, s in enumerate(sh.scales):
+        v.part_k[k] += k_row
+        v.part_v[k] += v_row
+        v.part_count[k] += 1
+        if v.part_count[k] == s:
+            j = v.n_seg[k]
+            v.seg_k[k][:, :, (j + 1) % sh.slots, :] = v.part_k[k] / s
+            v.seg_v[k][:, :, (j + 1) % sh.slots, :] = v.part_v[k] / s
+            v.n_seg[k] += 1
+            v.part_k[k] = np.zeros_like(v.part_k[k])
+            v.part_v[k] = np.zeros_like(v.part_v[k])
+            v.part_count[k] = 0
+    v.glob_k += k_row
+    v.glob_v += v_row
+    v.length = p + 1
+
+
+def _scratch_relative_alignment(sh, full_k, full_v, n, boundary=None):
+    # segments aligned to the end of the cache instead of absolute position 0
+    v = ORIG["views_from_scratch"](sh, full_k, full_v, n, boundary)
+    for k, s in enumerate(sh.scales):
+        off = n % s
+        n_c = n // s
+        for j in range(max(0, n_c - sh.slots), n_c):
+            lo = off + j * s
+            v.seg_k[k][:, :, j % sh.slots, :] = full_k[:, :, lo:lo + s, :].mean(axis=2)
+            v.seg_v[k][:, :, j % sh.slots, :] = full_v[:, :, lo:lo + s, :].mean(axis=2)
+    return v
+
+
+def _slots_without_partials(sh, v, l, g, bk, bv):
+    K, V, ok = ORIG["attention_slots"](sh, v, l, g, bk, bv)
+    ok = ok.copy()
+    for k in range(len(sh.scales)):
+        ok[1 + sh.window + k * (sh.slots + 1) + sh.slots] = False
+    return K, V, ok
+
+
+def _attend_wrong_group(sh, v, q, bk, bv, scale):
+    out = np.zeros_like(q)
+    for l in range(sh.n_layers):
+        for qh in range(sh.n_q_heads):
+            K, V, ok = M.attention_slots(sh, v, l, qh % sh.n_kv_heads, bk, bv)
+            lg = q[l, :, qh] @ K.T * scale
+            lg[:, ~ok] = -np.inf
+            w = np.exp(lg - lg.max(axis=1, keepdims=True))
+            out[l, :, qh] = (w / w.sum(axis=1, keepdims=True)) @ V
+    return out
+
+
+def _slots_window_mask_off_by_one(sh, v, l, g, bk, bv):
+    K, V, ok = ORIG["attention_slots"](sh, v, l, g, bk, bv)
+    ok = ok.copy()
+    for r in range(sh.window):
+        ok[1 + r] = r <= v.length
+    return K, V, ok
+
+
+def _retain_global_skips(sh, v, k_row, v_row):
+    ORIG["retain_row"](sh, v, k_row, v_row)
+    if v.length == 1:  # first row never reaches the global sum
+        v.glob_k -= k_row
+        v.glob_v -= v_row
+
+
+ORIG = {n: getattr(M, n) for n in ("accept_scan", "retain_row", "views_from_scratch",
+                                   "attention_slots", "draft_attend")}
+
+CASES = [
+    ("accept_scan", _scan_off_by_one, [P.test_scan_golden_examples]),
+    ("retain_row", _retain_wrong_slot, [lambda: P.test_ramp_closed_forms(513)]),
+    ("views_from_scratch", _scratch_relative_alignment, [lambda: P.test_incremental_equals_recompute(123)]),
+    ("attention_slots", _slots_without_partials, [P.test_golden_worked_example]),
+    ("draft_attend", _attend_wrong_group, [P.test_attend_matches_torch_sdpa]),
+    ("attention_slots", _slots_window_mask_off_by_one, [P.test_mask_counts]),
+    ("retain_row", _retain_global_skips, [lambda: P.test_ramp_closed_forms(200)]),
+]
+
+
+@pytest.mark.parametrize("name,fn,pins", CASES, ids=[f"{c[0]}:{c[1].__name__}" for c in CASES])
+def test_planted_mistake_is_caught(monkeypatch, name, fn, pins):
+    _patch(monkeypatch, name, fn)
+    for pin in pins:
+        with pytest.raises(AssertionError):
+            pin()

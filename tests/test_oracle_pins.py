@@ -1,0 +1,335 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test checks one piece of the oracle against a closed form, a brute-force
+enumeration, a hand-worked example (tests/golden/), an invariant the method states, or
+a library routine. The sources: LongSpark paper page (thelatestinai.com), Figure 2
+caption (round structure), Figure 3 caption (incremental summary, Delta <= B + 1),
+Figure 1 caption (fixed-size state), Table 3 caption (greedy T = 0 acceptance).
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _shapes(**kw):
+    base = dict(n_layers=2, n_kv_heads=2, n_q_heads=4, head_dim=8, hidden=32, block=4,
+                window=8, scales=(5, 10, 40), slots=3)
+    base.update(kw)
+    return O.Shapes(**base)
+
+
+def _rows(rng, L, H, n, D):
+    return rng.standard_normal((L, H, n, D))
+
+
+# ---------------------------------------------------------------------------------
+# accept scan
+# ---------------------------------------------------------------------------------
+def test_scan_exhaustive_b16():
+    """All 2^16 agreement patterns: a = count of leading agreements (cumulative product)."""
+    B = 16
+    masks = np.arange(1 << B, dtype=np.int64)
+    agree = ((masks[:, None] >> np.arange(B)[None, :]) & 1) == 0  # bit set = disagreement
+    brute = np.cumprod(agree, axis=1).sum(axis=1)
+    draft = np.arange(B) + 100
+    for m in range(1 << B):
+        target = np.concatenate([draft + ((m >> np.arange(B)) & 1) * 7, [9999]])
+        a, nxt = O.accept_scan(draft, target)
+        assert a == brute[m]
+        assert nxt == (target[a])
+        assert a + 1 <= B + 1
+
+
+def test_scan_golden_examples():
+    with open(os.path.join(GOLDEN, "accept_scan_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        a, nxt = O.accept_scan(c["draft"], c["target"])
+        assert (a, nxt, a + 1) == (c["a"], c["next"], c["delta"])
+
+
+# ---------------------------------------------------------------------------------
+# summary and window
+# ---------------------------------------------------------------------------------
+def _full_cache_run(sh, rng, P, accepts):
+    """Prefill P random rows, commit rounds with the given accepts; return (views, cache)."""
+    L, H, D, B = sh.n_layers, sh.n_kv_heads, sh.head_dim, sh.block
+    pk = rng.standard_normal((L, P, H, D))
+    pv = rng.standard_normal((L, P, H, D))
+    hid = rng.standard_normal((L, sh.hidden))
+    v = O.prefill(sh, pk, pv, P, hid)
+    cache_k = [np.transpose(pk, (0, 2, 1, 3))]
+    cache_v = [np.transpose(pv, (0, 2, 1, 3))]
+    for a in accepts:
+        draft = rng.integers(0, 50, B)
+        target = np.concatenate([draft, [0]]).copy()
+        if a < B:
+            target[a] = draft[a] + 1
+        vk = rng.standard_normal((L, B + 1, H, D))
+        vv = rng.standard_normal((L, B + 1, H, D))
+        vh = rng.standard_normal((L, B + 1, sh.hidden))
+        got_a, _ = O.commit_round(sh, v, draft, target, vk, vv, vh)
+        assert got_a == a
+        cache_k.append(np.transpose(vk[:, :a + 1], (0, 2, 1, 3)))
+        cache_v.append(np.transpose(vv[:, :a + 1], (0, 2, 1, 3)))
+    return v, np.concatenate(cache_k, axis=2), np.concatenate(cache_v, axis=2)
+
+
+def _assert_views_close(sh, a, b, rtol=1e-12):
+    assert a.length == b.length
+    assert a.n_seg == b.n_seg and a.part_count == b.part_count
+    np.testing.assert_array_equal(a.ring_k, b.ring_k)
+    np.testing.assert_array_equal(a.ring_v, b.ring_v)
+    for k in range(len(sh.scales)):
+        filled = min(a.n_seg[k], sh.slots)
+        np.testing.assert_allclose(a.seg_k[k][:, :, :filled], b.seg_k[k][:, :, :filled], rtol=rtol, atol=1e-12)
+        np.testing.assert_allclose(a.seg_v[k][:, :, :filled], b.seg_v[k][:, :, :filled], rtol=rtol, atol=1e-12)
+        np.testing.assert_allclose(a.part_k[k], b.part_k[k], rtol=rtol, atol=1e-11)
+        np.testing.assert_allclose(a.part_v[k], b.part_v[k], rtol=rtol, atol=1e-11)
+    np.testing.assert_allclose(a.glob_k, b.glob_k, rtol=rtol, atol=1e-10)
+    np.testing.assert_allclose(a.glob_v, b.glob_v, rtol=rtol, atol=1e-10)
+
+
+@pytest.mark.parametrize("P", [0, 1, 7, 40, 123])
+def test_incremental_equals_recompute(P):
+    """Figure 3: updating with only the new rows N equals the summary of the whole cache."""
+    sh = _shapes()
+    rng = np.random.default_rng(P)
+    accepts = rng.integers(0, sh.block + 1, 30)
+    v, ck, cv = _full_cache_run(sh, rng, P, accepts)
+    ref = O.views_from_scratch(sh, ck, cv, ck.shape[2])
+    _assert_views_close(sh, v, ref)
+
+
+def test_fold_from_empty_equals_recompute():
+    """Folding every row one by one from an empty state equals the definition."""
+    sh = _shapes(scales=(4, 8, 32), slots=2, window=5)
+    rng = np.random.default_rng(5)
+    n = 97
+    fk, fv = _rows(rng, 2, 2, n, 8), _rows(rng, 2, 2, n, 8)
+    v = O.empty_views(sh)
+    for p in range(n):
+        O.retain_row(sh, v, fk[:, :, p], fv[:, :, p])
+    _assert_views_close(sh, v, O.views_from_scratch(sh, fk, fv, n))
+
+
+def _ramp_cache(L, H, n, D):
+    p = np.arange(n).reshape(1, 1, n, 1).astype(np.float64)
+    h = np.arange(H).reshape(1, H, 1, 1)
+    l = np.arange(L).reshape(L, 1, 1, 1)
+    d = np.arange(D).reshape(1, 1, 1, D)
+    k = p + 1000.0 * h + 10000.0 * l + 0.25 * d + np.zeros((L, H, n, D))
+    return k, -3.0 * k
+
+
+@pytest.mark.parametrize("n", [0, 3, 64, 200, 511, 512, 513])
+def test_ramp_closed_forms(n):
+    """K = p + const: segment j of scale s has mean j*s + (s-1)/2 + const, exactly."""
+    sh = _shapes(scales=(8, 32, 128), slots=4, window=32, head_dim=4)
+    L, H, D = sh.n_layers, sh.n_kv_heads, sh.head_dim
+    fk, fv = _ramp_cache(L, H, n, D)
+    # incremental fold, the form the round uses
+    v = O.empty_views(sh)
+    for p in range(n):
+        O.retain_row(sh, v, fk[:, :, p], fv[:, :, p])
+    const = (1000.0 * np.arange(H)[None, :, None] + 10000.0 * np.arange(L)[:, None, None]
+             + 0.25 * np.arange(D)[None, None, :])
+    for k, s in enumerate(sh.scales):
+        n_c = n // s
+        assert v.n_seg[k] == n_c and v.part_count[k] == n - n_c * s
+        for j in range(max(0, n_c - sh.slots), n_c):
+            want = j * s + (s - 1) / 2.0 + const
+            assert np.array_equal(v.seg_k[k][:, :, j % sh.slots], want)
+            assert np.array_equal(v.seg_v[k][:, :, j % sh.slots], -3.0 * want)
+        c = n - n_c * s
+        # partial = sum of rows n_c*s .. n-1 = c*n_c*s + c(c-1)/2 + c*const
+        want_part = c * n_c * s + c * (c - 1) / 2.0 + c * const
+        assert np.array_equal(v.part_k[k], want_part)
+    assert np.array_equal(v.glob_k, n * (n - 1) / 2.0 + n * const)
+    # window: ring slot r holds row p with p = r mod W and len - W <= p < len
+    for r in range(sh.window):
+        ps = [p for p in range(max(0, n - sh.window), n) if p % sh.window == r]
+        if ps:
+            assert np.array_equal(v.ring_k[:, :, r], ps[0] + const)
+
+
+def test_constant_rows_give_exact_means():
+    sh = _shapes(scales=(3, 9, 27), slots=2)
+    c = 0.375
+    n = 100
+    fk = np.full((2, 2, n, 8), c)
+    v = O.views_from_scratch(sh, fk, -fk, n)
+    for k in range(3):
+        assert np.all(v.seg_k[k][:, :, :min(v.n_seg[k], 2)] == c)
+        if v.part_count[k]:
+            assert np.all(v.part_k[k] / v.part_count[k] == c)
+    assert np.all(v.glob_k / n == c)
+
+
+def test_window_is_last_w_rows():
+    sh = _shapes(window=7)
+    rng = np.random.default_rng(1)
+    v, ck, cv = _full_cache_run(sh, rng, 30, rng.integers(0, 5, 12))
+    n = v.length
+    for p in range(n - sh.window, n):
+        assert np.array_equal(v.ring_k[:, :, p % sh.window], ck[:, :, p])
+        assert np.array_equal(v.ring_v[:, :, p % sh.window], cv[:, :, p])
+
+
+def test_boundary_is_last_retained_position():
+    """The boundary view is the hidden state at position len - 1 after every round."""
+    sh = _shapes()
+    rng = np.random.default_rng(2)
+    L, H, D, B = sh.n_layers, sh.n_kv_heads, sh.head_dim, sh.block
+    P = 20
+    hid = np.full((L, sh.hidden), P - 1.0)
+    v = O.prefill(sh, np.zeros((L, P, H, D)), np.zeros((L, P, H, D)), P, hid)
+    assert np.all(v.boundary == v.length - 1)
+    for a in [0, 4, 2, 1, 3]:
+        draft = np.arange(B)
+        target = np.concatenate([draft, [0]])
+        if a < B:
+            target[a] += 1
+        # verify row i sits at absolute position len + i
+        vh = (v.length + np.arange(B + 1, dtype=np.float64)).reshape(1, B + 1, 1) * np.ones((L, 1, sh.hidden))
+        O.commit_round(sh, v, draft, target, np.zeros((L, B + 1, H, D)), np.zeros((L, B + 1, H, D)), vh)
+        assert np.all(v.boundary == v.length - 1)
+
+
+def test_golden_worked_example():
+    with open(os.path.join(GOLDEN, "ramp_worked_example.json")) as f:
+        g = json.load(f)
+    s = g["shapes"]
+    sh = O.Shapes(n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=1, hidden=1, block=1,
+                  window=s["window"], scales=tuple(s["scales"]), slots=s["slots"])
+    n = g["length"]
+    p = np.arange(n, dtype=np.float64).reshape(1, 1, n, 1)
+    v = O.views_from_scratch(sh, p, 10 * p, n)
+    assert v.ring_k[0, 0, :, 0].tolist() == g["ring_k"]
+    assert [v.seg_k[k][0, 0, :, 0].tolist() for k in range(2)] == g["seg_k"]
+    assert v.n_seg == g["n_seg"] and v.part_count == g["part_count"]
+    assert [float(v.part_k[k][0, 0, 0]) for k in range(2)] == g["part_k"]
+    assert float(v.glob_k[0, 0, 0]) == g["glob_k"]
+    # the same by folding row by row
+    w = O.empty_views(sh)
+    for i in range(n):
+        O.retain_row(sh, w, p[:, :, i], 10 * p[:, :, i])
+    _assert_views_close(sh, v, w)
+    out = O.draft_attend(sh, v, np.zeros((1, 1, 1, 1)), np.zeros((1, 1, 1)), np.full((1, 1, 1), 100.0), 1.0)
+    assert abs(out[0, 0, 0, 0] - g["attend_q0_out"]) < 1e-12
+
+
+def test_state_bytes_do_not_depend_on_prefix():
+    """Figure 1 caption: the drafter state does not grow with the prefix (4K vs 128K)."""
+    sh = _shapes(n_layers=1, n_kv_heads=1, n_q_heads=2, head_dim=4, hidden=16,
+                 window=512, scales=(64, 512, 4096), slots=32, block=16)
+    sizes = []
+    for n in (4096, 131072):
+        fk = np.ones((1, 1, n, 4))
+        v = O.views_from_scratch(sh, fk, fk, n)
+        sizes.append(O.state_bytes(sh, v))
+    assert sizes[0] == sizes[1]
+
+
+# ---------------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------------
+def _random_views(sh, rng, P, rounds):
+    v, _, _ = _full_cache_run(sh, rng, P, rng.integers(0, sh.block + 1, rounds))
+    return v
+
+
+def test_attend_matches_scalar_loops():
+    """Brute force with Python scalars and math.exp on a tiny case."""
+    sh = _shapes(n_layers=1, n_kv_heads=2, n_q_heads=4, head_dim=3, window=4,
+                 scales=(5, 10), slots=2, block=2)
+    rng = np.random.default_rng(3)
+    v = _random_views(sh, rng, 13, 4)
+    q = rng.standard_normal((1, 2, 4, 3))
+    bk, bv = rng.standard_normal((1, 2, 3)), rng.standard_normal((1, 2, 3))
+    scale = 0.7
+    out = O.draft_attend(sh, v, q, bk, bv, scale)
+    for qh in range(4):
+        g = qh // 2
+        K, V, ok = O.attention_slots(sh, v, 0, g, bk, bv)
+        for i in range(2):
+            logits = [sum(float(q[0, i, qh, d]) * float(K[s, d]) for d in range(3)) * scale
+                      for s in range(len(K))]
+            mx = max(lg for lg, o in zip(logits, ok) if o)
+            ws = [math.exp(lg - mx) if o else 0.0 for lg, o in zip(logits, ok)]
+            tot = sum(ws)
+            for d in range(3):
+                want = sum(w * float(V[s, d]) for s, w in enumerate(ws)) / tot
+                assert abs(out[0, i, qh, d] - want) < 1e-12
+
+
+def test_attend_matches_torch_sdpa():
+    """Library cross-check: torch scaled_dot_product_attention in fp64 with a mask."""
+    sh = _shapes(head_dim=16, window=16, scales=(5, 10, 20), slots=3, block=4)
+    rng = np.random.default_rng(4)
+    v = _random_views(sh, rng, 57, 9)
+    q = rng.standard_normal((2, 4, 4, 16))
+    bk, bv = rng.standard_normal((2, 2, 16)), rng.standard_normal((2, 2, 16))
+    out = O.draft_attend(sh, v, q, bk, bv, 0.25)
+    for l in range(2):
+        for qh in range(4):
+            K, V, ok = O.attention_slots(sh, v, l, qh // 2, bk, bv)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[l, :, qh][None]), torch.from_numpy(K[None]),
+                torch.from_numpy(V[None]), attn_mask=torch.from_numpy(ok)[None, None, :].expand(1, 4, -1),
+                scale=0.25)
+            np.testing.assert_allclose(out[l, :, qh], ref[0].numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_attend_special_cases():
+    sh = _shapes(n_layers=1, n_kv_heads=1, n_q_heads=2, head_dim=4, window=4,
+                 scales=(5, 10), slots=2, block=2)
+    rng = np.random.default_rng(6)
+    bk, bv = rng.standard_normal((1, 1, 4)), rng.standard_normal((1, 1, 4))
+    # empty state: only the boundary slot is valid -> output is exactly its value
+    v0 = O.empty_views(sh)
+    out = O.draft_attend(sh, v0, rng.standard_normal((1, 2, 2, 4)), bk, bv, 1.0)
+    assert np.array_equal(out[0, 0, 0], bv[0, 0]) and np.array_equal(out[0, 1, 1], bv[0, 0])
+    # q = 0: uniform weights -> mean of the valid values
+    v = _random_views(sh, rng, 23, 5)
+    K, V, ok = O.attention_slots(sh, v, 0, 0, bk, bv)
+    out = O.draft_attend(sh, v, np.zeros((1, 2, 2, 4)), bk, bv, 1.0)
+    np.testing.assert_allclose(out[0, 0, 0], V[ok].mean(axis=0), rtol=1e-12, atol=1e-14)
+    # identical keys everywhere -> again the mean of the valid values
+    n = 23
+    fk = np.ones((1, 1, n, 4))
+    fv = rng.standard_normal((1, 1, n, 4))
+    w = O.views_from_scratch(sh, fk, fv, n)
+    K, V, ok = O.attention_slots(sh, w, 0, 0, np.ones((1, 1, 4)), bv)
+    out = O.draft_attend(sh, w, rng.standard_normal((1, 2, 2, 4)), np.ones((1, 1, 4)), bv, 1.0)
+    np.testing.assert_allclose(out[0, 1, 0], V[ok].mean(axis=0), rtol=1e-12, atol=1e-14)
+    assert ok.sum() == 1 + 4 + (2 + 1) + (2 + 1) + 1
+
+
+def test_mask_counts():
+    """Valid slot count = boundary + min(len, W) + per scale min(n_c, slots) + [partial] + [len>0]."""
+    sh = _shapes(n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=2, window=16,
+                 scales=(4, 16, 64), slots=3)
+    for n in [0, 1, 3, 4, 15, 16, 17, 63, 64, 65, 200]:
+        fk = np.ones((1, 1, n, 2))
+        v = O.views_from_scratch(sh, fk, fk, n)
+        _, _, ok = O.attention_slots(sh, v, 0, 0, np.ones((1, 1, 2)), np.ones((1, 1, 2)))
+        want = 1 + min(n, 16) + sum(min(n // s, 3) + (1 if n % s else 0) for s in (4, 16, 64)) + (1 if n else 0)
+        assert ok.sum() == want and len(ok) == sh.n_attn_slots
+
+
+def test_to_f64_exact():
+    bits = np.array([0x3F80, 0xC000, 0x0001, 0x7F7F], dtype=np.uint16)
+    got = O.to_f64(bits, O.BF16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(got, ref)

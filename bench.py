@@ -1,0 +1,535 @@
+"""Benchmark of the LongSpark drafting round on B200.
+
+One step = one decoding round of the hot path over a batch of 16 sequences at Qwen3-8B
+shapes with a 64K-token prefix: ``ls_commit_round`` (accept scan, ring-window commit,
+summary update, boundary gather) followed by ``ls_draft_attend`` over all 4 tapped layers.
+The prefill summary over the prefix runs once per request before the rounds; it is timed
+separately in the same run and reported under ``prefill``.
+
+Timing: W untimed warm-up rounds, then K timed rounds. Before every round a 256 MB
+buffer is written (untimed) so that the round starts with a cold L2, as it would after
+the target's verification pass; each round is bracketed by CUDA events on the launching
+stream (a third event splits commit from attention). ``value`` is rounds per second over
+all ranks (weak scaling: every rank owns its own batch of 16 sequences).
+
+``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "draft rounds/s at batch 16 (Qwen3-8B shapes), 32K-128K prefix; % HBM roofline"
+WORKLOAD = "qwen3_8b_64k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------------------
+# multi-rank plumbing (host logic; covered by CPU gloo tests)
+# ---------------------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def sequence_offset(rank: int, batch_per_rank: int) -> int:
+    """First global sequence index owned by `rank` (weak scaling: disjoint batches)."""
+    return rank * batch_per_rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------
+# algorithmic bytes (the layout built: bf16 window and mean rows, fp32 summary sums)
+# ---------------------------------------------------------------------------------------
+def attend_bytes(wl) -> int:
+    e = wl.elem()
+    b, L, H, Hq, D, B = wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.block
+    summary_rows = len(wl.scales) * (wl.slots + 1) + 1
+    return (2 * b * L * B * Hq * D * e                # Q in, O out
+            + b * L * H * wl.window * 2 * D * e        # ring window K/V
+            + b * L * H * summary_rows * 2 * D * e     # summary mean rows K/V
+            + b * L * H * 2 * D * e                    # boundary K/V
+            + b * L * (1 + len(wl.scales)) * 8)        # counters
+
+
+def commit_bytes(wl, mean_delta: float) -> int:
+    e = wl.elem()
+    b, L, H, D, nsc = wl.batch, wl.n_layers, wl.n_kv_heads, wl.head_dim, len(wl.scales)
+    rows = b * mean_delta * L * H * 2 * D * e
+    return int(2 * rows                                          # read retained rows, write ring
+               + 2 * b * L * H * (nsc + 1) * 2 * D * 4           # fp32 partial + global RMW
+               + b * L * H * 2 * D * (4 + e) * sum(mean_delta / s for s in wl.scales)  # finalised means
+               + b * L * H * (nsc + 1) * 2 * D * e               # partial/global mean rows
+               + 2 * b * L * wl.hidden * e                       # boundary gather
+               + b * (2 * wl.block + 1) * 4 + 8 * b              # token ids, outputs
+               + 2 * b * L * (1 + nsc) * 8)                      # counters
+
+
+def prefill_bytes(wl, prefix_len) -> int:
+    return int(np.sum(prefix_len)) * wl.n_layers * wl.n_kv_heads * wl.head_dim * 2 * wl.elem()
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha(name: str) -> str:
+    p = os.path.join(ROOT, "fixed_cost_drafter_b200", "csrc", name)
+    h = hashlib.sha256()
+    for q in (p, os.path.join(ROOT, "fixed_cost_drafter_b200", "csrc", "ls_common.cuh")):
+        with open(q, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, key: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches the source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            rec = json.load(f)
+        ent = rec.get(key)
+        if ent and ent.get("source_sha") == kernel_source_sha(kernel_file):
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, path: str):
+        self.path, self.proc, self.gpu = path, None, gpu_index
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        rows = rows[1:] if len(rows) > 1 else rows  # the first sample may precede the load
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, v in enumerate(flags) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------------------
+class OracleSample:
+    """The CPU oracle on a bounded slice of the workload: one tapped layer of sequence 0.
+
+    The oracle's views are fixed-size, so its per-round work does not depend on the
+    prefix: the views are initialised (untimed) from the first ``prefix_rows`` prefix rows.
+    One step = the oracle's round for that (sequence, layer): commit of the retained rows
+    and the attention of all query heads; a full round is batch x layers such steps.
+    """
+
+    def __init__(self, wl, prefix_rows: int = 4096, n_inputs: int = 16):
+        import oracle as O
+        import synth as S
+        self.O, self.wl = O, wl
+        H, Hq, D, B = wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.block
+        self.sh = O.Shapes(n_layers=1, n_kv_heads=H, n_q_heads=Hq, head_dim=D, hidden=wl.hidden, block=B,
+                           window=wl.window, scales=tuple(wl.scales), slots=wl.slots)
+        scale = S.head_scales(wl.seed, wl.n_layers, H) if wl.head_scale else None
+        P = prefix_rows
+        f = lambda tid, shape, **kw: O.to_f64(S.fill_normal(wl.seed, tid, shape, **kw), wl.dtype)  # noqa: E731
+        pk = f(S.PREFIX_K, (1, 1, 1, P, H * D), head_dim=D, scale=scale)[0, 0]
+        pv = f(S.PREFIX_V, (1, 1, 1, P, H * D), head_dim=D, scale=scale)[0, 0]
+        hid = f(S.LAST_HIDDEN, (1, 1, 1, 1, wl.hidden))[0, 0, :, 0]
+        self.views = O.prefill(self.sh, pk.reshape(1, P, H, D), pv.reshape(1, P, H, D), P, hid)
+        acc = S.accept_lengths(wl.seed, n_inputs, 1, B, wl.accept_mean)
+        self.draft, self.target = S.token_ids(wl.seed, n_inputs, 1, B, acc, wl.vocab)
+        self.inputs = []
+        for r in range(n_inputs):
+            vk = f(S.VERIFY_K, (1, 1, 1, B + 1, H * D), r0=r, head_dim=D, scale=scale)[0, 0].reshape(1, B + 1, H, D)
+            vv = f(S.VERIFY_V, (1, 1, 1, B + 1, H * D), r0=r, head_dim=D, scale=scale)[0, 0].reshape(1, B + 1, H, D)
+            vh = f(S.VERIFY_HIDDEN, (1, 1, 1, B + 1, wl.hidden), r0=r)[0, 0]
+            q = f(S.QUERY, (1, 1, 1, B, Hq * D), r0=r, head_dim=D)[0, 0].reshape(1, B, Hq, D)
+            self.inputs.append((vk, vv, vh, q))
+        self.step_no = 0
+        self.sm = 1.0 / math.sqrt(D)
+
+    def step(self) -> float:
+        """Seconds for one oracle (sequence, layer) round slice."""
+        O, wl = self.O, self.wl
+        H, D = wl.n_kv_heads, wl.head_dim
+        r = self.step_no % len(self.inputs)
+        self.step_no += 1
+        vk, vv, vh, q = self.inputs[r]
+        t0 = time.perf_counter()
+        O.commit_round(self.sh, self.views, self.draft[r, 0], self.target[r, 0], vk, vv, vh)
+        bk = self.views.boundary[:, :H * D].reshape(1, H, D)
+        bv = self.views.boundary[:, H * D:2 * H * D].reshape(1, H, D)
+        O.draft_attend(self.sh, self.views, q, bk, bv, self.sm)
+        return time.perf_counter() - t0
+
+    def slices_per_round(self) -> int:
+        return self.wl.batch * self.wl.n_layers
+
+
+def cpu_baseline(wl, budget_s: float = 15.0):
+    from threadpoolctl import threadpool_limits
+    smp = OracleSample(wl)
+    with threadpool_limits(limits=1):
+        smp.step()
+        times = []
+        t_end = time.perf_counter() + budget_s
+        while time.perf_counter() < t_end or len(times) < 3:
+            times.append(smp.step())
+    per_round = float(np.mean(times)) * smp.slices_per_round()
+    return {"value": 1.0 / per_round, "unit": "rounds/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(times)} oracle round slices (commit + attention of all {wl.n_q_heads} query "
+                      f"heads for one tapped layer of sequence 0), mean x {smp.slices_per_round()} "
+                      f"(= {wl.batch} sequences x {wl.n_layers} layers); views initialised from a 4096-row "
+                      f"prefix (the oracle's per-round work does not depend on the prefix)"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from threadpoolctl import threadpool_limits
+    from fixed_cost_drafter_b200 import workloads as WLM
+    wl = WLM.CONFIGS[args.config]
+    smp = OracleSample(wl)
+    with threadpool_limits(limits=1):
+        for _ in range(args.warmup):
+            smp.step()
+        times = [smp.step() for _ in range(args.steps)]
+    per_round = float(np.mean(times)) * smp.slices_per_round()
+    v = 1.0 / per_round
+    sample = (f"each step: the oracle's round for one tapped layer of sequence 0 (commit + attention of "
+              f"all {wl.n_q_heads} query heads); a round of the workload = {smp.slices_per_round()} such "
+              f"slices ({wl.batch} sequences x {wl.n_layers} layers); 1 thread")
+    line = {"metric": METRIC, "value": v, "unit": "rounds/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": per_round * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": workload_config(wl),
+            "cpu_baseline": {"value": v, "unit": "rounds/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "rounds/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(wl):
+    return {"workload": f"{wl.name}: batch {wl.batch}, {wl.n_layers} tapped layers, {wl.n_kv_heads} KV / "
+                        f"{wl.n_q_heads} query heads, head_dim {wl.head_dim}, hidden {wl.hidden}, B {wl.block}, "
+                        f"W {wl.window}, summary scales {'/'.join(map(str, wl.scales))} x {wl.slots} slots + "
+                        f"partials + global mean, prefix {wl.prefix}",
+            "batch": wl.batch, "prefix": wl.prefix if not isinstance(wl.prefix, tuple) else list(wl.prefix),
+            "accept_mean": wl.accept_mean,
+            "l2": "flushed before every timed round (256 MB write, untimed)"}
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import fixed_cost_drafter_b200 as F
+    from fixed_cost_drafter_b200 import workloads as WLM
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = WLM.CONFIGS[args.config]
+    K, W = args.steps, args.warmup
+    # distinct rounds of generated inputs; the timed loop cycles through them (the state
+    # keeps growing, every round re-reads its inputs from HBM after the L2 flush)
+    n_rounds = min(K + W, args.distinct_rounds)
+    run = WLM.DeviceRun(wl, device=dev, rounds=n_rounds, seq_offset=sequence_offset(rank, wl.batch))
+
+    # prefill (timed separately)
+    pre = []
+    run.prefill(timer=lambda e0, e1, nbytes: pre.append((e0, e1, nbytes)))
+    torch.cuda.synchronize()
+    prefill_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in pre)
+    prefill_b = sum(n for _, _, n in pre)
+
+    inp = run.make_round_inputs(0, n_rounds)
+    out = run.new_out()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = run.stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    clock_path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "_build",
+                              f"clocks_rank{rank}.csv")
+    os.makedirs(os.path.dirname(clock_path), exist_ok=True)
+    # the sampler starts with the warm-up rounds so that its samples cover a loaded GPU
+    with ClockSampler(local, clock_path) as clk:
+        for r in range(W):
+            flush.zero_()
+            run.commit(inp, r % n_rounds)
+            run.attend(inp, r % n_rounds, out)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(K):
+            r = (W + i) % n_rounds
+            flush.zero_()
+            evs[i][0].record(stream)
+            run.commit(inp, r)
+            evs[i][1].record(stream)
+            run.attend(inp, r, out)
+            evs[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    commit_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    attend_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    round_ms = [a + c for a, c in zip(attend_ms, commit_ms)]
+    total_s = sum(round_ms) / 1e3
+    total_max = max_over_ranks(total_s, world, dev)
+    status, word = run.error()
+    if status != F.LS_OK:
+        raise RuntimeError(f"device error word {word:#x} after the timed rounds")
+
+    # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
+    graph_rps = None
+    if not args.no_graph:
+        g = torch.cuda.CUDAGraph()
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(gs):
+            run.stream = gs
+            with torch.cuda.graph(g, stream=gs):
+                for j in range(8):
+                    run.commit(inp, j % n_rounds)
+                    run.attend(inp, j % n_rounds, out)
+        run.stream = stream
+        torch.cuda.current_stream(dev).wait_stream(gs)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        reps = 20
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        graph_rps = 8 * reps / (e0.elapsed_time(e1) / 1e3)
+        del g
+
+    # end to end through the public API with host buffers (pinned), copies inside the region
+    e2e = e2e_measure(run, wl, dev, flush, K, world, inp)
+
+    # flatness over the prefix (b = 16) on a short sweep
+    flat = None
+    if not args.no_sweep and rank == 0:
+        flat = flatness_sweep(WLM, dev, flush, args.sweep_rounds)
+
+    peak, peak_kind = hbm_peak()
+    a_bytes = attend_bytes(wl)
+    deltas = run.accept_host[[(W + i) % n_rounds for i in range(K)]] + 1
+    c_bytes = commit_bytes(wl, float(deltas.mean()))
+    att_s = float(np.mean(attend_ms)) / 1e3
+    rnd_s = float(np.mean(round_ms)) / 1e3
+    achieved = a_bytes / att_s / 1e9
+    traffic = recorded_traffic("ls_attend_tc.cu" if F.ls_attend_uses_tensor_cores(run.state)
+                               else "ls_attend_simt.cu", f"attend_{wl.name}")
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * K / total_max, "unit": "rounds/s", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": total_max * 1e3 / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(wl),
+            "roofline": {"bound": "hbm", "kernel": "ls_draft_attend ("
+                         + ("tcgen05" if F.ls_attend_uses_tensor_cores(run.state) else "CUDA cores") + ")",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": a_bytes},
+            "round_roofline": {"bytes": a_bytes + c_bytes, "achieved": (a_bytes + c_bytes) / rnd_s / 1e9,
+                               "frac": (a_bytes + c_bytes) / rnd_s / 1e9 / peak, "unit": "GB/s"},
+            "us_per_round": {"median": float(np.median(round_ms)) * 1e3, "p90": float(np.percentile(round_ms, 90)) * 1e3,
+                             "commit_mean": float(np.mean(commit_ms)) * 1e3,
+                             "attend_mean": float(np.mean(attend_ms)) * 1e3},
+            "commit": {"bytes": c_bytes, "achieved_GBps": c_bytes / (np.mean(commit_ms) / 1e3) / 1e9},
+            "graph_rounds_per_s": graph_rps,
+            "prefill": {"ms": prefill_ms, "bytes": prefill_b, "achieved_GBps": prefill_b / (prefill_ms / 1e3) / 1e9,
+                        "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
+            "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch,
+            "flatness": flat,
+            "gpu_launches": 2 * K,
+            "e2e": e2e,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget)
+        print(json.dumps(line))
+    run.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_measure(run, wl, dev, flush, steps, world, inp):
+    """Rounds/s through the public entry points with inputs and results in pinned host memory."""
+    import torch
+    import fixed_cost_drafter_b200 as F
+    n_distinct = min(8, run.rounds)
+    host = []
+    for r in range(n_distinct):
+        host.append({k: inp[k][r].cpu().pin_memory() for k in ("vk", "vv", "vh", "q")}
+                    | {"draft": run.draft[r].cpu().pin_memory(), "target": run.target[r].cpu().pin_memory()})
+    dev_buf = {k: torch.empty_like(v, device=dev) for k, v in host[0].items()}
+    out = run.new_out()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_acc = torch.empty(wl.batch, dtype=torch.int32).pin_memory()
+    h_nxt = torch.empty(wl.batch, dtype=torch.int32).pin_memory()
+    s = run.stream
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+    d2h = h_out.numel() * h_out.element_size() + 8 * wl.batch
+    steps = max(3, min(steps, 50))
+    times = []
+    for i in range(steps + 3):
+        hb = host[i % n_distinct]
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for k, v in hb.items():
+            dev_buf[k].copy_(v, non_blocking=True)
+        F.ls_commit_round(run.state, dev_buf["draft"], dev_buf["target"], dev_buf["vk"], dev_buf["vv"],
+                          dev_buf["vh"], run.accept_len, run.next_token, s)
+        F.ls_draft_attend(run.state, 0, wl.n_layers, dev_buf["q"], run.boundary_k, run.boundary_v, wl.hidden,
+                          run.softmax_scale, out, s)
+        h_out.copy_(out, non_blocking=True)
+        h_acc.copy_(run.accept_len, non_blocking=True)
+        h_nxt.copy_(run.next_token, non_blocking=True)
+        e1.record(s)
+        e1.synchronize()
+        if i >= 3:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    tot = max_over_ranks(sum(times), world, dev)
+    return {"value": world * len(times) / tot, "unit": "rounds/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": len(times)}
+
+
+def flatness_sweep(WLM, dev, flush, rounds):
+    """Per-round time at batch 16 over prefixes 4K..128K (accept mean 4.0)."""
+    import torch
+    res = {}
+    for P in WLM.SWEEP_PREFIXES:
+        wl = WLM.sweep_point(P, 16, 4.0)
+        run = WLM.DeviceRun(wl, device=dev, rounds=rounds)
+        run.prefill()
+        inp = run.make_round_inputs(0, rounds)
+        out = run.new_out()
+        ms = []
+        for r in range(rounds):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(run.stream)
+            run.commit(inp, r)
+            run.attend(inp, r, out)
+            e1.record(run.stream)
+            e1.synchronize()
+            if r >= 3:
+                ms.append(e0.elapsed_time(e1))
+        res[str(P)] = float(np.median(ms)) * 1e3
+        run.close()
+        del run, inp, out
+        torch.cuda.empty_cache()
+    v = list(res.values())
+    return {"us_per_round": res, "flatness": (max(v) - min(v)) / min(v), "batch": 16, "accept_mean": 4.0}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--distinct-rounds", type=int, default=128)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=WORKLOAD)
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--sweep-rounds", type=int, default=40)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

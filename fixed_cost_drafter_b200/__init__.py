@@ -1,0 +1,200 @@
+"""Python binding of the LongSpark fixed-cost drafting round (C ABI: include/longspark.h).
+
+Argument marshalling only: every function forwards to the entry point of the same name
+in ``liblongspark.so``; every step of the path runs in the library's CUDA kernels.
+Device buffers may be given as torch tensors (their ``data_ptr()`` is passed) or as raw
+integer addresses; streams as ``torch.cuda.Stream`` or raw handles. A non-zero status
+raises :class:`LsError`. There is no fallback: if the library is missing, importing this
+package raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liblongspark.so")
+
+LS_OK = 0
+LS_ERR_INVALID_ARG = -1
+LS_ERR_SHAPE = -2
+LS_ERR_UNSUPPORTED = -3
+LS_ERR_CUDA = -4
+LS_ERR_DEVICE = -5
+LS_ERR_DEVICE_TIMEOUT = -6
+LS_DEVERR_PREFIX_LEN = 0x1
+LS_DEVERR_WAIT_TIMEOUT = 0x2
+LS_DEVERR_ORDER = 0x4
+LS_F32 = 0
+LS_BF16 = 1
+LS_FLAG_FORCE_SIMT = 0x1
+LS_MAX_SCALES = 4
+
+EXPORTED = (
+    "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",
+    "ls_prefill_summary", "ls_commit_round", "ls_draft_attend", "ls_attend_uses_tensor_cores",
+    "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
+)
+
+
+class LsError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: {status} ({ls_status_string(status)})")
+        self.status = status
+
+
+class ls_config(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_layers", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("hidden", ctypes.c_int32),
+        ("block", ctypes.c_int32), ("window", ctypes.c_int32), ("n_scales", ctypes.c_int32),
+        ("scales", ctypes.c_int32 * LS_MAX_SCALES), ("slots_per_scale", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32),
+    ]
+
+
+class ls_layout(ctypes.Structure):
+    _fields_ = [
+        ("total_bytes", ctypes.c_size_t), ("off_counters", ctypes.c_size_t),
+        ("off_error", ctypes.c_size_t), ("off_kv", ctypes.c_size_t),
+        ("off_seg_mean", ctypes.c_size_t), ("off_part_sum", ctypes.c_size_t),
+        ("off_glob_sum", ctypes.c_size_t), ("off_boundary", ctypes.c_size_t),
+        ("kv_rows", ctypes.c_int32), ("elem_bytes", ctypes.c_int32),
+    ]
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with __graft_entry__.build()")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    cfgp = ctypes.POINTER(ls_config)
+    sig = {
+        "ls_state_bytes": (sz, [cfgp]),
+        "ls_get_layout": (ctypes.c_int, [cfgp, ctypes.POINTER(ls_layout)]),
+        "ls_init_state": (ctypes.c_int, [cfgp, vp, sz, ctypes.POINTER(vp), vp]),
+        "ls_prefill_workspace_bytes": (sz, [cfgp, i64, i64]),
+        "ls_prefill_summary": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, i64, i64, vp, vp, sz, vp]),
+        "ls_commit_round": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "ls_draft_attend": (ctypes.c_int, [vp, i32, i32, vp, vp, vp, i64, ctypes.c_float, vp, vp]),
+        "ls_attend_uses_tensor_cores": (ctypes.c_int, [vp]),
+        "ls_read_state": (ctypes.c_int, [vp, vp, sz, vp]),
+        "ls_get_error": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
+        "ls_destroy_state": (None, [vp]),
+        "ls_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    raise TypeError(f"expected a tensor or an address, got {type(x)}")
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(fn, status):
+    if status != LS_OK:
+        raise LsError(fn, status)
+
+
+def make_config(batch, n_layers, n_kv_heads, n_q_heads, head_dim, hidden, block, window, scales,
+                slots_per_scale, dtype=LS_BF16, flags=0) -> ls_config:
+    c = ls_config()
+    c.batch, c.n_layers, c.n_kv_heads, c.n_q_heads = batch, n_layers, n_kv_heads, n_q_heads
+    c.head_dim, c.hidden, c.block, c.window = head_dim, hidden, block, window
+    c.n_scales = len(scales)
+    for i, s in enumerate(scales):
+        c.scales[i] = s
+    c.slots_per_scale, c.dtype, c.flags = slots_per_scale, dtype, flags
+    return c
+
+
+def ls_status_string(status: int) -> str:
+    return _lib.ls_status_string(status).decode()
+
+
+def ls_state_bytes(cfg: ls_config) -> int:
+    return int(_lib.ls_state_bytes(ctypes.byref(cfg)))
+
+
+def ls_get_layout(cfg: ls_config) -> ls_layout:
+    out = ls_layout()
+    _check("ls_get_layout", _lib.ls_get_layout(ctypes.byref(cfg), ctypes.byref(out)))
+    return out
+
+
+def ls_init_state(cfg: ls_config, arena, arena_bytes: int, stream=None) -> int:
+    """Returns the opaque state handle (an address)."""
+    h = ctypes.c_void_p()
+    _check("ls_init_state", _lib.ls_init_state(ctypes.byref(cfg), _ptr(arena), arena_bytes,
+                                               ctypes.byref(h), _stream(stream)))
+    return h.value
+
+
+def ls_prefill_workspace_bytes(cfg: ls_config, row_begin: int, row_end: int) -> int:
+    return int(_lib.ls_prefill_workspace_bytes(ctypes.byref(cfg), row_begin, row_end))
+
+
+def ls_prefill_summary(state, k, v, plane_stride, row_stride, prefix_len, row_begin, row_end,
+                       last_hidden, workspace, workspace_bytes, stream=None) -> None:
+    _check("ls_prefill_summary", _lib.ls_prefill_summary(
+        state, _ptr(k), _ptr(v), plane_stride, row_stride, _ptr(prefix_len), row_begin, row_end,
+        _ptr(last_hidden), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def ls_commit_round(state, draft_ids, target_ids, verify_k, verify_v, verify_hidden, accept_len,
+                    next_token, stream=None) -> None:
+    _check("ls_commit_round", _lib.ls_commit_round(
+        state, _ptr(draft_ids), _ptr(target_ids), _ptr(verify_k), _ptr(verify_v),
+        _ptr(verify_hidden), _ptr(accept_len), _ptr(next_token), _stream(stream)))
+
+
+def ls_draft_attend(state, layer_begin, layer_count, q, boundary_k, boundary_v, boundary_stride,
+                    softmax_scale, out, stream=None) -> None:
+    _check("ls_draft_attend", _lib.ls_draft_attend(
+        state, layer_begin, layer_count, _ptr(q), _ptr(boundary_k), _ptr(boundary_v),
+        boundary_stride, float(softmax_scale), _ptr(out), _stream(stream)))
+
+
+def ls_attend_uses_tensor_cores(state) -> bool:
+    return bool(_lib.ls_attend_uses_tensor_cores(state))
+
+
+def ls_read_state(state, host_dst, nbytes, stream=None) -> None:
+    _check("ls_read_state", _lib.ls_read_state(state, _ptr(host_dst), nbytes, _stream(stream)))
+
+
+def ls_get_error(state) -> tuple[int, int]:
+    """(status, device error word). Synchronises the device."""
+    code = ctypes.c_int32(0)
+    st = _lib.ls_get_error(state, ctypes.byref(code))
+    return st, code.value
+
+
+def ls_destroy_state(state) -> None:
+    _lib.ls_destroy_state(state)

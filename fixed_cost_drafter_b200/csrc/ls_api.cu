@@ -1,0 +1,240 @@
+// Host side of the C ABI declared in include/longspark.h: argument validation, the
+// state arena layout, and the kernel launches. No entry point allocates device memory.
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "ls_common.cuh"
+#include "ls_attend_tc.h"
+
+namespace ls {
+cudaError_t launch_commit(const Dev& p, const int32_t* draft, const int32_t* target, const void* vk,
+                          const void* vv, const void* vh, int32_t* accept_len, int32_t* next_token,
+                          cudaStream_t stream);
+bool simt_supported(const Dev& p);
+cudaError_t launch_attend_simt(const Dev& p, int lb, int lcount, const void* q, const void* bk,
+                               const void* bv, int64_t bstride, float scale, void* out,
+                               cudaStream_t stream);
+size_t prefill_workspace_bytes(const ls_config& c, int64_t row_begin, int64_t row_end);
+cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, const void* v,
+                           int64_t plane_stride, int64_t row_stride, const int64_t* prefix_len,
+                           int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws,
+                           int sms, cudaStream_t stream);
+}  // namespace ls
+
+struct ls_state {
+  ls_config cfg;
+  ls::Layout lay;
+  ls::Dev dev;
+  void* arena;
+  int device;
+  int sms;
+  int use_tc;
+  ls::TcPlan tc;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int validate(const ls_config* c) {
+  if (!c) return LS_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->n_layers < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 ||
+      c->head_dim < 1 || c->hidden < 1 || c->block < 1 || c->window < 1 || c->n_scales < 1 ||
+      c->slots_per_scale < 1)
+    return LS_ERR_INVALID_ARG;
+  if (c->dtype != LS_F32 && c->dtype != LS_BF16) return LS_ERR_INVALID_ARG;
+  if (c->n_scales > LS_MAX_SCALES) return LS_ERR_UNSUPPORTED;
+  if (c->n_q_heads % c->n_kv_heads != 0) return LS_ERR_SHAPE;
+  if (c->window < c->block + 1) return LS_ERR_SHAPE;  // a round's rows get distinct slots
+  for (int k = 0; k < c->n_scales; ++k) {
+    if (c->scales[k] < 1) return LS_ERR_INVALID_ARG;
+    if (k > 0 && c->scales[k] <= c->scales[k - 1]) return LS_ERR_SHAPE;
+  }
+  // GPU-path limits (valid for the method, not handled by these kernels)
+  if (c->scales[0] < c->block + 1) return LS_ERR_UNSUPPORTED;  // <= 1 close per scale per round
+  for (int k = 1; k < c->n_scales; ++k)
+    if (c->scales[k] % c->scales[k - 1] != 0) return LS_ERR_UNSUPPORTED;
+  const int elem = c->dtype == LS_BF16 ? 2 : 4;
+  if (c->head_dim % 8 != 0 || c->head_dim > 256 || c->hidden % 8 != 0) return LS_ERR_UNSUPPORTED;
+  const int lanes = c->head_dim * elem / 16;
+  if (!pow2(lanes) || lanes > 32) return LS_ERR_UNSUPPORTED;
+  if (c->n_kv_heads > 16 || c->block > 32) return LS_ERR_UNSUPPORTED;
+  if (c->flags & ~LS_FLAG_FORCE_SIMT) return LS_ERR_INVALID_ARG;
+  return LS_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? LS_OK : LS_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* ls_status_string(int s) {
+  switch (s) {
+    case LS_OK: return "ok";
+    case LS_ERR_INVALID_ARG: return "invalid argument";
+    case LS_ERR_SHAPE: return "inconsistent shapes";
+    case LS_ERR_UNSUPPORTED: return "unsupported by the GPU path";
+    case LS_ERR_CUDA: return "CUDA runtime error";
+    case LS_ERR_DEVICE: return "device error word set";
+    case LS_ERR_DEVICE_TIMEOUT: return "bounded device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t ls_state_bytes(const ls_config* cfg) {
+  if (validate(cfg) != LS_OK) return 0;
+  return size_t(ls::make_layout(*cfg).total);
+}
+
+int ls_get_layout(const ls_config* cfg, ls_layout* out) {
+  const int v = validate(cfg);
+  if (v != LS_OK) return v;
+  if (!out) return LS_ERR_INVALID_ARG;
+  const ls::Layout y = ls::make_layout(*cfg);
+  out->total_bytes = size_t(y.total);
+  out->off_counters = size_t(y.counters);
+  out->off_error = size_t(y.error);
+  out->off_kv = size_t(y.kv);
+  out->off_seg_mean = size_t(y.seg);
+  out->off_part_sum = size_t(y.part);
+  out->off_glob_sum = size_t(y.glob);
+  out->off_boundary = size_t(y.boundary);
+  out->kv_rows = y.R;
+  out->elem_bytes = y.elem;
+  return LS_OK;
+}
+
+int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_state** out,
+                  cudaStream_t stream) {
+  const int v = validate(cfg);
+  if (v != LS_OK) return v;
+  if (!d_arena || !out) return LS_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_arena) & 255) != 0) return LS_ERR_INVALID_ARG;
+  const ls::Layout y = ls::make_layout(*cfg);
+  if (arena_bytes < size_t(y.total)) return LS_ERR_SHAPE;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LS_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return LS_ERR_CUDA;
+  if (cudaMemsetAsync(d_arena, 0, size_t(y.total), stream) != cudaSuccess) return LS_ERR_CUDA;
+
+  ls_state* st = new (std::nothrow) ls_state;
+  if (!st) return LS_ERR_INVALID_ARG;
+  std::memset(static_cast<void*>(st), 0, sizeof(ls_state));
+  st->cfg = *cfg;
+  st->lay = y;
+  st->arena = d_arena;
+  st->device = dev;
+  st->sms = sms;
+  char* base = static_cast<char*>(d_arena);
+  ls::Dev& p = st->dev;
+  p.b = cfg->batch; p.L = cfg->n_layers; p.Hkv = cfg->n_kv_heads; p.Hq = cfg->n_q_heads;
+  p.D = cfg->head_dim; p.hidden = cfg->hidden; p.B = cfg->block; p.W = cfg->window;
+  p.nsc = cfg->n_scales; p.slots = cfg->slots_per_scale; p.R = y.R; p.dtype = cfg->dtype;
+  for (int k = 0; k < LS_MAX_SCALES; ++k) p.scales[k] = k < cfg->n_scales ? cfg->scales[k] : 1;
+  p.counters = reinterpret_cast<int64_t*>(base + y.counters);
+  p.err = reinterpret_cast<int32_t*>(base + y.error);
+  p.kv = base + y.kv;
+  p.seg = reinterpret_cast<float*>(base + y.seg);
+  p.part = reinterpret_cast<float*>(base + y.part);
+  p.glob = reinterpret_cast<float*>(base + y.glob);
+  p.boundary = base + y.boundary;
+
+  st->use_tc = 0;
+  if (!(cfg->flags & LS_FLAG_FORCE_SIMT) && ls::tc_supported(p)) {
+    const int r = ls::tc_prepare(p, &st->tc);
+    if (r != LS_OK) { delete st; return r; }
+    st->use_tc = 1;
+  } else if (!ls::simt_supported(p)) {
+    delete st;
+    return LS_ERR_UNSUPPORTED;
+  }
+  *out = st;
+  return LS_OK;
+}
+
+size_t ls_prefill_workspace_bytes(const ls_config* cfg, int64_t row_begin, int64_t row_end) {
+  if (validate(cfg) != LS_OK || row_begin < 0 || row_end < row_begin) return 0;
+  return ls::prefill_workspace_bytes(*cfg, row_begin, row_end);
+}
+
+int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t plane_stride,
+                       int64_t row_stride, const int64_t* d_prefix_len, int64_t row_begin,
+                       int64_t row_end, const void* d_last_hidden, void* d_workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+  if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
+  const ls_config& c = st->cfg;
+  if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
+  if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
+  const int64_t rowElems = int64_t(c.n_kv_heads) * c.head_dim;
+  if (row_end > row_begin) {
+    if (!d_k || !d_v || !d_workspace) return LS_ERR_INVALID_ARG;
+    if (row_stride < rowElems || row_stride % 8 != 0 || plane_stride % 8 != 0) return LS_ERR_SHAPE;
+    if (plane_stride < (row_end - row_begin) * row_stride && c.batch * c.n_layers > 1)
+      return LS_ERR_SHAPE;
+    if (!aligned16(d_k) || !aligned16(d_v) || !aligned16(d_workspace)) return LS_ERR_INVALID_ARG;
+    if (workspace_bytes < ls::prefill_workspace_bytes(c, row_begin, row_end)) return LS_ERR_SHAPE;
+  }
+  if (d_last_hidden && !aligned16(d_last_hidden)) return LS_ERR_INVALID_ARG;
+  return cuda_status(ls::launch_prefill(st->dev, c, d_k, d_v, plane_stride, row_stride,
+                                        d_prefix_len, row_begin, row_end, d_last_hidden,
+                                        d_workspace, st->sms, stream));
+}
+
+int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
+                    const void* d_verify_k, const void* d_verify_v, const void* d_verify_hidden,
+                    int32_t* d_accept_len, int32_t* d_next_token, cudaStream_t stream) {
+  if (!st || !d_draft_ids || !d_target_ids || !d_verify_k || !d_verify_v || !d_verify_hidden ||
+      !d_accept_len || !d_next_token)
+    return LS_ERR_INVALID_ARG;
+  if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden))
+    return LS_ERR_INVALID_ARG;
+  return cuda_status(ls::launch_commit(st->dev, d_draft_ids, d_target_ids, d_verify_k, d_verify_v,
+                                       d_verify_hidden, d_accept_len, d_next_token, stream));
+}
+
+int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count, const void* d_q,
+                    const void* d_boundary_k, const void* d_boundary_v, int64_t boundary_stride,
+                    float softmax_scale, void* d_out, cudaStream_t stream) {
+  if (!st || !d_q || !d_boundary_k || !d_boundary_v || !d_out) return LS_ERR_INVALID_ARG;
+  const ls_config& c = st->cfg;
+  if (layer_begin < 0 || layer_count < 1 || layer_begin + layer_count > c.n_layers)
+    return LS_ERR_INVALID_ARG;
+  if (boundary_stride < int64_t(c.n_kv_heads) * c.head_dim || boundary_stride % 8 != 0)
+    return LS_ERR_SHAPE;
+  if (!aligned16(d_q) || !aligned16(d_out) || !aligned16(d_boundary_k) || !aligned16(d_boundary_v))
+    return LS_ERR_INVALID_ARG;
+  if (st->use_tc)
+    return cuda_status(ls::launch_attend_tc(st->dev, st->tc, layer_begin, layer_count, d_q,
+                                            d_boundary_k, d_boundary_v, boundary_stride,
+                                            softmax_scale, d_out, st->sms, stream));
+  return cuda_status(ls::launch_attend_simt(st->dev, layer_begin, layer_count, d_q, d_boundary_k,
+                                            d_boundary_v, boundary_stride, softmax_scale, d_out,
+                                            stream));
+}
+
+int ls_attend_uses_tensor_cores(const ls_state* st) { return st && st->use_tc ? 1 : 0; }
+
+int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStream_t stream) {
+  if (!st || !h_dst) return LS_ERR_INVALID_ARG;
+  if (bytes > size_t(st->lay.total)) return LS_ERR_SHAPE;
+  if (cudaMemcpyAsync(h_dst, st->arena, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return LS_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(stream));
+}
+
+int ls_get_error(const ls_state* st, int32_t* h_code) {
+  if (!st || !h_code) return LS_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LS_ERR_CUDA;
+  if (cudaMemcpy(h_code, st->dev.err, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LS_ERR_CUDA;
+  if (*h_code & LS_DEVERR_WAIT_TIMEOUT) return LS_ERR_DEVICE_TIMEOUT;
+  return *h_code ? LS_ERR_DEVICE : LS_OK;
+}
+
+void ls_destroy_state(ls_state* st) { delete st; }
+
+}  // extern "C"

@@ -1,0 +1,19 @@
+// tcgen05 tensor-core path of the drafter block attention (sm_100a).
+#pragma once
+#include "ls_common.cuh"
+
+namespace ls {
+
+// Per-state constants of the tensor-core path (tensor map over the arena's K/V rows).
+struct alignas(64) TcPlan {
+  alignas(64) unsigned char kv_map[128];  // CUtensorMap of the kv region
+  int32_t n_chunks;                        // 128-row chunks of arena rows per tile
+};
+
+bool tc_supported(const Dev& p);
+int tc_prepare(const Dev& p, TcPlan* plan);
+cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
+                             const void* bk, const void* bv, int64_t bstride, float scale,
+                             void* out, int sms, cudaStream_t stream);
+
+}  // namespace ls

@@ -1,0 +1,177 @@
+// Shared definitions of the LongSpark drafting-round kernels (sm_100a).
+// State layout, slot validity, element conversion and the PTX wrappers used by the
+// bulk-copy pipelines and the tcgen05 attention kernel.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/longspark.h"
+
+namespace ls {
+
+constexpr int kMaxScales = LS_MAX_SCALES;
+
+// Device-side view of one drafting state: shapes plus region pointers in the arena.
+struct Dev {
+  int32_t b, L, Hkv, Hq, D, hidden, B, W, nsc, slots, R, dtype;
+  int32_t scales[kMaxScales];
+  int64_t* counters;  // [b][L][1+nsc]
+  int32_t* err;       // device error word
+  char* kv;           // [b][L][Hkv][2][R][D] elements
+  float* seg;         // [b][L][Hkv][nsc][slots][2][D]
+  float* part;        // [b][L][Hkv][nsc][2][D]
+  float* glob;        // [b][L][Hkv][2][D]
+  char* boundary;     // [b][L][hidden] elements
+};
+
+__host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+// Arena layout for a validated config (host and device agree by construction).
+struct Layout {
+  int64_t counters, error, kv, seg, part, glob, boundary, total;
+  int32_t R, elem;
+};
+
+__host__ inline Layout make_layout(const ls_config& c) {
+  Layout y{};
+  y.elem = c.dtype == LS_BF16 ? 2 : 4;
+  y.R = c.window + c.n_scales * (c.slots_per_scale + 1) + 1;
+  const int64_t tiles = int64_t(c.batch) * c.n_layers * c.n_kv_heads;
+  int64_t off = 0;
+  y.counters = off; off = align256(off + int64_t(c.batch) * c.n_layers * (1 + c.n_scales) * 8);
+  y.error = off;    off = align256(off + 16);
+  y.kv = off;       off = align256(off + tiles * 2 * y.R * c.head_dim * y.elem);
+  y.seg = off;      off = align256(off + tiles * c.n_scales * c.slots_per_scale * 2 * c.head_dim * 4);
+  y.part = off;     off = align256(off + tiles * c.n_scales * 2 * c.head_dim * 4);
+  y.glob = off;     off = align256(off + tiles * 2 * c.head_dim * 4);
+  y.boundary = off; off = align256(off + int64_t(c.batch) * c.n_layers * c.hidden * y.elem);
+  y.total = off;
+  return y;
+}
+
+// ---- element conversion -------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static constexpr int kVec = 4;  // elements per 16-byte vector
+  __device__ static inline void to_f32(const uint4& v, float* f) {
+    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+  }
+  __device__ static inline uint4 from_f32(const float* f) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+  __device__ static inline float load1(const void* p, int64_t i) {
+    return reinterpret_cast<const float*>(p)[i];
+  }
+  __device__ static inline void store1(void* p, int64_t i, float x) {
+    reinterpret_cast<float*>(p)[i] = x;
+  }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static constexpr int kVec = 8;
+  __device__ static inline void to_f32(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  __device__ static inline uint4 from_f32(const float* f) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);  // RNE
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  __device__ static inline float load1(const void* p, int64_t i) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  }
+  __device__ static inline void store1(void* p, int64_t i, float x) {
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(x);
+  }
+};
+
+// ---- slot validity of the arena rows of one tile --------------------------------
+// Row r < W: ring slot r, filled once len > r. Then per scale k: slots 0..slots-1
+// (filled once n_seg[k] > i) and the partial mean (non-empty when len - n_seg*s > 0).
+// Last row: the global mean (len > 0).
+__device__ inline bool arena_row_valid(const Dev& p, int r, int64_t len, const int64_t* nseg) {
+  if (r < p.W) return r < len;
+  int rr = r - p.W;
+  const int per = p.slots + 1;
+  int k = rr / per;
+  if (k >= p.nsc) return len > 0;  // global mean row
+  int i = rr - k * per;
+  if (i < p.slots) return i < nseg[k];
+  return len - nseg[k] * int64_t(p.scales[k]) > 0;
+}
+
+__device__ inline void set_err(int32_t* err, int32_t bits) { atomicOr(err, bits); }
+
+// ---- mbarrier / bulk-copy PTX ---------------------------------------------------
+__device__ inline uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ inline void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ inline void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: gives up after `limit` polls (each poll itself suspends for a
+// hardware-chosen interval) and reports false, so no kernel can spin forever.
+__device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// Bulk asynchronous global->shared copy on the TMA engine (no tensor map, no multicast).
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ inline void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ inline void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ inline uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+}  // namespace ls

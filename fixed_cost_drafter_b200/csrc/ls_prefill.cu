@@ -1,0 +1,509 @@
+// Summary initialisation over the full prefix at target prefill: LongSpark paper page,
+// Figure 3 caption ("initialized over the full prefix during target prefill").
+//
+// Pass 1 (prefill_units_kernel, persistent, one CTA per SM): the work items are units
+// of U prefix rows of one (sequence, layer); U is the largest scale <= 512. The TMA
+// engine streams each unit's K and V rows (all KV heads of a row are contiguous) into a
+// ring of shared-memory stages with cp.async.bulk + mbarrier transaction counts; every
+// thread owns one 16-byte column vector and keeps one fp32 sum per scale <= U. When a
+// segment of scale s_k closes, its sum is added into the next scale's sum (a tree,
+// not a long serial chain) and, if the segment is among the `slots` most recent ones of
+// the final prefix, its mean is written. A closed unit's sum goes to the workspace.
+// The last W prefix rows are copied into the ring window on the way through.
+// Pass 2 (prefill_finalize_kernel): per (sequence, layer, column block) the unit sums
+// are combined the same way into the segments of the scales > U, the partial sums, the
+// global sum (accumulated across chunk calls), the mean rows and the counters.
+#include "ls_common.cuh"
+
+namespace ls {
+
+struct PrefillArgs {
+  const char* k;
+  const char* v;
+  int64_t plane_stride, row_stride;  // elements
+  const int64_t* prefix_len;
+  int64_t row_begin, row_end;
+  float* ws;        // [b*L][n_units][2*Hkv*D] unit sums
+  int32_t n_units;  // units per (sequence, layer) in this chunk
+  int32_t U;        // unit rows (a scale)
+  int32_t kU;       // scales 0..kU-1 are <= U (scale kU-1 == U)
+  int32_t G;        // rows per stage
+  int32_t n_items;  // b * L * n_units
+};
+
+constexpr int kPrefillThreads = 256;
+constexpr int kPrefillStages = 3;
+
+__device__ inline int64_t clamp_prefix(const PrefillArgs& a, const Dev&, int b) {
+  int64_t P = a.prefix_len[b];
+  return P < 0 ? 0 : P;
+}
+
+// rows [r0, r1) of item `it` inside this chunk (empty when r1 <= r0)
+__device__ inline void item_rows(const PrefillArgs& a, const Dev& p, int it, int& bl, int& u,
+                                 int64_t& r0, int64_t& r1) {
+  bl = it / a.n_units;
+  u = it - bl * a.n_units;
+  const int b = bl / p.L;
+  const int64_t end = min(a.row_end, clamp_prefix(a, p, b));
+  r0 = a.row_begin + int64_t(u) * a.U;
+  r1 = min(r0 + a.U, end);
+}
+
+// Cursor over the flattened (item, row group) stage sequence of one CTA.
+struct Cursor {
+  int j;        // item ordinal within this CTA (item = blockIdx.x + j * gridDim.x)
+  int grp;      // row group within the item
+  bool valid;
+};
+
+__device__ inline void cursor_settle(const PrefillArgs& a, const Dev& p, Cursor& c) {
+  // move forward to the first item with rows left at group c.grp
+  while (true) {
+    const int it = blockIdx.x + c.j * gridDim.x;
+    if (it >= a.n_items) { c.valid = false; return; }
+    int bl, u; int64_t r0, r1;
+    item_rows(a, p, it, bl, u, r0, r1);
+    if (r1 > r0 + int64_t(c.grp) * a.G) { c.valid = true; return; }
+    c.j += 1; c.grp = 0;
+  }
+}
+__device__ inline void cursor_next(const PrefillArgs& a, const Dev& p, Cursor& c) {
+  c.grp += 1;
+  cursor_settle(a, p, c);
+}
+
+template <typename T, int CVT>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+prefill_units_kernel(Dev p, PrefillArgs a) {
+  using E = Elem<T>;
+  constexpr int VEC = E::kVec;
+  extern __shared__ __align__(128) char smem[];
+  __shared__ uint64_t full[kPrefillStages];
+
+  const int rowElems = p.Hkv * p.D;
+  const int rowBytes = rowElems * int(sizeof(T));
+  const int stageBytes = 2 * a.G * rowBytes;
+  const int ncv = 2 * rowElems / VEC;  // column vectors of K then V
+  const int cvPerRow = rowElems / VEC;
+  const int tid = threadIdx.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < kPrefillStages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // producer: thread 0 issues stage n into buffer n % kPrefillStages
+  Cursor prod{0, 0, false};
+  int issued = 0;
+  auto issue = [&](Cursor& c, int n) {
+    const int it = blockIdx.x + c.j * gridDim.x;
+    int bl, u; int64_t r0, r1;
+    item_rows(a, p, it, bl, u, r0, r1);
+    const int64_t g0 = r0 + int64_t(c.grp) * a.G;
+    const int nrows = int(min(int64_t(a.G), r1 - g0));
+    char* dst = smem + (n % kPrefillStages) * stageBytes;
+    uint64_t* bar = &full[n % kPrefillStages];
+    mbar_arrive_expect_tx(bar, uint32_t(2 * nrows * rowBytes));
+    for (int t = 0; t < 2; ++t) {
+      const char* base = (t == 0 ? a.k : a.v) +
+                         (int64_t(bl) * a.plane_stride + (g0 - a.row_begin) * a.row_stride) * int64_t(sizeof(T));
+      char* d = dst + t * a.G * rowBytes;
+      if (a.row_stride == rowElems) {
+        bulk_g2s(d, base, uint32_t(nrows * rowBytes), bar);
+      } else {
+        for (int r = 0; r < nrows; ++r)
+          bulk_g2s(d + r * rowBytes, base + int64_t(r) * a.row_stride * int64_t(sizeof(T)),
+                   uint32_t(rowBytes), bar);
+      }
+    }
+  };
+  if (tid == 0) {
+    cursor_settle(a, p, prod);
+    for (; issued < kPrefillStages && prod.valid; ++issued) {
+      issue(prod, issued);
+      cursor_next(a, p, prod);
+    }
+  }
+
+  Cursor cons{0, 0, false};
+  cursor_settle(a, p, cons);
+  int consumed = 0;
+
+  float acc[CVT][kMaxScales + 1][VEC];
+  int cnt[kMaxScales];  // rows (k = 0) or closes of scale k-1 until scale k closes
+  int cur_item = -1;
+  bool timed_out = false;
+
+  while (cons.valid) {
+    const int it = blockIdx.x + cons.j * gridDim.x;
+    int bl, u; int64_t r0, r1;
+    item_rows(a, p, it, bl, u, r0, r1);
+    const int b = bl / p.L;
+    const int64_t P = clamp_prefix(a, p, b);
+    if (it != cur_item) {  // new item: all sums start empty (r0 is a multiple of U)
+      cur_item = it;
+#pragma unroll
+      for (int q = 0; q < CVT; ++q)
+#pragma unroll
+        for (int k = 0; k <= kMaxScales; ++k)
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[q][k][e] = 0.f;
+#pragma unroll
+      for (int k = 0; k < kMaxScales; ++k)
+        cnt[k] = k >= a.kU ? 0 : (k == 0 ? p.scales[0] : p.scales[k] / p.scales[k - 1]);
+    }
+    const int64_t g0 = r0 + int64_t(cons.grp) * a.G;
+    const int nrows = int(min(int64_t(a.G), r1 - g0));
+    const int buf = consumed % kPrefillStages;
+    const bool ok = mbar_wait_bounded(&full[buf], uint32_t((consumed / kPrefillStages) & 1), kWaitLimit);
+    if (__syncthreads_or(!ok)) { timed_out = true; break; }
+
+    const char* st = smem + buf * stageBytes;
+    for (int r = 0; r < nrows; ++r) {
+      const int64_t pos = g0 + r;
+      const bool in_window = pos >= P - p.W;
+#pragma unroll
+      for (int q = 0; q < CVT; ++q) {
+        const int cv = tid + q * kPrefillThreads;
+        if (cv >= ncv) break;
+        const int t = cv / cvPerRow;
+        const int e0 = (cv - t * cvPerRow) * VEC;
+        const uint4 raw = *reinterpret_cast<const uint4*>(st + (t * a.G + r) * rowBytes + e0 * int(sizeof(T)));
+        float f[VEC];
+        E::to_f32(raw, f);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[q][0][e] += f[e];
+        if (in_window) {
+          const int h = e0 / p.D, d0 = e0 - h * p.D;
+          const int64_t tile = int64_t(bl) * p.Hkv + h;
+          T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + t) * int64_t(p.R) * p.D;
+          *reinterpret_cast<uint4*>(kvt + int64_t(pos % p.W) * p.D + d0) = raw;
+        }
+      }
+      // segment closes, smallest scale first; a closed scale feeds the next one
+#pragma unroll
+      for (int k = 0; k < kMaxScales; ++k) {
+        if (k >= a.kU) break;
+        if (--cnt[k] != 0) break;  // level k counts closes of level k-1 (rows for k = 0)
+        cnt[k] = k == 0 ? p.scales[0] : p.scales[k] / p.scales[k - 1];
+        const int s = p.scales[k];
+        const int64_t j = pos / s;  // segment that just closed
+        const bool keep = j >= P / s - p.slots;
+#pragma unroll
+        for (int q = 0; q < CVT; ++q) {
+          const int cv = tid + q * kPrefillThreads;
+          if (cv >= ncv) break;
+          const int t = cv / cvPerRow;
+          const int e0 = (cv - t * cvPerRow) * VEC;
+          const int h = e0 / p.D, d0 = e0 - h * p.D;
+          const int64_t tile = int64_t(bl) * p.Hkv + h;
+          if (keep) {
+            float m[VEC];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) m[e] = acc[q][k][e] / float(s);
+            const int slot = int(j % p.slots);
+            float* sg = p.seg + (((tile * p.nsc + k) * p.slots + slot) * 2 + t) * p.D + d0;
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+              *reinterpret_cast<float4*>(sg + e) = make_float4(m[e], m[e + 1], m[e + 2], m[e + 3]);
+            T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + t) * int64_t(p.R) * p.D;
+            *reinterpret_cast<uint4*>(kvt + (int64_t(p.W) + k * (p.slots + 1) + slot) * p.D + d0) =
+                E::from_f32(m);
+          }
+          if (k + 1 < a.kU) {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) { acc[q][k + 1][e] += acc[q][k][e]; acc[q][k][e] = 0.f; }
+          } else {  // the unit closed: its sum goes to the workspace
+            float* w = a.ws + (int64_t(bl) * a.n_units + u) * (2 * rowElems) + int64_t(cv) * VEC;
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+              *reinterpret_cast<float4*>(w + e) =
+                  make_float4(acc[q][k][e], acc[q][k][e + 1], acc[q][k][e + 2], acc[q][k][e + 3]);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[q][k][e] = 0.f;
+          }
+        }
+      }
+    }
+
+    const bool item_ends = g0 + nrows == r1;
+    if (item_ends) {
+      const bool unit_closed = r1 - r0 == a.U;
+#pragma unroll
+      for (int q = 0; q < CVT; ++q) {
+        const int cv = tid + q * kPrefillThreads;
+        if (cv >= ncv) break;
+        const int t = cv / cvPerRow;
+        const int e0 = (cv - t * cvPerRow) * VEC;
+        const int h = e0 / p.D, d0 = e0 - h * p.D;
+        const int64_t tile = int64_t(bl) * p.Hkv + h;
+        float run[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) run[e] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxScales; ++k) {
+          if (k >= a.kU) break;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) run[e] += acc[q][k][e];
+          if (r1 == P) {  // the sequence's prefix ends here: open partial of scale k
+            float* pp = p.part + ((tile * p.nsc + k) * 2 + t) * p.D + d0;
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+              *reinterpret_cast<float4*>(pp + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
+          }
+        }
+        if (!unit_closed) {
+          float* w = a.ws + (int64_t(bl) * a.n_units + u) * (2 * rowElems) + int64_t(cv) * VEC;
+#pragma unroll
+          for (int e = 0; e < VEC; e += 4)
+            *reinterpret_cast<float4*>(w + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
+        }
+      }
+    }
+
+    __syncthreads();  // buffer `buf` fully read by every thread
+    ++consumed;
+    if (tid == 0 && prod.valid) {
+      fence_proxy_async_smem();
+      issue(prod, issued);
+      ++issued;
+      cursor_next(a, p, prod);
+    }
+    cursor_next(a, p, cons);
+  }
+
+  if (timed_out) {
+    if (tid == 0) {
+      set_err(p.err, LS_DEVERR_WAIT_TIMEOUT);
+      // let every copy still in flight land before the CTA's shared memory goes away
+      for (int n = consumed; n < issued; ++n)
+        mbar_wait_bounded(&full[n % kPrefillStages], uint32_t((n / kPrefillStages) & 1), kWaitLimit);
+    }
+    __syncthreads();
+  }
+}
+
+// Pass 2: per (sequence*layer, column block of 64 column vectors).
+template <typename T>
+__global__ void __launch_bounds__(64)
+prefill_finalize_kernel(Dev p, PrefillArgs a, const T* __restrict__ last_hidden) {
+  using E = Elem<T>;
+  constexpr int VEC = E::kVec;
+  const int bl = blockIdx.x;
+  const int b = bl / p.L;
+  const int rowElems = p.Hkv * p.D;
+  const int ncv = 2 * rowElems / VEC;
+  const int cvPerRow = rowElems / VEC;
+  const int cv = blockIdx.y * blockDim.x + threadIdx.x;
+  int64_t* ctr = p.counters + int64_t(bl) * (1 + p.nsc);
+
+  const int64_t Praw = a.prefix_len[b];
+  const int64_t P = Praw < 0 ? 0 : Praw;
+  const int64_t len_prev = ctr[0];
+  const int64_t end = min(a.row_end, P);
+  const int64_t smax = p.scales[p.nsc - 1];
+  if (blockIdx.y == 0 && threadIdx.x == 0) {
+    if (Praw < 0) set_err(p.err, LS_DEVERR_PREFIX_LEN);
+    if (len_prev != min(a.row_begin, P)) set_err(p.err, LS_DEVERR_ORDER);
+    if (P > a.row_end && a.row_end % smax != 0) set_err(p.err, LS_DEVERR_ORDER);
+  }
+  const int64_t newlen = end > a.row_begin ? end : len_prev;
+
+  if (cv < ncv) {
+    const int t = cv / cvPerRow;
+    const int e0 = (cv - t * cvPerRow) * VEC;
+    const int h = e0 / p.D, d0 = e0 - h * p.D;
+    const int64_t tile = int64_t(bl) * p.Hkv + h;
+    T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + t) * int64_t(p.R) * p.D;
+
+    if (end > a.row_begin) {
+      const int nu = int((end - a.row_begin + a.U - 1) / a.U);
+      float acc[kMaxScales + 1][VEC], gs[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        gs[e] = 0.f;
+#pragma unroll
+        for (int k = 0; k <= kMaxScales; ++k) acc[k][e] = 0.f;
+      }
+      for (int uu = 0; uu < nu; ++uu) {
+        const float* w = a.ws + (int64_t(bl) * a.n_units + uu) * (2 * rowElems) + int64_t(cv) * VEC;
+        float x[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; e += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(w + e);
+          x[e] = v4.x; x[e + 1] = v4.y; x[e + 2] = v4.z; x[e + 3] = v4.w;
+        }
+        if (a.kU >= p.nsc) {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) gs[e] += x[e];
+          continue;
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[a.kU][e] += x[e];
+        const int64_t eu = a.row_begin + int64_t(uu + 1) * a.U;  // row after this unit
+        if (eu > end) continue;                                 // open unit
+        for (int k = a.kU; k < p.nsc; ++k) {
+          const int s = p.scales[k];
+          if (eu % s != 0) break;
+          const int64_t j = eu / s - 1;
+          if (j >= P / s - p.slots) {
+            float m[VEC];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) m[e] = acc[k][e] / float(s);
+            const int slot = int(j % p.slots);
+            float* sg = p.seg + (((tile * p.nsc + k) * p.slots + slot) * 2 + t) * p.D + d0;
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+              *reinterpret_cast<float4*>(sg + e) = make_float4(m[e], m[e + 1], m[e + 2], m[e + 3]);
+            *reinterpret_cast<uint4*>(kvt + (int64_t(p.W) + k * (p.slots + 1) + slot) * p.D + d0) =
+                E::from_f32(m);
+          }
+          if (k + 1 < p.nsc) {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) { acc[k + 1][e] += acc[k][e]; acc[k][e] = 0.f; }
+          } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) { gs[e] += acc[k][e]; acc[k][e] = 0.f; }
+          }
+        }
+      }
+      // open partials of the scales > U, then the rest of the global sum
+      float run[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) run[e] = 0.f;
+      for (int k = a.kU; k < p.nsc; ++k) {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) run[e] += acc[k][e];
+        if (end == P) {
+          float* pp = p.part + ((tile * p.nsc + k) * 2 + t) * p.D + d0;
+#pragma unroll
+          for (int e = 0; e < VEC; e += 4)
+            *reinterpret_cast<float4*>(pp + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
+        }
+      }
+      float* gp = p.glob + (tile * 2 + t) * p.D + d0;
+#pragma unroll
+      for (int e = 0; e < VEC; e += 4) {
+        float4 v4 = *reinterpret_cast<const float4*>(gp + e);
+        v4.x += gs[e] + run[e]; v4.y += gs[e + 1] + run[e + 1];
+        v4.z += gs[e + 2] + run[e + 2]; v4.w += gs[e + 3] + run[e + 3];
+        *reinterpret_cast<float4*>(gp + e) = v4;
+      }
+    }
+
+    // mean rows of the partials and of the global sum for the attention
+    float m[VEC];
+    for (int k = 0; k < p.nsc; ++k) {
+      const int64_t c = newlen % p.scales[k];
+      const float* pp = p.part + ((tile * p.nsc + k) * 2 + t) * p.D + d0;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) m[e] = c > 0 ? pp[e] / float(c) : 0.f;
+      *reinterpret_cast<uint4*>(kvt + (int64_t(p.W) + k * (p.slots + 1) + p.slots) * p.D + d0) =
+          E::from_f32(m);
+    }
+    const float* gp = p.glob + (tile * 2 + t) * p.D + d0;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) m[e] = newlen > 0 ? gp[e] / float(newlen) : 0.f;
+    *reinterpret_cast<uint4*>(kvt + int64_t(p.R - 1) * p.D + d0) = E::from_f32(m);
+  }
+
+  if (blockIdx.y == 0) {
+    if (last_hidden != nullptr) {
+      const T* src = last_hidden + int64_t(bl) * p.hidden;
+      T* dst = reinterpret_cast<T*>(p.boundary) + int64_t(bl) * p.hidden;
+      for (int x = threadIdx.x * VEC; x < p.hidden; x += blockDim.x * VEC)
+        *reinterpret_cast<uint4*>(dst + x) = ld_nc_v4(src + x);
+    }
+    __syncthreads();  // every thread of this block has read ctr[0]
+    if (threadIdx.x == 0) {
+      ctr[0] = newlen;
+      for (int k = 0; k < p.nsc; ++k) ctr[1 + k] = newlen / p.scales[k];
+    }
+  }
+}
+
+// ---- host side -------------------------------------------------------------------
+struct PrefillPlan {
+  int32_t U, kU, G, n_units;
+};
+
+PrefillPlan prefill_plan(const ls_config& c, int64_t row_begin, int64_t row_end) {
+  PrefillPlan pl{};
+  int kU = 0;
+  for (int k = 0; k < c.n_scales; ++k)
+    if (c.scales[k] <= 512) kU = k + 1;
+  if (kU == 0) kU = 1;
+  pl.kU = kU;
+  pl.U = c.scales[kU - 1];
+  const int elem = c.dtype == LS_BF16 ? 2 : 4;
+  const int rowBytes = c.n_kv_heads * c.head_dim * elem;
+  pl.G = max(1, min(64, 32768 / rowBytes));
+  const int64_t rows = row_end > row_begin ? row_end - row_begin : 0;
+  pl.n_units = int32_t((rows + pl.U - 1) / pl.U);
+  return pl;
+}
+
+size_t prefill_workspace_bytes(const ls_config& c, int64_t row_begin, int64_t row_end) {
+  const PrefillPlan pl = prefill_plan(c, row_begin, row_end);
+  return size_t(c.batch) * c.n_layers * size_t(pl.n_units) * 2 * c.n_kv_heads * c.head_dim * 4 + 256;
+}
+
+template <typename T, int CVT>
+static cudaError_t launch_units(const Dev& p, const PrefillArgs& a, int sms, cudaStream_t stream) {
+  const int rowBytes = p.Hkv * p.D * int(sizeof(T));
+  const size_t smem = size_t(kPrefillStages) * 2 * a.G * rowBytes;
+  auto kern = prefill_units_kernel<T, CVT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  const int grid = max(1, min(a.n_items, sms));
+  kern<<<grid, kPrefillThreads, smem, stream>>>(p, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, const void* v,
+                           int64_t plane_stride, int64_t row_stride, const int64_t* prefix_len,
+                           int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws,
+                           int sms, cudaStream_t stream) {
+  const PrefillPlan pl = prefill_plan(c, row_begin, row_end);
+  PrefillArgs a{};
+  a.k = static_cast<const char*>(k);
+  a.v = static_cast<const char*>(v);
+  a.plane_stride = plane_stride;
+  a.row_stride = row_stride;
+  a.prefix_len = prefix_len;
+  a.row_begin = row_begin;
+  a.row_end = row_end;
+  a.ws = static_cast<float*>(ws);
+  a.n_units = pl.n_units;
+  a.U = pl.U;
+  a.kU = pl.kU;
+  a.G = pl.G;
+  a.n_items = p.b * p.L * pl.n_units;
+  const int vec = p.dtype == LS_BF16 ? 8 : 4;
+  const int ncv = 2 * p.Hkv * p.D / vec;
+  const int cvt = (ncv + kPrefillThreads - 1) / kPrefillThreads;
+  cudaError_t e = cudaSuccess;
+  if (a.n_items > 0) {
+    if (p.dtype == LS_BF16) {
+      if (cvt <= 1) e = launch_units<__nv_bfloat16, 1>(p, a, sms, stream);
+      else if (cvt <= 2) e = launch_units<__nv_bfloat16, 2>(p, a, sms, stream);
+      else e = launch_units<__nv_bfloat16, 4>(p, a, sms, stream);
+    } else {
+      if (cvt <= 1) e = launch_units<float, 1>(p, a, sms, stream);
+      else if (cvt <= 2) e = launch_units<float, 2>(p, a, sms, stream);
+      else e = launch_units<float, 4>(p, a, sms, stream);
+    }
+    if (e != cudaSuccess) return e;
+  }
+  const dim3 grid(p.b * p.L, (ncv + 63) / 64);
+  if (p.dtype == LS_BF16)
+    prefill_finalize_kernel<__nv_bfloat16><<<grid, 64, 0, stream>>>(
+        p, a, static_cast<const __nv_bfloat16*>(last_hidden));
+  else
+    prefill_finalize_kernel<float><<<grid, 64, 0, stream>>>(p, a, static_cast<const float*>(last_hidden));
+  return cudaGetLastError();
+}
+
+}  // namespace ls

@@ -1,0 +1,268 @@
+"""Synthetic workloads of the drafting round and a device runner for them.
+
+The workloads take the shapes of the paper page's experiments only (Qwen3-4B/8B tapped
+state, prefix 32K/64K/128K, concurrency 16, accept means near the reported tau); the
+values are seeded synthetic draws from ``synth`` (no dataset, no trained weights).
+
+``DeviceRun`` owns the torch allocations of one run (state arena, prefix chunks, all
+rounds' inputs) and drives the library through the binding; it holds no arithmetic of
+the method.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import numpy as np
+
+import fixed_cost_drafter_b200 as F
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    seed: int
+    batch: int
+    n_layers: int
+    n_kv_heads: int
+    n_q_heads: int
+    head_dim: int
+    hidden: int
+    block: int
+    window: int
+    scales: tuple
+    slots: int
+    dtype: str  # "bf16" | "f32"
+    prefix: object  # int, or (lo, hi) for per-sequence lengths uniform on {lo..hi}
+    rounds: int
+    accept_mean: float | None  # None: uniform on 0..B
+    vocab: int
+    head_scale: bool = False
+    flags: int = 0
+
+    @property
+    def group(self):
+        return self.n_q_heads // self.n_kv_heads
+
+    def config(self):
+        return F.make_config(self.batch, self.n_layers, self.n_kv_heads, self.n_q_heads,
+                             self.head_dim, self.hidden, self.block, self.window, list(self.scales),
+                             self.slots, F.LS_BF16 if self.dtype == "bf16" else F.LS_F32, self.flags)
+
+    def prefix_lengths(self):
+        import synth
+        if isinstance(self.prefix, tuple):
+            return synth.prefix_lengths(self.seed, self.batch, *self.prefix)
+        return np.full(self.batch, int(self.prefix), dtype=np.int64)
+
+    def accepts(self):
+        import synth
+        return synth.accept_lengths(self.seed, self.rounds, self.batch, self.block, self.accept_mean)
+
+    def token_ids(self):
+        import synth
+        return synth.token_ids(self.seed, self.rounds, self.batch, self.block, self.accepts(), self.vocab)
+
+    def elem(self):
+        return 2 if self.dtype == "bf16" else 4
+
+
+QWEN3_8B = dict(n_layers=4, n_kv_heads=8, n_q_heads=32, head_dim=128, hidden=4096, block=16,
+                window=512, scales=(64, 512, 4096), slots=32, dtype="bf16", vocab=151936)
+
+CONFIGS = {
+    "tiny": Workload("tiny", 0, 1, 1, 2, 4, 64, 256, 4, 32, (8, 32, 128), 4, "f32", 512, 20, None, 1000),
+    "qwen3_4b_32k": Workload("qwen3_4b_32k", 1, 16, **{**QWEN3_8B, "hidden": 2560}, prefix=32768,
+                             rounds=256, accept_mean=4.7),
+    "qwen3_8b_64k": Workload("qwen3_8b_64k", 2, 16, **QWEN3_8B, prefix=65536, rounds=256,
+                             accept_mean=5.0, head_scale=True),
+    "qwen3_8b_128k_ragged": Workload("qwen3_8b_128k_ragged", 3, 16, **QWEN3_8B, prefix=(98304, 131072),
+                                     rounds=512, accept_mean=3.5),
+}
+
+
+def sweep_point(prefix: int, batch: int, accept_mean: float) -> Workload:
+    """One point of the prefix x concurrency x accept-mean sweep (Qwen3-8B shapes)."""
+    return Workload(f"sweep_p{prefix}_b{batch}_m{accept_mean}", 4, batch, **QWEN3_8B, prefix=prefix,
+                    rounds=128, accept_mean=accept_mean)
+
+
+SWEEP_PREFIXES = (4096, 16384, 32768, 65536, 131072)
+SWEEP_BATCHES = (1, 4, 16, 64)
+SWEEP_MEANS = (2.5, 4.0, 6.0)
+
+
+class DeviceRun:
+    """One workload on one GPU: state arena, generated inputs, calls into the library."""
+
+    def __init__(self, wl: Workload, device="cuda", rounds: int | None = None,
+                 prefill_chunk: int | None = None, prefix_override=None, accepts_override=None,
+                 seq_offset: int = 0):
+        import torch
+        import synth
+        self.torch, self.synth = torch, synth
+        self.wl = wl
+        self.dev = torch.device(device)
+        self.cfg = wl.config()
+        self.layout = F.ls_get_layout(self.cfg)
+        self.nbytes = F.ls_state_bytes(self.cfg)
+        self.arena = torch.empty(self.nbytes, dtype=torch.uint8, device=self.dev)
+        self.stream = torch.cuda.current_stream(self.dev)
+        self.state = F.ls_init_state(self.cfg, self.arena, self.nbytes, self.stream)
+        self.tdtype = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        self.rounds = wl.rounds if rounds is None else rounds
+        self.b0 = int(seq_offset)  # generator coordinates of this run's first sequence
+        self.prefix_len = (np.asarray(prefix_override, dtype=np.int64) if prefix_override is not None
+                           else replace(wl, batch=self.b0 + wl.batch).prefix_lengths()[self.b0:])
+        self.prefill_chunk = prefill_chunk
+        self.scale_host = synth.head_scales(wl.seed, wl.n_layers, wl.n_kv_heads) if wl.head_scale else None
+        self.scale_dev = (torch.from_numpy(self.scale_host).to(self.dev) if self.scale_host is not None
+                          else None)
+        nb = self.b0 + wl.batch
+        acc = synth.accept_lengths(wl.seed, max(self.rounds, 1), nb, wl.block, wl.accept_mean)[:, self.b0:]
+        if accepts_override is not None:
+            acc = np.broadcast_to(np.asarray(accepts_override, dtype=np.int32).reshape(-1, 1),
+                                  (max(self.rounds, 1), wl.batch)).copy() if np.ndim(accepts_override) == 1 \
+                else np.asarray(accepts_override, dtype=np.int32)
+        acc_all = np.zeros((max(self.rounds, 1), nb), dtype=np.int32)
+        acc_all[:, self.b0:] = acc
+        draft, target = synth.token_ids(wl.seed, max(self.rounds, 1), nb, wl.block, acc_all, wl.vocab)
+        draft, target = draft[:, self.b0:], target[:, self.b0:]
+        self.accept_host = acc[:self.rounds]
+        self.draft = torch.from_numpy(draft[:self.rounds].copy()).to(self.dev)
+        self.target = torch.from_numpy(target[:self.rounds].copy()).to(self.dev)
+        self.accept_len = torch.zeros(wl.batch, dtype=torch.int32, device=self.dev)
+        self.next_token = torch.zeros(wl.batch, dtype=torch.int32, device=self.dev)
+        self.round = 0
+        e = wl.elem()
+        self.boundary_k = self.arena.data_ptr() + self.layout.off_boundary
+        self.boundary_v = self.boundary_k + wl.n_kv_heads * wl.head_dim * e
+        self.softmax_scale = 1.0 / math.sqrt(wl.head_dim)
+
+    # ---- generated inputs -------------------------------------------------------
+    def _fill(self, t, tensor_id, shape, head_dim, r0=0, b0=0, l0=0, p0=0, scaled=False):
+        self.synth.device_fill_normal(
+            t.data_ptr(), self.wl.seed, tensor_id, shape, r0=r0, b0=self.b0 + b0, l0=l0, p0=p0,
+            head_dim=head_dim,
+            scale_ptr=self.scale_dev.data_ptr() if (scaled and self.scale_dev is not None) else None,
+            scale_heads=self.wl.n_kv_heads, dtype=self.wl.dtype, stream=self.stream.cuda_stream)
+
+    def prefill(self, timer=None):
+        """Generates the prefix (in chunks when asked) and runs ls_prefill_summary over it.
+
+        ``timer``, if given, is called as ``timer(start_event, end_event, bytes)`` around each
+        library call (generation excluded)."""
+        torch, wl = self.torch, self.wl
+        S = self.synth
+        P = self.prefix_len
+        pmax = int(P.max()) if len(P) else 0
+        chunk = self.prefill_chunk or max(pmax, 1)
+        smax = wl.scales[-1]
+        chunk = max(smax, (chunk // smax) * smax) if pmax > chunk else chunk
+        plen = torch.from_numpy(P).to(self.dev)
+        last_hidden = torch.empty((wl.batch, wl.n_layers, wl.hidden), dtype=self.tdtype, device=self.dev)
+        self._fill(last_hidden, S.LAST_HIDDEN, (1, wl.batch, wl.n_layers, 1, wl.hidden), 0)
+        rowel = wl.n_kv_heads * wl.head_dim
+        rb = 0
+        while True:
+            re_ = min(rb + chunk, pmax)
+            n = max(re_ - rb, 0)
+            k = torch.empty((wl.batch, wl.n_layers, max(n, 1), rowel), dtype=self.tdtype, device=self.dev)
+            v = torch.empty_like(k)
+            if n:
+                self._fill(k, S.PREFIX_K, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True)
+                self._fill(v, S.PREFIX_V, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True)
+            wsb = F.ls_prefill_workspace_bytes(self.cfg, rb, re_)
+            ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=self.dev)
+            last = re_ >= pmax
+            if timer is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+            F.ls_prefill_summary(self.state, k, v, max(n, 1) * rowel, rowel, plen, rb, re_,
+                                 last_hidden if last else None, ws, wsb, self.stream)
+            if timer is not None:
+                e1.record(self.stream)
+                rows = int(np.maximum(np.minimum(P, re_) - rb, 0).sum())
+                timer(e0, e1, rows * wl.n_layers * rowel * 2 * wl.elem())
+            del k, v, ws
+            if last:
+                break
+            rb = re_
+        self.last_hidden = last_hidden
+
+    def make_round_inputs(self, r0=0, n=None):
+        """All inputs of rounds [r0, r0+n): verify K/V/hidden and drafter queries."""
+        torch, wl, S = self.torch, self.wl, self.synth
+        n = self.rounds - r0 if n is None else n
+        B1 = wl.block + 1
+        rowel = wl.n_kv_heads * wl.head_dim
+        vk = torch.empty((n, wl.batch, wl.n_layers, B1, rowel), dtype=self.tdtype, device=self.dev)
+        vv = torch.empty_like(vk)
+        vh = torch.empty((n, wl.batch, wl.n_layers, B1, wl.hidden), dtype=self.tdtype, device=self.dev)
+        q = torch.empty((n, wl.batch, wl.n_layers, wl.block, wl.n_q_heads * wl.head_dim),
+                        dtype=self.tdtype, device=self.dev)
+        self._fill(vk, S.VERIFY_K, (n, wl.batch, wl.n_layers, B1, rowel), wl.head_dim, r0=r0, scaled=True)
+        self._fill(vv, S.VERIFY_V, (n, wl.batch, wl.n_layers, B1, rowel), wl.head_dim, r0=r0, scaled=True)
+        self._fill(vh, S.VERIFY_HIDDEN, (n, wl.batch, wl.n_layers, B1, wl.hidden), 0, r0=r0)
+        self._fill(q, S.QUERY, (n, wl.batch, wl.n_layers, wl.block, wl.n_q_heads * wl.head_dim),
+                   wl.head_dim, r0=r0)
+        return dict(vk=vk, vv=vv, vh=vh, q=q, r0=r0)
+
+    def commit(self, inputs, r):
+        i = r - inputs["r0"]
+        F.ls_commit_round(self.state, self.draft[r], self.target[r], inputs["vk"][i], inputs["vv"][i],
+                          inputs["vh"][i], self.accept_len, self.next_token, self.stream)
+
+    def attend(self, inputs, r, out, layer_begin=0, layer_count=None):
+        wl = self.wl
+        lc = wl.n_layers if layer_count is None else layer_count
+        i = r - inputs["r0"]
+        q = inputs["q"][i]
+        if lc != wl.n_layers or layer_begin != 0:
+            q = q[:, layer_begin:layer_begin + lc].contiguous()
+        F.ls_draft_attend(self.state, layer_begin, lc, q, self.boundary_k, self.boundary_v, wl.hidden,
+                          self.softmax_scale, out, self.stream)
+
+    def new_out(self, layer_count=None):
+        wl = self.wl
+        lc = wl.n_layers if layer_count is None else layer_count
+        return self.torch.empty((wl.batch, lc, wl.block, wl.n_q_heads * wl.head_dim), dtype=self.tdtype,
+                                device=self.dev)
+
+    # ---- readout ----------------------------------------------------------------
+    def read_state(self):
+        """The arena as numpy views: counters, kv rows, fp32 summary, boundary."""
+        torch, wl, y = self.torch, self.wl, self.layout
+        host = torch.empty(self.nbytes, dtype=torch.uint8, pin_memory=True)
+        F.ls_read_state(self.state, host, self.nbytes, self.stream)
+        raw = host.numpy()
+        b, L, H, D, nsc, sl = wl.batch, wl.n_layers, wl.n_kv_heads, wl.head_dim, len(wl.scales), wl.slots
+        ed = np.uint16 if wl.dtype == "bf16" else np.float32
+
+        def view(off, dt, shape):
+            n = int(np.prod(shape)) * np.dtype(dt).itemsize
+            return raw[off:off + n].view(dt).reshape(shape)
+
+        return dict(
+            counters=view(y.off_counters, np.int64, (b, L, 1 + nsc)).copy(),
+            kv=view(y.off_kv, ed, (b, L, H, 2, y.kv_rows, D)).copy(),
+            seg=view(y.off_seg_mean, np.float32, (b, L, H, nsc, sl, 2, D)).copy(),
+            part=view(y.off_part_sum, np.float32, (b, L, H, nsc, 2, D)).copy(),
+            glob=view(y.off_glob_sum, np.float32, (b, L, H, 2, D)).copy(),
+            boundary=view(y.off_boundary, ed, (b, L, wl.hidden)).copy(),
+        )
+
+    def error(self):
+        return F.ls_get_error(self.state)
+
+    def close(self):
+        if self.state:
+            F.ls_destroy_state(self.state)
+            self.state = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -46,6 +46,12 @@
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
+#if defined(__GNUC__)
+#define LS_API __attribute__((visibility("default")))
+#else
+#define LS_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -75,7 +81,7 @@ extern "C" {
 /* Shapes of one drafting state (one batch of sequences).
  *   batch b, n_layers L (tapped layers), n_kv_heads Hkv, n_q_heads Hq (multiple of Hkv),
  *   head_dim D (multiple of 8, <= 256), hidden (multiple of 8), block B (1..32),
- *   window W (>= B+1, multiple of 8), n_scales (1..4), scales ascending, each >= B+1,
+ *   window W (>= B+1), n_scales (1..4), scales ascending, each >= B+1,
  *   each dividing the next (so no segment of any scale straddles a larger one),
  *   slots_per_scale >= 1, dtype LS_F32 | LS_BF16, flags LS_FLAG_*.              */
 typedef struct {
@@ -116,19 +122,19 @@ typedef struct ls_state ls_state; /* opaque host handle */
 
 /* Bytes of the state arena for `cfg`. Depends on the shapes only, never on a prefix
  * length (the views are fixed-size: Figure 1 caption, abstract). 0 if cfg is invalid. */
-size_t ls_state_bytes(const ls_config* cfg);
+LS_API size_t ls_state_bytes(const ls_config* cfg);
 
 /* Fills *out with the arena layout for `cfg` (host-only computation). */
-int ls_get_layout(const ls_config* cfg, ls_layout* out);
+LS_API int ls_get_layout(const ls_config* cfg, ls_layout* out);
 
 /* Validates cfg, records d_arena (>= ls_state_bytes(cfg) bytes, 256-byte aligned,
  * caller-owned), zeroes it on `stream` (len = 0, every view empty) and creates the
  * host handle in *out. The arena must stay allocated until ls_destroy_state.        */
-int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_state** out,
+LS_API int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_state** out,
                   cudaStream_t stream);
 
 /* Workspace bytes that ls_prefill_summary needs for rows [row_begin, row_end). */
-size_t ls_prefill_workspace_bytes(const ls_config* cfg, int64_t row_begin, int64_t row_end);
+LS_API size_t ls_prefill_workspace_bytes(const ls_config* cfg, int64_t row_begin, int64_t row_end);
 
 /* Summary initialisation over the prefix at target prefill (Figure 3 caption).
  * Appends prefix rows p in [row_begin, min(row_end, prefix_len[b])) of every sequence.
@@ -145,7 +151,7 @@ size_t ls_prefill_workspace_bytes(const ls_config* cfg, int64_t row_begin, int64
  *   d_workspace    >= ls_prefill_workspace_bytes(...) bytes of caller scratch.
  * After the call len = min(row_end, P_b), the window holds the last min(len, W) rows,
  * the summary covers rows [0, len).                                                  */
-int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t plane_stride,
+LS_API int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t plane_stride,
                        int64_t row_stride, const int64_t* d_prefix_len, int64_t row_begin,
                        int64_t row_end, const void* d_last_hidden, void* d_workspace,
                        size_t workspace_bytes, cudaStream_t stream);
@@ -159,7 +165,7 @@ int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t p
  *   d_accept_len    int32 [b] out: a;  d_next_token int32 [b] out: target_ids[a]
  * Retains verify rows 0..a (Delta = a + 1 <= B + 1): ring window, summary sums,
  * segment finalisation and mean rows, boundary = verify_hidden[a], len += Delta.   */
-int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
+LS_API int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
                     const void* d_verify_k, const void* d_verify_v,
                     const void* d_verify_hidden, int32_t* d_accept_len,
                     int32_t* d_next_token, cudaStream_t stream);
@@ -172,26 +178,26 @@ int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_t
  *   softmax_scale  logit multiplier (1/sqrt(D) for the usual attention).
  * Uses the tcgen05 tensor-core kernel when dtype is bf16, (Hq/Hkv)*B == 64, D == 128 and
  * kv_rows <= 768 (unless LS_FLAG_FORCE_SIMT), otherwise a CUDA-core kernel.          */
-int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count,
+LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count,
                     const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
                     int64_t boundary_stride, float softmax_scale, void* d_out,
                     cudaStream_t stream);
 
 /* 1 if ls_draft_attend takes the tcgen05 path for this state, 0 if the CUDA-core one. */
-int ls_attend_uses_tensor_cores(const ls_state* st);
+LS_API int ls_attend_uses_tensor_cores(const ls_state* st);
 
 /* Copies the first `bytes` bytes of the arena to h_dst; synchronises `stream`. */
-int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStream_t stream);
+LS_API int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStream_t stream);
 
 /* Reads the device error word into *h_code (synchronous). Returns LS_ERR_DEVICE or
  * LS_ERR_DEVICE_TIMEOUT when it is non-zero, LS_OK otherwise.                      */
-int ls_get_error(const ls_state* st, int32_t* h_code);
+LS_API int ls_get_error(const ls_state* st, int32_t* h_code);
 
 /* Frees the host handle only; the arena stays the caller's. */
-void ls_destroy_state(ls_state* st);
+LS_API void ls_destroy_state(ls_state* st);
 
 /* Static description of a status code. */
-const char* ls_status_string(int status);
+LS_API const char* ls_status_string(int status);
 
 #ifdef __cplusplus
 }

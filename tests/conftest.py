@@ -10,6 +10,9 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # the in-tree libraries are built (or found up to date) before any test imports them
+    from fixed_cost_drafter_b200 import build as _build
+    _build.build()
 
 
 @pytest.fixture(scope="session")

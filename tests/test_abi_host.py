@@ -1,0 +1,96 @@
+"""CPU checks of the C ABI: the library loads without a GPU, exports every declared entry
+point, validates configurations and lays out a fixed-size state arena."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import fixed_cost_drafter_b200 as F
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "longspark.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LS_API\s+[\w\s\*]+?\b(ls_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(F.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(F.EXPORTED) == names
+
+
+def _cfg(**kw):
+    base = dict(batch=16, n_layers=4, n_kv_heads=8, n_q_heads=32, head_dim=128, hidden=4096, block=16,
+                window=512, scales=[64, 512, 4096], slots_per_scale=32, dtype=F.LS_BF16)
+    base.update(kw)
+    return F.make_config(**base)
+
+
+def test_layout_sizes():
+    c = _cfg()
+    y = F.ls_get_layout(c)
+    b, L, H, D, nsc, sl = 16, 4, 8, 128, 3, 32
+    R = 512 + nsc * (sl + 1) + 1
+    assert y.kv_rows == R == 612 and y.elem_bytes == 2
+    assert y.off_seg_mean - y.off_kv >= b * L * H * 2 * R * D * 2
+    assert y.off_part_sum - y.off_seg_mean >= b * L * H * nsc * sl * 2 * D * 4
+    assert y.off_glob_sum - y.off_part_sum >= b * L * H * nsc * 2 * D * 4
+    assert y.off_boundary - y.off_glob_sum >= b * L * H * 2 * D * 4
+    assert y.total_bytes - y.off_boundary >= b * L * 4096 * 2
+    for off in (y.off_counters, y.off_error, y.off_kv, y.off_seg_mean, y.off_part_sum, y.off_glob_sum,
+                y.off_boundary, y.total_bytes):
+        assert off % 256 == 0
+    assert F.ls_state_bytes(c) == y.total_bytes
+    # about 13.3 MB per sequence at Qwen3-8B shapes, whatever the prefix
+    assert 13.2e6 < y.total_bytes / 16 < 13.5e6
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), F.LS_ERR_INVALID_ARG),
+    (dict(n_q_heads=30), F.LS_ERR_SHAPE),
+    (dict(window=16), F.LS_ERR_SHAPE),             # W < B + 1
+    (dict(scales=[64, 64, 4096]), F.LS_ERR_SHAPE),  # not ascending
+    (dict(scales=[16, 512, 4096]), F.LS_ERR_UNSUPPORTED),  # smallest scale < B + 1
+    (dict(scales=[64, 500, 4096]), F.LS_ERR_UNSUPPORTED),  # does not divide the next
+    (dict(head_dim=96), F.LS_ERR_UNSUPPORTED),
+    (dict(dtype=7), F.LS_ERR_INVALID_ARG),
+    (dict(n_kv_heads=32, n_q_heads=64), F.LS_ERR_UNSUPPORTED),
+])
+def test_config_validation(kw, status):
+    c = _cfg(**kw)
+    assert F.ls_state_bytes(c) == 0
+    with pytest.raises(F.LsError) as e:
+        F.ls_get_layout(c)
+    assert e.value.status == status
+
+
+def test_init_rejects_null_and_misaligned_arena():
+    c = _cfg(batch=1)
+    with pytest.raises(F.LsError) as e:
+        F.ls_init_state(c, None, 1 << 30, 0)
+    assert e.value.status == F.LS_ERR_INVALID_ARG
+    with pytest.raises(F.LsError) as e:
+        F.ls_init_state(c, 0x1000 + 8, 1 << 30, 0)
+    assert e.value.status == F.LS_ERR_INVALID_ARG
+    with pytest.raises(F.LsError) as e:
+        F.ls_init_state(c, 0x10000, 16, 0)
+    assert e.value.status == F.LS_ERR_SHAPE
+
+
+def test_prefill_workspace_bytes():
+    c = _cfg()
+    # one fp32 sum per (sequence, layer, 512-row unit, K/V column)
+    assert F.ls_prefill_workspace_bytes(c, 0, 65536) >= 16 * 4 * 128 * 2 * 8 * 128 * 4
+    assert F.ls_prefill_workspace_bytes(c, 10, 5) == 0
+
+
+def test_status_strings():
+    for s in (0, -1, -2, -3, -4, -5, -6):
+        assert F.ls_status_string(s) != "unknown status"

@@ -1,0 +1,87 @@
+"""Parity at the full workload sizes, on sampled tiles the oracle computes one by one.
+
+Each run uses the same launch sequence the bench times (one ls_commit_round and one
+ls_draft_attend over all tapped layers per round, batch 16). The sampled tiles cover
+first/last sequences, layers and KV heads; the oracle rebuilds their whole K/V cache
+(prefix + retained verify rows) from the generator and recomputes the views by their
+definition. Properties that hold at any size are checked on every tile.
+"""
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from tests import oracle_side as OS  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import fixed_cost_drafter_b200 as F
+    from fixed_cost_drafter_b200 import workloads as WL
+
+
+def _run_full(wl, rounds=None, prefill_chunk=None, check_every_round=False):
+    run = WL.DeviceRun(wl, rounds=rounds, prefill_chunk=prefill_chunk)
+    run.prefill()
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    acc_gpu = []
+    for r in range(run.rounds):
+        run.commit(inp, r)
+        run.attend(inp, r, out)
+        if check_every_round:
+            acc_gpu.append(run.accept_len.clone())
+    torch.cuda.synchronize()
+    return run, out, acc_gpu
+
+
+def _sampled_check(run, wl, out, tiles):
+    st = run.read_state()
+    R = run.rounds
+    draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
+    acc = OS.accepts_from_ids(draft, target)
+    assert np.array_equal(acc, run.accept_host), "generator accepts vs oracle scan"
+    # any-size properties on every tile: len and counters consistent, all layers equal
+    P = run.prefix_len
+    want_len = P + (acc + 1).sum(axis=0)
+    assert np.array_equal(st["counters"][:, :, 0], np.repeat(want_len[:, None], wl.n_layers, 1))
+    for k, s in enumerate(wl.scales):
+        assert np.array_equal(st["counters"][:, :, 1 + k], st["counters"][:, :, 0] // s)
+    assert np.all(np.isfinite(out.float().cpu().numpy()))
+    for b, l, h in tiles:
+        sh, views = OS.tile_views(wl, b, l, h, int(P[b]), acc[:, b], run.scale_host)
+        OS.check_tile_state(wl, st, b, l, h, views)
+        hid = OS.boundary_hidden(wl, b, l, R - 1, int(acc[R - 1, b]))
+        assert np.array_equal(st["boundary"][b, l], hid)
+        ref = OS.tile_attend(wl, sh, views, b, l, h, R - 1, hid)
+        o = out[b, l].view(wl.block, wl.n_q_heads, wl.head_dim)[:, h * wl.group:(h + 1) * wl.group]
+        err = np.abs(o.float().cpu().numpy() - ref).max()
+        assert err <= OS.ATTEND_ATOL, ("attend", b, l, h, float(err))
+
+
+TILES = [(0, 0, 0), (7, 2, 5), (15, 3, 7)]
+
+
+@pytest.mark.parametrize("name", ["qwen3_4b_32k", "qwen3_8b_64k", "qwen3_8b_128k_ragged"])
+def test_full_config(name):
+    wl = WL.CONFIGS[name]
+    run, out, _ = _run_full(wl)
+    assert run.error() == (F.LS_OK, 0)
+    _sampled_check(run, wl, out, TILES)
+
+
+@pytest.mark.parametrize("prefix,batch,mean", [(4096, 1, 2.5), (16384, 4, 4.0), (131072, 64, 6.0)])
+def test_sweep_points(prefix, batch, mean):
+    wl = WL.sweep_point(prefix, batch, mean)
+    chunk = 32768 if prefix * batch > 4 * 1024 * 1024 else None
+    run, out, _ = _run_full(wl, prefill_chunk=chunk)
+    assert run.error() == (F.LS_OK, 0)
+    _sampled_check(run, wl, out, [(0, 0, 0), (batch - 1, 3, 7)])
+
+
+def test_state_bytes_fixed_across_sweep():
+    """Drafter state bytes depend on batch and shapes only, never on the prefix."""
+    for batch in WL.SWEEP_BATCHES:
+        sizes = {F.ls_state_bytes(WL.sweep_point(p, batch, 4.0).config()) for p in WL.SWEEP_PREFIXES}
+        assert len(sizes) == 1

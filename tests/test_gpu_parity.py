@@ -1,0 +1,198 @@
+"""Parity of the CUDA path with the oracle at sizes the oracle finishes in seconds.
+
+Integers (accept length, next token, len, per-scale segment counts, ring contents and
+mean-row roundings) are compared bit for bit; summary means within 1e-3 normwise
+relative error per slot vector; attention outputs within 1e-2 max absolute error.
+"""
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle as O  # noqa: E402
+import synth as S  # noqa: E402
+from tests import oracle_side as OS  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import fixed_cost_drafter_b200 as F
+    from fixed_cost_drafter_b200 import workloads as WL
+
+
+MID = dict(seed=5, batch=3, n_layers=2, n_kv_heads=2, n_q_heads=8, head_dim=128, hidden=512, block=16,
+           window=128, scales=(32, 64, 256), slots=4, dtype="bf16", prefix=(300, 1400), rounds=40,
+           accept_mean=None, vocab=1000, head_scale=True)
+
+
+def _mid(**kw):
+    return WL.Workload(name="mid", **{**MID, **kw})
+
+
+def _out_tile(out, wl, b, l, g):
+    """GPU output [B][grp][D] of tile (b, l, g) from out [b][L][B][Hq*D]."""
+    o = out[b, l].view(wl.block, wl.n_q_heads, wl.head_dim)[:, g * wl.group:(g + 1) * wl.group]
+    return o.float().cpu().numpy().astype(np.float64)
+
+
+def _check_run_against_oracle(run, wl, rounds_done, out, r_last, tiles=None):
+    """Every (or the given) tile's state and attention output vs oracle recompute."""
+    st = run.read_state()
+    draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
+    acc = (OS.accepts_from_ids(draft[:rounds_done], target[:rounds_done]) if rounds_done
+           else np.zeros((0, wl.batch), dtype=np.int64))
+    tiles = tiles or [(b, l, h) for b in range(wl.batch) for l in range(wl.n_layers)
+                      for h in range(wl.n_kv_heads)]
+    for b, l, h in tiles:
+        P = int(run.prefix_len[b])
+        sh, views = OS.tile_views(wl, b, l, h, P, acc[:, b], run.scale_host)
+        OS.check_tile_state(wl, st, b, l, h, views)
+        hid = OS.boundary_hidden(wl, b, l, rounds_done - 1, int(acc[rounds_done - 1, b]) if rounds_done else 0)
+        assert np.array_equal(st["boundary"][b, l], hid), ("boundary", b, l)
+        if out is not None:
+            ref = OS.tile_attend(wl, sh, views, b, l, h, r_last, hid)
+            got = _out_tile(out, wl, b, l, h)
+            err = np.abs(got - ref).max()
+            assert err <= OS.ATTEND_ATOL, ("attend", b, l, h, float(err))
+    return acc
+
+
+def test_tiny_round_by_round():
+    """Config 1 (fp32): every round against the incremental oracle (Figure 3's form)."""
+    wl = WL.CONFIGS["tiny"]
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    inp = run.make_round_inputs()
+    sh = O.Shapes(n_layers=wl.n_layers, n_kv_heads=wl.n_kv_heads, n_q_heads=wl.n_q_heads,
+                  head_dim=wl.head_dim, hidden=wl.hidden, block=wl.block, window=wl.window,
+                  scales=tuple(wl.scales), slots=wl.slots)
+    L, H, D, P = wl.n_layers, wl.n_kv_heads, wl.head_dim, int(run.prefix_len[0])
+    pk = S.fill_normal(wl.seed, S.PREFIX_K, (1, 1, L, P, H * D), head_dim=D, dtype="f32")[0, 0]
+    pv = S.fill_normal(wl.seed, S.PREFIX_V, (1, 1, L, P, H * D), head_dim=D, dtype="f32")[0, 0]
+    hid = S.fill_normal(wl.seed, S.LAST_HIDDEN, (1, 1, L, 1, wl.hidden), dtype="f32")[0, 0, :, 0]
+    views = O.prefill(sh, O.to_f64(pk, "f32").reshape(L, P, H, D), O.to_f64(pv, "f32").reshape(L, P, H, D), P,
+                      O.to_f64(hid, "f32"))
+    st = run.read_state()
+    for l in range(L):
+        for h in range(H):
+            OS.check_tile_state(wl, st, 0, l, h, OS.slice_views(views, l, h))
+    out = run.new_out()
+    draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
+    vk_all, vv_all, vh_all, q_all = (inp[k].cpu().numpy() for k in ("vk", "vv", "vh", "q"))
+    for r in range(wl.rounds):
+        run.commit(inp, r)
+        run.attend(inp, r, out)
+        torch.cuda.synchronize()
+        a, nxt = O.commit_round(sh, views, draft[r, 0], target[r, 0],
+                                O.to_f64(vk_all[r, 0], "f32").reshape(L, wl.block + 1, H, D),
+                                O.to_f64(vv_all[r, 0], "f32").reshape(L, wl.block + 1, H, D),
+                                O.to_f64(vh_all[r, 0], "f32"))
+        assert int(run.accept_len[0]) == a and int(run.next_token[0]) == nxt
+        st = run.read_state()
+        for l in range(L):
+            for h in range(H):
+                OS.check_tile_state(wl, st, 0, l, h, OS.slice_views(views, l, h))
+        assert np.array_equal(st["boundary"][0], O.to_f64(vh_all[r, 0, :, a], "f32"))
+        bk = views.boundary[:, :H * D].reshape(L, H, D)
+        bv = views.boundary[:, H * D:2 * H * D].reshape(L, H, D)
+        ref = O.draft_attend(sh, views, O.to_f64(q_all[r, 0], "f32").reshape(L, wl.block, wl.n_q_heads, D),
+                             bk, bv, 1.0 / np.sqrt(D))
+        got = out[0].view(L, wl.block, wl.n_q_heads, D).double().cpu().numpy()
+        assert np.abs(got - ref).max() <= OS.ATTEND_ATOL
+    assert run.error() == (F.LS_OK, 0)
+
+
+@pytest.mark.parametrize("force_simt", [False, True], ids=["default_path", "cuda_cores"])
+def test_mid_ragged_all_tiles(force_simt):
+    """Ragged prefixes, several tiles; bf16; GQA group 4 x B 16 = a 64-row tile."""
+    wl = _mid(flags=F.LS_FLAG_FORCE_SIMT if force_simt else 0)
+    run = WL.DeviceRun(wl)
+    if force_simt:
+        assert not F.ls_attend_uses_tensor_cores(run.state)
+    run.prefill()
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    _check_run_against_oracle(run, wl, 0, None, -1)
+    for r in range(wl.rounds):
+        run.commit(inp, r)
+        run.attend(inp, r, out)
+        if r in (0, 7, wl.rounds - 1):
+            torch.cuda.synchronize()
+            _check_run_against_oracle(run, wl, r + 1, out, r)
+    assert run.error() == (F.LS_OK, 0)
+
+
+def test_paths_agree():
+    """Tensor-core and CUDA-core attention on the same state agree within tolerance."""
+    wl = _mid(rounds=5)
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    inp = run.make_round_inputs()
+    for r in range(wl.rounds):
+        run.commit(inp, r)
+    out_a = run.new_out()
+    run.attend(inp, wl.rounds - 1, out_a)
+    wl2 = _mid(rounds=5, flags=F.LS_FLAG_FORCE_SIMT)
+    run2 = WL.DeviceRun(wl2)
+    run2.prefill()
+    inp2 = run2.make_round_inputs()
+    for r in range(wl.rounds):
+        run2.commit(inp2, r)
+    out_b = run2.new_out()
+    run2.attend(inp2, wl.rounds - 1, out_b)
+    torch.cuda.synchronize()
+    assert (out_a.float() - out_b.float()).abs().max().item() <= OS.ATTEND_ATOL
+
+
+def test_per_layer_calls_match_one_call():
+    wl = _mid(rounds=3)
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    inp = run.make_round_inputs()
+    for r in range(3):
+        run.commit(inp, r)
+    full = run.new_out()
+    run.attend(inp, 2, full)
+    for l in range(wl.n_layers):
+        one = run.new_out(1)
+        run.attend(inp, 2, one, layer_begin=l, layer_count=1)
+        torch.cuda.synchronize()
+        assert torch.equal(one[:, 0], full[:, l])
+
+
+def test_chunked_prefill_matches_oracle():
+    wl = _mid(rounds=6, prefix=(700, 1337))
+    run = WL.DeviceRun(wl, prefill_chunk=256)
+    run.prefill()
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    for r in range(wl.rounds):
+        run.commit(inp, r)
+        run.attend(inp, r, out)
+    torch.cuda.synchronize()
+    _check_run_against_oracle(run, wl, wl.rounds, out, wl.rounds - 1)
+    assert run.error() == (F.LS_OK, 0)
+
+
+@pytest.mark.parametrize("prefix,accepts", [
+    (0, None),                 # empty prefix: every view starts empty
+    (5, None),                 # prefix shorter than the window and every scale
+    (512, None),               # prefix a multiple of every scale: all partials empty
+    (256 - 3, 16),             # one round crosses the 32-, 64- and 256-row boundaries at once
+    (1000, 0),                 # a = 0 every round: Delta = 1
+    (1000, 16),                # a = B every round: Delta = B + 1
+], ids=["empty", "short", "aligned", "multi_crossing", "a0", "aB"])
+def test_edge_cases(prefix, accepts):
+    wl = _mid(rounds=12, prefix=prefix)
+    run = WL.DeviceRun(wl, accepts_override=None if accepts is None else [accepts] * 12)
+    run.prefill()
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    for r in range(wl.rounds):
+        run.commit(inp, r)
+        run.attend(inp, r, out)
+        if r in (0, wl.rounds - 1):
+            torch.cuda.synchronize()
+            _check_run_against_oracle(run, wl, r + 1, out, r)
+    assert run.error() == (F.LS_OK, 0)

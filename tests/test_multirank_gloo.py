@@ -1,0 +1,56 @@
+"""World-size-2 gloo run of the bench's multi-rank host logic on CPU.
+
+The path shards by sequence with no data-path collective: every rank owns a disjoint
+batch (weak scaling) and the only collective is the max over ranks of the timed region.
+"""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    r, w, _ = bench.dist_env()
+    off = bench.sequence_offset(r, 16)
+    t = bench.max_over_ranks(1.0 + r, w, torch.device("cpu"))
+    bench.barrier(w)
+    q.put((r, off, t))
+    dist.destroy_process_group()
+
+
+def test_two_ranks_shard_and_max():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [o for _, o, _ in res] == [0, 16]       # disjoint sequence ranges
+    assert all(t == 2.0 for _, _, t in res)         # every rank sees the slowest rank's time
+
+
+def test_reference_arm_other_ranks_exit(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0

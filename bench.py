@@ -309,6 +309,9 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     wl = WLM.CONFIGS[args.config]
+    if args.prefix:  # profiling runs: same per-round work, smaller prefix to generate
+        from dataclasses import replace
+        wl = replace(wl, prefix=args.prefix)
     K, W = args.steps, args.warmup
     # distinct rounds of generated inputs; the timed loop cycles through them (the state
     # keeps growing, every round re-reads its inputs from HBM after the L2 flush)
@@ -523,6 +526,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--sweep-rounds", type=int, default=40)
+    ap.add_argument("--prefix", type=int, default=0, help="override the workload's prefix length")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

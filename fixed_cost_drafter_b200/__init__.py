@@ -29,6 +29,7 @@ LS_DEVERR_ORDER = 0x4
 LS_F32 = 0
 LS_BF16 = 1
 LS_FLAG_FORCE_SIMT = 0x1
+LS_FLAG_OUT_F32 = 0x2
 LS_MAX_SCALES = 4
 
 EXPORTED = (

@@ -61,7 +61,7 @@ int validate(const ls_config* c) {
   const int lanes = c->head_dim * elem / 16;
   if (!pow2(lanes) || lanes > 32) return LS_ERR_UNSUPPORTED;
   if (c->n_kv_heads > 16 || c->block > 32) return LS_ERR_UNSUPPORTED;
-  if (c->flags & ~LS_FLAG_FORCE_SIMT) return LS_ERR_INVALID_ARG;
+  if (c->flags & ~(LS_FLAG_FORCE_SIMT | LS_FLAG_OUT_F32)) return LS_ERR_INVALID_ARG;
   return LS_OK;
 }
 
@@ -134,6 +134,7 @@ int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_st
   p.b = cfg->batch; p.L = cfg->n_layers; p.Hkv = cfg->n_kv_heads; p.Hq = cfg->n_q_heads;
   p.D = cfg->head_dim; p.hidden = cfg->hidden; p.B = cfg->block; p.W = cfg->window;
   p.nsc = cfg->n_scales; p.slots = cfg->slots_per_scale; p.R = y.R; p.dtype = cfg->dtype;
+  p.out_f32 = (cfg->flags & LS_FLAG_OUT_F32) ? 1 : 0;
   for (int k = 0; k < LS_MAX_SCALES; ++k) p.scales[k] = k < cfg->n_scales ? cfg->scales[k] : 1;
   p.counters = reinterpret_cast<int64_t*>(base + y.counters);
   p.err = reinterpret_cast<int32_t*>(base + y.error);

@@ -18,7 +18,7 @@ template <typename T, int DV>
 __global__ void __launch_bounds__(kSimtWarps * 32)
 attend_simt_kernel(Dev p, int layer_begin, int layer_count, const T* __restrict__ q,
                    const T* __restrict__ bk, const T* __restrict__ bv, int64_t bstride,
-                   float scale, T* __restrict__ out) {
+                   float scale, void* __restrict__ out) {
   using E = Elem<T>;
   const int g = blockIdx.x, lc = blockIdx.y, b = blockIdx.z;
   const int l = layer_begin + lc;
@@ -116,7 +116,10 @@ attend_simt_kernel(Dev p, int layer_begin, int layer_count, const T* __restrict_
     const float inv = 1.0f / lrun[r];
     const int64_t ob = (((int64_t(b) * layer_count + lc) * p.B + i) * p.Hq + g * grp + j) * D;
 #pragma unroll
-    for (int dd = 0; dd < DV; ++dd) E::store1(out, ob + lane + 32 * dd, o[r][dd] * inv);
+    for (int dd = 0; dd < DV; ++dd) {
+      if (p.out_f32) static_cast<float*>(out)[ob + lane + 32 * dd] = o[r][dd] * inv;
+      else E::store1(out, ob + lane + 32 * dd, o[r][dd] * inv);
+    }
   }
 }
 
@@ -137,7 +140,7 @@ static cudaError_t launch_simt_t(const Dev& p, int lb, int lcount, const void* q
   const dim3 grid(p.Hkv, lcount, p.b);
   kern<<<grid, kSimtWarps * 32, smem, stream>>>(p, lb, lcount, static_cast<const T*>(q),
                                                 static_cast<const T*>(bk), static_cast<const T*>(bv),
-                                                bstride, scale, static_cast<T*>(out));
+                                                bstride, scale, out);
   return cudaGetLastError();
 }
 

@@ -4,10 +4,13 @@
 
 namespace ls {
 
-// Per-state constants of the tensor-core path (tensor map over the arena's K/V rows).
+// Per-state constants of the tensor-core path: tensor maps over the arena's K/V rows
+// (128-row chunks, and the shorter last chunk of each tile).
 struct alignas(64) TcPlan {
-  alignas(64) unsigned char kv_map[128];  // CUtensorMap of the kv region
-  int32_t n_chunks;                        // 128-row chunks of arena rows per tile
+  alignas(64) unsigned char kv_map[128];       // CUtensorMap, box 64 x 128 rows
+  alignas(64) unsigned char kv_tail_map[128];  // CUtensorMap, box 64 x tail_rows
+  int32_t n_chunks;                             // 128-row chunks of arena rows per tile
+  int32_t tail_rows;                            // rows of the last chunk, rounded up to 16
 };
 
 bool tc_supported(const Dev& p);

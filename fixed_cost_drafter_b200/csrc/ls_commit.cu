@@ -6,10 +6,13 @@
 //   1. greedy accept scan (every warp, one ballot per 32 drafts): a, Delta = a + 1;
 //   2. verify rows 0..a are read once with 16-byte loads (D*e/16 lanes per row, several
 //      rows per warp instruction) and written to ring slot (len + i) mod W;
-//   3. the same registers are summed per scale into the part that closes the open
-//      segment (rows i < c_k) and the part that opens the next one, reduced across the
-//      row groups of the warp with shuffles, and folded into the fp32 partial / global
-//      sums; a segment whose last row arrived becomes a slot mean (fp32 + dtype copy);
+//   3. the same registers are summed into the rows that close the open segments (i < c)
+//      and the rows that open the next ones (i >= c), reduced across the row groups of
+//      the warp with shuffles, and folded into the fp32 partial / global sums; a segment
+//      whose last row arrived becomes a slot mean (fp32 + dtype copy). One split row c
+//      serves every scale: the scales divide each other and Delta <= s_0, so the only
+//      segment boundaries a round can cross all sit at the single multiple of s_0 in
+//      (len, len + Delta], i.e. at c = s_0 - len mod s_0;
 //   4. the CTA copies the hidden vector of verify row a into the boundary view.
 // Counters are read by every warp before the CTA barrier and written once after it.
 #include "ls_common.cuh"
@@ -46,11 +49,13 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
   const int delta = a + 1;
   const int64_t newlen = len + delta;
 
-  // rows that close the open segment of each scale
-  int ck[kMaxScales];
+  // rows before the split row close the open segments; scale k closes one this round
+  // exactly when its own distance to the next boundary is <= Delta (then it equals c)
+  const int c_split = int(p.scales[0] - (len - nseg[0] * p.scales[0]));
+  unsigned closes = 0;
 #pragma unroll
   for (int k = 0; k < kMaxScales; ++k)
-    ck[k] = k < nsc ? int(p.scales[k] - (len - nseg[k] * p.scales[k])) : 0x7fffffff;
+    if (k < nsc && p.scales[k] - (len - nseg[k] * p.scales[k]) <= delta) closes |= 1u << k;
 
   if (warp < 2 * p.Hkv) {
     const int h = warp >> 1, t = warp & 1;
@@ -62,38 +67,31 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
     const int rpi = 32 / lpr;   // rows per warp instruction
     const int c = lane & (lpr - 1), rg = lane / lpr;
 
-    float all[VEC], lo[kMaxScales][VEC], hi[kMaxScales][VEC];
+    float lo[VEC], hi[VEC];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      all[e] = 0.f;
-#pragma unroll
-      for (int k = 0; k < kMaxScales; ++k) lo[k][e] = hi[k][e] = 0.f;
-    }
+    for (int e = 0; e < VEC; ++e) lo[e] = hi[e] = 0.f;
+    const int ring0 = int(len % p.W);
     for (int i = rg; i < delta; i += rpi) {
       const uint4 raw = ld_nc_v4(src + int64_t(i) * row_stride + c * VEC);
-      const int slot = int((len + i) % p.W);
+      int slot = ring0 + i;
+      if (slot >= p.W) slot -= p.W;  // Delta <= W
       *reinterpret_cast<uint4*>(kvt + int64_t(slot) * p.D + c * VEC) = raw;
       float f[VEC];
       E::to_f32(raw, f);
+      if (i < c_split) {
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        all[e] += f[e];
+        for (int e = 0; e < VEC; ++e) lo[e] += f[e];
+      } else {
 #pragma unroll
-        for (int k = 0; k < kMaxScales; ++k) {
-          if (i < ck[k]) lo[k][e] += f[e]; else hi[k][e] += f[e];
-        }
+        for (int e = 0; e < VEC; ++e) hi[e] += f[e];
       }
     }
     // segmented reduction across the row groups of the warp
     for (int off = lpr; off < 32; off <<= 1) {
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
-        all[e] += __shfl_xor_sync(0xffffffffu, all[e], off);
-#pragma unroll
-        for (int k = 0; k < kMaxScales; ++k) {
-          lo[k][e] += __shfl_xor_sync(0xffffffffu, lo[k][e], off);
-          hi[k][e] += __shfl_xor_sync(0xffffffffu, hi[k][e], off);
-        }
+        lo[e] += __shfl_xor_sync(0xffffffffu, lo[e], off);
+        hi[e] += __shfl_xor_sync(0xffffffffu, hi[e], off);
       }
     }
     if (rg == 0) {
@@ -104,8 +102,8 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
 #pragma unroll
       for (int e = 0; e < VEC; e += 4) {
         float4 v4 = *reinterpret_cast<const float4*>(gp + e);
-        g[e] = v4.x + all[e]; g[e + 1] = v4.y + all[e + 1];
-        g[e + 2] = v4.z + all[e + 2]; g[e + 3] = v4.w + all[e + 3];
+        g[e] = v4.x + (lo[e] + hi[e]); g[e + 1] = v4.y + (lo[e + 1] + hi[e + 1]);
+        g[e + 2] = v4.z + (lo[e + 2] + hi[e + 2]); g[e + 3] = v4.w + (lo[e + 3] + hi[e + 3]);
         *reinterpret_cast<float4*>(gp + e) = make_float4(g[e], g[e + 1], g[e + 2], g[e + 3]);
       }
 #pragma unroll
@@ -123,22 +121,22 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
           float4 v4 = *reinterpret_cast<const float4*>(pp + e);
           pr[e] = v4.x; pr[e + 1] = v4.y; pr[e + 2] = v4.z; pr[e + 3] = v4.w;
         }
-        const bool completes = ck[k] <= delta;
+        const bool completes = (closes >> k) & 1u;
         const int64_t row0 = int64_t(p.W) + int64_t(k) * (p.slots + 1);
         if (completes) {
           const int slot = int(nseg[k] % p.slots);
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) m[e] = (pr[e] + lo[k][e]) / float(s);
+          for (int e = 0; e < VEC; ++e) m[e] = (pr[e] + lo[e]) / float(s);
           float* sg = p.seg + (((tile * nsc + k) * p.slots + slot) * 2 + t) * p.D + cb;
 #pragma unroll
           for (int e = 0; e < VEC; e += 4)
             *reinterpret_cast<float4*>(sg + e) = make_float4(m[e], m[e + 1], m[e + 2], m[e + 3]);
           *reinterpret_cast<uint4*>(kvt + (row0 + slot) * p.D + cb) = E::from_f32(m);
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) pr[e] = hi[k][e];
-        } else {
+          for (int e = 0; e < VEC; ++e) pr[e] = hi[e];
+        } else {  // no boundary crossed at this scale: every row extends the open segment
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) pr[e] += lo[k][e];
+          for (int e = 0; e < VEC; ++e) pr[e] += lo[e] + hi[e];
         }
 #pragma unroll
         for (int e = 0; e < VEC; e += 4)
@@ -162,7 +160,7 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
   __syncthreads();  // every warp has read the counters
   if (threadIdx.x == 0) {
     ctr[0] = newlen;
-    for (int k = 0; k < nsc; ++k) ctr[1 + k] = nseg[k] + (ck[k] <= delta ? 1 : 0);
+    for (int k = 0; k < nsc; ++k) ctr[1 + k] = nseg[k] + ((closes >> k) & 1u);
     if (l == 0) {
       accept_len[b] = a;
       next_token[b] = target[int64_t(b) * (p.B + 1) + a];

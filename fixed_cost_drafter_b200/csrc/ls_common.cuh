@@ -16,6 +16,7 @@ constexpr int kMaxScales = LS_MAX_SCALES;
 // Device-side view of one drafting state: shapes plus region pointers in the arena.
 struct Dev {
   int32_t b, L, Hkv, Hq, D, hidden, B, W, nsc, slots, R, dtype;
+  int32_t out_f32;  // attention output in fp32 instead of dtype
   int32_t scales[kMaxScales];
   int64_t* counters;  // [b][L][1+nsc]
   int32_t* err;       // device error word

@@ -227,8 +227,8 @@ class DeviceRun:
     def new_out(self, layer_count=None):
         wl = self.wl
         lc = wl.n_layers if layer_count is None else layer_count
-        return self.torch.empty((wl.batch, lc, wl.block, wl.n_q_heads * wl.head_dim), dtype=self.tdtype,
-                                device=self.dev)
+        dt = self.torch.float32 if (wl.flags & F.LS_FLAG_OUT_F32) else self.tdtype
+        return self.torch.empty((wl.batch, lc, wl.block, wl.n_q_heads * wl.head_dim), dtype=dt, device=self.dev)
 
     # ---- readout ----------------------------------------------------------------
     def read_state(self):

@@ -75,6 +75,9 @@ extern "C" {
 #define LS_BF16 1
 #define LS_FLAG_FORCE_SIMT 0x1      /* run draft attention on CUDA cores even where the
                                        tcgen05 tensor-core kernel applies              */
+#define LS_FLAG_OUT_F32    0x2      /* ls_draft_attend writes fp32 outputs (otherwise
+                                       `dtype`); a bf16 output adds its own rounding of
+                                       up to 2^-9 |out| to the attention's error       */
 
 #define LS_MAX_SCALES 4
 
@@ -172,7 +175,8 @@ LS_API int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32
 
 /* The drafter's block attention over the three views (Figure 2 (c)).
  *   layers [layer_begin, layer_begin + layer_count)
- *   d_q, d_out     `dtype` [b][layer_count][B][Hq][D]
+ *   d_q            `dtype` [b][layer_count][B][Hq][D]
+ *   d_out          same shape; fp32 with LS_FLAG_OUT_F32, else `dtype`
  *   d_boundary_k/v `dtype`, element (b, l, g, d) at [(b*L + l)*boundary_stride + g*D + d]
  *                  with l the absolute layer; boundary_stride >= Hkv*D, multiple of 8.
  *   softmax_scale  logit multiplier (1/sqrt(D) for the usual attention).

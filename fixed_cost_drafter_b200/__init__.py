@@ -23,6 +23,7 @@ LS_ERR_UNSUPPORTED = -3
 LS_ERR_CUDA = -4
 LS_ERR_DEVICE = -5
 LS_ERR_DEVICE_TIMEOUT = -6
+LS_ERR_SCRATCH_LIMIT = -7
 LS_DEVERR_PREFIX_LEN = 0x1
 LS_DEVERR_WAIT_TIMEOUT = 0x2
 LS_DEVERR_ORDER = 0x4
@@ -34,7 +35,7 @@ LS_MAX_SCALES = 4
 
 EXPORTED = (
     "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",
-    "ls_prefill_summary", "ls_commit_round", "ls_draft_attend", "ls_attend_uses_tensor_cores",
+    "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend", "ls_attend_uses_tensor_cores",
     "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
 )
 
@@ -77,6 +78,7 @@ def _load():
         "ls_init_state": (ctypes.c_int, [cfgp, vp, sz, ctypes.POINTER(vp), vp]),
         "ls_prefill_workspace_bytes": (sz, [cfgp, i64, i64]),
         "ls_prefill_summary": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, i64, i64, vp, vp, sz, vp]),
+        "ls_prefill_summary_noalloc": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, i64, i64, vp, vp]),
         "ls_commit_round": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ls_draft_attend": (ctypes.c_int, [vp, i32, i32, vp, vp, vp, i64, ctypes.c_float, vp, vp]),
         "ls_attend_uses_tensor_cores": (ctypes.c_int, [vp]),
@@ -166,6 +168,15 @@ def ls_prefill_summary(state, k, v, plane_stride, row_stride, prefix_len, row_be
     _check("ls_prefill_summary", _lib.ls_prefill_summary(
         state, _ptr(k), _ptr(v), plane_stride, row_stride, _ptr(prefix_len), row_begin, row_end,
         _ptr(last_hidden), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def ls_prefill_summary_noalloc(state, k, v, plane_stride, row_stride, prefix_len, row_begin, row_end,
+                               last_hidden, stream=None) -> None:
+    """ls_prefill_summary without a workspace argument: the library's fixed 16 MiB scratch
+    is used instead, for callers that cannot allocate device memory."""
+    _check("ls_prefill_summary_noalloc", _lib.ls_prefill_summary_noalloc(
+        state, _ptr(k), _ptr(v), plane_stride, row_stride, _ptr(prefix_len), row_begin, row_end,
+        _ptr(last_hidden), _stream(stream)))
 
 
 def ls_commit_round(state, draft_ids, target_ids, verify_k, verify_v, verify_hidden, accept_len,

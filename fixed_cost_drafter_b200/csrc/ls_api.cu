@@ -20,6 +20,8 @@ cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, cons
                            int64_t plane_stride, int64_t row_stride, const int64_t* prefix_len,
                            int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws,
                            int sms, cudaStream_t stream);
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_scratch(void** out);
 }  // namespace ls
 
 struct ls_state {
@@ -80,6 +82,7 @@ const char* ls_status_string(int s) {
     case LS_ERR_CUDA: return "CUDA runtime error";
     case LS_ERR_DEVICE: return "device error word set";
     case LS_ERR_DEVICE_TIMEOUT: return "bounded device wait timed out";
+    case LS_ERR_SCRATCH_LIMIT: return "needs more than the library's fixed 16 MiB scratch: split the prefix into chunks";
     default: return "unknown status";
   }
 }
@@ -183,6 +186,30 @@ int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t p
   return cuda_status(ls::launch_prefill(st->dev, c, d_k, d_v, plane_stride, row_stride,
                                         d_prefix_len, row_begin, row_end, d_last_hidden,
                                         d_workspace, st->sms, stream));
+}
+
+int ls_prefill_summary_noalloc(ls_state* st, const void* d_k, const void* d_v, int64_t plane_stride,
+                               int64_t row_stride, const int64_t* d_prefix_len, int64_t row_begin,
+                               int64_t row_end, const void* d_last_hidden, cudaStream_t stream) {
+  if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
+  const ls_config& c = st->cfg;
+  if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
+  if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
+  const int64_t rowElems = int64_t(c.n_kv_heads) * c.head_dim;
+  if (row_end > row_begin) {
+    if (!d_k || !d_v) return LS_ERR_INVALID_ARG;
+    if (row_stride < rowElems || row_stride % 8 != 0 || plane_stride % 8 != 0) return LS_ERR_SHAPE;
+    if (plane_stride < (row_end - row_begin) * row_stride && c.batch * c.n_layers > 1)
+      return LS_ERR_SHAPE;
+    if (!aligned16(d_k) || !aligned16(d_v)) return LS_ERR_INVALID_ARG;
+  }
+  if (d_last_hidden && !aligned16(d_last_hidden)) return LS_ERR_INVALID_ARG;
+  if (ls::prefill_workspace_bytes(c, row_begin, row_end) > ls::noalloc_scratch_bytes())
+    return LS_ERR_SCRATCH_LIMIT;
+  void* ws = nullptr;
+  if (ls::noalloc_scratch(&ws) != cudaSuccess) return LS_ERR_CUDA;
+  return cuda_status(ls::launch_prefill(st->dev, c, d_k, d_v, plane_stride, row_stride, d_prefix_len,
+                                        row_begin, row_end, d_last_hidden, ws, st->sms, stream));
 }
 
 int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,

@@ -13,6 +13,8 @@
 // Pass 2 (prefill_finalize_kernel): per (sequence, layer, column block) the unit sums
 // are combined the same way into the segments of the scales > U, the partial sums, the
 // global sum (accumulated across chunk calls), the mean rows and the counters.
+#include <mutex>
+
 #include "ls_common.cuh"
 
 namespace ls {
@@ -504,6 +506,37 @@ cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, cons
   else
     prefill_finalize_kernel<float><<<grid, 64, 0, stream>>>(p, a, static_cast<const float*>(last_hidden));
   return cudaGetLastError();
+}
+
+// ---- fixed scratch for callers that cannot allocate ----------------------------------
+// The unit sums of pass 1 live here instead of in a caller workspace. Every GPU that
+// loads the library holds this array until the process exits. Nothing in it has to start
+// at zero: pass 2 only reads unit sums that pass 1 of the same call wrote. Calls share it,
+// so calls that overlap on the GPU race.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of the array on the current device, looked up once per device (the
+// host-side name of the array is not a device address).
+cudaError_t noalloc_scratch(void** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace ls

@@ -64,6 +64,8 @@ extern "C" {
 #define LS_ERR_CUDA           (-4)  /* a CUDA runtime call failed                       */
 #define LS_ERR_DEVICE         (-5)  /* the device error word holds a non-zero code      */
 #define LS_ERR_DEVICE_TIMEOUT (-6)  /* a bounded device wait gave up                    */
+#define LS_ERR_SCRATCH_LIMIT  (-7)  /* ls_prefill_summary_noalloc: the chunk needs more
+                                       than the library's fixed 16 MiB scratch        */
 
 /* ---- device error word bits (ls_get_error) ----------------------------------- */
 #define LS_DEVERR_PREFIX_LEN   0x1  /* prefix_len[b] < 0 or beyond what the buffers hold */
@@ -158,6 +160,27 @@ LS_API int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, in
                        int64_t row_stride, const int64_t* d_prefix_len, int64_t row_begin,
                        int64_t row_end, const void* d_last_hidden, void* d_workspace,
                        size_t workspace_bytes, cudaStream_t stream);
+
+/* Prefill that allocates nothing (the paper has no counterpart: this is an interface
+ * for callers that cannot allocate device memory when they prefill, e.g. an inference
+ * engine that reserves nearly all of the GPU's memory for its own KV-cache pool at
+ * start-up, so a cudaMalloc would fail or break up that pool, or a C host that links
+ * only this library and has no device allocator of its own).
+ * Same arguments and result as ls_prefill_summary, without the workspace: the unit sums
+ * live in a fixed array of 16 MiB compiled into the library; every GPU that loads the
+ * library holds it until the process exits. Each call needs
+ * ls_prefill_workspace_bytes(cfg, row_begin, row_end) <= 16 MiB, otherwise it returns
+ * LS_ERR_SCRATCH_LIMIT and does nothing: split the prefix into chunks (row_begin a
+ * multiple of the largest scale) that each fit. The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress); make that first call before any stream
+ * capture. Every call uses the same array, which keeps the last call's contents (nothing
+ * in it has to start at zero), so calls that overlap on the GPU race: order them on one
+ * stream or with events. Calls no cudaMalloc/cudaFree and no allocating routine.      */
+LS_API int ls_prefill_summary_noalloc(ls_state* st, const void* d_k, const void* d_v,
+                                      int64_t plane_stride, int64_t row_stride,
+                                      const int64_t* d_prefix_len, int64_t row_begin,
+                                      int64_t row_end, const void* d_last_hidden,
+                                      cudaStream_t stream);
 
 /* One round's view extraction from the target's verification pass (Figure 2 (a)-(b),
  * Figure 3 caption). Verify row 0 is the previous round's bonus token, rows 1..B the

@@ -6,10 +6,11 @@ summary update, boundary gather) followed by ``ls_draft_attend`` over all 4 tapp
 The prefill summary over the prefix runs once per request before the rounds; it is timed
 separately in the same run and reported under ``prefill``.
 
-Timing: W untimed warm-up rounds, then K timed rounds. Before every round a 256 MB
-buffer is written (untimed) so that the round starts with a cold L2, as it would after
-the target's verification pass; each round is bracketed by CUDA events on the launching
-stream (a third event splits commit from attention). ``value`` is rounds per second over
+Timing: W untimed warm-up rounds, then K timed rounds. Before every round (untimed) a
+256 MB buffer is written and a second 256 MB buffer is read, so the round starts with a
+cold L2 that holds no dirty lines of the flush (as after the target's verification pass,
+whose big reads leave clean lines); each round is bracketed by CUDA events on the
+launching stream (a third event splits commit from attention). ``value`` is rounds per second over
 all ranks (weak scaling: every rank owns its own batch of 16 sequences).
 
 ``--impl reference`` times the CPU oracle instead (rank 0 only).
@@ -289,7 +290,8 @@ def workload_config(wl):
                         f"partials + global mean, prefix {wl.prefix}",
             "batch": wl.batch, "prefix": wl.prefix if not isinstance(wl.prefix, tuple) else list(wl.prefix),
             "accept_mean": wl.accept_mean,
-            "l2": "flushed before every timed round (256 MB write, untimed)"}
+            "l2": "flushed before every timed round: 256 MB written then 256 MB read (untimed), "
+                  "so the round starts cold with no dirty flush lines to write back"}
 
 
 # ---------------------------------------------------------------------------------------
@@ -327,7 +329,7 @@ def run_gpu(args):
 
     inp = run.make_round_inputs(0, n_rounds)
     out = run.new_out()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = run.stream
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
 
@@ -440,6 +442,19 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+class L2Flush:
+    """Evicts L2 between rounds: writes a buffer larger than L2, then reads another one."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+
+    def zero_(self):  # same call shape as the plain write-only buffer it replaces
+        self.w.zero_()
+        self.r.sum()
 
 
 def e2e_measure(run, wl, dev, flush, steps, world, inp):

@@ -59,7 +59,7 @@ class ls_config(ctypes.Structure):
 class ls_layout(ctypes.Structure):
     _fields_ = [
         ("total_bytes", ctypes.c_size_t), ("off_counters", ctypes.c_size_t),
-        ("off_error", ctypes.c_size_t), ("off_kv", ctypes.c_size_t),
+        ("off_error", ctypes.c_size_t), ("off_sync", ctypes.c_size_t), ("off_kv", ctypes.c_size_t),
         ("off_seg_mean", ctypes.c_size_t), ("off_part_sum", ctypes.c_size_t),
         ("off_glob_sum", ctypes.c_size_t), ("off_boundary", ctypes.c_size_t),
         ("kv_rows", ctypes.c_int32), ("elem_bytes", ctypes.c_int32),

@@ -62,7 +62,7 @@ int validate(const ls_config* c) {
   if (c->head_dim % 8 != 0 || c->head_dim > 256 || c->hidden % 8 != 0) return LS_ERR_UNSUPPORTED;
   const int lanes = c->head_dim * elem / 16;
   if (!pow2(lanes) || lanes > 32) return LS_ERR_UNSUPPORTED;
-  if (c->n_kv_heads > 16 || c->block > 32) return LS_ERR_UNSUPPORTED;
+  if (c->n_kv_heads > 8 || c->block > 32) return LS_ERR_UNSUPPORTED;
   if (c->flags & ~(LS_FLAG_FORCE_SIMT | LS_FLAG_OUT_F32)) return LS_ERR_INVALID_ARG;
   return LS_OK;
 }
@@ -100,6 +100,7 @@ int ls_get_layout(const ls_config* cfg, ls_layout* out) {
   out->total_bytes = size_t(y.total);
   out->off_counters = size_t(y.counters);
   out->off_error = size_t(y.error);
+  out->off_sync = size_t(y.sync);
   out->off_kv = size_t(y.kv);
   out->off_seg_mean = size_t(y.seg);
   out->off_part_sum = size_t(y.part);
@@ -141,6 +142,7 @@ int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_st
   for (int k = 0; k < LS_MAX_SCALES; ++k) p.scales[k] = k < cfg->n_scales ? cfg->scales[k] : 1;
   p.counters = reinterpret_cast<int64_t*>(base + y.counters);
   p.err = reinterpret_cast<int32_t*>(base + y.error);
+  p.arrive = reinterpret_cast<int32_t*>(base + y.sync);
   p.kv = base + y.kv;
   p.seg = reinterpret_cast<float*>(base + y.seg);
   p.part = reinterpret_cast<float*>(base + y.part);
@@ -233,6 +235,7 @@ int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count
     return LS_ERR_INVALID_ARG;
   if (boundary_stride < int64_t(c.n_kv_heads) * c.head_dim || boundary_stride % 8 != 0)
     return LS_ERR_SHAPE;
+  if (!(softmax_scale > 0.0f) || softmax_scale == INFINITY) return LS_ERR_INVALID_ARG;
   if (!aligned16(d_q) || !aligned16(d_out) || !aligned16(d_boundary_k) || !aligned16(d_boundary_v))
     return LS_ERR_INVALID_ARG;
   if (st->use_tc)

@@ -5,25 +5,31 @@
 // One tile = (sequence, layer, KV head g): M = (Hq/Hkv) * B = 64 query rows (the GQA
 // group's heads x the block's queries, row m = i * group + j) against the tile's
 // kv_rows <= 768 arena rows (ring window + summary mean rows) plus the boundary row.
-// Because the views are fixed-size, the whole score matrix S = Q K^T of a tile fits in
-// tensor memory at once, so the softmax is exact (global row max first, then one pass of
-// exponentials) and the output accumulator is never rescaled.
+// The arena rows stream through in chunks of 128 rows with an online softmax.
 //
-// Persistent kernel, one CTA per SM, 6 warps:
-//   warp 0    TMA producer: Q of each tile through a 3-D tensor map (two 64-column
-//             swizzled halves), then the tile's K rows and V rows in chunks of 128 rows
-//             through a ring of shared-memory stages (tensor map over the state arena).
-//   warp 1    TMEM allocator and the single MMA-issuing thread: tcgen05.mma kind::f16
-//             (bf16 in, fp32 accumulate), M = 64. S chunk c goes to TMEM columns
-//             128*(c/2) at lane offset 16*(c%2) (the M = 64 accumulator fills lanes 0-15
-//             of each 32-lane subpartition; the odd chunk uses lanes 16-31). O (64 x 128
-//             fp32) sits in columns 384..511.
-//   warps 2-5 softmax and epilogue, one TMEM subpartition each: per row the boundary
-//             logit on CUDA cores, row max over all chunks, exp2, bf16 P written to shared
-//             memory in the MMA's swizzled K-major layout; after P V, the boundary value's
-//             share, 1/rowsum, bf16 output.
-// Every wait is bounded; a wait that runs out sets LS_DEVERR_WAIT_TIMEOUT and the CTA
-// stops, lets its issued copies land, frees its tensor memory and returns.
+// Persistent kernel, one CTA per SM, 8 warps; the roles only meet at mbarriers, so no
+// role's order of work can hold up another's:
+//   warp 0    TMA producer of Q (3-D tensor map, two 64-column swizzled halves) and of
+//             the K rows of every chunk (ring of K stages, tensor map over the arena).
+//   warp 6    TMA producer of the V rows of every chunk (its own ring of V stages).
+//   warp 1    TMEM allocator and the QK-issuing thread (tcgen05.mma kind::f16, bf16 in,
+//             fp32 accumulate, M = 64). The M = 64 accumulator fills lanes 0-15 of each
+//             32-lane TMEM subpartition; a second accumulator at lane offset 16 fills
+//             lanes 16-31. S_c = Q K_c^T is issued as two N = 64 halves (keys 0-63 to
+//             lanes 0-15, keys 64-127 to lanes 16-31 of the same 64 columns), so the two
+//             threads of a row pair each own half of the chunk's keys. Four S buffers.
+//   warp 7    the PV-issuing thread: P_c V_c accumulates into the tile's output O, split
+//             over the output columns the same way; O is double-buffered by tile.
+//             512 TMEM columns in all.
+//   warps 2-5 softmax, one TMEM subpartition each, thread pairs (t, t+16) per query row.
+//             Per chunk: scaled logits, row max, exp2 against the row's reference max,
+//             bf16 P into shared memory in the MMA's swizzled K-major layout. The
+//             reference max only moves when a chunk exceeds it by more than 2^8 (then the
+//             row's O in TMEM and its running sum are rescaled once), so no chunk's P V
+//             has to come back to registers. Epilogue: O from TMEM, the boundary row's
+//             share (its logit is computed on CUDA cores), 1/rowsum.
+// Every wait is bounded and warp-uniform; a wait that runs out sets
+// LS_DEVERR_WAIT_TIMEOUT, all roles stop, the copies in flight land, TMEM is freed.
 #include <cuda.h>
 
 #include "ls_attend_tc.h"
@@ -32,16 +38,21 @@ namespace ls {
 
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kKStages = 3;           // K ring
+constexpr int kVStages = 2;           // V ring
 constexpr int kChunk = 128;            // arena rows per chunk
 constexpr int kMaxChunks = 6;          // kv_rows <= 768
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
 constexpr int kQBytes = 64 * 128 * 2;  // one Q tile (two 8 KB halves)
-constexpr int kPBytes = 64 * 128 * 2;  // one P chunk (two 8 KB halves)
-constexpr int kStageBytes = kChunk * 128 * 2;  // one K or V chunk (two 16 KB halves)
-constexpr int kSmemBytes = 2 * kQBytes + 2 * kPBytes + kStages * kStageBytes + 1024;
+constexpr int kPBytes = 64 * 128 * 2;  // one P chunk (two 8 KB halves: keys 0-63 / 64-127)
+constexpr int kStageBytes = kChunk * 128 * 2;  // one K or V chunk (two 16 KB halves: d 0-63 / 64-127)
+constexpr int kBRowBytes = 2 * 128 * 2;  // the tile's boundary key and value rows (bf16)
+constexpr int kSmemBytes =
+    2 * kQBytes + 2 * kPBytes + (kKStages + kVStages) * kStageBytes + 2 * kBRowBytes + 1024;
+constexpr int kSBufs = 4;              // S buffers: QK may run up to four chunks ahead
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 384;
+constexpr uint32_t kOCol = 256;        // O buffers at columns 256 + 64 * (tile & 1)
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
 
 struct TcArgs {
   int32_t lb, lcount, n_tiles, n_chunks, tail_rows;
@@ -53,13 +64,15 @@ struct TcArgs {
 };
 
 struct Bars {
-  uint64_t full[kStages], empty[kStages];
+  uint64_t kfull[kKStages], kempty[kKStages];
+  uint64_t vfull[kVStages], vempty[kVStages];
   uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[kSBufs], s_free[kSBufs];
   uint64_t p_full[2], p_empty[2];
-  uint64_t s_full, s_free, o_full, o_empty;
+  uint64_t pv_done;
+  uint64_t o_full[2], o_free[2];
   uint32_t tmem_base;
   uint32_t abort;
-  uint32_t vmask[kMaxChunks * kChunk / 32];
 };
 
 // ---- PTX wrappers -------------------------------------------------------------------
@@ -135,14 +148,26 @@ __device__ inline void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ inline void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ inline float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-__device__ inline void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 __device__ inline uint32_t pack_bf16(float a, float b) {
@@ -168,28 +193,61 @@ __device__ inline void tile_coords(int t, const Dev& p, int lcount, int& b, int&
   b = rest / lcount;
 }
 
+// Validity of the 64 arena rows [r0, r0 + 64) of a tile as a bit mask (bit i = row r0+i):
+// the ring slots below min(len, W), per scale the first min(n_seg, slots) segment slots
+// and the partial mean when its segment is non-empty, and the global mean when len > 0.
+__device__ inline uint64_t range_bits(int lo, int hi, int r0) {
+  lo = max(lo, r0);
+  hi = min(hi, r0 + 64);
+  if (hi <= lo) return 0ull;
+  const int n = hi - lo;
+  const uint64_t m = n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+  return m << (lo - r0);
+}
+__device__ inline uint64_t rows_mask64(const Dev& p, int r0, int64_t len, const int64_t* nseg) {
+  uint64_t m = range_bits(0, int(len < p.W ? len : int64_t(p.W)), r0);
+  int base = p.W;
+#pragma unroll
+  for (int k = 0; k < kMaxScales; ++k) {
+    if (k < p.nsc) {
+      m |= range_bits(base, base + int(nseg[k] < p.slots ? nseg[k] : int64_t(p.slots)), r0);
+      if (len - nseg[k] * int64_t(p.scales[k]) > 0) m |= range_bits(base + p.slots, base + p.slots + 1, r0);
+      base += p.slots + 1;
+    }
+  }
+  if (len > 0) m |= range_bits(base, base + 1, r0);  // base == R - 1
+  return m;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMap kv_map,
                  const __grid_constant__ CUtensorMap kv_tail_map, const __grid_constant__ CUtensorMap q_map) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ Bars s;
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_buf = smem;                           // [2][kQBytes]
   unsigned char* p_buf = q_buf + 2 * kQBytes;            // [2][kPBytes]
-  unsigned char* st_buf = p_buf + 2 * kPBytes;           // [kStages][kStageBytes]
+  unsigned char* k_buf = p_buf + 2 * kPBytes;            // [kKStages][kStageBytes]
+  unsigned char* v_buf = k_buf + kKStages * kStageBytes; // [kVStages][kStageBytes]
+  unsigned char* b_buf = v_buf + kVStages * kStageBytes; // [2][boundary k row, v row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nC = a.n_chunks;
+  int my_tiles = 0;
+  for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) ++my_tiles;
+  const int total = my_tiles * nC;  // chunks this CTA processes, in order
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+    for (int i = 0; i < kKStages; ++i) { mbar_init(&s.kfull[i], 1); mbar_init(&s.kempty[i], 1); }
+    for (int i = 0; i < kVStages; ++i) { mbar_init(&s.vfull[i], 1); mbar_init(&s.vempty[i], 1); }
+    for (int i = 0; i < kSBufs; ++i) { mbar_init(&s.s_full[i], 1); mbar_init(&s.s_free[i], 128); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.q_full[i], 1); mbar_init(&s.q_empty[i], 2);
-      mbar_init(&s.p_full[i], 1); mbar_init(&s.p_empty[i], 1);
+      mbar_init(&s.q_full[i], 1); mbar_init(&s.q_empty[i], 1 + 128);
+      mbar_init(&s.p_full[i], 128); mbar_init(&s.p_empty[i], 1);
+      mbar_init(&s.o_full[i], 1); mbar_init(&s.o_free[i], 128);
     }
-    mbar_init(&s.s_full, 1); mbar_init(&s.s_free, 1);
-    mbar_init(&s.o_full, 1); mbar_init(&s.o_empty, 1);
+    mbar_init(&s.pv_done, 1);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -204,282 +262,287 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  int issued = 0;  // producers: loads issued into their ring (for the drain after an abort)
+  auto chunk_rows = [&](int k) { return (k % nC) == nC - 1 ? a.tail_rows : kChunk; };
+  auto chunk_y = [&](int k, int t2) {  // first arena row of chunk k's K (t2 = 0) or V (t2 = 1)
+    const int it = k / nC, c = k - it * nC;
+    int b, lc, g;
+    tile_coords(blockIdx.x + it * gridDim.x, p, a.lcount, b, lc, g);
+    const int64_t tile = (int64_t(b) * p.L + (a.lb + lc)) * p.Hkv + g;
+    return int((tile * 2 + t2) * p.R + int64_t(c) * kChunk);
+  };
 
-  int issued_stages = 0, landed_stages = 0;  // producer bookkeeping for the drain
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 6) {
+    // ------------------------------------------------------------ TMA producers
     if (lane == 0) {
-      prefetch_map(&kv_map); prefetch_map(&kv_tail_map); prefetch_map(&q_map);
-      int st = 0, it = 0;
-      for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
-        int b, lc, g;
-        tile_coords(t, p, a.lcount, b, lc, g);
-        const int qb = it & 1;
-        if (!wait_or_abort(s, &s.q_empty[qb], ((it >> 1) & 1) ^ 1, p.err)) break;
-        mbar_arrive_expect_tx(&s.q_full[qb], kQBytes);
-        const int grp = p.Hq / p.Hkv;
-        const int zrow = (b * a.lcount + lc) * p.B;
-        tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
-        tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
-        const int l = a.lb + lc;
-        const int64_t tile = (int64_t(b) * p.L + l) * p.Hkv + g;
-        bool ok = true;
-        for (int t2 = 0; t2 < 2 && ok; ++t2) {
-          for (int c = 0; c < nC; ++c, ++st) {
-            const int sidx = st % kStages;
-            if (!wait_or_abort(s, &s.empty[sidx], ((st / kStages) & 1) ^ 1, p.err)) { ok = false; break; }
-            const bool tail = c == nC - 1;
-            const int rows = tail ? a.tail_rows : kChunk;
-            mbar_arrive_expect_tx(&s.full[sidx], uint32_t(rows * 256));
-            const int y = int((tile * 2 + t2) * p.R + int64_t(c) * kChunk);
-            unsigned char* dst = st_buf + sidx * kStageBytes;
-            const CUtensorMap* m = tail ? &kv_tail_map : &kv_map;
-            tma_load_2d(dst, m, 0, y, &s.full[sidx]);
-            tma_load_2d(dst + kStageBytes / 2, m, 64, y, &s.full[sidx]);
-            ++issued_stages;
-          }
+      const bool is_k = warp == 0;
+      const int nst = is_k ? kKStages : kVStages;
+      uint64_t* fullb = is_k ? s.kfull : s.vfull;
+      uint64_t* emptyb = is_k ? s.kempty : s.vempty;
+      unsigned char* ring = is_k ? k_buf : v_buf;
+      prefetch_map(&kv_map); prefetch_map(&kv_tail_map);
+      if (is_k) prefetch_map(&q_map);
+      const int grp = p.Hq / p.Hkv;
+      for (int k = 0; k < total; ++k) {
+        const int it = k / nC, c = k - it * nC;
+        if (is_k && c == 0) {  // Q of the tile first
+          const int qb = it & 1;
+          if (!wait_or_abort(s, &s.q_empty[qb], ((it >> 1) & 1) ^ 1, p.err)) break;
+          int b, lc, g;
+          tile_coords(blockIdx.x + it * gridDim.x, p, a.lcount, b, lc, g);
+          mbar_arrive_expect_tx(&s.q_full[qb], kQBytes + kBRowBytes);
+          const int zrow = (b * a.lcount + lc) * p.B;
+          tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
+          tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
+          // the tile's boundary key and value rows travel with Q
+          const int64_t boff = (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + int64_t(g) * 128;
+          bulk_g2s(b_buf + qb * kBRowBytes, a.bk + boff, 256, &s.q_full[qb]);
+          bulk_g2s(b_buf + qb * kBRowBytes + 256, a.bv + boff, 256, &s.q_full[qb]);
         }
-        if (!ok) break;
+        const int st = k % nst;
+        if (!wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err)) break;
+        const int rows = chunk_rows(k);
+        const CUtensorMap* m = c == nC - 1 ? &kv_tail_map : &kv_map;
+        const int y = chunk_y(k, is_k ? 0 : 1);
+        mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
+        unsigned char* dst = ring + st * kStageBytes;
+        tma_load_2d(dst, m, 0, y, &fullb[st]);
+        tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
+        ++issued;
       }
-      landed_stages = st;
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ QK issuer
     if (lane == 0) {
-      int st = 0, it = 0, pu[2] = {0, 0};
-      const uint32_t q_base = smem_u32(q_buf), p_base = smem_u32(p_buf), s_base = smem_u32(st_buf);
-      const uint32_t id_qk_full = idesc_bf16(kChunk, false);
-      const uint32_t id_qk_tail = idesc_bf16(a.tail_rows, false);
-      const uint32_t id_pv = idesc_bf16(128, true);
-      bool ok = true;
-      for (int t = blockIdx.x; t < a.n_tiles && ok; t += gridDim.x, ++it) {
-        const int qb = it & 1;
-        if (!wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err)) break;
-        if (!wait_or_abort(s, &s.s_free, (it & 1) ^ 1, p.err)) break;
+      const uint32_t q_base = smem_u32(q_buf), k_base = smem_u32(k_buf);
+      for (int k = 0; k < total; ++k) {
+        const int it = k / nC, c = k - it * nC, qb = it & 1, sb = k % kSBufs, st = k % kKStages;
+        if (c == 0 && !wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err)) break;
+        if (!wait_or_abort(s, &s.kfull[st], (k / kKStages) & 1, p.err)) break;
+        if (!wait_or_abort(s, &s.s_free[sb], ((k / kSBufs) & 1) ^ 1, p.err)) break;
         tc_fence_after();
-        // S = Q K^T, chunk by chunk
-        for (int c = 0; c < nC; ++c, ++st) {
-          const int sidx = st % kStages;
-          if (!wait_or_abort(s, &s.full[sidx], (st / kStages) & 1, p.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + (uint32_t(16 * (c & 1)) << 16) + uint32_t(128 * (c >> 1));
-          const uint32_t idesc = c == nC - 1 ? id_qk_tail : id_qk_full;
-          const uint32_t kb = s_base + sidx * kStageBytes;
+        const int rows = chunk_rows(k);
+        const int n0 = rows < 64 ? rows : 64, n1 = rows - n0;
+        const uint32_t id0 = idesc_bf16(n0, false), id1 = idesc_bf16(n1 > 0 ? n1 : 8, false);
+        const uint32_t kb = k_base + st * kStageBytes;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t off = (k >> 2) * (kQBytes / 2) + (k & 3) * 32;
-            const uint32_t koff = (k >> 2) * (kStageBytes / 2) + (k & 3) * 32;
-            mma_bf16(d, sdesc(q_base + qb * kQBytes + off, 16, 1024), sdesc(kb + koff, 16, 1024), idesc,
-                     k > 0);
-          }
-          mma_commit(&s.empty[sidx]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t qa = sdesc(q_base + qb * kQBytes + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
+          const uint32_t koff = (kk >> 2) * (kStageBytes / 2) + (kk & 3) * 32;
+          mma_bf16(tmem + 64 * sb, qa, sdesc(kb + koff, 16, 1024), id0, kk > 0);
+          if (n1 > 0) mma_bf16(tmem + (16u << 16) + 64 * sb, qa, sdesc(kb + koff + 64 * 128, 16, 1024), id1, kk > 0);
         }
-        if (!ok) break;
-        mma_commit(&s.q_empty[qb]);
-        mma_commit(&s.s_full);
-        // O = P V, chunk by chunk, once the softmax has written P_c
-        if (!wait_or_abort(s, &s.o_empty, (it & 1) ^ 1, p.err)) break;
-        for (int c = 0; c < nC; ++c, ++st) {
-          const int sidx = st % kStages;
-          const int pb = c & 1;
-          if (!wait_or_abort(s, &s.full[sidx], (st / kStages) & 1, p.err)) { ok = false; break; }
-          if (!wait_or_abort(s, &s.p_full[pb], pu[pb] & 1, p.err)) { ok = false; break; }
-          ++pu[pb];
-          tc_fence_after();
-          const int rows = c == nC - 1 ? a.tail_rows : kChunk;
-          const uint32_t vb = s_base + sidx * kStageBytes;
-          for (int k = 0; k < rows / 16; ++k) {
-            const uint32_t poff = (k >> 2) * (kPBytes / 2) + (k & 3) * 32;
-            // V chunk: rows = keys (K dim), 128-byte rows per 64-column half: MN-major B,
-            // LBO = distance to the second half, SBO = 8 rows.
-            mma_bf16(tmem + kOCol, sdesc(p_base + pb * kPBytes + poff, 16, 1024),
-                     sdesc(vb + k * 2048, kStageBytes / 2, 1024), id_pv, (c > 0 || k > 0));
-          }
-          mma_commit(&s.empty[sidx]);
-          mma_commit(&s.p_empty[pb]);
+        mma_commit(&s.kempty[st]);
+        mma_commit(&s.s_full[sb]);
+        if (c == nC - 1) mma_commit(&s.q_empty[qb]);
+      }
+    }
+  } else if (warp == 7) {
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      const uint32_t p_base = smem_u32(p_buf), v_base = smem_u32(v_buf);
+      const uint32_t id_pv = idesc_bf16(64, true);
+      for (int k = 0; k < total; ++k) {
+        const int it = k / nC, c = k - it * nC, ob = it & 1, pb = k & 1, st = k % kVStages;
+        if (c == 0 && !wait_or_abort(s, &s.o_free[ob], ((it >> 1) & 1) ^ 1, p.err)) break;
+        if (!wait_or_abort(s, &s.vfull[st], (k / kVStages) & 1, p.err)) break;
+        if (!wait_or_abort(s, &s.p_full[pb], (k >> 1) & 1, p.err)) break;
+        tc_fence_after();
+        const uint32_t vb = v_base + st * kStageBytes;
+        const int rows = chunk_rows(k);
+        for (int kk = 0; kk < rows / 16; ++kk) {
+          const uint64_t pa = sdesc(p_base + pb * kPBytes + (kk >> 2) * (kPBytes / 2) + (kk & 3) * 32, 16, 1024);
+          const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+          // V: rows = keys (K dim), 128-byte rows per 64-column half: MN-major B, SBO = 8 rows
+          mma_bf16(tmem + kOCol + 64 * ob, pa, sdesc(vb + kk * 2048, kStageBytes / 2, 1024), id_pv, acc);
+          mma_bf16(tmem + (16u << 16) + kOCol + 64 * ob, pa,
+                   sdesc(vb + kStageBytes / 2 + kk * 2048, kStageBytes / 2, 1024), id_pv, acc);
         }
-        if (!ok) break;
-        mma_commit(&s.o_full);
+        mma_commit(&s.vempty[st]);
+        mma_commit(&s.p_empty[pb]);
+        mma_commit(&s.pv_done);
+        if (c == nC - 1) mma_commit(&s.o_full[ob]);
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue
-    // The four warps leave the tile loop only together, right after a named barrier,
-    // when the shared abort flag is set (a wait that ran out sets it before the barrier).
-    const int sw = warp - 2;            // 0..3
+    // ------------------------------------------------------------ softmax
     const int sub = warp & 3;           // TMEM subpartition this warp may access
-    const int half = lane >> 4;         // 0: even chunks, 1: odd chunks
+    const int half = lane >> 4;         // 0: keys / output columns 0-63, 1: 64-127
     const int row = 16 * sub + (lane & 15);
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
     const int grp = p.Hq / p.Hkv;
-    const int tid = sw * 32 + lane;     // 0..127
-    const int ncb = (nC + 1) >> 1;
-    volatile uint32_t* abort_flag = &s.abort;
-    auto group_sync_ok = [&]() {
-      named_sync(1, 128);
-      return *abort_flag == 0;
+    const float sl2 = a.scale_log2;     // > 0 (checked by the caller)
+    int it = 0, k = 0;
+    // counters of the tile after this one are read one tile ahead (their load latency
+    // then never sits between two tiles)
+    auto load_counters = [&](int t, int64_t* dst) {
+      if (t >= a.n_tiles) return;
+      int b, lc, g;
+      tile_coords(t, p, a.lcount, b, lc, g);
+      const int64_t* ctr = p.counters + (int64_t(b) * p.L + a.lb + lc) * (1 + p.nsc);
+#pragma unroll
+      for (int kk = 0; kk <= kMaxScales; ++kk) dst[kk] = kk <= p.nsc ? ctr[kk] : 0;
     };
-    int it = 0, pu[2] = {0, 0};
+    int64_t cnt_next[kMaxScales + 1];
+    load_counters(blockIdx.x, cnt_next);
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
       int b, lc, g;
       tile_coords(t, p, a.lcount, b, lc, g);
-      const int l = a.lb + lc;
-      const int qb = it & 1;
-      // validity of the tile's arena rows as a bit mask
-      {
-        const int64_t* ctr = p.counters + (int64_t(b) * p.L + l) * (1 + p.nsc);
-        const int64_t len = ctr[0];
-        int64_t nseg[kMaxScales];
+      const int qb = it & 1, ob = it & 1;
+      const int64_t len = cnt_next[0];
+      int64_t nseg[kMaxScales];
 #pragma unroll
-        for (int k = 0; k < kMaxScales; ++k) nseg[k] = k < p.nsc ? ctr[1 + k] : 0;
-        for (int base = 0; base < nC * kChunk; base += 128) {
-          const int r = base + tid;
-          const bool v = r < p.R && arena_row_valid(p, r, len, nseg);
-          const unsigned bal = __ballot_sync(0xffffffffu, v);
-          if (lane == 0) s.vmask[(base >> 5) + sw] = bal;
-        }
-      }
-      // boundary logit on CUDA cores: q_row . boundary_k (each half of the pair does 64 d)
-      const bool q_ok = wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err);
-      float blog = 0.f;
-      const int64_t boff = (int64_t(b) * p.L + l) * a.bstride + int64_t(g) * 128;
-      if (q_ok) {
+      for (int kk = 0; kk < kMaxScales; ++kk) nseg[kk] = cnt_next[1 + kk];
+      load_counters(t + gridDim.x, cnt_next);
+
+      // boundary logit on CUDA cores (each thread of the pair does 64 of the 128 d)
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err))) break;
+      float bpart[4] = {0.f, 0.f, 0.f, 0.f};
+      {
         const unsigned char* qrow = q_buf + qb * kQBytes + half * (kQBytes / 2) + row * 128;
+        const uint4* bkrow = reinterpret_cast<const uint4*>(b_buf + qb * kBRowBytes + half * 128);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const uint4 qv = *reinterpret_cast<const uint4*>(qrow + ((ch ^ (row & 7)) << 4));
-          const uint4 kv4 = ld_nc_v4(a.bk + boff + half * 64 + ch * 8);
           float qf[8], kf[8];
           Elem<__nv_bfloat16>::to_f32(qv, qf);
-          Elem<__nv_bfloat16>::to_f32(kv4, kf);
+          Elem<__nv_bfloat16>::to_f32(bkrow[ch], kf);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) blog = fmaf(qf[e], kf[e], blog);
+          for (int e = 0; e < 8; ++e) bpart[e & 3] = fmaf(qf[e], kf[e], bpart[e & 3]);
         }
       }
+      uint4 bvv[8];  // boundary value row (this thread's 64 columns), kept for the epilogue
+      {
+        const uint4* bvrow = reinterpret_cast<const uint4*>(b_buf + qb * kBRowBytes + 256 + half * 128);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) bvv[ch] = bvrow[ch];
+      }
+      mbar_arrive(&s.q_empty[qb]);
+      float blog = (bpart[0] + bpart[1]) + (bpart[2] + bpart[3]);
       blog += __shfl_xor_sync(0xffffffffu, blog, 16);
-      if (!group_sync_ok()) break;
-      if (tid == 0) mbar_arrive(&s.q_empty[qb]);
+      const float blog_s = blog * sl2;
+      float mref = blog_s;  // reference max (log2 units) the P values are taken against
+      float lsum = 0.f;     // sum of the arena rows' weights against mref
 
-      // all S chunks of this tile are in TMEM: row max over every valid slot
-      const bool s_ok = wait_or_abort(s, &s.s_full, it & 1, p.err);
-      tc_fence_after();
-      float mx = -INFINITY;
-      if (__all_sync(0xffffffffu, s_ok)) {
-        for (int cb = 0; cb < ncb; ++cb) {
-          const int c = 2 * cb + half;
-#pragma unroll 1
-          for (int q4 = 0; q4 < 4; ++q4) {
-            float v[32];
-            tmem_ld32(trow + uint32_t(cb * 128 + q4 * 32), v);
-            const uint32_t m = c < nC ? s.vmask[(c * kChunk + q4 * 32) >> 5] : 0u;
+      bool ok = true;
+      for (int c = 0; c < nC; ++c, ++k) {
+        const int sb = k % kSBufs, pb = k & 1;
+        const uint64_t vm = rows_mask64(p, c * kChunk + 64 * half, len, nseg);
+        const bool all_valid = __all_sync(0xffffffffu, vm == ~0ull);
+        if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.s_full[sb], (k / kSBufs) & 1, p.err))) { ok = false; break; }
+        tc_fence_after();
+        float sv[64];
+        tmem_ld32(trow + 64 * sb, sv);
+        tmem_ld32(trow + 64 * sb + 32, sv + 32);
+        tc_fence_before();
+        mbar_arrive(&s.s_free[sb]);
+        // row max over the valid raw logits (scale > 0 keeps the order), 8-way tree
+        float mx8[8];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if ((m >> j) & 1u) mx = fmaxf(mx, v[j]);
+        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+        if (all_valid) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            if (!((vm >> i) & 1ull)) sv[i] = -INFINITY;
+            mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
           }
         }
-      }
-      if (!group_sync_ok()) break;
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      mx = fmaxf(mx, blog);
-      const float mscaled = mx * a.scale_log2;
-      // exponentials, row sums, bf16 P into the swizzled K-major tile of its chunk
-      float sum = 0.f;
-      bool aborted = false;
-      for (int cb = 0; cb < ncb; ++cb) {
-        const int c = 2 * cb + half;
-        const bool mine = c < nC;
-        const bool pe_ok = !mine || wait_or_abort(s, &s.p_empty[half], (pu[half] & 1) ^ 1, p.err);
-        const bool go = __all_sync(0xffffffffu, pe_ok);
-        unsigned char* prow = p_buf + half * kPBytes + row * 128;
+        float cmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 16)) * sl2;
+        // P buffer pb free again means P_{k-2} V_{k-2} has landed; only after that does the
+        // parity wait on pv_done below identify P_{k-1} V_{k-1} unambiguously
+        if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.p_empty[pb], ((k >> 1) & 1) ^ 1, p.err))) { ok = false; break; }
+        if (c == 0) {
+          mref = fmaxf(mref, cmax);  // O is still empty: the reference moves for free
+        } else if (__any_sync(0xffffffffu, cmax > mref + kRescaleThreshold)) {
+          // rows whose max grew by more than 2^8: rescale their O (after the P V MMAs
+          // issued so far have landed) and their running sum to the new reference
+          const float mnew = cmax > mref + kRescaleThreshold ? cmax : mref;
+          const float alpha = ex2(mref - mnew);
+          if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.pv_done, (k - 1) & 1, p.err))) { ok = false; break; }
+          tc_fence_after();
+          float ov[32];
 #pragma unroll 1
-        for (int q4 = 0; q4 < 4 && go; ++q4) {
-          float v[32];
-          tmem_ld32(trow + uint32_t(cb * 128 + q4 * 32), v);
-          if (!mine) continue;
-          const uint32_t m = s.vmask[(c * kChunk + q4 * 32) >> 5];
-          uint32_t pk[16];
+          for (int h2 = 0; h2 < 2; ++h2) {
+            tmem_ld32(trow + kOCol + 64 * ob + 32 * h2, ov);
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float p0 = ((m >> j) & 1u) ? ex2(fmaf(v[j], a.scale_log2, -mscaled)) : 0.f;
-            const float p1 = ((m >> (j + 1)) & 1u) ? ex2(fmaf(v[j + 1], a.scale_log2, -mscaled)) : 0.f;
-            sum += p0 + p1;
-            pk[j >> 1] = pack_bf16(p0, p1);
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            tmem_st32(trow + kOCol + 64 * ob + 32 * h2, ov);
           }
-          // keys q4*32 .. q4*32+31 of this chunk: half (q4 >> 1) of the P tile, 16-byte
-          // pieces (q4 & 1)*4 .. +3 of the row, swizzled by the row's position in its atom
-          unsigned char* dst = prow + (q4 >> 1) * (kPBytes / 2);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int piece = (q4 & 1) * 4 + u;
-            *reinterpret_cast<uint4*>(dst + ((piece ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          }
+          tc_fence_before();
+          lsum *= alpha;
+          mref = mnew;
         }
+        // weights 2^(s * scale - mref) (masked slots hold -inf: weight 0), bf16 P, 8-way sums
+        float ps8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ps8[u] = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          const float p0 = ex2(fmaf(sv[i], sl2, -mref));
+          const float p1 = ex2(fmaf(sv[i + 1], sl2, -mref));
+          ps8[(i >> 1) & 7] += p0 + p1;
+          pk[i >> 1] = pack_bf16(p0, p1);
+        }
+        const float psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+        lsum += psum + __shfl_xor_sync(0xffffffffu, psum, 16);
+        // this thread's 64 keys: half `half` of the P tile, 8 swizzled 16-byte pieces
+        unsigned char* prow = p_buf + pb * kPBytes + half * (kPBytes / 2) + row * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) << 4)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         fence_proxy_async_smem();
-        if (!group_sync_ok()) { aborted = true; break; }
-        if (tid == 0) {
-          mbar_arrive(&s.p_full[0]);
-          if (2 * cb + 1 < nC) mbar_arrive(&s.p_full[1]);
-        }
-        if (2 * cb < nC) ++pu[0];
-        if (2 * cb + 1 < nC) ++pu[1];
+        mbar_arrive(&s.p_full[pb]);
       }
-      if (aborted) break;
-      tc_fence_before();
-      if (!group_sync_ok()) break;
-      if (tid == 0) mbar_arrive(&s.s_free);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-      const float pbd = ex2(fmaf(blog, a.scale_log2, -mscaled));
-      sum += pbd;
-      const float inv = 1.0f / sum;
-
-      // epilogue: O row (lanes 0-15 of each subpartition) + boundary share, normalised
-      const bool o_ok = wait_or_abort(s, &s.o_full, it & 1, p.err);
+      if (!ok) break;
+      // epilogue: O from TMEM plus the boundary row's share, normalised
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.o_full[ob], (it >> 1) & 1, p.err))) break;
       tc_fence_after();
-      const int i = row / grp, j = row - (row / grp) * grp;
-      const int64_t orow = (((int64_t(b) * a.lcount + lc) * p.B + i) * p.Hq + g * grp + j) * 128;
-      const bool o_go = __all_sync(0xffffffffu, o_ok);
-#pragma unroll 1
-      for (int q4 = 0; q4 < 4 && o_go; ++q4) {
-        float v[32];
-        tmem_ld32(trow + kOCol + uint32_t(q4 * 32), v);
-        if (half == 0) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 bv4 = ld_nc_v4(a.bv + boff + q4 * 32 + u * 8);
-            float bf[8];
-            Elem<__nv_bfloat16>::to_f32(bv4, bf);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[u * 8 + e] = fmaf(pbd, bf[e], v[u * 8 + e]) * inv;
-          }
-          if (p.out_f32) {
-            float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow + q4 * 32);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) o4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-          } else {
-            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow + q4 * 32);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              o4[u] = make_uint4(pack_bf16(v[8 * u], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
-                                 pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
-          }
-        }
-      }
+      float o[64];
+      tmem_ld32(trow + kOCol + 64 * ob, o);
+      tmem_ld32(trow + kOCol + 64 * ob + 32, o + 32);
       tc_fence_before();
-      if (!group_sync_ok()) break;
-      if (tid == 0) mbar_arrive(&s.o_empty);
+      mbar_arrive(&s.o_free[ob]);
+      const float pbd = ex2(blog_s - mref);
+      const float inv = 1.0f / (lsum + pbd);
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        float bf[8];
+        Elem<__nv_bfloat16>::to_f32(bvv[ch], bf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[8 * ch + e] = fmaf(pbd, bf[e], o[8 * ch + e]) * inv;
+      }
+      const int i = row / grp, jj = row - (row / grp) * grp;
+      const int64_t orow = (((int64_t(b) * a.lcount + lc) * p.B + i) * p.Hq + g * grp + jj) * 128 + 64 * half;
+      if (p.out_f32) {
+        float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) o4[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+      } else {
+        uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          o4[u] = make_uint4(pack_bf16(o[8 * u], o[8 * u + 1]), pack_bf16(o[8 * u + 2], o[8 * u + 3]),
+                             pack_bf16(o[8 * u + 4], o[8 * u + 5]), pack_bf16(o[8 * u + 6], o[8 * u + 7]));
+      }
     }
   }
 
   __syncthreads();
-  if (warp == 0 && lane == 0 && s.abort) {
-    // let the copies still in flight (at most the last kStages issued) land before the
-    // CTA's shared memory is released
-    for (int st = landed_stages > kStages ? landed_stages - kStages : 0; st < landed_stages; ++st)
-      mbar_wait_bounded(&s.full[st % kStages], (st / kStages) & 1, kWaitLimit);
+  if ((warp == 0 || warp == 6) && lane == 0 && s.abort) {
+    // let the copies still in flight (at most the last ring's worth issued) land before
+    // the CTA's shared memory is released
+    const int nst = warp == 0 ? kKStages : kVStages;
+    uint64_t* fullb = warp == 0 ? s.kfull : s.vfull;
+    for (int n = issued > nst ? issued - nst : 0; n < issued; ++n)
+      mbar_wait_bounded(&fullb[n % nst], (n / nst) & 1, kWaitLimit);
   }
-  (void)issued_stages;
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -20,6 +20,7 @@ struct Dev {
   int32_t scales[kMaxScales];
   int64_t* counters;  // [b][L][1+nsc]
   int32_t* err;       // device error word
+  int32_t* arrive;    // [b][L] arrivals of the (sequence, layer)'s KV-head CTAs in a commit
   char* kv;           // [b][L][Hkv][2][R][D] elements
   float* seg;         // [b][L][Hkv][nsc][slots][2][D]
   float* part;        // [b][L][Hkv][nsc][2][D]
@@ -31,7 +32,7 @@ __host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int
 
 // Arena layout for a validated config (host and device agree by construction).
 struct Layout {
-  int64_t counters, error, kv, seg, part, glob, boundary, total;
+  int64_t counters, error, sync, kv, seg, part, glob, boundary, total;
   int32_t R, elem;
 };
 
@@ -43,6 +44,7 @@ __host__ inline Layout make_layout(const ls_config& c) {
   int64_t off = 0;
   y.counters = off; off = align256(off + int64_t(c.batch) * c.n_layers * (1 + c.n_scales) * 8);
   y.error = off;    off = align256(off + 16);
+  y.sync = off;     off = align256(off + int64_t(c.batch) * c.n_layers * 4);
   y.kv = off;       off = align256(off + tiles * 2 * y.R * c.head_dim * y.elem);
   y.seg = off;      off = align256(off + tiles * c.n_scales * c.slots_per_scale * 2 * c.head_dim * 4);
   y.part = off;     off = align256(off + tiles * c.n_scales * 2 * c.head_dim * 4);

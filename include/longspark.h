@@ -84,7 +84,7 @@ extern "C" {
 #define LS_MAX_SCALES 4
 
 /* Shapes of one drafting state (one batch of sequences).
- *   batch b, n_layers L (tapped layers), n_kv_heads Hkv, n_q_heads Hq (multiple of Hkv),
+ *   batch b, n_layers L (tapped layers), n_kv_heads Hkv (<= 8), n_q_heads Hq (multiple of Hkv),
  *   head_dim D (multiple of 8, <= 256), hidden (multiple of 8), block B (1..32),
  *   window W (>= B+1), n_scales (1..4), scales ascending, each >= B+1,
  *   each dividing the next (so no segment of any scale straddles a larger one),
@@ -105,6 +105,7 @@ typedef struct {
  *   counters  int64 [b][L][1 + n_scales]: retained length len, then for each scale the
  *             number of segments finalised so far (floor(len / s_k)).
  *   error     int32 [4]: word 0 is the device error word.
+ *   sync      int32 [b][L]: zero between calls (arrival counts inside a commit).
  *   kv        e     [b][L][Hkv][2][kv_rows][D]: for K (index 0) and V (index 1) of each
  *             (sequence, layer, KV head) tile, rows 0..W-1 are the ring window, then for
  *             each scale k rows W + k*(slots+1) + i hold the mean of the segment in slot i
@@ -117,7 +118,7 @@ typedef struct {
  *   boundary  e     [b][L][hidden]: hidden vectors at the last retained position.     */
 typedef struct {
   size_t total_bytes;
-  size_t off_counters, off_error, off_kv, off_seg_mean, off_part_sum, off_glob_sum,
+  size_t off_counters, off_error, off_sync, off_kv, off_seg_mean, off_part_sum, off_glob_sum,
          off_boundary;
   int32_t kv_rows;
   int32_t elem_bytes;
@@ -202,7 +203,7 @@ LS_API int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32
  *   d_out          same shape; fp32 with LS_FLAG_OUT_F32, else `dtype`
  *   d_boundary_k/v `dtype`, element (b, l, g, d) at [(b*L + l)*boundary_stride + g*D + d]
  *                  with l the absolute layer; boundary_stride >= Hkv*D, multiple of 8.
- *   softmax_scale  logit multiplier (1/sqrt(D) for the usual attention).
+ *   softmax_scale  logit multiplier, finite and > 0 (1/sqrt(D) for the usual attention).
  * Uses the tcgen05 tensor-core kernel when dtype is bf16, (Hq/Hkv)*B == 64, D == 128 and
  * kv_rows <= 768 (unless LS_FLAG_FORCE_SIMT), otherwise a CUDA-core kernel.          */
 LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count,

@@ -44,7 +44,7 @@ def test_layout_sizes():
     assert y.off_glob_sum - y.off_part_sum >= b * L * H * nsc * 2 * D * 4
     assert y.off_boundary - y.off_glob_sum >= b * L * H * 2 * D * 4
     assert y.total_bytes - y.off_boundary >= b * L * 4096 * 2
-    for off in (y.off_counters, y.off_error, y.off_kv, y.off_seg_mean, y.off_part_sum, y.off_glob_sum,
+    for off in (y.off_counters, y.off_error, y.off_sync, y.off_kv, y.off_seg_mean, y.off_part_sum, y.off_glob_sum,
                 y.off_boundary, y.total_bytes):
         assert off % 256 == 0
     assert F.ls_state_bytes(c) == y.total_bytes
@@ -61,7 +61,7 @@ def test_layout_sizes():
     (dict(scales=[64, 500, 4096]), F.LS_ERR_UNSUPPORTED),  # does not divide the next
     (dict(head_dim=96), F.LS_ERR_UNSUPPORTED),
     (dict(dtype=7), F.LS_ERR_INVALID_ARG),
-    (dict(n_kv_heads=32, n_q_heads=64), F.LS_ERR_UNSUPPORTED),
+    (dict(n_kv_heads=16, n_q_heads=64), F.LS_ERR_UNSUPPORTED),
 ])
 def test_config_validation(kw, status):
     c = _cfg(**kw)

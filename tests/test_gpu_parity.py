@@ -197,3 +197,45 @@ def test_edge_cases(prefix, accepts):
             torch.cuda.synchronize()
             _check_run_against_oracle(run, wl, r + 1, out, r)
     assert run.error() == (F.LS_OK, 0)
+
+
+def test_large_logit_spread_takes_rescale_path():
+    """Queries x16: later chunks raise rows' max by more than 2^8, so the tensor-core
+    kernel must rescale its running output and sum; the result still matches the oracle."""
+    wl = WL.Workload("spread", 7, 2, 1, 2, 8, 128, 512, 16, 512, (64, 512, 4096), 32, "bf16", (5000, 9000), 3,
+                     None, 1000, head_scale=True, flags=F.LS_FLAG_OUT_F32)
+    run = WL.DeviceRun(wl)
+    assert F.ls_attend_uses_tensor_cores(run.state)
+    run.prefill()
+    inp = run.make_round_inputs()
+    inp["q"].mul_(16.0)  # exact in bf16 (power of two)
+    out = run.new_out()
+    for r in range(wl.rounds):
+        run.commit(inp, r)
+    run.attend(inp, wl.rounds - 1, out)
+    torch.cuda.synchronize()
+    st = run.read_state()
+    draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
+    acc = OS.accepts_from_ids(draft, target)
+    jumped = 0
+    for b in range(wl.batch):
+        for h in range(wl.n_kv_heads):
+            sh, views = OS.tile_views(wl, b, 0, h, int(run.prefix_len[b]), acc[:, b], run.scale_host)
+            OS.check_tile_state(wl, st, b, 0, h, views)
+            hid = OS.boundary_hidden(wl, b, 0, wl.rounds - 1, int(acc[-1, b]))
+            hv = O.to_f64(hid, wl.dtype)
+            bk = hv[h * 128:(h + 1) * 128].reshape(1, 1, 128)
+            bv = hv[wl.n_kv_heads * 128 + h * 128:wl.n_kv_heads * 128 + (h + 1) * 128].reshape(1, 1, 128)
+            q = OS.queries(wl, wl.rounds - 1, b, 0, h) * 16.0
+            ref = O.draft_attend(sh, views, q, bk, bv, 1.0 / np.sqrt(128))[0]
+            got = _out_tile(out, wl, b, 0, h)
+            assert OS.attend_error_excess(got, ref, True) <= 0, float(np.abs(got - ref).max())
+            # the kernel's chunks are the tile's arena rows in blocks of 128: boundary and
+            # chunk 0 set the first reference, later chunks exceed it by > 8 log2 units?
+            K, _, ok = O.attention_slots(sh, views, 0, 0, bk, bv)
+            lg = (q[0].reshape(-1, 128) @ K.T) / np.sqrt(128) / np.log(2.0)
+            lg[:, ~ok] = -np.inf
+            first = np.maximum(lg[:, 0], lg[:, 1:129].max(axis=1))
+            later = lg[:, 129:].max(axis=1)
+            jumped += int(np.sum(later > first + 8.0))
+    assert jumped > 0, "inputs never exercise the rescale path"

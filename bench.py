@@ -1,8 +1,12 @@
 """Benchmark of the LongSpark drafting round on B200.
 
 One step = one decoding round of the hot path over a batch of 16 sequences at Qwen3-8B
-shapes with a 64K-token prefix: ``ls_commit_round`` (accept scan, ring-window commit,
-summary update, boundary gather) followed by ``ls_draft_attend`` over all 4 tapped layers.
+shapes with a 64K-token prefix: ``ls_round``, i.e. the commit (accept scan, ring-window
+commit, summary update, boundary gather) and the drafter's block attention over all 4
+tapped layers, the attention kernel launched as a programmatic dependent of the commit
+kernel. The same round as two plain calls (``ls_commit_round`` then ``ls_draft_attend``,
+CUDA events around each) gives the per-kernel times; ``roofline`` is the attention kernel's
+(the dominant one) and ``round_roofline`` the whole round's.
 The prefill summary over the prefix runs once per request before the rounds; it is timed
 separately in the same run and reported under ``prefill``.
 
@@ -336,12 +340,12 @@ def run_gpu(args):
     clock_path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "_build",
                               f"clocks_rank{rank}.csv")
     os.makedirs(os.path.dirname(clock_path), exist_ok=True)
+    overlapped = F.ls_round_overlaps(run.state)
     # the sampler starts with the warm-up rounds so that its samples cover a loaded GPU
     with ClockSampler(local, clock_path) as clk:
         for r in range(W):
             flush.zero_()
-            run.commit(inp, r % n_rounds)
-            run.attend(inp, r % n_rounds, out)
+            run.round(inp, r % n_rounds, out)
         torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
@@ -349,17 +353,26 @@ def run_gpu(args):
             r = (W + i) % n_rounds
             flush.zero_()
             evs[i][0].record(stream)
-            run.commit(inp, r)
+            run.round(inp, r, out)
             evs[i][1].record(stream)
-            run.attend(inp, r, out)
-            evs[i][2].record(stream)
         torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    commit_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    attend_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    round_ms = [a + c for a, c in zip(attend_ms, commit_ms)]
+    round_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_s = sum(round_ms) / 1e3
+    # the same round as two calls, for the per-kernel split
+    KS = min(K, 500)
+    for i in range(KS):
+        r = (W + K + i) % n_rounds
+        flush.zero_()
+        evs[i][0].record(stream)
+        run.commit(inp, r)
+        evs[i][1].record(stream)
+        run.attend(inp, r, out)
+        evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    commit_ms = [e[0].elapsed_time(e[1]) for e in evs[:KS]]
+    attend_ms = [e[1].elapsed_time(e[2]) for e in evs[:KS]]
     total_max = max_over_ranks(total_s, world, dev)
     status, word = run.error()
     if status != F.LS_OK:
@@ -375,8 +388,7 @@ def run_gpu(args):
             run.stream = gs
             with torch.cuda.graph(g, stream=gs):
                 for j in range(8):
-                    run.commit(inp, j % n_rounds)
-                    run.attend(inp, j % n_rounds, out)
+                    run.round(inp, j % n_rounds, out)
         run.stream = stream
         torch.cuda.current_stream(dev).wait_stream(gs)
         g.replay()
@@ -405,9 +417,10 @@ def run_gpu(args):
     c_bytes = commit_bytes(wl, float(deltas.mean()))
     att_s = float(np.mean(attend_ms)) / 1e3
     rnd_s = float(np.mean(round_ms)) / 1e3
+    r_bytes = a_bytes + c_bytes
     achieved = a_bytes / att_s / 1e9
-    traffic = recorded_traffic("ls_attend_tc.cu" if F.ls_attend_uses_tensor_cores(run.state)
-                               else "ls_attend_simt.cu", f"attend_{wl.name}")
+    tc = F.ls_attend_uses_tensor_cores(run.state)
+    traffic = recorded_traffic("ls_attend_tc.cu" if tc else "ls_attend_simt.cu", f"attend_{wl.name}")
 
     if rank == 0:
         line = {
@@ -415,16 +428,20 @@ def run_gpu(args):
             "steps": K, "warmup": W, "ms_per_step": total_max * 1e3 / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(wl),
-            "roofline": {"bound": "hbm", "kernel": "ls_draft_attend ("
-                         + ("tcgen05" if F.ls_attend_uses_tensor_cores(run.state) else "CUDA cores") + ")",
+            "roofline": {"bound": "hbm",
+                         "kernel": "ls_draft_attend (" + ("tcgen05" if tc else "CUDA cores") + ")",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": a_bytes},
-            "round_roofline": {"bytes": a_bytes + c_bytes, "achieved": (a_bytes + c_bytes) / rnd_s / 1e9,
-                               "frac": (a_bytes + c_bytes) / rnd_s / 1e9 / peak, "unit": "GB/s"},
-            "us_per_round": {"median": float(np.median(round_ms)) * 1e3, "p90": float(np.percentile(round_ms, 90)) * 1e3,
-                             "commit_mean": float(np.mean(commit_ms)) * 1e3,
-                             "attend_mean": float(np.mean(attend_ms)) * 1e3},
-            "commit": {"bytes": c_bytes, "achieved_GBps": c_bytes / (np.mean(commit_ms) / 1e3) / 1e9},
+                         "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": a_bytes,
+                         "us": att_s * 1e6, "timed_launches": KS},
+            "round_roofline": {"kernels": "ls_round: commit + attention" + (
+                                   " (programmatic dependent launch)" if overlapped else " (two launches)"),
+                               "bytes": r_bytes, "achieved": r_bytes / rnd_s / 1e9,
+                               "frac": r_bytes / rnd_s / 1e9 / peak, "unit": "GB/s"},
+            "us_per_round": {"median": float(np.median(round_ms)) * 1e3, "mean": rnd_s * 1e6,
+                             "p90": float(np.percentile(round_ms, 90)) * 1e3},
+            "split": {"steps": KS, "commit_us": float(np.mean(commit_ms)) * 1e3,
+                      "attend_us": att_s * 1e6, "commit_bytes": c_bytes,
+                      "commit_GBps": c_bytes / (float(np.mean(commit_ms)) / 1e3) / 1e9},
             "graph_rounds_per_s": graph_rps,
             "prefill": {"ms": prefill_ms, "bytes": prefill_b, "achieved_GBps": prefill_b / (prefill_ms / 1e3) / 1e9,
                         "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
@@ -483,10 +500,9 @@ def e2e_measure(run, wl, dev, flush, steps, world, inp):
         e0.record(s)
         for k, v in hb.items():
             dev_buf[k].copy_(v, non_blocking=True)
-        F.ls_commit_round(run.state, dev_buf["draft"], dev_buf["target"], dev_buf["vk"], dev_buf["vv"],
-                          dev_buf["vh"], run.accept_len, run.next_token, s)
-        F.ls_draft_attend(run.state, 0, wl.n_layers, dev_buf["q"], run.boundary_k, run.boundary_v, wl.hidden,
-                          run.softmax_scale, out, s)
+        F.ls_round(run.state, dev_buf["draft"], dev_buf["target"], dev_buf["vk"], dev_buf["vv"], dev_buf["vh"],
+                   run.accept_len, run.next_token, dev_buf["q"], 0, wl.n_kv_heads * wl.head_dim,
+                   run.softmax_scale, out, s)
         h_out.copy_(out, non_blocking=True)
         h_acc.copy_(run.accept_len, non_blocking=True)
         h_nxt.copy_(run.next_token, non_blocking=True)
@@ -514,8 +530,7 @@ def flatness_sweep(WLM, dev, flush, rounds):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(run.stream)
-            run.commit(inp, r)
-            run.attend(inp, r, out)
+            run.round(inp, r, out)
             e1.record(run.stream)
             e1.synchronize()
             if r >= 3:

@@ -35,7 +35,8 @@ LS_MAX_SCALES = 4
 
 EXPORTED = (
     "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",
-    "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend", "ls_attend_uses_tensor_cores",
+    "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend", "ls_round",
+    "ls_round_overlaps", "ls_attend_uses_tensor_cores",
     "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
 )
 
@@ -81,6 +82,8 @@ def _load():
         "ls_prefill_summary_noalloc": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, i64, i64, vp, vp]),
         "ls_commit_round": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ls_draft_attend": (ctypes.c_int, [vp, i32, i32, vp, vp, vp, i64, ctypes.c_float, vp, vp]),
+        "ls_round": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, ctypes.c_float, vp, vp]),
+        "ls_round_overlaps": (ctypes.c_int, [vp]),
         "ls_attend_uses_tensor_cores": (ctypes.c_int, [vp]),
         "ls_read_state": (ctypes.c_int, [vp, vp, sz, vp]),
         "ls_get_error": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
@@ -191,6 +194,18 @@ def ls_draft_attend(state, layer_begin, layer_count, q, boundary_k, boundary_v, 
     _check("ls_draft_attend", _lib.ls_draft_attend(
         state, layer_begin, layer_count, _ptr(q), _ptr(boundary_k), _ptr(boundary_v),
         boundary_stride, float(softmax_scale), _ptr(out), _stream(stream)))
+
+
+def ls_round(state, draft_ids, target_ids, verify_k, verify_v, verify_hidden, accept_len, next_token, q,
+             boundary_k_offset, boundary_v_offset, softmax_scale, out, stream=None) -> None:
+    _check("ls_round", _lib.ls_round(
+        state, _ptr(draft_ids), _ptr(target_ids), _ptr(verify_k), _ptr(verify_v), _ptr(verify_hidden),
+        _ptr(accept_len), _ptr(next_token), _ptr(q), boundary_k_offset, boundary_v_offset,
+        float(softmax_scale), _ptr(out), _stream(stream)))
+
+
+def ls_round_overlaps(state) -> bool:
+    return bool(_lib.ls_round_overlaps(state))
 
 
 def ls_attend_uses_tensor_cores(state) -> bool:

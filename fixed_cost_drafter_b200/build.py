@@ -4,6 +4,8 @@
 * ``synth/libls_synth.so`` — the device twin of the seeded input generator.
 
 Each library is rebuilt only when one of its sources (or a header) is newer than it.
+Load this file by path (``load_builder()`` in the repository's entry points does), not as
+``fixed_cost_drafter_b200.build``: importing the package loads the library it builds.
 The CUDA runtime is linked statically, so loading a library needs no GPU driver.
 """
 

@@ -241,11 +241,42 @@ int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count
   if (st->use_tc)
     return cuda_status(ls::launch_attend_tc(st->dev, st->tc, layer_begin, layer_count, d_q,
                                             d_boundary_k, d_boundary_v, boundary_stride,
-                                            softmax_scale, d_out, st->sms, stream));
+                                            softmax_scale, d_out, st->sms, false, stream));
   return cuda_status(ls::launch_attend_simt(st->dev, layer_begin, layer_count, d_q, d_boundary_k,
                                             d_boundary_v, boundary_stride, softmax_scale, d_out,
                                             stream));
 }
+
+int ls_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids, const void* d_verify_k,
+             const void* d_verify_v, const void* d_verify_hidden, int32_t* d_accept_len, int32_t* d_next_token,
+             const void* d_q, int64_t boundary_k_offset, int64_t boundary_v_offset, float softmax_scale,
+             void* d_out, cudaStream_t stream) {
+  if (!st || !d_draft_ids || !d_target_ids || !d_verify_k || !d_verify_v || !d_verify_hidden || !d_accept_len ||
+      !d_next_token || !d_q || !d_out)
+    return LS_ERR_INVALID_ARG;
+  const ls_config& c = st->cfg;
+  const int64_t span = int64_t(c.n_kv_heads) * c.head_dim;
+  if (boundary_k_offset < 0 || boundary_v_offset < 0 || boundary_k_offset % 8 != 0 ||
+      boundary_v_offset % 8 != 0 || boundary_k_offset + span > c.hidden || boundary_v_offset + span > c.hidden)
+    return LS_ERR_SHAPE;
+  if (!(softmax_scale > 0.0f) || softmax_scale == INFINITY) return LS_ERR_INVALID_ARG;
+  if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden) || !aligned16(d_q) ||
+      !aligned16(d_out))
+    return LS_ERR_INVALID_ARG;
+  int r = ls_commit_round(st, d_draft_ids, d_target_ids, d_verify_k, d_verify_v, d_verify_hidden, d_accept_len,
+                          d_next_token, stream);
+  if (r != LS_OK) return r;
+  const char* bnd = static_cast<const char*>(st->dev.boundary);
+  const int64_t e = st->lay.elem;
+  if (st->use_tc)  // the attention kernel is scheduled while the commit runs
+    return cuda_status(ls::launch_attend_tc(st->dev, st->tc, 0, c.n_layers, d_q, bnd + boundary_k_offset * e,
+                                            bnd + boundary_v_offset * e, c.hidden, softmax_scale, d_out, st->sms,
+                                            true, stream));
+  return ls_draft_attend(st, 0, c.n_layers, d_q, bnd + boundary_k_offset * e, bnd + boundary_v_offset * e, c.hidden,
+                         softmax_scale, d_out, stream);
+}
+
+int ls_round_overlaps(const ls_state* st) { return st && st->use_tc ? 1 : 0; }
 
 int ls_attend_uses_tensor_cores(const ls_state* st) { return st && st->use_tc ? 1 : 0; }
 

@@ -28,6 +28,10 @@
 //             row's O in TMEM and its running sum are rescaled once), so no chunk's P V
 //             has to come back to registers. Epilogue: O from TMEM, the boundary row's
 //             share (its logit is computed on CUDA cores), 1/rowsum.
+// ls_round launches this kernel programmatically dependent on the commit kernel: it is
+// scheduled while the commit runs, allocates TMEM, sets up its barriers and issues the
+// first tile's Q (complete before the commit started), then waits on the device
+// (griddepcontrol.wait) for the commit's writes before it reads any state.
 // Every wait is bounded and warp-uniform; a wait that runs out sets
 // LS_DEVERR_WAIT_TIMEOUT, all roles stop, the copies in flight land, TMEM is freed.
 #include <cuda.h>
@@ -177,6 +181,7 @@ __device__ inline uint32_t pack_bf16(float a, float b) {
 
 // Bounded wait that also gives up when another role has already aborted.
 __device__ inline bool wait_or_abort(Bars& s, uint64_t* bar, uint32_t parity, int32_t* err) {
+#pragma unroll 1  // one copy per call site: the kernel's code must stay small for the instruction cache
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 1023) == 1023 && *reinterpret_cast<volatile uint32_t*>(&s.abort)) return false;
@@ -204,7 +209,13 @@ __device__ inline uint64_t range_bits(int lo, int hi, int r0) {
   const uint64_t m = n >= 64 ? ~0ull : ((1ull << n) - 1ull);
   return m << (lo - r0);
 }
-__device__ inline uint64_t rows_mask64(const Dev& p, int r0, int64_t len, const int64_t* nseg) {
+// Out of line: only tiles with an empty view slot (short prefix, a scale with fewer than
+// `slots` segments, an empty partial segment) need it, and the softmax loop's code must
+// stay small for the instruction cache.
+__device__ __noinline__ uint64_t rows_mask64(const Dev& p, int r0, int64_t len, int64_t n0, int64_t n1,
+                                             int64_t n2, int64_t n3) {
+  static_assert(kMaxScales == 4, "one argument per scale");
+  const int64_t nseg[kMaxScales] = {n0, n1, n2, n3};
   uint64_t m = range_bits(0, int(len < p.W ? len : int64_t(p.W)), r0);
   int base = p.W;
 #pragma unroll
@@ -218,6 +229,8 @@ __device__ inline uint64_t rows_mask64(const Dev& p, int r0, int64_t len, const 
   if (len > 0) m |= range_bits(base, base + 1, r0);  // base == R - 1
   return m;
 }
+// Rows [r0, r0 + 64) below R (the last chunk's box reaches past the tile's rows).
+__device__ inline uint64_t rows_below(int n) { return n >= 64 ? ~0ull : (n <= 0 ? 0ull : (1ull << n) - 1ull); }
 
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMap kv_map,
@@ -282,10 +295,11 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       unsigned char* ring = is_k ? k_buf : v_buf;
       prefetch_map(&kv_map); prefetch_map(&kv_tail_map);
       if (is_k) prefetch_map(&q_map);
+      if (!is_k) grid_dependency_wait();
       const int grp = p.Hq / p.Hkv;
       for (int k = 0; k < total; ++k) {
         const int it = k / nC, c = k - it * nC;
-        if (is_k && c == 0) {  // Q of the tile first
+        if (is_k && c == 0) {  // Q of the tile first, then its boundary key and value rows
           const int qb = it & 1;
           if (!wait_or_abort(s, &s.q_empty[qb], ((it >> 1) & 1) ^ 1, p.err)) break;
           int b, lc, g;
@@ -294,7 +308,8 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           const int zrow = (b * a.lcount + lc) * p.B;
           tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
           tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
-          // the tile's boundary key and value rows travel with Q
+          // Q is an input; the boundary rows and the arena are state a preceding commit writes
+          if (it == 0) grid_dependency_wait();
           const int64_t boff = (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + int64_t(g) * 128;
           bulk_g2s(b_buf + qb * kBRowBytes, a.bk + boff, 256, &s.q_full[qb]);
           bulk_g2s(b_buf + qb * kBRowBytes + 256, a.bv + boff, 256, &s.q_full[qb]);
@@ -314,7 +329,9 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   } else if (warp == 1) {
     // ------------------------------------------------------------ QK issuer
     if (lane == 0) {
-      const uint32_t q_base = smem_u32(q_buf), k_base = smem_u32(k_buf);
+      // descriptors of the buffers' first bytes; an operand further in adds its offset / 16
+      // to the start-address field (shared addresses stay below 256 KB: no carry out)
+      const uint64_t dq0 = sdesc(smem_u32(q_buf), 16, 1024), dk0 = sdesc(smem_u32(k_buf), 16, 1024);
       for (int k = 0; k < total; ++k) {
         const int it = k / nC, c = k - it * nC, qb = it & 1, sb = k % kSBufs, st = k % kKStages;
         if (c == 0 && !wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err)) break;
@@ -324,13 +341,13 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         const int rows = chunk_rows(k);
         const int n0 = rows < 64 ? rows : 64, n1 = rows - n0;
         const uint32_t id0 = idesc_bf16(n0, false), id1 = idesc_bf16(n1 > 0 ? n1 : 8, false);
-        const uint32_t kb = k_base + st * kStageBytes;
+        const uint64_t dq = dq0 + uint32_t(qb * kQBytes >> 4), dk = dk0 + uint32_t(st * kStageBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t qa = sdesc(q_base + qb * kQBytes + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
-          const uint32_t koff = (kk >> 2) * (kStageBytes / 2) + (kk & 3) * 32;
-          mma_bf16(tmem + 64 * sb, qa, sdesc(kb + koff, 16, 1024), id0, kk > 0);
-          if (n1 > 0) mma_bf16(tmem + (16u << 16) + 64 * sb, qa, sdesc(kb + koff + 64 * 128, 16, 1024), id1, kk > 0);
+          const uint32_t qo = ((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4;
+          const uint32_t ko = ((kk >> 2) * (kStageBytes / 2) + (kk & 3) * 32) >> 4;
+          mma_bf16(tmem + 64 * sb, dq + qo, dk + ko, id0, kk > 0);
+          if (n1 > 0) mma_bf16(tmem + (16u << 16) + 64 * sb, dq + qo, dk + ko + (64 * 128 >> 4), id1, kk > 0);
         }
         mma_commit(&s.kempty[st]);
         mma_commit(&s.s_full[sb]);
@@ -340,7 +357,8 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   } else if (warp == 7) {
     // ------------------------------------------------------------ PV issuer
     if (lane == 0) {
-      const uint32_t p_base = smem_u32(p_buf), v_base = smem_u32(v_buf);
+      const uint64_t dp0 = sdesc(smem_u32(p_buf), 16, 1024);
+      const uint64_t dv0 = sdesc(smem_u32(v_buf), kStageBytes / 2, 1024);
       const uint32_t id_pv = idesc_bf16(64, true);
       for (int k = 0; k < total; ++k) {
         const int it = k / nC, c = k - it * nC, ob = it & 1, pb = k & 1, st = k % kVStages;
@@ -348,15 +366,15 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         if (!wait_or_abort(s, &s.vfull[st], (k / kVStages) & 1, p.err)) break;
         if (!wait_or_abort(s, &s.p_full[pb], (k >> 1) & 1, p.err)) break;
         tc_fence_after();
-        const uint32_t vb = v_base + st * kStageBytes;
+        const uint64_t dv = dv0 + uint32_t(st * kStageBytes >> 4), dp = dp0 + uint32_t(pb * kPBytes >> 4);
         const int rows = chunk_rows(k);
         for (int kk = 0; kk < rows / 16; ++kk) {
-          const uint64_t pa = sdesc(p_base + pb * kPBytes + (kk >> 2) * (kPBytes / 2) + (kk & 3) * 32, 16, 1024);
+          const uint64_t pa = dp + uint32_t(((kk >> 2) * (kPBytes / 2) + (kk & 3) * 32) >> 4);
           const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
           // V: rows = keys (K dim), 128-byte rows per 64-column half: MN-major B, SBO = 8 rows
-          mma_bf16(tmem + kOCol + 64 * ob, pa, sdesc(vb + kk * 2048, kStageBytes / 2, 1024), id_pv, acc);
-          mma_bf16(tmem + (16u << 16) + kOCol + 64 * ob, pa,
-                   sdesc(vb + kStageBytes / 2 + kk * 2048, kStageBytes / 2, 1024), id_pv, acc);
+          mma_bf16(tmem + kOCol + 64 * ob, pa, dv + uint32_t(kk * 2048 >> 4), id_pv, acc);
+          mma_bf16(tmem + (16u << 16) + kOCol + 64 * ob, pa, dv + uint32_t((kStageBytes / 2 + kk * 2048) >> 4), id_pv,
+                   acc);
         }
         mma_commit(&s.vempty[st]);
         mma_commit(&s.p_empty[pb]);
@@ -364,7 +382,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         if (c == nC - 1) mma_commit(&s.o_full[ob]);
       }
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ softmax
     const int sub = warp & 3;           // TMEM subpartition this warp may access
     const int half = lane >> 4;         // 0: keys / output columns 0-63, 1: 64-127
@@ -384,16 +402,20 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       for (int kk = 0; kk <= kMaxScales; ++kk) dst[kk] = kk <= p.nsc ? ctr[kk] : 0;
     };
     int64_t cnt_next[kMaxScales + 1];
+    grid_dependency_wait();  // the counters are state a preceding commit writes
     load_counters(blockIdx.x, cnt_next);
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
       int b, lc, g;
       tile_coords(t, p, a.lcount, b, lc, g);
       const int qb = it & 1, ob = it & 1;
-      const int64_t len = cnt_next[0];
+      int64_t len;
       int64_t nseg[kMaxScales];
+      {
+        len = cnt_next[0];
 #pragma unroll
-      for (int kk = 0; kk < kMaxScales; ++kk) nseg[kk] = cnt_next[1 + kk];
-      load_counters(t + gridDim.x, cnt_next);
+        for (int kk = 0; kk < kMaxScales; ++kk) nseg[kk] = cnt_next[1 + kk];
+        load_counters(t + gridDim.x, cnt_next);
+      }
 
       // boundary logit on CUDA cores (each thread of the pair does 64 of the 128 d)
       if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err))) break;
@@ -401,7 +423,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       {
         const unsigned char* qrow = q_buf + qb * kQBytes + half * (kQBytes / 2) + row * 128;
         const uint4* bkrow = reinterpret_cast<const uint4*>(b_buf + qb * kBRowBytes + half * 128);
-#pragma unroll
+#pragma unroll 2
         for (int ch = 0; ch < 8; ++ch) {
           const uint4 qv = *reinterpret_cast<const uint4*>(qrow + ((ch ^ (row & 7)) << 4));
           float qf[8], kf[8];
@@ -418,6 +440,12 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         for (int ch = 0; ch < 8; ++ch) bvv[ch] = bvrow[ch];
       }
       mbar_arrive(&s.q_empty[qb]);
+      // every view slot of the tile holds a row (the steady state): no masks beyond R
+      const int ring_valid = len < p.W ? int(len) : p.W;
+      bool tile_full = len >= p.W;
+#pragma unroll
+      for (int kk = 0; kk < kMaxScales; ++kk)
+        if (kk < p.nsc) tile_full = tile_full && nseg[kk] >= p.slots && len - nseg[kk] * p.scales[kk] > 0;
       float blog = (bpart[0] + bpart[1]) + (bpart[2] + bpart[3]);
       blog += __shfl_xor_sync(0xffffffffu, blog, 16);
       const float blog_s = blog * sl2;
@@ -427,7 +455,10 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       bool ok = true;
       for (int c = 0; c < nC; ++c, ++k) {
         const int sb = k % kSBufs, pb = k & 1;
-        const uint64_t vm = rows_mask64(p, c * kChunk + 64 * half, len, nseg);
+        const int r0 = c * kChunk + 64 * half;
+        const uint64_t vm = r0 + 64 <= p.W ? rows_below(ring_valid - r0)  // ring slots only
+                            : tile_full ? rows_below(p.R - r0)
+                                        : rows_mask64(p, r0, len, nseg[0], nseg[1], nseg[2], nseg[3]);
         const bool all_valid = __all_sync(0xffffffffu, vm == ~0ull);
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.s_full[sb], (k / kSBufs) & 1, p.err))) { ok = false; break; }
         tc_fence_after();
@@ -615,7 +646,7 @@ int tc_prepare(const Dev& p, TcPlan* plan) {
 
 cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
                              const void* bk, const void* bv, int64_t bstride, float scale, void* out,
-                             int sms, cudaStream_t stream) {
+                             int sms, bool after_commit, cudaStream_t stream) {
   CUtensorMap qmap;
   if (!encode_q(p, lcount, q, &qmap)) return cudaErrorInvalidValue;
   TcArgs a{};
@@ -629,11 +660,20 @@ cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcoun
   a.bstride = bstride;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
-  const int grid = a.n_tiles < sms ? a.n_tiles : sms;
-  attend_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
-      p, a, *reinterpret_cast<const CUtensorMap*>(plan.kv_map),
-      *reinterpret_cast<const CUtensorMap*>(plan.kv_tail_map), qmap);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(a.n_tiles < sms ? a.n_tiles : sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (after_commit) {  // scheduled while the commit kernel just launched on `stream` runs
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, attend_tc_kernel, p, a, *reinterpret_cast<const CUtensorMap*>(plan.kv_map),
+                            *reinterpret_cast<const CUtensorMap*>(plan.kv_tail_map), qmap);
 }
 
 }  // namespace ls

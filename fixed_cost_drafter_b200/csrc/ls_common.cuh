@@ -155,6 +155,15 @@ __device__ inline bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_
 }
 constexpr uint32_t kWaitLimit = 1u << 22;
 
+// Programmatic dependent launch. A kernel launched with the programmatic-serialization
+// attribute may start while the kernel before it on the stream still runs; its threads
+// call grid_dependency_wait() before they read anything that kernel writes (the wait
+// returns once that grid has completed and its writes are visible; without the launch
+// attribute it returns at once). The earlier kernel calls allow_dependent_launch() to let
+// the dependent be scheduled before it completes.
+__device__ inline void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Bulk asynchronous global->shared copy on the TMA engine (no tensor map, no multicast).
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ inline void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -134,7 +134,6 @@ class DeviceRun:
         self.target = torch.from_numpy(target[:self.rounds].copy()).to(self.dev)
         self.accept_len = torch.zeros(wl.batch, dtype=torch.int32, device=self.dev)
         self.next_token = torch.zeros(wl.batch, dtype=torch.int32, device=self.dev)
-        self.round = 0
         e = wl.elem()
         self.boundary_k = self.arena.data_ptr() + self.layout.off_boundary
         self.boundary_v = self.boundary_k + wl.n_kv_heads * wl.head_dim * e
@@ -223,6 +222,15 @@ class DeviceRun:
             q = q[:, layer_begin:layer_begin + lc].contiguous()
         F.ls_draft_attend(self.state, layer_begin, lc, q, self.boundary_k, self.boundary_v, wl.hidden,
                           self.softmax_scale, out, self.stream)
+
+    def round(self, inputs, r, out):
+        """ls_round: commit and attention over all layers in one call (boundary keys and
+        values are the slices [0, Hkv*D) and [Hkv*D, 2*Hkv*D) of the boundary hidden)."""
+        wl = self.wl
+        i = r - inputs["r0"]
+        F.ls_round(self.state, self.draft[r], self.target[r], inputs["vk"][i], inputs["vv"][i], inputs["vh"][i],
+                   self.accept_len, self.next_token, inputs["q"][i], 0, wl.n_kv_heads * wl.head_dim,
+                   self.softmax_scale, out, self.stream)
 
     def new_out(self, layer_count=None):
         wl = self.wl

@@ -211,6 +211,27 @@ LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t laye
                     int64_t boundary_stride, float softmax_scale, void* d_out,
                     cudaStream_t stream);
 
+/* One whole decoding round: ls_commit_round, then ls_draft_attend over all layers, for
+ * drafters whose boundary keys/values are slices of the new boundary hidden vector:
+ * element (b, l, g, d) of the boundary key is hidden_b,l[boundary_k_offset + g*D + d] and
+ * of the value hidden_b,l[boundary_v_offset + g*D + d], hidden_b,l being verify row a's
+ * hidden vector (offsets multiples of 8, each slice inside `hidden`). Arguments as in the
+ * two calls; the result (state, accept_len, next_token, out) is the same as theirs.
+ * Where the tcgen05 kernel applies (ls_round_overlaps) the attention kernel is launched
+ * as a programmatic dependent of the commit kernel: it is scheduled while the commit runs,
+ * sets itself up and loads its first Q tile, then waits on the device for the commit's
+ * writes. d_q must therefore be complete when the call is issued (stream order gives
+ * that), and must not be written by the commit's outputs.                              */
+LS_API int ls_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
+                    const void* d_verify_k, const void* d_verify_v, const void* d_verify_hidden,
+                    int32_t* d_accept_len, int32_t* d_next_token, const void* d_q,
+                    int64_t boundary_k_offset, int64_t boundary_v_offset, float softmax_scale,
+                    void* d_out, cudaStream_t stream);
+
+/* 1 if ls_round overlaps the attention kernel's launch with the commit for this state
+ * (programmatic dependent launch), 0 if it makes the two calls in turn.              */
+LS_API int ls_round_overlaps(const ls_state* st);
+
 /* 1 if ls_draft_attend takes the tcgen05 path for this state, 0 if the CUDA-core one. */
 LS_API int ls_attend_uses_tensor_cores(const ls_state* st);
 

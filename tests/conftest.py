@@ -11,8 +11,8 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     # the in-tree libraries are built (or found up to date) before any test imports them
-    from fixed_cost_drafter_b200 import build as _build
-    _build.build()
+    from __graft_entry__ import load_builder
+    load_builder().build()
 
 
 @pytest.fixture(scope="session")

@@ -4,14 +4,19 @@
 //
 // One tile = (sequence, layer, KV head g): M = (Hq/Hkv) * B = 64 query rows (the GQA
 // group's heads x the block's queries, row m = i * group + j) against the tile's
-// kv_rows <= 768 arena rows (ring window + summary mean rows) plus the boundary row.
-// The arena rows stream through in chunks of 128 rows with an online softmax.
+// kv_rows arena rows (ring window + summary mean rows) followed by the boundary row:
+// R + 1 <= 768 key/value rows stream through in chunks of 128 with an online softmax. The
+// boundary row (a per-tile vector given by the caller) is written by the producer warps
+// into the last chunk's stage right after the tile's rows, so every row of the views is
+// handled the same way.
 //
 // Persistent kernel, one CTA per SM, 8 warps; the roles only meet at mbarriers, so no
 // role's order of work can hold up another's:
 //   warp 0    TMA producer of Q (3-D tensor map, two 64-column swizzled halves) and of
-//             the K rows of every chunk (ring of K stages, tensor map over the arena).
-//   warp 6    TMA producer of the V rows of every chunk (its own ring of V stages).
+//             the K rows of every chunk (ring of K stages, tensor map over the arena),
+//             plus the boundary key row.
+//   warp 6    TMA producer of the V rows of every chunk (its own ring of V stages), plus
+//             the boundary value row.
 //   warp 1    TMEM allocator and the QK-issuing thread (tcgen05.mma kind::f16, bf16 in,
 //             fp32 accumulate, M = 64). The M = 64 accumulator fills lanes 0-15 of each
 //             32-lane TMEM subpartition; a second accumulator at lane offset 16 fills
@@ -26,8 +31,7 @@
 //             bf16 P into shared memory in the MMA's swizzled K-major layout. The
 //             reference max only moves when a chunk exceeds it by more than 2^8 (then the
 //             row's O in TMEM and its running sum are rescaled once), so no chunk's P V
-//             has to come back to registers. Epilogue: O from TMEM, the boundary row's
-//             share (its logit is computed on CUDA cores), 1/rowsum.
+//             has to come back to registers. Epilogue: O from TMEM times 1/rowsum.
 // ls_round launches this kernel programmatically dependent on the commit kernel: it is
 // scheduled while the commit runs, allocates TMEM, sets up its barriers and issues the
 // first tile's Q (complete before the commit started), then waits on the device
@@ -45,21 +49,21 @@ namespace {
 constexpr int kKStages = 3;           // K ring
 constexpr int kVStages = 2;           // V ring
 constexpr int kChunk = 128;            // arena rows per chunk
-constexpr int kMaxChunks = 6;          // kv_rows <= 768
+constexpr int kMaxChunks = 6;          // kv_rows + 1 <= 768
 constexpr int kThreads = 256;
 constexpr int kQBytes = 64 * 128 * 2;  // one Q tile (two 8 KB halves)
 constexpr int kPBytes = 64 * 128 * 2;  // one P chunk (two 8 KB halves: keys 0-63 / 64-127)
 constexpr int kStageBytes = kChunk * 128 * 2;  // one K or V chunk (two 16 KB halves: d 0-63 / 64-127)
-constexpr int kBRowBytes = 2 * 128 * 2;  // the tile's boundary key and value rows (bf16)
-constexpr int kSmemBytes =
-    2 * kQBytes + 2 * kPBytes + (kKStages + kVStages) * kStageBytes + 2 * kBRowBytes + 1024;
+constexpr int kSmemBytes = 2 * kQBytes + 2 * kPBytes + (kKStages + kVStages) * kStageBytes + 1024;
 constexpr int kSBufs = 4;              // S buffers: QK may run up to four chunks ahead
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 256;        // O buffers at columns 256 + 64 * (tile & 1)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
 
 struct TcArgs {
-  int32_t lb, lcount, n_tiles, n_chunks, tail_rows;
+  int32_t lb, lcount, n_tiles;
+  int32_t n_chunks;   // chunks per tile: floor(R / 128) + 1, the last holding the boundary row
+  int32_t tail_rows;  // R mod 128: the tile's arena rows in its last chunk
   const __nv_bfloat16* bk;
   const __nv_bfloat16* bv;
   int64_t bstride;
@@ -198,9 +202,11 @@ __device__ inline void tile_coords(int t, const Dev& p, int lcount, int& b, int&
   b = rest / lcount;
 }
 
-// Validity of the 64 arena rows [r0, r0 + 64) of a tile as a bit mask (bit i = row r0+i):
-// the ring slots below min(len, W), per scale the first min(n_seg, slots) segment slots
-// and the partial mean when its segment is non-empty, and the global mean when len > 0.
+// Validity of the 64 rows [r0, r0 + 64) of a tile's key/value stream as a bit mask
+// (bit i = row r0 + i). The stream is the tile's arena rows followed by the boundary row
+// (row R): ring slots below min(len, W), per scale the first min(n_seg, slots) segment
+// slots and the partial mean when its segment is non-empty, the global mean when len > 0,
+// and the boundary row always.
 __device__ inline uint64_t range_bits(int lo, int hi, int r0) {
   lo = max(lo, r0);
   hi = min(hi, r0 + 64);
@@ -209,28 +215,22 @@ __device__ inline uint64_t range_bits(int lo, int hi, int r0) {
   const uint64_t m = n >= 64 ? ~0ull : ((1ull << n) - 1ull);
   return m << (lo - r0);
 }
-// Out of line: only tiles with an empty view slot (short prefix, a scale with fewer than
-// `slots` segments, an empty partial segment) need it, and the softmax loop's code must
-// stay small for the instruction cache.
-__device__ __noinline__ uint64_t rows_mask64(const Dev& p, int r0, int64_t len, int64_t n0, int64_t n1,
-                                             int64_t n2, int64_t n3) {
-  static_assert(kMaxScales == 4, "one argument per scale");
-  const int64_t nseg[kMaxScales] = {n0, n1, n2, n3};
-  uint64_t m = range_bits(0, int(len < p.W ? len : int64_t(p.W)), r0);
-  int base = p.W;
-#pragma unroll
-  for (int k = 0; k < kMaxScales; ++k) {
-    if (k < p.nsc) {
-      m |= range_bits(base, base + int(nseg[k] < p.slots ? nseg[k] : int64_t(p.slots)), r0);
-      if (len - nseg[k] * int64_t(p.scales[k]) > 0) m |= range_bits(base + p.slots, base + p.slots + 1, r0);
-      base += p.slots + 1;
-    }
-  }
-  if (len > 0) m |= range_bits(base, base + 1, r0);  // base == R - 1
-  return m;
-}
-// Rows [r0, r0 + 64) below R (the last chunk's box reaches past the tile's rows).
+// Rows below n of [r0, r0 + 64), r0 already subtracted.
 __device__ inline uint64_t rows_below(int n) { return n >= 64 ? ~0ull : (n <= 0 ? 0ull : (1ull << n) - 1ull); }
+// sinfo: 16 bits per scale k at bit 16k: valid segment slots (bits 0-14), partial non-empty (bit 15).
+__device__ inline uint64_t view_mask(const Dev& p, int r0, int ring_valid, uint64_t sinfo, bool has_glob) {
+  uint64_t m = range_bits(0, ring_valid, r0);
+  int base = p.W;
+#pragma unroll 1
+  for (int k = 0; k < p.nsc; ++k) {
+    const uint32_t e = uint32_t(sinfo >> (16 * k));
+    m |= range_bits(base, base + int(e & 0x7fffu), r0);
+    if (e & 0x8000u) m |= range_bits(base + p.slots, base + p.slots + 1, r0);
+    base += p.slots + 1;
+  }
+  if (has_glob) m |= range_bits(base, base + 1, r0);  // global mean, row R - 1
+  return m | range_bits(base + 1, base + 2, r0);       // boundary row, row R
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMap kv_map,
@@ -243,10 +243,11 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   unsigned char* p_buf = q_buf + 2 * kQBytes;            // [2][kPBytes]
   unsigned char* k_buf = p_buf + 2 * kPBytes;            // [kKStages][kStageBytes]
   unsigned char* v_buf = k_buf + kKStages * kStageBytes; // [kVStages][kStageBytes]
-  unsigned char* b_buf = v_buf + kVStages * kStageBytes; // [2][boundary k row, v row]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nC = a.n_chunks;
+  const int tail = a.tail_rows;                   // the tile's arena rows in its last chunk
+  const int last_rows = (tail + 1 + 15) & ~15;    // rows the last chunk's MMAs take (+ boundary)
   int my_tiles = 0;
   for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) ++my_tiles;
   const int total = my_tiles * nC;  // chunks this CTA processes, in order
@@ -256,13 +257,26 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     for (int i = 0; i < kVStages; ++i) { mbar_init(&s.vfull[i], 1); mbar_init(&s.vempty[i], 1); }
     for (int i = 0; i < kSBufs; ++i) { mbar_init(&s.s_full[i], 1); mbar_init(&s.s_free[i], 128); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.q_full[i], 1); mbar_init(&s.q_empty[i], 1 + 128);
+      mbar_init(&s.q_full[i], 1); mbar_init(&s.q_empty[i], 1);
       mbar_init(&s.p_full[i], 128); mbar_init(&s.p_empty[i], 1);
       mbar_init(&s.o_full[i], 1); mbar_init(&s.o_free[i], 128);
     }
     mbar_init(&s.pv_done, 1);
     s.abort = 0;
     fence_mbar_init();
+  }
+  {
+    // rows of the last chunk past the boundary row are read by its MMAs (masked): they
+    // must hold finite values, zeros until a full chunk has used the stage
+    const int zr = last_rows - tail - 1;
+    if (zr > 0) {
+      const int n = (kKStages + kVStages) * 2 * zr * 8;
+      for (int i = threadIdx.x; i < n; i += kThreads) {
+        const int piece = i & 7, r = tail + 1 + (i >> 3) % zr, sh = (i >> 3) / zr;
+        *reinterpret_cast<uint4*>(k_buf + sh * (kStageBytes / 2) + r * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+    }
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -276,7 +290,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   int issued = 0;  // producers: loads issued into their ring (for the drain after an abort)
-  auto chunk_rows = [&](int k) { return (k % nC) == nC - 1 ? a.tail_rows : kChunk; };
+  auto chunk_rows = [&](int k) { return (k % nC) == nC - 1 ? last_rows : kChunk; };
   auto chunk_y = [&](int k, int t2) {  // first arena row of chunk k's K (t2 = 0) or V (t2 = 1)
     const int it = k / nC, c = k - it * nC;
     int b, lc, g;
@@ -286,45 +300,65 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   };
 
   if (warp == 0 || warp == 6) {
-    // ------------------------------------------------------------ TMA producers
+    // ------------------------------------------------------------ producers
+    // The whole warp runs the loop; lane 0 issues the copies. Lanes 0-15 carry the tile's
+    // boundary row (16 bytes each), loaded when the tile starts and written into the
+    // last chunk's stage right after the tile's rows, in the TMA's 128-byte swizzle.
+    const bool is_k = warp == 0;
+    const int nst = is_k ? kKStages : kVStages;
+    uint64_t* fullb = is_k ? s.kfull : s.vfull;
+    uint64_t* emptyb = is_k ? s.kempty : s.vempty;
+    unsigned char* ring = is_k ? k_buf : v_buf;
+    const __nv_bfloat16* bsrc = is_k ? a.bk : a.bv;
     if (lane == 0) {
-      const bool is_k = warp == 0;
-      const int nst = is_k ? kKStages : kVStages;
-      uint64_t* fullb = is_k ? s.kfull : s.vfull;
-      uint64_t* emptyb = is_k ? s.kempty : s.vempty;
-      unsigned char* ring = is_k ? k_buf : v_buf;
-      prefetch_map(&kv_map); prefetch_map(&kv_tail_map);
+      prefetch_map(&kv_map);
+      if (tail > 0) prefetch_map(&kv_tail_map);
       if (is_k) prefetch_map(&q_map);
-      if (!is_k) grid_dependency_wait();
-      const int grp = p.Hq / p.Hkv;
-      for (int k = 0; k < total; ++k) {
-        const int it = k / nC, c = k - it * nC;
-        if (is_k && c == 0) {  // Q of the tile first, then its boundary key and value rows
+    }
+    if (!is_k) grid_dependency_wait();
+    const int grp = p.Hq / p.Hkv;
+    uint4 brow = make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < total; ++k) {
+      const int it = k / nC, c = k - it * nC;
+      if (c == 0) {
+        int b, lc, g;
+        tile_coords(blockIdx.x + it * gridDim.x, p, a.lcount, b, lc, g);
+        if (is_k) {  // Q of the tile first
           const int qb = it & 1;
-          if (!wait_or_abort(s, &s.q_empty[qb], ((it >> 1) & 1) ^ 1, p.err)) break;
-          int b, lc, g;
-          tile_coords(blockIdx.x + it * gridDim.x, p, a.lcount, b, lc, g);
-          mbar_arrive_expect_tx(&s.q_full[qb], kQBytes + kBRowBytes);
-          const int zrow = (b * a.lcount + lc) * p.B;
-          tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
-          tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
+          if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_empty[qb], ((it >> 1) & 1) ^ 1, p.err))) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&s.q_full[qb], kQBytes);
+            const int zrow = (b * a.lcount + lc) * p.B;
+            tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
+            tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
+          }
           // Q is an input; the boundary rows and the arena are state a preceding commit writes
           if (it == 0) grid_dependency_wait();
-          const int64_t boff = (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + int64_t(g) * 128;
-          bulk_g2s(b_buf + qb * kBRowBytes, a.bk + boff, 256, &s.q_full[qb]);
-          bulk_g2s(b_buf + qb * kBRowBytes + 256, a.bv + boff, 256, &s.q_full[qb]);
         }
-        const int st = k % nst;
-        if (!wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err)) break;
-        const int rows = chunk_rows(k);
-        const CUtensorMap* m = c == nC - 1 ? &kv_tail_map : &kv_map;
-        const int y = chunk_y(k, is_k ? 0 : 1);
-        mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
-        unsigned char* dst = ring + st * kStageBytes;
-        tma_load_2d(dst, m, 0, y, &fullb[st]);
-        tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
-        ++issued;
+        if (lane < 16) brow = ld_nc_v4(bsrc + (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + g * 128 + lane * 8);
       }
+      const int st = k % nst;
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err))) break;
+      unsigned char* dst = ring + st * kStageBytes;
+      const bool last = c == nC - 1;
+      if (last) {  // the boundary row, row `tail` of the stage
+        if (lane < 16)
+          *reinterpret_cast<uint4*>(dst + (lane >> 3) * (kStageBytes / 2) + tail * 128 +
+                                    (((lane & 7) ^ (tail & 7)) << 4)) = brow;
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (lane == 0) {
+        const int rows = last ? tail : kChunk;
+        mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
+        if (rows > 0) {
+          const CUtensorMap* m = last ? &kv_tail_map : &kv_map;
+          const int y = chunk_y(k, is_k ? 0 : 1);
+          tma_load_2d(dst, m, 0, y, &fullb[st]);
+          tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
+        }
+      }
+      ++issued;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ QK issuer
@@ -340,7 +374,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         tc_fence_after();
         const int rows = chunk_rows(k);
         const int n0 = rows < 64 ? rows : 64, n1 = rows - n0;
-        const uint32_t id0 = idesc_bf16(n0, false), id1 = idesc_bf16(n1 > 0 ? n1 : 8, false);
+        const uint32_t id0 = idesc_bf16(n0, false), id1 = idesc_bf16(n1 > 0 ? n1 : 16, false);
         const uint64_t dq = dq0 + uint32_t(qb * kQBytes >> 4), dk = dk0 + uint32_t(st * kStageBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -407,58 +441,29 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
       int b, lc, g;
       tile_coords(t, p, a.lcount, b, lc, g);
-      const int qb = it & 1, ob = it & 1;
-      int64_t len;
-      int64_t nseg[kMaxScales];
-      {
-        len = cnt_next[0];
+      const int ob = it & 1;
+      const int64_t len = cnt_next[0];
+      const int ring_valid = len < p.W ? int(len) : p.W;
+      uint64_t sinfo = 0;
 #pragma unroll
-        for (int kk = 0; kk < kMaxScales; ++kk) nseg[kk] = cnt_next[1 + kk];
-        load_counters(t + gridDim.x, cnt_next);
-      }
-
-      // boundary logit on CUDA cores (each thread of the pair does 64 of the 128 d)
-      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err))) break;
-      float bpart[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        const unsigned char* qrow = q_buf + qb * kQBytes + half * (kQBytes / 2) + row * 128;
-        const uint4* bkrow = reinterpret_cast<const uint4*>(b_buf + qb * kBRowBytes + half * 128);
-#pragma unroll 2
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 qv = *reinterpret_cast<const uint4*>(qrow + ((ch ^ (row & 7)) << 4));
-          float qf[8], kf[8];
-          Elem<__nv_bfloat16>::to_f32(qv, qf);
-          Elem<__nv_bfloat16>::to_f32(bkrow[ch], kf);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) bpart[e & 3] = fmaf(qf[e], kf[e], bpart[e & 3]);
+      for (int kk = 0; kk < kMaxScales; ++kk) {
+        if (kk < p.nsc) {
+          const int64_t n = cnt_next[1 + kk];
+          const uint64_t e = uint64_t(n < p.slots ? n : int64_t(p.slots)) |
+                             (len - n * p.scales[kk] > 0 ? 0x8000ull : 0ull);
+          sinfo |= e << (16 * kk);
         }
       }
-      uint4 bvv[8];  // boundary value row (this thread's 64 columns), kept for the epilogue
-      {
-        const uint4* bvrow = reinterpret_cast<const uint4*>(b_buf + qb * kBRowBytes + 256 + half * 128);
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) bvv[ch] = bvrow[ch];
-      }
-      mbar_arrive(&s.q_empty[qb]);
-      // every view slot of the tile holds a row (the steady state): no masks beyond R
-      const int ring_valid = len < p.W ? int(len) : p.W;
-      bool tile_full = len >= p.W;
-#pragma unroll
-      for (int kk = 0; kk < kMaxScales; ++kk)
-        if (kk < p.nsc) tile_full = tile_full && nseg[kk] >= p.slots && len - nseg[kk] * p.scales[kk] > 0;
-      float blog = (bpart[0] + bpart[1]) + (bpart[2] + bpart[3]);
-      blog += __shfl_xor_sync(0xffffffffu, blog, 16);
-      const float blog_s = blog * sl2;
-      float mref = blog_s;  // reference max (log2 units) the P values are taken against
-      float lsum = 0.f;     // sum of the arena rows' weights against mref
+      load_counters(t + gridDim.x, cnt_next);
 
+      float mref = -INFINITY;  // reference max (log2 units) the P values are taken against
+      float lsum = 0.f;        // sum of the rows' weights against mref
       bool ok = true;
       for (int c = 0; c < nC; ++c, ++k) {
         const int sb = k % kSBufs, pb = k & 1;
         const int r0 = c * kChunk + 64 * half;
         const uint64_t vm = r0 + 64 <= p.W ? rows_below(ring_valid - r0)  // ring slots only
-                            : tile_full ? rows_below(p.R - r0)
-                                        : rows_mask64(p, r0, len, nseg[0], nseg[1], nseg[2], nseg[3]);
+                                           : view_mask(p, r0, ring_valid, sinfo, len > 0);
         const bool all_valid = __all_sync(0xffffffffu, vm == ~0ull);
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.s_full[sb], (k / kSBufs) & 1, p.err))) { ok = false; break; }
         tc_fence_after();
@@ -488,12 +493,12 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         // parity wait on pv_done below identify P_{k-1} V_{k-1} unambiguously
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.p_empty[pb], ((k >> 1) & 1) ^ 1, p.err))) { ok = false; break; }
         if (c == 0) {
-          mref = fmaxf(mref, cmax);  // O is still empty: the reference moves for free
+          mref = cmax;  // O is still empty: the reference moves for free
         } else if (__any_sync(0xffffffffu, cmax > mref + kRescaleThreshold)) {
           // rows whose max grew by more than 2^8: rescale their O (after the P V MMAs
           // issued so far have landed) and their running sum to the new reference
           const float mnew = cmax > mref + kRescaleThreshold ? cmax : mref;
-          const float alpha = ex2(mref - mnew);
+          const float alpha = ex2(mref - mnew);  // 0 while no row was valid yet
           if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.pv_done, (k - 1) & 1, p.err))) { ok = false; break; }
           tc_fence_after();
           float ov[32];
@@ -508,15 +513,17 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           lsum *= alpha;
           mref = mnew;
         }
-        // weights 2^(s * scale - mref) (masked slots hold -inf: weight 0), bf16 P, 8-way sums
+        // weights 2^(s * scale - mref) (masked slots hold -inf: weight 0), bf16 P, 8-way sums;
+        // before any valid row the reference is -inf and every slot so far is masked
+        const float mu = mref == -INFINITY ? 0.f : mref;
         float ps8[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) ps8[u] = 0.f;
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 64; i += 2) {
-          const float p0 = ex2(fmaf(sv[i], sl2, -mref));
-          const float p1 = ex2(fmaf(sv[i + 1], sl2, -mref));
+          const float p0 = ex2(fmaf(sv[i], sl2, -mu));
+          const float p1 = ex2(fmaf(sv[i + 1], sl2, -mu));
           ps8[(i >> 1) & 7] += p0 + p1;
           pk[i >> 1] = pack_bf16(p0, p1);
         }
@@ -532,7 +539,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         mbar_arrive(&s.p_full[pb]);
       }
       if (!ok) break;
-      // epilogue: O from TMEM plus the boundary row's share, normalised
+      // epilogue: O from TMEM over the row sum (the boundary row is one of the summed rows)
       if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.o_full[ob], (it >> 1) & 1, p.err))) break;
       tc_fence_after();
       float o[64];
@@ -540,27 +547,21 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       tmem_ld32(trow + kOCol + 64 * ob + 32, o + 32);
       tc_fence_before();
       mbar_arrive(&s.o_free[ob]);
-      const float pbd = ex2(blog_s - mref);
-      const float inv = 1.0f / (lsum + pbd);
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        float bf[8];
-        Elem<__nv_bfloat16>::to_f32(bvv[ch], bf);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[8 * ch + e] = fmaf(pbd, bf[e], o[8 * ch + e]) * inv;
-      }
+      const float inv = 1.0f / lsum;
       const int i = row / grp, jj = row - (row / grp) * grp;
       const int64_t orow = (((int64_t(b) * a.lcount + lc) * p.B + i) * p.Hq + g * grp + jj) * 128 + 64 * half;
       if (p.out_f32) {
         float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) o4[u] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        for (int u = 0; u < 16; ++u)
+          o4[u] = make_float4(o[4 * u] * inv, o[4 * u + 1] * inv, o[4 * u + 2] * inv, o[4 * u + 3] * inv);
       } else {
         uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow);
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          o4[u] = make_uint4(pack_bf16(o[8 * u], o[8 * u + 1]), pack_bf16(o[8 * u + 2], o[8 * u + 3]),
-                             pack_bf16(o[8 * u + 4], o[8 * u + 5]), pack_bf16(o[8 * u + 6], o[8 * u + 7]));
+          o4[u] = make_uint4(pack_bf16(o[8 * u] * inv, o[8 * u + 1] * inv), pack_bf16(o[8 * u + 2] * inv, o[8 * u + 3] * inv),
+                             pack_bf16(o[8 * u + 4] * inv, o[8 * u + 5] * inv),
+                             pack_bf16(o[8 * u + 6] * inv, o[8 * u + 7] * inv));
       }
     }
   }
@@ -628,16 +629,16 @@ bool encode_q(const Dev& p, int lcount, const void* q, CUtensorMap* out) {
 
 bool tc_supported(const Dev& p) {
   const int grp = p.Hq / p.Hkv;
-  return p.dtype == LS_BF16 && p.D == 128 && grp * p.B == 64 && p.R <= kMaxChunks * kChunk;
+  return p.dtype == LS_BF16 && p.D == 128 && grp * p.B == 64 && p.R + 1 <= kMaxChunks * kChunk;
 }
 
 int tc_prepare(const Dev& p, TcPlan* plan) {
   static_assert(sizeof(CUtensorMap) <= sizeof(plan->kv_map), "tensor map size");
-  plan->n_chunks = (p.R + kChunk - 1) / kChunk;
-  const int tail = p.R - (plan->n_chunks - 1) * kChunk;
-  plan->tail_rows = (tail + 15) / 16 * 16;
+  plan->n_chunks = p.R / kChunk + 1;
+  plan->tail_rows = p.R % kChunk;
   if (!encode_kv(p, kChunk, reinterpret_cast<CUtensorMap*>(plan->kv_map))) return LS_ERR_CUDA;
-  if (!encode_kv(p, plan->tail_rows, reinterpret_cast<CUtensorMap*>(plan->kv_tail_map))) return LS_ERR_CUDA;
+  if (plan->tail_rows > 0 && !encode_kv(p, plan->tail_rows, reinterpret_cast<CUtensorMap*>(plan->kv_tail_map)))
+    return LS_ERR_CUDA;
   if (cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
       cudaSuccess)
     return LS_ERR_CUDA;

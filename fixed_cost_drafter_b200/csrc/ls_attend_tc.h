@@ -8,9 +8,9 @@ namespace ls {
 // (128-row chunks, and the shorter last chunk of each tile).
 struct alignas(64) TcPlan {
   alignas(64) unsigned char kv_map[128];       // CUtensorMap, box 64 x 128 rows
-  alignas(64) unsigned char kv_tail_map[128];  // CUtensorMap, box 64 x tail_rows
-  int32_t n_chunks;                             // 128-row chunks of arena rows per tile
-  int32_t tail_rows;                            // rows of the last chunk, rounded up to 16
+  alignas(64) unsigned char kv_tail_map[128];  // CUtensorMap, box 64 x tail_rows (if tail_rows > 0)
+  int32_t n_chunks;                             // 128-row chunks per tile: floor(R / 128) + 1
+  int32_t tail_rows;                            // R mod 128: arena rows of the last chunk
 };
 
 bool tc_supported(const Dev& p);

@@ -10,7 +10,7 @@
 // into the last chunk's stage right after the tile's rows, so every row of the views is
 // handled the same way.
 //
-// Persistent kernel, one CTA per SM, 8 warps; the roles only meet at mbarriers, so no
+// Persistent kernel, one CTA per SM, 12 warps; the roles only meet at mbarriers, so no
 // role's order of work can hold up another's:
 //   warp 0    TMA producer of Q (3-D tensor map, two 64-column swizzled halves) and of
 //             the K rows of every chunk (ring of K stages, tensor map over the arena),
@@ -31,7 +31,11 @@
 //             bf16 P into shared memory in the MMA's swizzled K-major layout. The
 //             reference max only moves when a chunk exceeds it by more than 2^8 (then the
 //             row's O in TMEM and its running sum are rescaled once), so no chunk's P V
-//             has to come back to registers. Epilogue: O from TMEM times 1/rowsum.
+//             has to come back to registers. After a tile's last chunk the row sums go
+//             to the epilogue warps through shared memory.
+//   warps 8-11 epilogue, one TMEM subpartition each: O of a tile from TMEM (O is
+//             double-buffered by tile) times 1/rowsum, to global memory, while the
+//             softmax warps already work on the next tile.
 // ls_round launches this kernel programmatically dependent on the commit kernel: it is
 // scheduled while the commit runs, allocates TMEM, sets up its barriers and issues the
 // first tile's Q (complete before the commit started), then waits on the device
@@ -50,7 +54,7 @@ constexpr int kKStages = 3;           // K ring
 constexpr int kVStages = 2;           // V ring
 constexpr int kChunk = 128;            // arena rows per chunk
 constexpr int kMaxChunks = 6;          // kv_rows + 1 <= 768
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;          // 12 warps: 3 per SM sub-partition, <= 168 registers
 constexpr int kQBytes = 64 * 128 * 2;  // one Q tile (two 8 KB halves)
 constexpr int kPBytes = 64 * 128 * 2;  // one P chunk (two 8 KB halves: keys 0-63 / 64-127)
 constexpr int kStageBytes = kChunk * 128 * 2;  // one K or V chunk (two 16 KB halves: d 0-63 / 64-127)
@@ -79,6 +83,8 @@ struct Bars {
   uint64_t p_full[2], p_empty[2];
   uint64_t pv_done;
   uint64_t o_full[2], o_free[2];
+  uint64_t lsum_full[2], lsum_free[2];
+  float lsum_buf[2][64];  // row sums of the last two tiles, softmax -> epilogue
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -260,6 +266,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       mbar_init(&s.q_full[i], 1); mbar_init(&s.q_empty[i], 1);
       mbar_init(&s.p_full[i], 128); mbar_init(&s.p_empty[i], 1);
       mbar_init(&s.o_full[i], 1); mbar_init(&s.o_free[i], 128);
+      mbar_init(&s.lsum_full[i], 128); mbar_init(&s.lsum_free[i], 128);
     }
     mbar_init(&s.pv_done, 1);
     s.abort = 0;
@@ -422,7 +429,6 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     const int half = lane >> 4;         // 0: keys / output columns 0-63, 1: 64-127
     const int row = 16 * sub + (lane & 15);
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
-    const int grp = p.Hq / p.Hkv;
     const float sl2 = a.scale_log2;     // > 0 (checked by the caller)
     int it = 0, k = 0;
     // counters of the tile after this one are read one tile ahead (their load latency
@@ -439,8 +445,6 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     grid_dependency_wait();  // the counters are state a preceding commit writes
     load_counters(blockIdx.x, cnt_next);
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
-      int b, lc, g;
-      tile_coords(t, p, a.lcount, b, lc, g);
       const int ob = it & 1;
       const int64_t len = cnt_next[0];
       const int ring_valid = len < p.W ? int(len) : p.W;
@@ -539,7 +543,27 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         mbar_arrive(&s.p_full[pb]);
       }
       if (!ok) break;
-      // epilogue: O from TMEM over the row sum (the boundary row is one of the summed rows)
+      // the row sum goes to the epilogue warps, which read this tile's O once its last
+      // P V has landed; the softmax goes on with the next tile
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.lsum_free[ob], ((it >> 1) & 1) ^ 1, p.err))) break;
+      if (half == 0) s.lsum_buf[ob][row] = lsum;
+      mbar_arrive(&s.lsum_full[ob]);
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ epilogue
+    const int sub = warp & 3;
+    const int half = lane >> 4;
+    const int row = 16 * sub + (lane & 15);
+    const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
+    const int grp = p.Hq / p.Hkv;
+    int it = 0;
+    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
+      int b, lc, g;
+      tile_coords(t, p, a.lcount, b, lc, g);
+      const int ob = it & 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.lsum_full[ob], (it >> 1) & 1, p.err))) break;
+      const float inv = 1.0f / s.lsum_buf[ob][row];  // the boundary row is one of the summed rows
+      mbar_arrive(&s.lsum_free[ob]);
       if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.o_full[ob], (it >> 1) & 1, p.err))) break;
       tc_fence_after();
       float o[64];
@@ -547,7 +571,6 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       tmem_ld32(trow + kOCol + 64 * ob + 32, o + 32);
       tc_fence_before();
       mbar_arrive(&s.o_free[ob]);
-      const float inv = 1.0f / lsum;
       const int i = row / grp, jj = row - (row / grp) * grp;
       const int64_t orow = (((int64_t(b) * a.lcount + lc) * p.B + i) * p.Hq + g * grp + jj) * 128 + 64 * half;
       if (p.out_f32) {

@@ -238,6 +238,12 @@ __device__ inline uint64_t view_mask(const Dev& p, int r0, int ring_valid, uint6
   return m | range_bits(base + 1, base + 2, r0);       // boundary row, row R
 }
 
+// Work of one CTA: tiles blockIdx.x, blockIdx.x + gridDim.x, ... (each all nC chunks).
+__device__ inline int item_count(const TcArgs& a) {
+  return blockIdx.x < a.n_tiles ? (a.n_tiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+}
+__device__ inline int item_tile(int i) { return int(blockIdx.x) + i * int(gridDim.x); }
+
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMap kv_map,
                  const __grid_constant__ CUtensorMap kv_tail_map, const __grid_constant__ CUtensorMap q_map) {
@@ -254,9 +260,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   const int nC = a.n_chunks;
   const int tail = a.tail_rows;                   // the tile's arena rows in its last chunk
   const int last_rows = (tail + 1 + 15) & ~15;    // rows the last chunk's MMAs take (+ boundary)
-  int my_tiles = 0;
-  for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x) ++my_tiles;
-  const int total = my_tiles * nC;  // chunks this CTA processes, in order
+  const int n_items = item_count(a);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kKStages; ++i) { mbar_init(&s.kfull[i], 1); mbar_init(&s.kempty[i], 1); }
@@ -297,14 +301,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   int issued = 0;  // producers: loads issued into their ring (for the drain after an abort)
-  auto chunk_rows = [&](int k) { return (k % nC) == nC - 1 ? last_rows : kChunk; };
-  auto chunk_y = [&](int k, int t2) {  // first arena row of chunk k's K (t2 = 0) or V (t2 = 1)
-    const int it = k / nC, c = k - it * nC;
-    int b, lc, g;
-    tile_coords(blockIdx.x + it * gridDim.x, p, a.lcount, b, lc, g);
-    const int64_t tile = (int64_t(b) * p.L + (a.lb + lc)) * p.Hkv + g;
-    return int((tile * 2 + t2) * p.R + int64_t(c) * kChunk);
-  };
+  auto chunk_rows = [&](int c) { return c == nC - 1 ? last_rows : kChunk; };
 
   if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------ producers
@@ -324,48 +321,51 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     }
     if (!is_k) grid_dependency_wait();
     const int grp = p.Hq / p.Hkv;
-    uint4 brow = make_uint4(0, 0, 0, 0);
-    for (int k = 0; k < total; ++k) {
-      const int it = k / nC, c = k - it * nC;
-      if (c == 0) {
-        int b, lc, g;
-        tile_coords(blockIdx.x + it * gridDim.x, p, a.lcount, b, lc, g);
-        if (is_k) {  // Q of the tile first
-          const int qb = it & 1;
-          if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_empty[qb], ((it >> 1) & 1) ^ 1, p.err))) break;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&s.q_full[qb], kQBytes);
-            const int zrow = (b * a.lcount + lc) * p.B;
-            tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
-            tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
+    bool ok = true;
+    int k = 0;  // chunks of this CTA so far: ring stage and phase
+    for (int i = 0; i < n_items && ok; ++i) {
+      int b, lc, g;
+      tile_coords(item_tile(i), p, a.lcount, b, lc, g);
+      const int64_t tile = (int64_t(b) * p.L + (a.lb + lc)) * p.Hkv + g;
+      if (is_k) {  // Q of the item first
+        const int qb = i & 1;
+        if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_empty[qb], ((i >> 1) & 1) ^ 1, p.err))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&s.q_full[qb], kQBytes);
+          const int zrow = (b * a.lcount + lc) * p.B;
+          tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
+          tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
+        }
+        // Q is an input; the boundary rows and the arena are state a preceding commit writes
+        if (i == 0) grid_dependency_wait();
+      }
+      uint4 brow = make_uint4(0, 0, 0, 0);
+      if (lane < 16)
+        brow = ld_nc_v4(bsrc + (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + g * 128 + lane * 8);
+      for (int c = 0; c < nC; ++c, ++k) {
+        const int st = k % nst;
+        if (!__all_sync(0xffffffffu, wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err))) { ok = false; break; }
+        unsigned char* dst = ring + st * kStageBytes;
+        const bool last = c == nC - 1;
+        if (last) {  // the boundary row, row `tail` of the stage
+          if (lane < 16)
+            *reinterpret_cast<uint4*>(dst + (lane >> 3) * (kStageBytes / 2) + tail * 128 +
+                                      (((lane & 7) ^ (tail & 7)) << 4)) = brow;
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          const int rows = last ? tail : kChunk;
+          mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
+          if (rows > 0) {
+            const CUtensorMap* m = last ? &kv_tail_map : &kv_map;
+            const int y = int((tile * 2 + (is_k ? 0 : 1)) * p.R + int64_t(c) * kChunk);
+            tma_load_2d(dst, m, 0, y, &fullb[st]);
+            tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
           }
-          // Q is an input; the boundary rows and the arena are state a preceding commit writes
-          if (it == 0) grid_dependency_wait();
         }
-        if (lane < 16) brow = ld_nc_v4(bsrc + (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + g * 128 + lane * 8);
+        ++issued;
       }
-      const int st = k % nst;
-      if (!__all_sync(0xffffffffu, wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err))) break;
-      unsigned char* dst = ring + st * kStageBytes;
-      const bool last = c == nC - 1;
-      if (last) {  // the boundary row, row `tail` of the stage
-        if (lane < 16)
-          *reinterpret_cast<uint4*>(dst + (lane >> 3) * (kStageBytes / 2) + tail * 128 +
-                                    (((lane & 7) ^ (tail & 7)) << 4)) = brow;
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-      if (lane == 0) {
-        const int rows = last ? tail : kChunk;
-        mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
-        if (rows > 0) {
-          const CUtensorMap* m = last ? &kv_tail_map : &kv_map;
-          const int y = chunk_y(k, is_k ? 0 : 1);
-          tma_load_2d(dst, m, 0, y, &fullb[st]);
-          tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
-        }
-      }
-      ++issued;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ QK issuer
@@ -373,26 +373,31 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       // descriptors of the buffers' first bytes; an operand further in adds its offset / 16
       // to the start-address field (shared addresses stay below 256 KB: no carry out)
       const uint64_t dq0 = sdesc(smem_u32(q_buf), 16, 1024), dk0 = sdesc(smem_u32(k_buf), 16, 1024);
-      for (int k = 0; k < total; ++k) {
-        const int it = k / nC, c = k - it * nC, qb = it & 1, sb = k % kSBufs, st = k % kKStages;
-        if (c == 0 && !wait_or_abort(s, &s.q_full[qb], (it >> 1) & 1, p.err)) break;
-        if (!wait_or_abort(s, &s.kfull[st], (k / kKStages) & 1, p.err)) break;
-        if (!wait_or_abort(s, &s.s_free[sb], ((k / kSBufs) & 1) ^ 1, p.err)) break;
-        tc_fence_after();
-        const int rows = chunk_rows(k);
-        const int n0 = rows < 64 ? rows : 64, n1 = rows - n0;
-        const uint32_t id0 = idesc_bf16(n0, false), id1 = idesc_bf16(n1 > 0 ? n1 : 16, false);
-        const uint64_t dq = dq0 + uint32_t(qb * kQBytes >> 4), dk = dk0 + uint32_t(st * kStageBytes >> 4);
+      bool ok = true;
+      int k = 0;
+      for (int i = 0; i < n_items && ok; ++i) {
+        const int qb = i & 1;
+        if (!wait_or_abort(s, &s.q_full[qb], (i >> 1) & 1, p.err)) break;
+        for (int c = 0; c < nC; ++c, ++k) {
+          const int sb = k % kSBufs, st = k % kKStages;
+          if (!wait_or_abort(s, &s.kfull[st], (k / kKStages) & 1, p.err)) { ok = false; break; }
+          if (!wait_or_abort(s, &s.s_free[sb], ((k / kSBufs) & 1) ^ 1, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const int rows = chunk_rows(c);
+          const int n0 = rows < 64 ? rows : 64, n1 = rows - n0;
+          const uint32_t id0 = idesc_bf16(n0, false), id1 = idesc_bf16(n1 > 0 ? n1 : 16, false);
+          const uint64_t dq = dq0 + uint32_t(qb * kQBytes >> 4), dk = dk0 + uint32_t(st * kStageBytes >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t qo = ((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4;
-          const uint32_t ko = ((kk >> 2) * (kStageBytes / 2) + (kk & 3) * 32) >> 4;
-          mma_bf16(tmem + 64 * sb, dq + qo, dk + ko, id0, kk > 0);
-          if (n1 > 0) mma_bf16(tmem + (16u << 16) + 64 * sb, dq + qo, dk + ko + (64 * 128 >> 4), id1, kk > 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t qo = ((kk >> 2) * (kQBytes / 2) + (kk & 3) * 32) >> 4;
+            const uint32_t ko = ((kk >> 2) * (kStageBytes / 2) + (kk & 3) * 32) >> 4;
+            mma_bf16(tmem + 64 * sb, dq + qo, dk + ko, id0, kk > 0);
+            if (n1 > 0) mma_bf16(tmem + (16u << 16) + 64 * sb, dq + qo, dk + ko + (64 * 128 >> 4), id1, kk > 0);
+          }
+          mma_commit(&s.kempty[st]);
+          mma_commit(&s.s_full[sb]);
+          if (c == nC - 1) mma_commit(&s.q_empty[qb]);
         }
-        mma_commit(&s.kempty[st]);
-        mma_commit(&s.s_full[sb]);
-        if (c == nC - 1) mma_commit(&s.q_empty[qb]);
       }
     }
   } else if (warp == 7) {
@@ -401,26 +406,31 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       const uint64_t dp0 = sdesc(smem_u32(p_buf), 16, 1024);
       const uint64_t dv0 = sdesc(smem_u32(v_buf), kStageBytes / 2, 1024);
       const uint32_t id_pv = idesc_bf16(64, true);
-      for (int k = 0; k < total; ++k) {
-        const int it = k / nC, c = k - it * nC, ob = it & 1, pb = k & 1, st = k % kVStages;
-        if (c == 0 && !wait_or_abort(s, &s.o_free[ob], ((it >> 1) & 1) ^ 1, p.err)) break;
-        if (!wait_or_abort(s, &s.vfull[st], (k / kVStages) & 1, p.err)) break;
-        if (!wait_or_abort(s, &s.p_full[pb], (k >> 1) & 1, p.err)) break;
-        tc_fence_after();
-        const uint64_t dv = dv0 + uint32_t(st * kStageBytes >> 4), dp = dp0 + uint32_t(pb * kPBytes >> 4);
-        const int rows = chunk_rows(k);
-        for (int kk = 0; kk < rows / 16; ++kk) {
-          const uint64_t pa = dp + uint32_t(((kk >> 2) * (kPBytes / 2) + (kk & 3) * 32) >> 4);
-          const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
-          // V: rows = keys (K dim), 128-byte rows per 64-column half: MN-major B, SBO = 8 rows
-          mma_bf16(tmem + kOCol + 64 * ob, pa, dv + uint32_t(kk * 2048 >> 4), id_pv, acc);
-          mma_bf16(tmem + (16u << 16) + kOCol + 64 * ob, pa, dv + uint32_t((kStageBytes / 2 + kk * 2048) >> 4), id_pv,
-                   acc);
+      bool ok = true;
+      int k = 0;
+      for (int i = 0; i < n_items && ok; ++i) {
+        const int ob = i & 1;
+        if (!wait_or_abort(s, &s.o_free[ob], ((i >> 1) & 1) ^ 1, p.err)) break;
+        for (int c = 0; c < nC; ++c, ++k) {
+          const int pb = k & 1, st = k % kVStages;
+          if (!wait_or_abort(s, &s.vfull[st], (k / kVStages) & 1, p.err)) { ok = false; break; }
+          if (!wait_or_abort(s, &s.p_full[pb], (k >> 1) & 1, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t dv = dv0 + uint32_t(st * kStageBytes >> 4), dp = dp0 + uint32_t(pb * kPBytes >> 4);
+          const int rows = chunk_rows(c);
+          for (int kk = 0; kk < rows / 16; ++kk) {
+            const uint64_t pa = dp + uint32_t(((kk >> 2) * (kPBytes / 2) + (kk & 3) * 32) >> 4);
+            const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+            // V: rows = keys (K dim), 128-byte rows per 64-column half: MN-major B, SBO = 8 rows
+            mma_bf16(tmem + kOCol + 64 * ob, pa, dv + uint32_t(kk * 2048 >> 4), id_pv, acc);
+            mma_bf16(tmem + (16u << 16) + kOCol + 64 * ob, pa, dv + uint32_t((kStageBytes / 2 + kk * 2048) >> 4),
+                     id_pv, acc);
+          }
+          mma_commit(&s.vempty[st]);
+          mma_commit(&s.p_empty[pb]);
+          mma_commit(&s.pv_done);
+          if (c == nC - 1) mma_commit(&s.o_full[ob]);
         }
-        mma_commit(&s.vempty[st]);
-        mma_commit(&s.p_empty[pb]);
-        mma_commit(&s.pv_done);
-        if (c == nC - 1) mma_commit(&s.o_full[ob]);
       }
     }
   } else if (warp >= 2 && warp <= 5) {
@@ -430,22 +440,22 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     const int row = 16 * sub + (lane & 15);
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
     const float sl2 = a.scale_log2;     // > 0 (checked by the caller)
-    int it = 0, k = 0;
-    // counters of the tile after this one are read one tile ahead (their load latency
-    // then never sits between two tiles)
-    auto load_counters = [&](int t, int64_t* dst) {
-      if (t >= a.n_tiles) return;
+    // counters of the next item's tile are read one item ahead (their load latency then
+    // never sits between two items)
+    auto load_counters = [&](int i, int64_t* dst) {
+      if (i >= n_items) return;
       int b, lc, g;
-      tile_coords(t, p, a.lcount, b, lc, g);
+      tile_coords(item_tile(i), p, a.lcount, b, lc, g);
       const int64_t* ctr = p.counters + (int64_t(b) * p.L + a.lb + lc) * (1 + p.nsc);
 #pragma unroll
       for (int kk = 0; kk <= kMaxScales; ++kk) dst[kk] = kk <= p.nsc ? ctr[kk] : 0;
     };
     int64_t cnt_next[kMaxScales + 1];
     grid_dependency_wait();  // the counters are state a preceding commit writes
-    load_counters(blockIdx.x, cnt_next);
-    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
-      const int ob = it & 1;
+    load_counters(0, cnt_next);
+    int k = 0;
+    for (int i = 0; i < n_items; ++i) {
+      const int ob = i & 1;
       const int64_t len = cnt_next[0];
       const int ring_valid = len < p.W ? int(len) : p.W;
       uint64_t sinfo = 0;
@@ -458,7 +468,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           sinfo |= e << (16 * kk);
         }
       }
-      load_counters(t + gridDim.x, cnt_next);
+      load_counters(i + 1, cnt_next);
 
       float mref = -INFINITY;  // reference max (log2 units) the P values are taken against
       float lsum = 0.f;        // sum of the rows' weights against mref
@@ -482,12 +492,12 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
         if (all_valid) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+          for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], sv[e]);
         } else {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            if (!((vm >> i) & 1ull)) sv[i] = -INFINITY;
-            mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+          for (int e = 0; e < 64; ++e) {
+            if (!((vm >> e) & 1ull)) sv[e] = -INFINITY;
+            mx8[e & 7] = fmaxf(mx8[e & 7], sv[e]);
           }
         }
         float cmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
@@ -510,7 +520,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           for (int h2 = 0; h2 < 2; ++h2) {
             tmem_ld32(trow + kOCol + 64 * ob + 32 * h2, ov);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
             tmem_st32(trow + kOCol + 64 * ob + 32 * h2, ov);
           }
           tc_fence_before();
@@ -525,11 +535,11 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         for (int u = 0; u < 8; ++u) ps8[u] = 0.f;
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const float p0 = ex2(fmaf(sv[i], sl2, -mu));
-          const float p1 = ex2(fmaf(sv[i + 1], sl2, -mu));
-          ps8[(i >> 1) & 7] += p0 + p1;
-          pk[i >> 1] = pack_bf16(p0, p1);
+        for (int e = 0; e < 64; e += 2) {
+          const float p0 = ex2(fmaf(sv[e], sl2, -mu));
+          const float p1 = ex2(fmaf(sv[e + 1], sl2, -mu));
+          ps8[(e >> 1) & 7] += p0 + p1;
+          pk[e >> 1] = pack_bf16(p0, p1);
         }
         const float psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
         lsum += psum + __shfl_xor_sync(0xffffffffu, psum, 16);
@@ -545,47 +555,54 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       if (!ok) break;
       // the row sum goes to the epilogue warps, which read this tile's O once its last
       // P V has landed; the softmax goes on with the next tile
-      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.lsum_free[ob], ((it >> 1) & 1) ^ 1, p.err))) break;
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.lsum_free[ob], ((i >> 1) & 1) ^ 1, p.err))) break;
       if (half == 0) s.lsum_buf[ob][row] = lsum;
       mbar_arrive(&s.lsum_full[ob]);
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------ epilogue
+    // Each thread owns an output slice (row, half): 64 columns of one row.
     const int sub = warp & 3;
     const int half = lane >> 4;
     const int row = 16 * sub + (lane & 15);
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
     const int grp = p.Hq / p.Hkv;
-    int it = 0;
-    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++it) {
+    const int qi = row / grp, jj = row - qi * grp;
+    // 32 output columns (col0 + 0..31 of this thread's 64) of the slice, times inv
+    auto store32 = [&](const float* v, float inv, int b, int lc, int g, int col0) {
+      const int64_t orow =
+          (((int64_t(b) * a.lcount + lc) * p.B + qi) * p.Hq + g * grp + jj) * 128 + 64 * half + col0;
+      if (p.out_f32) {
+        float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          o4[u] = make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
+      } else {
+        uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          o4[u] = make_uint4(pack_bf16(v[8 * u] * inv, v[8 * u + 1] * inv), pack_bf16(v[8 * u + 2] * inv, v[8 * u + 3] * inv),
+                             pack_bf16(v[8 * u + 4] * inv, v[8 * u + 5] * inv),
+                             pack_bf16(v[8 * u + 6] * inv, v[8 * u + 7] * inv));
+      }
+    };
+    for (int i = 0; i < n_items; ++i) {
       int b, lc, g;
-      tile_coords(t, p, a.lcount, b, lc, g);
-      const int ob = it & 1;
-      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.lsum_full[ob], (it >> 1) & 1, p.err))) break;
-      const float inv = 1.0f / s.lsum_buf[ob][row];  // the boundary row is one of the summed rows
+      tile_coords(item_tile(i), p, a.lcount, b, lc, g);
+      const int ob = i & 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.lsum_full[ob], (i >> 1) & 1, p.err))) break;
+      const float lsum = s.lsum_buf[ob][row];  // the boundary row is one of the summed rows
       mbar_arrive(&s.lsum_free[ob]);
-      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.o_full[ob], (it >> 1) & 1, p.err))) break;
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.o_full[ob], (i >> 1) & 1, p.err))) break;
       tc_fence_after();
       float o[64];
       tmem_ld32(trow + kOCol + 64 * ob, o);
       tmem_ld32(trow + kOCol + 64 * ob + 32, o + 32);
       tc_fence_before();
       mbar_arrive(&s.o_free[ob]);
-      const int i = row / grp, jj = row - (row / grp) * grp;
-      const int64_t orow = (((int64_t(b) * a.lcount + lc) * p.B + i) * p.Hq + g * grp + jj) * 128 + 64 * half;
-      if (p.out_f32) {
-        float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow);
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          o4[u] = make_float4(o[4 * u] * inv, o[4 * u + 1] * inv, o[4 * u + 2] * inv, o[4 * u + 3] * inv);
-      } else {
-        uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          o4[u] = make_uint4(pack_bf16(o[8 * u] * inv, o[8 * u + 1] * inv), pack_bf16(o[8 * u + 2] * inv, o[8 * u + 3] * inv),
-                             pack_bf16(o[8 * u + 4] * inv, o[8 * u + 5] * inv),
-                             pack_bf16(o[8 * u + 6] * inv, o[8 * u + 7] * inv));
-      }
+      const float inv = 1.0f / lsum;
+      store32(o, inv, b, lc, g, 0);
+      store32(o + 32, inv, b, lc, g, 32);
     }
   }
 
@@ -684,8 +701,10 @@ cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcoun
   a.bstride = bstride;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
+  // one CTA per SM, tiles round robin
+  const int grid = a.n_tiles < sms ? a.n_tiles : sms;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(a.n_tiles < sms ? a.n_tiles : sms);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;

@@ -23,6 +23,7 @@ all ranks (weak scaling: every rank owns its own batch of 16 sequences).
 from __future__ import annotations
 
 import argparse
+import glob
 import hashlib
 import json
 import math
@@ -114,9 +115,10 @@ def hbm_peak():
 
 
 def kernel_source_sha(name: str) -> str:
-    p = os.path.join(ROOT, "fixed_cost_drafter_b200", "csrc", name)
+    """Hash of a kernel's source file and every shared header it may include."""
+    csrc = os.path.join(ROOT, "fixed_cost_drafter_b200", "csrc")
     h = hashlib.sha256()
-    for q in (p, os.path.join(ROOT, "fixed_cost_drafter_b200", "csrc", "ls_common.cuh")):
+    for q in [os.path.join(csrc, name)] + sorted(glob.glob(os.path.join(csrc, "*.cuh"))):
         with open(q, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

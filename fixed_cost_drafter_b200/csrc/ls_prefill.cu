@@ -133,6 +133,21 @@ prefill_units_kernel(Dev p, PrefillArgs a) {
   cursor_settle(a, p, cons);
   int consumed = 0;
 
+  // this thread's column vectors (fixed for the whole kernel): K (0) or V (1), head,
+  // element offset in the head, byte offset in the row
+  bool col_ok[CVT];
+  int col_t[CVT], col_h[CVT], col_d0[CVT], col_byte[CVT], col_kv[CVT];
+#pragma unroll
+  for (int q = 0; q < CVT; ++q) {
+    const int cv = tid + q * kPrefillThreads;
+    col_ok[q] = cv < ncv;
+    const int t = cv / cvPerRow, e0 = (cv - t * cvPerRow) * VEC;
+    col_t[q] = t;
+    col_h[q] = e0 / p.D;
+    col_d0[q] = e0 - col_h[q] * p.D;
+    col_byte[q] = e0 * int(sizeof(T));
+    col_kv[q] = col_h[q] * 2 + t;  // (head, K|V) tile-plane index within the (sequence, layer)
+  }
   float acc[CVT][kMaxScales + 1][VEC];
   int cnt[kMaxScales];  // rows (k = 0) or closes of scale k-1 until scale k closes
   int cur_item = -1;
@@ -163,55 +178,51 @@ prefill_units_kernel(Dev p, PrefillArgs a) {
     if (__syncthreads_or(!ok)) { timed_out = true; break; }
 
     const char* st = smem + buf * stageBytes;
+    // ring-window rows of this stage: positions >= P - W go to ring slot pos mod W
+    const int64_t wfirst = P - p.W > g0 ? P - p.W - g0 : 0;  // first stage row in the window
+    int wslot = wfirst < nrows ? int((g0 + wfirst) % p.W) : 0;
     for (int r = 0; r < nrows; ++r) {
-      const int64_t pos = g0 + r;
-      const bool in_window = pos >= P - p.W;
 #pragma unroll
       for (int q = 0; q < CVT; ++q) {
-        const int cv = tid + q * kPrefillThreads;
-        if (cv >= ncv) break;
-        const int t = cv / cvPerRow;
-        const int e0 = (cv - t * cvPerRow) * VEC;
-        const uint4 raw = *reinterpret_cast<const uint4*>(st + (t * a.G + r) * rowBytes + e0 * int(sizeof(T)));
+        if (!col_ok[q]) continue;
+        const uint4 raw = *reinterpret_cast<const uint4*>(st + (col_t[q] * a.G + r) * rowBytes + col_byte[q]);
         float f[VEC];
         E::to_f32(raw, f);
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[q][0][e] += f[e];
-        if (in_window) {
-          const int h = e0 / p.D, d0 = e0 - h * p.D;
-          const int64_t tile = int64_t(bl) * p.Hkv + h;
-          T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + t) * int64_t(p.R) * p.D;
-          *reinterpret_cast<uint4*>(kvt + int64_t(pos % p.W) * p.D + d0) = raw;
+        if (r >= wfirst) {
+          T* kvt = reinterpret_cast<T*>(p.kv) + (int64_t(bl) * p.Hkv * 2 + col_kv[q]) * int64_t(p.R) * p.D;
+          *reinterpret_cast<uint4*>(kvt + int64_t(wslot) * p.D + col_d0[q]) = raw;
         }
       }
+      if (r >= wfirst && ++wslot == p.W) wslot = 0;
+      if (--cnt[0] != 0) continue;  // no segment of the smallest scale closes at this row
       // segment closes, smallest scale first; a closed scale feeds the next one
+      const int64_t pos = g0 + r;
 #pragma unroll
       for (int k = 0; k < kMaxScales; ++k) {
         if (k >= a.kU) break;
-        if (--cnt[k] != 0) break;  // level k counts closes of level k-1 (rows for k = 0)
+        if (k > 0 && --cnt[k] != 0) break;  // level k counts closes of level k-1
         cnt[k] = k == 0 ? p.scales[0] : p.scales[k] / p.scales[k - 1];
         const int s = p.scales[k];
         const int64_t j = pos / s;  // segment that just closed
         const bool keep = j >= P / s - p.slots;
 #pragma unroll
         for (int q = 0; q < CVT; ++q) {
+          if (!col_ok[q]) continue;
           const int cv = tid + q * kPrefillThreads;
-          if (cv >= ncv) break;
-          const int t = cv / cvPerRow;
-          const int e0 = (cv - t * cvPerRow) * VEC;
-          const int h = e0 / p.D, d0 = e0 - h * p.D;
-          const int64_t tile = int64_t(bl) * p.Hkv + h;
+          const int64_t tile = int64_t(bl) * p.Hkv + col_h[q];
           if (keep) {
             float m[VEC];
 #pragma unroll
             for (int e = 0; e < VEC; ++e) m[e] = acc[q][k][e] / float(s);
             const int slot = int(j % p.slots);
-            float* sg = p.seg + (((tile * p.nsc + k) * p.slots + slot) * 2 + t) * p.D + d0;
+            float* sg = p.seg + (((tile * p.nsc + k) * p.slots + slot) * 2 + col_t[q]) * p.D + col_d0[q];
 #pragma unroll
             for (int e = 0; e < VEC; e += 4)
               *reinterpret_cast<float4*>(sg + e) = make_float4(m[e], m[e + 1], m[e + 2], m[e + 3]);
-            T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + t) * int64_t(p.R) * p.D;
-            *reinterpret_cast<uint4*>(kvt + (int64_t(p.W) + k * (p.slots + 1) + slot) * p.D + d0) =
+            T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + col_t[q]) * int64_t(p.R) * p.D;
+            *reinterpret_cast<uint4*>(kvt + (int64_t(p.W) + k * (p.slots + 1) + slot) * p.D + col_d0[q]) =
                 E::from_f32(m);
           }
           if (k + 1 < a.kU) {

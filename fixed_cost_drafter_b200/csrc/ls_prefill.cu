@@ -2,10 +2,12 @@
 // Figure 3 caption ("initialized over the full prefix during target prefill").
 //
 // Pass 1 (prefill_units_kernel, persistent, one CTA per SM): the work items are units
-// of U prefix rows of one (sequence, layer); U is the largest scale <= 512. The TMA
-// engine streams each unit's K and V rows (all KV heads of a row are contiguous) into a
-// ring of shared-memory stages with cp.async.bulk + mbarrier transaction counts; every
-// thread owns one 16-byte column vector and keeps one fp32 sum per scale <= U. When a
+// of U prefix rows of one (sequence, layer); U is the largest scale <= 512. A producer
+// warp streams each unit's K and V rows (all KV heads of a row are contiguous) through
+// the TMA engine into a ring of shared-memory stages (cp.async.bulk + mbarrier
+// transaction counts; the consumers release a stage through an "empty" mbarrier, no
+// block-wide barrier); every consumer thread owns one 16-byte column vector and keeps
+// one fp32 sum per scale <= U, adding rows in runs between segment closes. When a
 // segment of scale s_k closes, its sum is added into the next scale's sum (a tree,
 // not a long serial chain) and, if the segment is among the `slots` most recent ones of
 // the final prefix, its mean is written. A closed unit's sum goes to the workspace.
@@ -33,7 +35,8 @@ struct PrefillArgs {
   int32_t n_items;  // b * L * n_units
 };
 
-constexpr int kPrefillThreads = 256;
+constexpr int kPrefillThreads = 256;                 // consumer threads
+constexpr int kPrefillBlock = kPrefillThreads + 32;  // + one producer warp
 constexpr int kPrefillStages = 3;
 
 __device__ inline int64_t clamp_prefix(const PrefillArgs& a, const Dev&, int b) {
@@ -76,12 +79,13 @@ __device__ inline void cursor_next(const PrefillArgs& a, const Dev& p, Cursor& c
 }
 
 template <typename T, int CVT>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+__global__ void __launch_bounds__(kPrefillBlock, 1)
 prefill_units_kernel(Dev p, PrefillArgs a) {
   using E = Elem<T>;
   constexpr int VEC = E::kVec;
   extern __shared__ __align__(128) char smem[];
-  __shared__ uint64_t full[kPrefillStages];
+  __shared__ uint64_t full[kPrefillStages], empty[kPrefillStages];
+  __shared__ uint32_t abort_flag;
 
   const int rowElems = p.Hkv * p.D;
   const int rowBytes = rowElems * int(sizeof(T));
@@ -91,210 +95,233 @@ prefill_units_kernel(Dev p, PrefillArgs a) {
   const int tid = threadIdx.x;
 
   if (tid == 0) {
-    for (int s = 0; s < kPrefillStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < kPrefillStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kPrefillThreads); }
+    abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
+  // bounded wait that also gives up once another thread has given up
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+#pragma unroll 1
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if ((i & 1023) == 1023 && *reinterpret_cast<volatile uint32_t*>(&abort_flag)) return false;
+    }
+    set_err(p.err, LS_DEVERR_WAIT_TIMEOUT);
+    *reinterpret_cast<volatile uint32_t*>(&abort_flag) = 1;
+    return false;
+  };
 
-  // producer: thread 0 issues stage n into buffer n % kPrefillStages
-  Cursor prod{0, 0, false};
-  int issued = 0;
-  auto issue = [&](Cursor& c, int n) {
-    const int it = blockIdx.x + c.j * gridDim.x;
-    int bl, u; int64_t r0, r1;
-    item_rows(a, p, it, bl, u, r0, r1);
-    const int64_t g0 = r0 + int64_t(c.grp) * a.G;
-    const int nrows = int(min(int64_t(a.G), r1 - g0));
-    char* dst = smem + (n % kPrefillStages) * stageBytes;
-    uint64_t* bar = &full[n % kPrefillStages];
-    mbar_arrive_expect_tx(bar, uint32_t(2 * nrows * rowBytes));
-    for (int t = 0; t < 2; ++t) {
-      const char* base = (t == 0 ? a.k : a.v) +
-                         (int64_t(bl) * a.plane_stride + (g0 - a.row_begin) * a.row_stride) * int64_t(sizeof(T));
-      char* d = dst + t * a.G * rowBytes;
-      if (a.row_stride == rowElems) {
-        bulk_g2s(d, base, uint32_t(nrows * rowBytes), bar);
-      } else {
-        for (int r = 0; r < nrows; ++r)
-          bulk_g2s(d + r * rowBytes, base + int64_t(r) * a.row_stride * int64_t(sizeof(T)),
-                   uint32_t(rowBytes), bar);
+  if (tid >= kPrefillThreads) {
+    // ------------------------------------------------------------ producer (one lane)
+    // stage n goes into buffer n % kPrefillStages once the consumers released it
+    if (tid == kPrefillThreads) {
+      Cursor prod{0, 0, false};
+      cursor_settle(a, p, prod);
+      int n = 0;
+      int last_issue[kPrefillStages];
+      for (int s = 0; s < kPrefillStages; ++s) last_issue[s] = -1;
+      for (; prod.valid; ++n) {
+        const int buf = n % kPrefillStages;
+        if (!wait(&empty[buf], ((n / kPrefillStages) & 1) ^ 1)) break;
+        fence_proxy_async_smem();  // the consumers' reads of the buffer come before its refill
+        const int it = blockIdx.x + prod.j * gridDim.x;
+        int bl, u; int64_t r0, r1;
+        item_rows(a, p, it, bl, u, r0, r1);
+        const int64_t g0 = r0 + int64_t(prod.grp) * a.G;
+        const int nrows = int(min(int64_t(a.G), r1 - g0));
+        char* dst = smem + buf * stageBytes;
+        mbar_arrive_expect_tx(&full[buf], uint32_t(2 * nrows * rowBytes));
+        for (int t = 0; t < 2; ++t) {
+          const char* base = (t == 0 ? a.k : a.v) +
+                             (int64_t(bl) * a.plane_stride + (g0 - a.row_begin) * a.row_stride) * int64_t(sizeof(T));
+          char* d = dst + t * a.G * rowBytes;
+          if (a.row_stride == rowElems) {
+            bulk_g2s(d, base, uint32_t(nrows * rowBytes), &full[buf]);
+          } else {
+            for (int r = 0; r < nrows; ++r)
+              bulk_g2s(d + r * rowBytes, base + int64_t(r) * a.row_stride * int64_t(sizeof(T)), uint32_t(rowBytes),
+                       &full[buf]);
+          }
+        }
+        last_issue[buf] = n;
+        cursor_next(a, p, prod);
+      }
+      if (*reinterpret_cast<volatile uint32_t*>(&abort_flag)) {
+        // let every copy still in flight land before the CTA's shared memory goes away
+        for (int s = 0; s < kPrefillStages; ++s)
+          if (last_issue[s] >= 0)
+            mbar_wait_bounded(&full[s], uint32_t((last_issue[s] / kPrefillStages) & 1), kWaitLimit);
       }
     }
-  };
-  if (tid == 0) {
-    cursor_settle(a, p, prod);
-    for (; issued < kPrefillStages && prod.valid; ++issued) {
-      issue(prod, issued);
-      cursor_next(a, p, prod);
+  } else {
+    // ------------------------------------------------------------ consumers
+    // this thread's column vectors (fixed for the whole kernel): K (0) or V (1), head,
+    // element offset in the head, byte offset in the row
+    bool col_ok[CVT];
+    int col_t[CVT], col_h[CVT], col_d0[CVT], col_byte[CVT], col_kv[CVT];
+#pragma unroll
+    for (int q = 0; q < CVT; ++q) {
+      const int cv = tid + q * kPrefillThreads;
+      col_ok[q] = cv < ncv;
+      const int t = cv / cvPerRow, e0 = (cv - t * cvPerRow) * VEC;
+      col_t[q] = t;
+      col_h[q] = e0 / p.D;
+      col_d0[q] = e0 - col_h[q] * p.D;
+      col_byte[q] = e0 * int(sizeof(T));
+      col_kv[q] = col_h[q] * 2 + t;  // (head, K|V) plane of the (sequence, layer)
     }
-  }
+    Cursor cons{0, 0, false};
+    cursor_settle(a, p, cons);
+    int consumed = 0;
+    float acc[CVT][kMaxScales + 1][VEC];
+    int cnt[kMaxScales];  // rows (k = 0) or closes of scale k-1 until scale k closes
+    int cur_item = -1;
 
-  Cursor cons{0, 0, false};
-  cursor_settle(a, p, cons);
-  int consumed = 0;
+    while (cons.valid) {
+      const int it = blockIdx.x + cons.j * gridDim.x;
+      int bl, u; int64_t r0, r1;
+      item_rows(a, p, it, bl, u, r0, r1);
+      const int b = bl / p.L;
+      const int64_t P = clamp_prefix(a, p, b);
+      if (it != cur_item) {  // new item: all sums start empty (r0 is a multiple of U)
+        cur_item = it;
+#pragma unroll
+        for (int q = 0; q < CVT; ++q)
+#pragma unroll
+          for (int k = 0; k <= kMaxScales; ++k)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[q][k][e] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxScales; ++k)
+          cnt[k] = k >= a.kU ? 0 : (k == 0 ? p.scales[0] : p.scales[k] / p.scales[k - 1]);
+      }
+      const int64_t g0 = r0 + int64_t(cons.grp) * a.G;
+      const int nrows = int(min(int64_t(a.G), r1 - g0));
+      const int buf = consumed % kPrefillStages;
+      if (!wait(&full[buf], uint32_t((consumed / kPrefillStages) & 1))) break;
 
-  // this thread's column vectors (fixed for the whole kernel): K (0) or V (1), head,
-  // element offset in the head, byte offset in the row
-  bool col_ok[CVT];
-  int col_t[CVT], col_h[CVT], col_d0[CVT], col_byte[CVT], col_kv[CVT];
+      const char* st = smem + buf * stageBytes;
+      // rows >= wfirst of this stage are among the prefix's last W: ring slot pos mod W
+      const int64_t wf = P - p.W > g0 ? P - p.W - g0 : 0;
+      const int wfirst = wf < nrows ? int(wf) : nrows;
+      int wslot = wfirst < nrows ? int((g0 + wfirst) % p.W) : 0;
+      int r = 0;
+      while (r < nrows) {
+        // rows up to and including the next close of the smallest scale
+        const int run = nrows - r < cnt[0] ? nrows - r : cnt[0];
+        const int rend = r + run;
+        if (rend <= wfirst) {  // no ring-window row in this run
+#pragma unroll 4
+          for (; r < rend; ++r) {
 #pragma unroll
-  for (int q = 0; q < CVT; ++q) {
-    const int cv = tid + q * kPrefillThreads;
-    col_ok[q] = cv < ncv;
-    const int t = cv / cvPerRow, e0 = (cv - t * cvPerRow) * VEC;
-    col_t[q] = t;
-    col_h[q] = e0 / p.D;
-    col_d0[q] = e0 - col_h[q] * p.D;
-    col_byte[q] = e0 * int(sizeof(T));
-    col_kv[q] = col_h[q] * 2 + t;  // (head, K|V) tile-plane index within the (sequence, layer)
-  }
-  float acc[CVT][kMaxScales + 1][VEC];
-  int cnt[kMaxScales];  // rows (k = 0) or closes of scale k-1 until scale k closes
-  int cur_item = -1;
-  bool timed_out = false;
-
-  while (cons.valid) {
-    const int it = blockIdx.x + cons.j * gridDim.x;
-    int bl, u; int64_t r0, r1;
-    item_rows(a, p, it, bl, u, r0, r1);
-    const int b = bl / p.L;
-    const int64_t P = clamp_prefix(a, p, b);
-    if (it != cur_item) {  // new item: all sums start empty (r0 is a multiple of U)
-      cur_item = it;
+            for (int q = 0; q < CVT; ++q) {
+              if (!col_ok[q]) continue;
+              const uint4 raw = *reinterpret_cast<const uint4*>(st + (col_t[q] * a.G + r) * rowBytes + col_byte[q]);
+              float f[VEC];
+              E::to_f32(raw, f);
 #pragma unroll
-      for (int q = 0; q < CVT; ++q)
+              for (int e = 0; e < VEC; ++e) acc[q][0][e] += f[e];
+            }
+          }
+        } else {
+          for (; r < rend; ++r) {
 #pragma unroll
-        for (int k = 0; k <= kMaxScales; ++k)
+            for (int q = 0; q < CVT; ++q) {
+              if (!col_ok[q]) continue;
+              const uint4 raw = *reinterpret_cast<const uint4*>(st + (col_t[q] * a.G + r) * rowBytes + col_byte[q]);
+              float f[VEC];
+              E::to_f32(raw, f);
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) acc[q][k][e] = 0.f;
+              for (int e = 0; e < VEC; ++e) acc[q][0][e] += f[e];
+              if (r >= wfirst) {
+                T* kvt = reinterpret_cast<T*>(p.kv) + (int64_t(bl) * p.Hkv * 2 + col_kv[q]) * int64_t(p.R) * p.D;
+                *reinterpret_cast<uint4*>(kvt + int64_t(wslot) * p.D + col_d0[q]) = raw;
+              }
+            }
+            if (r >= wfirst && ++wslot == p.W) wslot = 0;
+          }
+        }
+        cnt[0] -= run;
+        if (cnt[0] != 0) break;  // r == nrows: no close in the rest of the stage
+        // segment closes at row rend - 1, smallest scale first; a closed scale feeds the next
+        const int64_t pos = g0 + rend - 1;
 #pragma unroll
-      for (int k = 0; k < kMaxScales; ++k)
-        cnt[k] = k >= a.kU ? 0 : (k == 0 ? p.scales[0] : p.scales[k] / p.scales[k - 1]);
-    }
-    const int64_t g0 = r0 + int64_t(cons.grp) * a.G;
-    const int nrows = int(min(int64_t(a.G), r1 - g0));
-    const int buf = consumed % kPrefillStages;
-    const bool ok = mbar_wait_bounded(&full[buf], uint32_t((consumed / kPrefillStages) & 1), kWaitLimit);
-    if (__syncthreads_or(!ok)) { timed_out = true; break; }
-
-    const char* st = smem + buf * stageBytes;
-    // ring-window rows of this stage: positions >= P - W go to ring slot pos mod W
-    const int64_t wfirst = P - p.W > g0 ? P - p.W - g0 : 0;  // first stage row in the window
-    int wslot = wfirst < nrows ? int((g0 + wfirst) % p.W) : 0;
-    for (int r = 0; r < nrows; ++r) {
+        for (int k = 0; k < kMaxScales; ++k) {
+          if (k >= a.kU) break;
+          if (k > 0 && --cnt[k] != 0) break;  // level k counts closes of level k-1
+          cnt[k] = k == 0 ? p.scales[0] : p.scales[k] / p.scales[k - 1];
+          const int s = p.scales[k];
+          const int64_t j = pos / s;  // segment that just closed
+          const bool keep = j >= P / s - p.slots;
 #pragma unroll
-      for (int q = 0; q < CVT; ++q) {
-        if (!col_ok[q]) continue;
-        const uint4 raw = *reinterpret_cast<const uint4*>(st + (col_t[q] * a.G + r) * rowBytes + col_byte[q]);
-        float f[VEC];
-        E::to_f32(raw, f);
+          for (int q = 0; q < CVT; ++q) {
+            if (!col_ok[q]) continue;
+            const int cv = tid + q * kPrefillThreads;
+            const int64_t tile = int64_t(bl) * p.Hkv + col_h[q];
+            if (keep) {
+              float m[VEC];
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[q][0][e] += f[e];
-        if (r >= wfirst) {
-          T* kvt = reinterpret_cast<T*>(p.kv) + (int64_t(bl) * p.Hkv * 2 + col_kv[q]) * int64_t(p.R) * p.D;
-          *reinterpret_cast<uint4*>(kvt + int64_t(wslot) * p.D + col_d0[q]) = raw;
+              for (int e = 0; e < VEC; ++e) m[e] = acc[q][k][e] / float(s);
+              const int slot = int(j % p.slots);
+              float* sg = p.seg + (((tile * p.nsc + k) * p.slots + slot) * 2 + col_t[q]) * p.D + col_d0[q];
+#pragma unroll
+              for (int e = 0; e < VEC; e += 4)
+                *reinterpret_cast<float4*>(sg + e) = make_float4(m[e], m[e + 1], m[e + 2], m[e + 3]);
+              T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + col_t[q]) * int64_t(p.R) * p.D;
+              *reinterpret_cast<uint4*>(kvt + (int64_t(p.W) + k * (p.slots + 1) + slot) * p.D + col_d0[q]) =
+                  E::from_f32(m);
+            }
+            if (k + 1 < a.kU) {
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) { acc[q][k + 1][e] += acc[q][k][e]; acc[q][k][e] = 0.f; }
+            } else {  // the unit closed: its sum goes to the workspace
+              float* w = a.ws + (int64_t(bl) * a.n_units + u) * (2 * rowElems) + int64_t(cv) * VEC;
+#pragma unroll
+              for (int e = 0; e < VEC; e += 4)
+                *reinterpret_cast<float4*>(w + e) =
+                    make_float4(acc[q][k][e], acc[q][k][e + 1], acc[q][k][e + 2], acc[q][k][e + 3]);
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) acc[q][k][e] = 0.f;
+            }
+          }
         }
       }
-      if (r >= wfirst && ++wslot == p.W) wslot = 0;
-      if (--cnt[0] != 0) continue;  // no segment of the smallest scale closes at this row
-      // segment closes, smallest scale first; a closed scale feeds the next one
-      const int64_t pos = g0 + r;
-#pragma unroll
-      for (int k = 0; k < kMaxScales; ++k) {
-        if (k >= a.kU) break;
-        if (k > 0 && --cnt[k] != 0) break;  // level k counts closes of level k-1
-        cnt[k] = k == 0 ? p.scales[0] : p.scales[k] / p.scales[k - 1];
-        const int s = p.scales[k];
-        const int64_t j = pos / s;  // segment that just closed
-        const bool keep = j >= P / s - p.slots;
+      mbar_arrive(&empty[buf]);  // this thread's reads of the stage are done
+
+      if (g0 + nrows == r1) {  // the item ends with this stage
+        const bool unit_closed = r1 - r0 == a.U;
 #pragma unroll
         for (int q = 0; q < CVT; ++q) {
           if (!col_ok[q]) continue;
           const int cv = tid + q * kPrefillThreads;
           const int64_t tile = int64_t(bl) * p.Hkv + col_h[q];
-          if (keep) {
-            float m[VEC];
+          float run[VEC];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) m[e] = acc[q][k][e] / float(s);
-            const int slot = int(j % p.slots);
-            float* sg = p.seg + (((tile * p.nsc + k) * p.slots + slot) * 2 + col_t[q]) * p.D + col_d0[q];
+          for (int e = 0; e < VEC; ++e) run[e] = 0.f;
 #pragma unroll
-            for (int e = 0; e < VEC; e += 4)
-              *reinterpret_cast<float4*>(sg + e) = make_float4(m[e], m[e + 1], m[e + 2], m[e + 3]);
-            T* kvt = reinterpret_cast<T*>(p.kv) + (tile * 2 + col_t[q]) * int64_t(p.R) * p.D;
-            *reinterpret_cast<uint4*>(kvt + (int64_t(p.W) + k * (p.slots + 1) + slot) * p.D + col_d0[q]) =
-                E::from_f32(m);
+          for (int k = 0; k < kMaxScales; ++k) {
+            if (k >= a.kU) break;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) run[e] += acc[q][k][e];
+            if (r1 == P) {  // the sequence's prefix ends here: open partial of scale k
+              float* pp = p.part + ((tile * p.nsc + k) * 2 + col_t[q]) * p.D + col_d0[q];
+#pragma unroll
+              for (int e = 0; e < VEC; e += 4)
+                *reinterpret_cast<float4*>(pp + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
+            }
           }
-          if (k + 1 < a.kU) {
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) { acc[q][k + 1][e] += acc[q][k][e]; acc[q][k][e] = 0.f; }
-          } else {  // the unit closed: its sum goes to the workspace
+          if (!unit_closed) {
             float* w = a.ws + (int64_t(bl) * a.n_units + u) * (2 * rowElems) + int64_t(cv) * VEC;
 #pragma unroll
             for (int e = 0; e < VEC; e += 4)
-              *reinterpret_cast<float4*>(w + e) =
-                  make_float4(acc[q][k][e], acc[q][k][e + 1], acc[q][k][e + 2], acc[q][k][e + 3]);
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) acc[q][k][e] = 0.f;
+              *reinterpret_cast<float4*>(w + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
           }
         }
       }
+      ++consumed;
+      cursor_next(a, p, cons);
     }
-
-    const bool item_ends = g0 + nrows == r1;
-    if (item_ends) {
-      const bool unit_closed = r1 - r0 == a.U;
-#pragma unroll
-      for (int q = 0; q < CVT; ++q) {
-        const int cv = tid + q * kPrefillThreads;
-        if (cv >= ncv) break;
-        const int t = cv / cvPerRow;
-        const int e0 = (cv - t * cvPerRow) * VEC;
-        const int h = e0 / p.D, d0 = e0 - h * p.D;
-        const int64_t tile = int64_t(bl) * p.Hkv + h;
-        float run[VEC];
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) run[e] = 0.f;
-#pragma unroll
-        for (int k = 0; k < kMaxScales; ++k) {
-          if (k >= a.kU) break;
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) run[e] += acc[q][k][e];
-          if (r1 == P) {  // the sequence's prefix ends here: open partial of scale k
-            float* pp = p.part + ((tile * p.nsc + k) * 2 + t) * p.D + d0;
-#pragma unroll
-            for (int e = 0; e < VEC; e += 4)
-              *reinterpret_cast<float4*>(pp + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
-          }
-        }
-        if (!unit_closed) {
-          float* w = a.ws + (int64_t(bl) * a.n_units + u) * (2 * rowElems) + int64_t(cv) * VEC;
-#pragma unroll
-          for (int e = 0; e < VEC; e += 4)
-            *reinterpret_cast<float4*>(w + e) = make_float4(run[e], run[e + 1], run[e + 2], run[e + 3]);
-        }
-      }
-    }
-
-    __syncthreads();  // buffer `buf` fully read by every thread
-    ++consumed;
-    if (tid == 0 && prod.valid) {
-      fence_proxy_async_smem();
-      issue(prod, issued);
-      ++issued;
-      cursor_next(a, p, prod);
-    }
-    cursor_next(a, p, cons);
-  }
-
-  if (timed_out) {
-    if (tid == 0) {
-      set_err(p.err, LS_DEVERR_WAIT_TIMEOUT);
-      // let every copy still in flight land before the CTA's shared memory goes away
-      for (int n = consumed; n < issued; ++n)
-        mbar_wait_bounded(&full[n % kPrefillStages], uint32_t((n / kPrefillStages) & 1), kWaitLimit);
-    }
-    __syncthreads();
   }
 }
 
@@ -471,7 +498,7 @@ static cudaError_t launch_units(const Dev& p, const PrefillArgs& a, int sms, cud
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int grid = max(1, min(a.n_items, sms));
-  kern<<<grid, kPrefillThreads, smem, stream>>>(p, a);
+  kern<<<grid, kPrefillBlock, smem, stream>>>(p, a);
   return cudaGetLastError();
 }
 

@@ -701,8 +701,12 @@ cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcoun
   a.bstride = bstride;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
-  // one CTA per SM, tiles round robin
-  const int grid = a.n_tiles < sms ? a.n_tiles : sms;
+  // at most one CTA per SM, tiles round robin, and no more CTAs than needed for the
+  // fewest tiles per CTA: every CTA then gets the same number of tiles (512 tiles on 148
+  // SMs: 128 CTAs x 4 instead of 68 x 4 + 80 x 3). The stream is bandwidth-bound, so the
+  // idle SMs cost nothing while the ragged last wave would have.
+  const int waves = (a.n_tiles + sms - 1) / sms;
+  const int grid = (a.n_tiles + waves - 1) / waves;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);

@@ -13,9 +13,9 @@
 // Persistent kernel, one CTA per SM, 12 warps; the roles only meet at mbarriers, so no
 // role's order of work can hold up another's:
 //   warp 0    TMA producer of Q (3-D tensor map, two 64-column swizzled halves) and of
-//             the K rows of every chunk (ring of K stages, tensor map over the arena),
+//             the K rows of every chunk (ring of 2 K stages, tensor map over the arena),
 //             plus the boundary key row.
-//   warp 6    TMA producer of the V rows of every chunk (its own ring of V stages), plus
+//   warp 6    TMA producer of the V rows of every chunk (its own ring of 3 stages), plus
 //             the boundary value row.
 //   warp 1    TMEM allocator and the QK-issuing thread (tcgen05.mma kind::f16, bf16 in,
 //             fp32 accumulate, M = 64). The M = 64 accumulator fills lanes 0-15 of each
@@ -50,8 +50,8 @@ namespace ls {
 
 namespace {
 
-constexpr int kKStages = 3;           // K ring
-constexpr int kVStages = 2;           // V ring
+constexpr int kKStages = 2;           // K ring (QK runs ahead of the softmax anyway)
+constexpr int kVStages = 3;           // V ring (a V chunk waits for the softmax's P: deeper)
 constexpr int kChunk = 128;            // arena rows per chunk
 constexpr int kMaxChunks = 6;          // kv_rows + 1 <= 768
 constexpr int kThreads = 384;          // 12 warps: 3 per SM sub-partition, <= 168 registers

@@ -24,18 +24,25 @@
 //             lanes 0-15, keys 64-127 to lanes 16-31 of the same 64 columns), so the two
 //             threads of a row pair each own half of the chunk's keys. Four S buffers.
 //   warp 7    the PV-issuing thread: P_c V_c accumulates into the tile's output O, split
-//             over the output columns the same way; O is double-buffered by tile.
-//             512 TMEM columns in all.
+//             over the output columns the same way; O is double-buffered by tile. P is the
+//             MMA's A operand straight from TMEM (two P buffers), V its B operand in shared
+//             memory. 512 TMEM columns in all: S 0-255, O 256-383, P 384-511.
 //   warps 2-5 softmax, one TMEM subpartition each, thread pairs (t, t+16) per query row.
-//             Per chunk: scaled logits, row max, exp2 against the row's reference max,
-//             bf16 P into shared memory in the MMA's swizzled K-major layout. The
+//             Per chunk: the chunk's key mask (from a table the epilogue warps fill one
+//             tile ahead), scaled logits, row max, exp2 against the row's reference max,
+//             bf16 P into TMEM (a row's 128 keys as 64 packed columns of its lane, once in
+//             lanes 0-15 and once in lanes 16-31 for the two output halves). The
 //             reference max only moves when a chunk exceeds it by more than 2^8 (then the
 //             row's O in TMEM and its running sum are rescaled once), so no chunk's P V
 //             has to come back to registers. After a tile's last chunk the row sums go
 //             to the epilogue warps through shared memory.
 //   warps 8-11 epilogue, one TMEM subpartition each: O of a tile from TMEM (O is
 //             double-buffered by tile) times 1/rowsum, to global memory, while the
-//             softmax warps already work on the next tile.
+//             softmax warps already work on the next tile. A bf16 O goes through the
+//             tile's own Q buffer (free once its last P V has landed) and leaves with one
+//             TMA tensor store, so no global store instruction competes with the softmax's
+//             exp2 for the SM sub-partitions' shared-function queue. Warp 8 also turns the
+//             counters of the tile two ahead into the key masks of its chunks.
 // ls_round launches this kernel programmatically dependent on the commit kernel: it is
 // scheduled while the commit runs, allocates TMEM, sets up its barriers and issues the
 // first tile's Q (complete before the commit started), then waits on the device
@@ -50,18 +57,18 @@ namespace ls {
 
 namespace {
 
-constexpr int kKStages = 2;           // K ring (QK runs ahead of the softmax anyway)
-constexpr int kVStages = 3;           // V ring (a V chunk waits for the softmax's P: deeper)
+constexpr int kKStages = 3;           // K ring
+constexpr int kVStages = 3;           // V ring
 constexpr int kChunk = 128;            // arena rows per chunk
 constexpr int kMaxChunks = 6;          // kv_rows + 1 <= 768
 constexpr int kThreads = 384;          // 12 warps: 3 per SM sub-partition, <= 168 registers
 constexpr int kQBytes = 64 * 128 * 2;  // one Q tile (two 8 KB halves)
-constexpr int kPBytes = 64 * 128 * 2;  // one P chunk (two 8 KB halves: keys 0-63 / 64-127)
 constexpr int kStageBytes = kChunk * 128 * 2;  // one K or V chunk (two 16 KB halves: d 0-63 / 64-127)
-constexpr int kSmemBytes = 2 * kQBytes + 2 * kPBytes + (kKStages + kVStages) * kStageBytes + 1024;
+constexpr int kSmemBytes = 2 * kQBytes + (kKStages + kVStages) * kStageBytes + 1024;
 constexpr int kSBufs = 4;              // S buffers: QK may run up to four chunks ahead
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 256;        // O buffers at columns 256 + 64 * (tile & 1)
+constexpr uint32_t kPCol = 384;        // P buffers at columns 384 + 64 * (chunk & 1)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P values stay <= 2^8
 
 struct TcArgs {
@@ -84,7 +91,10 @@ struct Bars {
   uint64_t pv_done;
   uint64_t o_full[2], o_free[2];
   uint64_t lsum_full[2], lsum_free[2];
+  uint64_t info_full[2], info_free[2];
+  uint64_t o_staged;
   float lsum_buf[2][64];  // row sums of the last two tiles, softmax -> epilogue
+  uint64_t vmask[2][kMaxChunks][2];  // key masks of the last two tiles: [chunk][64-row half]
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -104,6 +114,15 @@ __device__ inline void tma_load_3d(void* dst, const CUtensorMap* map, int x, int
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ inline void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ inline void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ inline void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ inline void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ inline void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -136,6 +155,16 @@ __device__ inline void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// The same with A (M x K, bf16 pairs packed per 32-bit column, row m in the lane of
+// accumulator row m) read from TMEM.
+__device__ inline void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 __device__ inline void mma_commit(uint64_t* bar) {
@@ -176,6 +205,19 @@ __device__ inline void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 16 lanes from taddr on: lanes 0-15 of the warp write columns 0-31 of their lane, lanes
+// 16-31 columns 32-63 of the same 16 lanes (the 16x32bx2 shape, half split at 32 columns).
+__device__ inline void tmem_st_pairs(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
 }
 
 __device__ inline float ex2(float x) {
@@ -221,8 +263,6 @@ __device__ inline uint64_t range_bits(int lo, int hi, int r0) {
   const uint64_t m = n >= 64 ? ~0ull : ((1ull << n) - 1ull);
   return m << (lo - r0);
 }
-// Rows below n of [r0, r0 + 64), r0 already subtracted.
-__device__ inline uint64_t rows_below(int n) { return n >= 64 ? ~0ull : (n <= 0 ? 0ull : (1ull << n) - 1ull); }
 // sinfo: 16 bits per scale k at bit 16k: valid segment slots (bits 0-14), partial non-empty (bit 15).
 __device__ inline uint64_t view_mask(const Dev& p, int r0, int ring_valid, uint64_t sinfo, bool has_glob) {
   uint64_t m = range_bits(0, ring_valid, r0);
@@ -244,16 +284,18 @@ __device__ inline int item_count(const TcArgs& a) {
 }
 __device__ inline int item_tile(int i) { return int(blockIdx.x) + i * int(gridDim.x); }
 
+// kOutF32: fp32 output written with plain stores; otherwise bf16 output through a TMA store.
+template <bool kOutF32>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMap kv_map,
-                 const __grid_constant__ CUtensorMap kv_tail_map, const __grid_constant__ CUtensorMap q_map) {
+                 const __grid_constant__ CUtensorMap kv_tail_map, const __grid_constant__ CUtensorMap q_map,
+                 const __grid_constant__ CUtensorMap o_map) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ Bars s;
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_buf = smem;                           // [2][kQBytes]
-  unsigned char* p_buf = q_buf + 2 * kQBytes;            // [2][kPBytes]
-  unsigned char* k_buf = p_buf + 2 * kPBytes;            // [kKStages][kStageBytes]
+  unsigned char* k_buf = q_buf + 2 * kQBytes;            // [kKStages][kStageBytes]
   unsigned char* v_buf = k_buf + kKStages * kStageBytes; // [kVStages][kStageBytes]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -267,12 +309,16 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     for (int i = 0; i < kVStages; ++i) { mbar_init(&s.vfull[i], 1); mbar_init(&s.vempty[i], 1); }
     for (int i = 0; i < kSBufs; ++i) { mbar_init(&s.s_full[i], 1); mbar_init(&s.s_free[i], 128); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.q_full[i], 1); mbar_init(&s.q_empty[i], 1);
+      // a Q buffer is free once its tile's QK is done and, for a bf16 output, once the
+      // tile's O staged in it has been read by the TMA store
+      mbar_init(&s.q_full[i], 1); mbar_init(&s.q_empty[i], kOutF32 ? 1 : 2);
+      mbar_init(&s.info_full[i], 32); mbar_init(&s.info_free[i], 128);
       mbar_init(&s.p_full[i], 128); mbar_init(&s.p_empty[i], 1);
       mbar_init(&s.o_full[i], 1); mbar_init(&s.o_free[i], 128);
       mbar_init(&s.lsum_full[i], 128); mbar_init(&s.lsum_free[i], 128);
     }
     mbar_init(&s.pv_done, 1);
+    mbar_init(&s.o_staged, 128);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -403,7 +449,6 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   } else if (warp == 7) {
     // ------------------------------------------------------------ PV issuer
     if (lane == 0) {
-      const uint64_t dp0 = sdesc(smem_u32(p_buf), 16, 1024);
       const uint64_t dv0 = sdesc(smem_u32(v_buf), kStageBytes / 2, 1024);
       const uint32_t id_pv = idesc_bf16(64, true);
       bool ok = true;
@@ -416,15 +461,15 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           if (!wait_or_abort(s, &s.vfull[st], (k / kVStages) & 1, p.err)) { ok = false; break; }
           if (!wait_or_abort(s, &s.p_full[pb], (k >> 1) & 1, p.err)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dv = dv0 + uint32_t(st * kStageBytes >> 4), dp = dp0 + uint32_t(pb * kPBytes >> 4);
+          const uint64_t dv = dv0 + uint32_t(st * kStageBytes >> 4);
+          const uint32_t pa = tmem + kPCol + 64 * pb;  // 16 keys = 8 packed columns per step
           const int rows = chunk_rows(c);
           for (int kk = 0; kk < rows / 16; ++kk) {
-            const uint64_t pa = dp + uint32_t(((kk >> 2) * (kPBytes / 2) + (kk & 3) * 32) >> 4);
             const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
             // V: rows = keys (K dim), 128-byte rows per 64-column half: MN-major B, SBO = 8 rows
-            mma_bf16(tmem + kOCol + 64 * ob, pa, dv + uint32_t(kk * 2048 >> 4), id_pv, acc);
-            mma_bf16(tmem + (16u << 16) + kOCol + 64 * ob, pa, dv + uint32_t((kStageBytes / 2 + kk * 2048) >> 4),
-                     id_pv, acc);
+            mma_bf16_ta(tmem + kOCol + 64 * ob, pa + 8 * kk, dv + uint32_t(kk * 2048 >> 4), id_pv, acc);
+            mma_bf16_ta(tmem + (16u << 16) + kOCol + 64 * ob, pa + (16u << 16) + 8 * kk,
+                        dv + uint32_t((kStageBytes / 2 + kk * 2048) >> 4), id_pv, acc);
           }
           mma_commit(&s.vempty[st]);
           mma_commit(&s.p_empty[pb]);
@@ -440,44 +485,17 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     const int row = 16 * sub + (lane & 15);
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
     const float sl2 = a.scale_log2;     // > 0 (checked by the caller)
-    // counters of the next item's tile are read one item ahead (their load latency then
-    // never sits between two items)
-    auto load_counters = [&](int i, int64_t* dst) {
-      if (i >= n_items) return;
-      int b, lc, g;
-      tile_coords(item_tile(i), p, a.lcount, b, lc, g);
-      const int64_t* ctr = p.counters + (int64_t(b) * p.L + a.lb + lc) * (1 + p.nsc);
-#pragma unroll
-      for (int kk = 0; kk <= kMaxScales; ++kk) dst[kk] = kk <= p.nsc ? ctr[kk] : 0;
-    };
-    int64_t cnt_next[kMaxScales + 1];
-    grid_dependency_wait();  // the counters are state a preceding commit writes
-    load_counters(0, cnt_next);
     int k = 0;
     for (int i = 0; i < n_items; ++i) {
       const int ob = i & 1;
-      const int64_t len = cnt_next[0];
-      const int ring_valid = len < p.W ? int(len) : p.W;
-      uint64_t sinfo = 0;
-#pragma unroll
-      for (int kk = 0; kk < kMaxScales; ++kk) {
-        if (kk < p.nsc) {
-          const int64_t n = cnt_next[1 + kk];
-          const uint64_t e = uint64_t(n < p.slots ? n : int64_t(p.slots)) |
-                             (len - n * p.scales[kk] > 0 ? 0x8000ull : 0ull);
-          sinfo |= e << (16 * kk);
-        }
-      }
-      load_counters(i + 1, cnt_next);
-
+      // the key masks of this tile's chunks (epilogue warp 8 fills them from the counters)
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.info_full[ob], (i >> 1) & 1, p.err))) break;
       float mref = -INFINITY;  // reference max (log2 units) the P values are taken against
       float lsum = 0.f;        // sum of the rows' weights against mref
       bool ok = true;
       for (int c = 0; c < nC; ++c, ++k) {
         const int sb = k % kSBufs, pb = k & 1;
-        const int r0 = c * kChunk + 64 * half;
-        const uint64_t vm = r0 + 64 <= p.W ? rows_below(ring_valid - r0)  // ring slots only
-                                           : view_mask(p, r0, ring_valid, sinfo, len > 0);
+        const uint64_t vm = s.vmask[ob][c][half];
         const bool all_valid = __all_sync(0xffffffffu, vm == ~0ull);
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.s_full[sb], (k / kSBufs) & 1, p.err))) { ok = false; break; }
         tc_fence_after();
@@ -543,16 +561,16 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         }
         const float psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
         lsum += psum + __shfl_xor_sync(0xffffffffu, psum, 16);
-        // this thread's 64 keys: half `half` of the P tile, 8 swizzled 16-byte pieces
-        unsigned char* prow = p_buf + pb * kPBytes + half * (kPBytes / 2) + row * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) << 4)) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        fence_proxy_async_smem();
+        // the row's 128 keys as 64 packed columns (this thread's 64 keys at columns
+        // 32 * half ...), in lanes 0-15 and again in lanes 16-31 of the subpartition
+        tmem_st_pairs(trow + kPCol + 64 * pb, pk);
+        tmem_st_pairs(trow + (16u << 16) + kPCol + 64 * pb, pk);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
         mbar_arrive(&s.p_full[pb]);
       }
       if (!ok) break;
+      mbar_arrive(&s.info_free[ob]);
       // the row sum goes to the epilogue warps, which read this tile's O once its last
       // P V has landed; the softmax goes on with the next tile
       if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.lsum_free[ob], ((i >> 1) & 1) ^ 1, p.err))) break;
@@ -567,25 +585,32 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
     const int row = 16 * sub + (lane & 15);
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
     const int grp = p.Hq / p.Hkv;
-    const int qi = row / grp, jj = row - qi * grp;
-    // 32 output columns (col0 + 0..31 of this thread's 64) of the slice, times inv
-    auto store32 = [&](const float* v, float inv, int b, int lc, int g, int col0) {
-      const int64_t orow =
-          (((int64_t(b) * a.lcount + lc) * p.B + qi) * p.Hq + g * grp + jj) * 128 + 64 * half + col0;
-      if (p.out_f32) {
-        float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          o4[u] = make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
-      } else {
-        uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          o4[u] = make_uint4(pack_bf16(v[8 * u] * inv, v[8 * u + 1] * inv), pack_bf16(v[8 * u + 2] * inv, v[8 * u + 3] * inv),
-                             pack_bf16(v[8 * u + 4] * inv, v[8 * u + 5] * inv),
-                             pack_bf16(v[8 * u + 6] * inv, v[8 * u + 7] * inv));
+    // Warp 8: key masks of item i's chunks into table slot i & 1. Lane 2c + h takes the
+    // 64 rows [128 c + 64 h, +64) of the tile's key/value stream (see view_mask).
+    auto fill_masks = [&](int i) {
+      int b, lc, g;
+      tile_coords(item_tile(i), p, a.lcount, b, lc, g);
+      const int64_t* ctr = p.counters + (int64_t(b) * p.L + a.lb + lc) * (1 + p.nsc);
+      const int64_t len = ctr[0];
+      uint64_t sinfo = 0;
+#pragma unroll 1
+      for (int kk = 0; kk < p.nsc; ++kk) {
+        const int64_t n = ctr[1 + kk];
+        const uint64_t e = uint64_t(n < p.slots ? n : int64_t(p.slots)) |
+                           (len - n * p.scales[kk] > 0 ? 0x8000ull : 0ull);
+        sinfo |= e << (16 * kk);
       }
+      if (lane < 2 * nC)
+        s.vmask[i & 1][lane >> 1][lane & 1] =
+            view_mask(p, 64 * lane, len < p.W ? int(len) : p.W, sinfo, len > 0);
     };
+    if (warp == 8) {
+      grid_dependency_wait();  // the counters are state a preceding commit writes
+      for (int i = 0; i < 2 && i < n_items; ++i) {
+        fill_masks(i);
+        mbar_arrive(&s.info_full[i]);
+      }
+    }
     for (int i = 0; i < n_items; ++i) {
       int b, lc, g;
       tile_coords(item_tile(i), p, a.lcount, b, lc, g);
@@ -601,9 +626,43 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       tc_fence_before();
       mbar_arrive(&s.o_free[ob]);
       const float inv = 1.0f / lsum;
-      store32(o, inv, b, lc, g, 0);
-      store32(o + 32, inv, b, lc, g, 32);
+      const int zrow = (b * a.lcount + lc) * p.B;  // the tile's first query of the block
+      if constexpr (kOutF32) {
+        const int qi = row / grp, jj = row - qi * grp;
+        float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                               ((int64_t(zrow) + qi) * p.Hq + g * grp + jj) * 128 + 64 * half);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          o4[u] = make_float4(o[4 * u] * inv, o[4 * u + 1] * inv, o[4 * u + 2] * inv, o[4 * u + 3] * inv);
+      } else {
+        // O into the tile's Q buffer (row m = i_q * group + j, two swizzled 64-column
+        // halves: the layout of the output tensor map's box), then one TMA store
+        unsigned char* orow = q_buf + ob * kQBytes + half * (kQBytes / 2) + row * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(orow + ((u ^ (row & 7)) << 4)) =
+              make_uint4(pack_bf16(o[8 * u] * inv, o[8 * u + 1] * inv), pack_bf16(o[8 * u + 2] * inv, o[8 * u + 3] * inv),
+                         pack_bf16(o[8 * u + 4] * inv, o[8 * u + 5] * inv),
+                         pack_bf16(o[8 * u + 6] * inv, o[8 * u + 7] * inv));
+        fence_proxy_async_smem();
+        mbar_arrive(&s.o_staged);
+        // (after an abort the store is skipped; the warp leaves at its next wait)
+        if (threadIdx.x == 256 && wait_or_abort(s, &s.o_staged, i & 1, p.err)) {
+          tma_store_3d(&o_map, q_buf + ob * kQBytes, 0, g * grp, zrow);
+          tma_store_3d(&o_map, q_buf + ob * kQBytes + kQBytes / 2, 64, g * grp, zrow);
+          bulk_commit_group();
+          bulk_wait_read_all();  // the buffer is read: Q of the tile two ahead may land
+          mbar_arrive(&s.q_empty[ob]);
+        }
+      }
+      if (warp == 8 && i + 2 < n_items) {
+        // the softmax is done with slot ob's masks: they become those of tile i + 2
+        if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.info_free[ob], (i >> 1) & 1, p.err))) break;
+        fill_masks(i + 2);
+        mbar_arrive(&s.info_full[ob]);
+      }
     }
+    if (!kOutF32 && threadIdx.x == 256) bulk_wait_all();  // the output stores are complete
   }
 
   __syncthreads();
@@ -679,8 +738,10 @@ int tc_prepare(const Dev& p, TcPlan* plan) {
   if (!encode_kv(p, kChunk, reinterpret_cast<CUtensorMap*>(plan->kv_map))) return LS_ERR_CUDA;
   if (plan->tail_rows > 0 && !encode_kv(p, plan->tail_rows, reinterpret_cast<CUtensorMap*>(plan->kv_tail_map)))
     return LS_ERR_CUDA;
-  if (cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(attend_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(attend_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+          cudaSuccess)
     return LS_ERR_CUDA;
   return LS_OK;
 }
@@ -688,8 +749,14 @@ int tc_prepare(const Dev& p, TcPlan* plan) {
 cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
                              const void* bk, const void* bv, int64_t bstride, float scale, void* out,
                              int sms, bool after_commit, cudaStream_t stream) {
-  CUtensorMap qmap;
+  // Q in, and a bf16 O out, are [b, lcount, B, Hq, D]: one tile is the box (64 columns,
+  // the group's heads, the block's queries) at (0 or 64, g * group, first query)
+  CUtensorMap qmap, omap;
   if (!encode_q(p, lcount, q, &qmap)) return cudaErrorInvalidValue;
+  if (p.out_f32)
+    omap = qmap;  // unused: fp32 output is stored directly
+  else if (!encode_q(p, lcount, out, &omap))
+    return cudaErrorInvalidValue;
   TcArgs a{};
   a.lb = lb;
   a.lcount = lcount;
@@ -719,8 +786,10 @@ cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcoun
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  return cudaLaunchKernelEx(&cfg, attend_tc_kernel, p, a, *reinterpret_cast<const CUtensorMap*>(plan.kv_map),
-                            *reinterpret_cast<const CUtensorMap*>(plan.kv_tail_map), qmap);
+  const CUtensorMap& kv = *reinterpret_cast<const CUtensorMap*>(plan.kv_map);
+  const CUtensorMap& kv_tail = *reinterpret_cast<const CUtensorMap*>(plan.kv_tail_map);
+  return p.out_f32 ? cudaLaunchKernelEx(&cfg, attend_tc_kernel<true>, p, a, kv, kv_tail, qmap, omap)
+                   : cudaLaunchKernelEx(&cfg, attend_tc_kernel<false>, p, a, kv, kv_tail, qmap, omap);
 }
 
 }  // namespace ls

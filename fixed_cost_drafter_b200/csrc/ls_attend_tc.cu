@@ -385,15 +385,17 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         // Q is an input; the boundary rows and the arena are state a preceding commit writes
         if (i == 0) grid_dependency_wait();
       }
+      // the boundary row is loaded once the tile's first chunk is on its way (its latency
+      // then overlaps the stream), or before a one-chunk tile's only chunk
+      const __nv_bfloat16* bptr = bsrc + (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + g * 128 + lane * 8;
       uint4 brow = make_uint4(0, 0, 0, 0);
-      if (lane < 16)
-        brow = ld_nc_v4(bsrc + (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + g * 128 + lane * 8);
       for (int c = 0; c < nC; ++c, ++k) {
         const int st = k % nst;
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err))) { ok = false; break; }
         unsigned char* dst = ring + st * kStageBytes;
         const bool last = c == nC - 1;
         if (last) {  // the boundary row, row `tail` of the stage
+          if (c == 0 && lane < 16) brow = ld_nc_v4(bptr);
           if (lane < 16)
             *reinterpret_cast<uint4*>(dst + (lane >> 3) * (kStageBytes / 2) + tail * 128 +
                                       (((lane & 7) ^ (tail & 7)) << 4)) = brow;
@@ -410,6 +412,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
             tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
           }
         }
+        if (c == 0 && !last && lane < 16) brow = ld_nc_v4(bptr);
         ++issued;
       }
     }

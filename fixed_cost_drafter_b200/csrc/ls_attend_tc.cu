@@ -13,7 +13,7 @@
 // Persistent kernel, one CTA per SM, 12 warps; the roles only meet at mbarriers, so no
 // role's order of work can hold up another's:
 //   warp 0    TMA producer of Q (3-D tensor map, two 64-column swizzled halves) and of
-//             the K rows of every chunk (ring of 2 K stages, tensor map over the arena),
+//             the K rows of every chunk (ring of 3 K stages, tensor map over the arena),
 //             plus the boundary key row.
 //   warp 6    TMA producer of the V rows of every chunk (its own ring of 3 stages), plus
 //             the boundary value row.

@@ -26,6 +26,7 @@ import argparse
 import glob
 import hashlib
 import json
+import re
 import math
 import os
 import statistics
@@ -77,15 +78,24 @@ def barrier(world):
 # ---------------------------------------------------------------------------------------
 # algorithmic bytes (the layout built: bf16 window and mean rows, fp32 summary sums)
 # ---------------------------------------------------------------------------------------
-def attend_bytes(wl) -> int:
+VIEW_BOUNDARY, VIEW_WINDOW, VIEW_SUMMARY, VIEW_ALL = 0x1, 0x2, 0x4, 0x7  # LS_VIEW_*
+
+# Table 5's component ablations: the views each variant keeps
+ABLATIONS = {"full": VIEW_ALL, "without_global_summary": VIEW_BOUNDARY | VIEW_WINDOW,
+             "without_boundary_state": VIEW_WINDOW | VIEW_SUMMARY,
+             "without_recent_kv_window": VIEW_BOUNDARY | VIEW_SUMMARY}
+
+
+def attend_bytes(wl, views: int = VIEW_ALL) -> int:
+    """Algorithmic bytes of one attention launch over the given views."""
     e = wl.elem()
     b, L, H, Hq, D, B = wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.block
     summary_rows = len(wl.scales) * (wl.slots + 1) + 1
-    return (2 * b * L * B * Hq * D * e                # Q in, O out
-            + b * L * H * wl.window * 2 * D * e        # ring window K/V
-            + b * L * H * summary_rows * 2 * D * e     # summary mean rows K/V
-            + b * L * H * 2 * D * e                    # boundary K/V
-            + b * L * (1 + len(wl.scales)) * 8)        # counters
+    return (2 * b * L * B * Hq * D * e                                        # Q in, O out
+            + (b * L * H * wl.window * 2 * D * e if views & VIEW_WINDOW else 0)  # ring window K/V
+            + (b * L * H * summary_rows * 2 * D * e if views & VIEW_SUMMARY else 0)  # summary mean rows
+            + (b * L * H * 2 * D * e if views & VIEW_BOUNDARY else 0)          # boundary K/V
+            + b * L * (1 + len(wl.scales)) * 8)                                # counters
 
 
 def commit_bytes(wl, mean_delta: float) -> int:
@@ -115,10 +125,25 @@ def hbm_peak():
 
 
 def kernel_source_sha(name: str) -> str:
-    """Hash of a kernel's source file and every shared header it may include."""
+    """Hash of a kernel's source file and of the package headers it includes (recursively)."""
     csrc = os.path.join(ROOT, "fixed_cost_drafter_b200", "csrc")
+    inc = os.path.join(ROOT, "include")
+    seen, order, todo = set(), [], [os.path.join(csrc, name)]
+    while todo:
+        q = todo.pop(0)
+        if q in seen:
+            continue
+        seen.add(q)
+        order.append(q)
+        with open(q, encoding="utf-8") as f:
+            for m in re.finditer(r'^\s*#\s*include\s+"([^"]+)"', f.read(), re.M):
+                for d in (os.path.dirname(q), csrc, inc):
+                    cand = os.path.join(d, m.group(1))
+                    if os.path.exists(cand):
+                        todo.append(os.path.normpath(cand))
+                        break
     h = hashlib.sha256()
-    for q in [os.path.join(csrc, name)] + sorted(glob.glob(os.path.join(csrc, "*.cuh"))):
+    for q in order:
         with open(q, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -380,6 +405,29 @@ def run_gpu(args):
     if status != F.LS_OK:
         raise RuntimeError(f"device error word {word:#x} after the timed rounds")
 
+    # the cost side of Table 5's component ablations: the attention over fewer views
+    ablations = None
+    if not args.no_ablations:
+        KA = min(K, 200)
+        ablations = {}
+        for name, views in ABLATIONS.items():
+            ms = []
+            for i in range(KA):
+                r = (W + i) % n_rounds
+                flush.zero_()
+                evs[i][0].record(stream)
+                run.attend(inp, r, out, views=views)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize()
+            ms = [e[0].elapsed_time(e[1]) for e in evs[:KA]]
+            us = float(np.mean(ms)) * 1e3
+            nb = attend_bytes(wl, views)
+            ablations[name] = {"views": views, "attend_us": us, "bytes": nb, "GBps": nb / us / 1e3,
+                               "state_bytes_per_sequence": F.ls_view_state_bytes(run.cfg, views) / wl.batch}
+        status, word = run.error()
+        if status != F.LS_OK:
+            raise RuntimeError(f"device error word {word:#x} after the ablation launches")
+
     # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
     graph_rps = None
     if not args.no_graph:
@@ -445,6 +493,7 @@ def run_gpu(args):
                       "attend_us": att_s * 1e6, "commit_bytes": c_bytes,
                       "commit_GBps": c_bytes / (float(np.mean(commit_ms)) / 1e3) / 1e9},
             "graph_rounds_per_s": graph_rps,
+            "view_ablations": ablations,
             "prefill": {"ms": prefill_ms, "bytes": prefill_b, "achieved_GBps": prefill_b / (prefill_ms / 1e3) / 1e9,
                         "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
             "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch,
@@ -589,6 +638,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=WORKLOAD)
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-ablations", action="store_true", help="skip the view-ablation attention timings")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

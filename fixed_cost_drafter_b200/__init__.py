@@ -32,10 +32,15 @@ LS_BF16 = 1
 LS_FLAG_FORCE_SIMT = 0x1
 LS_FLAG_OUT_F32 = 0x2
 LS_MAX_SCALES = 4
+LS_VIEW_BOUNDARY = 0x1
+LS_VIEW_WINDOW = 0x2
+LS_VIEW_SUMMARY = 0x4
+LS_VIEW_ALL = 0x7
 
 EXPORTED = (
     "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",
-    "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend", "ls_round",
+    "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend",
+    "ls_draft_attend_views", "ls_view_state_bytes", "ls_round",
     "ls_round_overlaps", "ls_attend_uses_tensor_cores",
     "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
 )
@@ -75,6 +80,7 @@ def _load():
     cfgp = ctypes.POINTER(ls_config)
     sig = {
         "ls_state_bytes": (sz, [cfgp]),
+        "ls_view_state_bytes": (sz, [cfgp, i32]),
         "ls_get_layout": (ctypes.c_int, [cfgp, ctypes.POINTER(ls_layout)]),
         "ls_init_state": (ctypes.c_int, [cfgp, vp, sz, ctypes.POINTER(vp), vp]),
         "ls_prefill_workspace_bytes": (sz, [cfgp, i64, i64]),
@@ -82,6 +88,7 @@ def _load():
         "ls_prefill_summary_noalloc": (ctypes.c_int, [vp, vp, vp, i64, i64, vp, i64, i64, vp, vp]),
         "ls_commit_round": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "ls_draft_attend": (ctypes.c_int, [vp, i32, i32, vp, vp, vp, i64, ctypes.c_float, vp, vp]),
+        "ls_draft_attend_views": (ctypes.c_int, [vp, i32, i32, vp, vp, vp, i64, ctypes.c_float, i32, vp, vp]),
         "ls_round": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, ctypes.c_float, vp, vp]),
         "ls_round_overlaps": (ctypes.c_int, [vp]),
         "ls_attend_uses_tensor_cores": (ctypes.c_int, [vp]),
@@ -148,6 +155,10 @@ def ls_state_bytes(cfg: ls_config) -> int:
     return int(_lib.ls_state_bytes(ctypes.byref(cfg)))
 
 
+def ls_view_state_bytes(cfg: ls_config, views: int) -> int:
+    return int(_lib.ls_view_state_bytes(ctypes.byref(cfg), views))
+
+
 def ls_get_layout(cfg: ls_config) -> ls_layout:
     out = ls_layout()
     _check("ls_get_layout", _lib.ls_get_layout(ctypes.byref(cfg), ctypes.byref(out)))
@@ -194,6 +205,13 @@ def ls_draft_attend(state, layer_begin, layer_count, q, boundary_k, boundary_v, 
     _check("ls_draft_attend", _lib.ls_draft_attend(
         state, layer_begin, layer_count, _ptr(q), _ptr(boundary_k), _ptr(boundary_v),
         boundary_stride, float(softmax_scale), _ptr(out), _stream(stream)))
+
+
+def ls_draft_attend_views(state, layer_begin, layer_count, q, boundary_k, boundary_v, boundary_stride,
+                          softmax_scale, views, out, stream=None) -> None:
+    _check("ls_draft_attend_views", _lib.ls_draft_attend_views(
+        state, layer_begin, layer_count, _ptr(q), _ptr(boundary_k), _ptr(boundary_v),
+        boundary_stride, float(softmax_scale), views, _ptr(out), _stream(stream)))
 
 
 def ls_round(state, draft_ids, target_ids, verify_k, verify_v, verify_hidden, accept_len, next_token, q,

@@ -13,7 +13,7 @@ cudaError_t launch_commit(const Dev& p, const int32_t* draft, const int32_t* tar
                           cudaStream_t stream);
 bool simt_supported(const Dev& p);
 cudaError_t launch_attend_simt(const Dev& p, int lb, int lcount, const void* q, const void* bk,
-                               const void* bv, int64_t bstride, float scale, void* out,
+                               const void* bv, int64_t bstride, float scale, int views, void* out,
                                cudaStream_t stream);
 size_t prefill_workspace_bytes(const ls_config& c, int64_t row_begin, int64_t row_end);
 cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, const void* v,
@@ -90,6 +90,19 @@ const char* ls_status_string(int s) {
 size_t ls_state_bytes(const ls_config* cfg) {
   if (validate(cfg) != LS_OK) return 0;
   return size_t(ls::make_layout(*cfg).total);
+}
+
+size_t ls_view_state_bytes(const ls_config* cfg, int32_t views) {
+  if (validate(cfg) != LS_OK || (views & ~LS_VIEW_ALL)) return 0;
+  const ls_config& c = *cfg;
+  const int64_t e = c.dtype == LS_BF16 ? 2 : 4;
+  const int64_t bl = int64_t(c.batch) * c.n_layers, tiles = bl * c.n_kv_heads;
+  const int64_t summary_rows = int64_t(c.n_scales) * (c.slots_per_scale + 1) + 1;
+  int64_t n = bl * (1 + c.n_scales) * 8;  // counters
+  if (views & LS_VIEW_WINDOW) n += tiles * 2 * c.window * c.head_dim * e;
+  if (views & LS_VIEW_SUMMARY) n += tiles * 2 * summary_rows * c.head_dim * (4 + e);
+  if (views & LS_VIEW_BOUNDARY) n += bl * c.hidden * e;
+  return size_t(n);
 }
 
 int ls_get_layout(const ls_config* cfg, ls_layout* out) {
@@ -229,7 +242,15 @@ int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_t
 int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count, const void* d_q,
                     const void* d_boundary_k, const void* d_boundary_v, int64_t boundary_stride,
                     float softmax_scale, void* d_out, cudaStream_t stream) {
+  return ls_draft_attend_views(st, layer_begin, layer_count, d_q, d_boundary_k, d_boundary_v, boundary_stride,
+                               softmax_scale, LS_VIEW_ALL, d_out, stream);
+}
+
+int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer_count, const void* d_q,
+                          const void* d_boundary_k, const void* d_boundary_v, int64_t boundary_stride,
+                          float softmax_scale, int32_t views, void* d_out, cudaStream_t stream) {
   if (!st || !d_q || !d_boundary_k || !d_boundary_v || !d_out) return LS_ERR_INVALID_ARG;
+  if (views == 0 || (views & ~LS_VIEW_ALL)) return LS_ERR_INVALID_ARG;
   const ls_config& c = st->cfg;
   if (layer_begin < 0 || layer_count < 1 || layer_begin + layer_count > c.n_layers)
     return LS_ERR_INVALID_ARG;
@@ -241,9 +262,9 @@ int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count
   if (st->use_tc)
     return cuda_status(ls::launch_attend_tc(st->dev, st->tc, layer_begin, layer_count, d_q,
                                             d_boundary_k, d_boundary_v, boundary_stride,
-                                            softmax_scale, d_out, st->sms, false, stream));
+                                            softmax_scale, views, d_out, st->sms, false, stream));
   return cuda_status(ls::launch_attend_simt(st->dev, layer_begin, layer_count, d_q, d_boundary_k,
-                                            d_boundary_v, boundary_stride, softmax_scale, d_out,
+                                            d_boundary_v, boundary_stride, softmax_scale, views, d_out,
                                             stream));
 }
 
@@ -270,8 +291,8 @@ int ls_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_i
   const int64_t e = st->lay.elem;
   if (st->use_tc)  // the attention kernel is scheduled while the commit runs
     return cuda_status(ls::launch_attend_tc(st->dev, st->tc, 0, c.n_layers, d_q, bnd + boundary_k_offset * e,
-                                            bnd + boundary_v_offset * e, c.hidden, softmax_scale, d_out, st->sms,
-                                            true, stream));
+                                            bnd + boundary_v_offset * e, c.hidden, softmax_scale, LS_VIEW_ALL,
+                                            d_out, st->sms, true, stream));
   return ls_draft_attend(st, 0, c.n_layers, d_q, bnd + boundary_k_offset * e, bnd + boundary_v_offset * e, c.hidden,
                          softmax_scale, d_out, stream);
 }

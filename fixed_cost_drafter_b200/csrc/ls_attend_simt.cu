@@ -7,6 +7,8 @@
 // 32 slots at a time (slot 0 = boundary, slot 1 + r = arena row r of the tile); each
 // warp keeps an online softmax (running max, running sum, output in registers) for
 // its query rows, one key per lane for the logits and D/32 output columns per lane.
+// `views` (LS_VIEW_*) selects the views that take part (Table 5's component ablations);
+// a row with no valid slot at all writes zeros.
 #include "ls_common.cuh"
 
 namespace ls {
@@ -18,7 +20,7 @@ template <typename T, int DV>
 __global__ void __launch_bounds__(kSimtWarps * 32)
 attend_simt_kernel(Dev p, int layer_begin, int layer_count, const T* __restrict__ q,
                    const T* __restrict__ bk, const T* __restrict__ bv, int64_t bstride,
-                   float scale, void* __restrict__ out) {
+                   float scale, int views, void* __restrict__ out) {
   using E = Elem<T>;
   const int g = blockIdx.x, lc = blockIdx.y, b = blockIdx.z;
   const int l = layer_begin + lc;
@@ -76,7 +78,11 @@ attend_simt_kernel(Dev p, int layer_begin, int layer_count, const T* __restrict_
     }
     if (threadIdx.x < 32) {
       const int s = s0 + threadIdx.x;
-      valid_s[threadIdx.x] = s == 0 ? 1 : (s < S ? int(arena_row_valid(p, s - 1, len, nseg)) : 0);
+      bool ok = false;
+      if (s == 0) ok = (views & LS_VIEW_BOUNDARY) != 0;
+      else if (s < S) ok = ((views & (s - 1 < p.W ? LS_VIEW_WINDOW : LS_VIEW_SUMMARY)) != 0) &&
+                           arena_row_valid(p, s - 1, len, nseg);
+      valid_s[threadIdx.x] = int(ok);
     }
     __syncthreads();
     const bool ok = valid_s[lane] != 0;
@@ -113,7 +119,7 @@ attend_simt_kernel(Dev p, int layer_begin, int layer_count, const T* __restrict_
     const int m = warp + r * kSimtWarps;
     if (m >= M) break;
     const int i = m / grp, j = m - i * grp;
-    const float inv = 1.0f / lrun[r];
+    const float inv = lrun[r] > 0.f ? 1.0f / lrun[r] : 0.f;  // no valid slot: zeros
     const int64_t ob = (((int64_t(b) * layer_count + lc) * p.B + i) * p.Hq + g * grp + j) * D;
 #pragma unroll
     for (int dd = 0; dd < DV; ++dd) {
@@ -125,7 +131,7 @@ attend_simt_kernel(Dev p, int layer_begin, int layer_count, const T* __restrict_
 
 template <typename T, int DV>
 static cudaError_t launch_simt_t(const Dev& p, int lb, int lcount, const void* q, const void* bk,
-                                 const void* bv, int64_t bstride, float scale, void* out,
+                                 const void* bv, int64_t bstride, float scale, int views, void* out,
                                  cudaStream_t stream) {
   const int D = DV * 32;
   const int M = (p.Hq / p.Hkv) * p.B;
@@ -140,19 +146,19 @@ static cudaError_t launch_simt_t(const Dev& p, int lb, int lcount, const void* q
   const dim3 grid(p.Hkv, lcount, p.b);
   kern<<<grid, kSimtWarps * 32, smem, stream>>>(p, lb, lcount, static_cast<const T*>(q),
                                                 static_cast<const T*>(bk), static_cast<const T*>(bv),
-                                                bstride, scale, out);
+                                                bstride, scale, views, out);
   return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_simt_dt(const Dev& p, int lb, int lcount, const void* q, const void* bk,
-                                  const void* bv, int64_t bstride, float scale, void* out,
+                                  const void* bv, int64_t bstride, float scale, int views, void* out,
                                   cudaStream_t stream) {
   switch (p.D / 32) {
-    case 1: return launch_simt_t<T, 1>(p, lb, lcount, q, bk, bv, bstride, scale, out, stream);
-    case 2: return launch_simt_t<T, 2>(p, lb, lcount, q, bk, bv, bstride, scale, out, stream);
-    case 4: return launch_simt_t<T, 4>(p, lb, lcount, q, bk, bv, bstride, scale, out, stream);
-    case 8: return launch_simt_t<T, 8>(p, lb, lcount, q, bk, bv, bstride, scale, out, stream);
+    case 1: return launch_simt_t<T, 1>(p, lb, lcount, q, bk, bv, bstride, scale, views, out, stream);
+    case 2: return launch_simt_t<T, 2>(p, lb, lcount, q, bk, bv, bstride, scale, views, out, stream);
+    case 4: return launch_simt_t<T, 4>(p, lb, lcount, q, bk, bv, bstride, scale, views, out, stream);
+    case 8: return launch_simt_t<T, 8>(p, lb, lcount, q, bk, bv, bstride, scale, views, out, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -165,11 +171,11 @@ bool simt_supported(const Dev& p) {
 }
 
 cudaError_t launch_attend_simt(const Dev& p, int lb, int lcount, const void* q, const void* bk,
-                               const void* bv, int64_t bstride, float scale, void* out,
+                               const void* bv, int64_t bstride, float scale, int views, void* out,
                                cudaStream_t stream) {
   if (p.dtype == LS_BF16)
-    return launch_simt_dt<__nv_bfloat16>(p, lb, lcount, q, bk, bv, bstride, scale, out, stream);
-  return launch_simt_dt<float>(p, lb, lcount, q, bk, bv, bstride, scale, out, stream);
+    return launch_simt_dt<__nv_bfloat16>(p, lb, lcount, q, bk, bv, bstride, scale, views, out, stream);
+  return launch_simt_dt<float>(p, lb, lcount, q, bk, bv, bstride, scale, views, out, stream);
 }
 
 }  // namespace ls

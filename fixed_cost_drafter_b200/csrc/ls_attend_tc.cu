@@ -80,7 +80,16 @@ struct TcArgs {
   int64_t bstride;
   float scale_log2;  // softmax_scale * log2(e)
   void* out;         // bf16, or fp32 when Dev::out_f32
+  int32_t views;         // LS_VIEW_* taking part in the softmax
+  uint32_t chunk_mask;   // bit c: chunk c is streamed (the last chunk always is)
+  int32_t tail_load;     // the last chunk's arena rows are loaded (else only its boundary row)
 };
+
+// Chunks streamed after chunk c (c = -1: the first one): nC or more when none is left.
+__device__ inline int next_chunk(uint32_t mask, int c) {
+  const uint32_t m = mask >> (c + 1);
+  return m ? c + __ffs(int(m)) : 32;
+}
 
 struct Bars {
   uint64_t kfull[kKStages], kempty[kKStages];
@@ -254,7 +263,7 @@ __device__ inline void tile_coords(int t, const Dev& p, int lcount, int& b, int&
 // (bit i = row r0 + i). The stream is the tile's arena rows followed by the boundary row
 // (row R): ring slots below min(len, W), per scale the first min(n_seg, slots) segment
 // slots and the partial mean when its segment is non-empty, the global mean when len > 0,
-// and the boundary row always.
+// and the boundary row always; then only the rows of the views in `views` (LS_VIEW_*).
 __device__ inline uint64_t range_bits(int lo, int hi, int r0) {
   lo = max(lo, r0);
   hi = min(hi, r0 + 64);
@@ -264,18 +273,22 @@ __device__ inline uint64_t range_bits(int lo, int hi, int r0) {
   return m << (lo - r0);
 }
 // sinfo: 16 bits per scale k at bit 16k: valid segment slots (bits 0-14), partial non-empty (bit 15).
-__device__ inline uint64_t view_mask(const Dev& p, int r0, int ring_valid, uint64_t sinfo, bool has_glob) {
-  uint64_t m = range_bits(0, ring_valid, r0);
+__device__ inline uint64_t view_mask(const Dev& p, int r0, int ring_valid, uint64_t sinfo, bool has_glob,
+                                    int views) {
+  uint64_t m = (views & LS_VIEW_WINDOW) ? range_bits(0, ring_valid, r0) : 0ull;
   int base = p.W;
+  if (views & LS_VIEW_SUMMARY) {
 #pragma unroll 1
-  for (int k = 0; k < p.nsc; ++k) {
-    const uint32_t e = uint32_t(sinfo >> (16 * k));
-    m |= range_bits(base, base + int(e & 0x7fffu), r0);
-    if (e & 0x8000u) m |= range_bits(base + p.slots, base + p.slots + 1, r0);
-    base += p.slots + 1;
+    for (int k = 0; k < p.nsc; ++k) {
+      const uint32_t e = uint32_t(sinfo >> (16 * k));
+      m |= range_bits(base, base + int(e & 0x7fffu), r0);
+      if (e & 0x8000u) m |= range_bits(base + p.slots, base + p.slots + 1, r0);
+      base += p.slots + 1;
+    }
+    if (has_glob) m |= range_bits(base, base + 1, r0);  // global mean, row R - 1
   }
-  if (has_glob) m |= range_bits(base, base + 1, r0);  // global mean, row R - 1
-  return m | range_bits(base + 1, base + 2, r0);       // boundary row, row R
+  if (views & LS_VIEW_BOUNDARY) m |= range_bits(p.R, p.R + 1, r0);  // boundary row, row R
+  return m;
 }
 
 // Work of one CTA: tiles blockIdx.x, blockIdx.x + gridDim.x, ... (each all nC chunks).
@@ -303,6 +316,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   const int tail = a.tail_rows;                   // the tile's arena rows in its last chunk
   const int last_rows = (tail + 1 + 15) & ~15;    // rows the last chunk's MMAs take (+ boundary)
   const int n_items = item_count(a);
+  const int c_first = next_chunk(a.chunk_mask, -1);  // chunks of left-out views are skipped
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kKStages; ++i) { mbar_init(&s.kfull[i], 1); mbar_init(&s.kempty[i], 1); }
@@ -325,11 +339,13 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   {
     // rows of the last chunk past the boundary row are read by its MMAs (masked): they
     // must hold finite values, zeros until a full chunk has used the stage
-    const int zr = last_rows - tail - 1;
+    // (with the last chunk's arena rows not loaded, all of its rows but the boundary row)
+    const int z0 = a.tail_load ? tail + 1 : 0;
+    const int zr = last_rows - z0;
     if (zr > 0) {
       const int n = (kKStages + kVStages) * 2 * zr * 8;
       for (int i = threadIdx.x; i < n; i += kThreads) {
-        const int piece = i & 7, r = tail + 1 + (i >> 3) % zr, sh = (i >> 3) / zr;
+        const int piece = i & 7, r = z0 + (i >> 3) % zr, sh = (i >> 3) / zr;
         *reinterpret_cast<uint4*>(k_buf + sh * (kStageBytes / 2) + r * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();
@@ -389,13 +405,13 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       // then overlaps the stream), or before a one-chunk tile's only chunk
       const __nv_bfloat16* bptr = bsrc + (int64_t(b) * p.L + (a.lb + lc)) * a.bstride + g * 128 + lane * 8;
       uint4 brow = make_uint4(0, 0, 0, 0);
-      for (int c = 0; c < nC; ++c, ++k) {
+      for (int c = c_first; c < nC; c = next_chunk(a.chunk_mask, c), ++k) {
         const int st = k % nst;
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err))) { ok = false; break; }
         unsigned char* dst = ring + st * kStageBytes;
         const bool last = c == nC - 1;
         if (last) {  // the boundary row, row `tail` of the stage
-          if (c == 0 && lane < 16) brow = ld_nc_v4(bptr);
+          if (c == c_first && lane < 16) brow = ld_nc_v4(bptr);
           if (lane < 16)
             *reinterpret_cast<uint4*>(dst + (lane >> 3) * (kStageBytes / 2) + tail * 128 +
                                       (((lane & 7) ^ (tail & 7)) << 4)) = brow;
@@ -403,7 +419,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           __syncwarp();
         }
         if (lane == 0) {
-          const int rows = last ? tail : kChunk;
+          const int rows = last ? (a.tail_load ? tail : 0) : kChunk;
           mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
           if (rows > 0) {
             const CUtensorMap* m = last ? &kv_tail_map : &kv_map;
@@ -412,7 +428,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
             tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
           }
         }
-        if (c == 0 && !last && lane < 16) brow = ld_nc_v4(bptr);
+        if (c == c_first && !last && lane < 16) brow = ld_nc_v4(bptr);
         ++issued;
       }
     }
@@ -427,7 +443,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       for (int i = 0; i < n_items && ok; ++i) {
         const int qb = i & 1;
         if (!wait_or_abort(s, &s.q_full[qb], (i >> 1) & 1, p.err)) break;
-        for (int c = 0; c < nC; ++c, ++k) {
+        for (int c = c_first; c < nC; c = next_chunk(a.chunk_mask, c), ++k) {
           const int sb = k % kSBufs, st = k % kKStages;
           if (!wait_or_abort(s, &s.kfull[st], (k / kKStages) & 1, p.err)) { ok = false; break; }
           if (!wait_or_abort(s, &s.s_free[sb], ((k / kSBufs) & 1) ^ 1, p.err)) { ok = false; break; }
@@ -459,7 +475,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       for (int i = 0; i < n_items && ok; ++i) {
         const int ob = i & 1;
         if (!wait_or_abort(s, &s.o_free[ob], ((i >> 1) & 1) ^ 1, p.err)) break;
-        for (int c = 0; c < nC; ++c, ++k) {
+        for (int c = c_first; c < nC; c = next_chunk(a.chunk_mask, c), ++k) {
           const int pb = k & 1, st = k % kVStages;
           if (!wait_or_abort(s, &s.vfull[st], (k / kVStages) & 1, p.err)) { ok = false; break; }
           if (!wait_or_abort(s, &s.p_full[pb], (k >> 1) & 1, p.err)) { ok = false; break; }
@@ -468,7 +484,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           const uint32_t pa = tmem + kPCol + 64 * pb;  // 16 keys = 8 packed columns per step
           const int rows = chunk_rows(c);
           for (int kk = 0; kk < rows / 16; ++kk) {
-            const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (c != c_first || kk > 0) ? 1u : 0u;
             // V: rows = keys (K dim), 128-byte rows per 64-column half: MN-major B, SBO = 8 rows
             mma_bf16_ta(tmem + kOCol + 64 * ob, pa + 8 * kk, dv + uint32_t(kk * 2048 >> 4), id_pv, acc);
             mma_bf16_ta(tmem + (16u << 16) + kOCol + 64 * ob, pa + (16u << 16) + 8 * kk,
@@ -496,7 +512,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       float mref = -INFINITY;  // reference max (log2 units) the P values are taken against
       float lsum = 0.f;        // sum of the rows' weights against mref
       bool ok = true;
-      for (int c = 0; c < nC; ++c, ++k) {
+      for (int c = c_first; c < nC; c = next_chunk(a.chunk_mask, c), ++k) {
         const int sb = k % kSBufs, pb = k & 1;
         const uint64_t vm = s.vmask[ob][c][half];
         const bool all_valid = __all_sync(0xffffffffu, vm == ~0ull);
@@ -527,7 +543,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
         // P buffer pb free again means P_{k-2} V_{k-2} has landed; only after that does the
         // parity wait on pv_done below identify P_{k-1} V_{k-1} unambiguously
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.p_empty[pb], ((k >> 1) & 1) ^ 1, p.err))) { ok = false; break; }
-        if (c == 0) {
+        if (c == c_first) {
           mref = cmax;  // O is still empty: the reference moves for free
         } else if (__any_sync(0xffffffffu, cmax > mref + kRescaleThreshold)) {
           // rows whose max grew by more than 2^8: rescale their O (after the P V MMAs
@@ -605,7 +621,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       }
       if (lane < 2 * nC)
         s.vmask[i & 1][lane >> 1][lane & 1] =
-            view_mask(p, 64 * lane, len < p.W ? int(len) : p.W, sinfo, len > 0);
+            view_mask(p, 64 * lane, len < p.W ? int(len) : p.W, sinfo, len > 0, a.views);
     };
     if (warp == 8) {
       grid_dependency_wait();  // the counters are state a preceding commit writes
@@ -628,7 +644,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       tmem_ld32(trow + kOCol + 64 * ob + 32, o + 32);
       tc_fence_before();
       mbar_arrive(&s.o_free[ob]);
-      const float inv = 1.0f / lsum;
+      const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;  // no valid row in the views: zeros
       const int zrow = (b * a.lcount + lc) * p.B;  // the tile's first query of the block
       if constexpr (kOutF32) {
         const int qi = row / grp, jj = row - qi * grp;
@@ -750,8 +766,8 @@ int tc_prepare(const Dev& p, TcPlan* plan) {
 }
 
 cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
-                             const void* bk, const void* bv, int64_t bstride, float scale, void* out,
-                             int sms, bool after_commit, cudaStream_t stream) {
+                             const void* bk, const void* bv, int64_t bstride, float scale, int views,
+                             void* out, int sms, bool after_commit, cudaStream_t stream) {
   // Q in, and a bf16 O out, are [b, lcount, B, Hq, D]: one tile is the box (64 columns,
   // the group's heads, the block's queries) at (0 or 64, g * group, first query)
   CUtensorMap qmap, omap;
@@ -771,6 +787,20 @@ cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcoun
   a.bstride = bstride;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
+  // chunks holding rows of a view that takes part are streamed; the last chunk always is
+  // (it carries the boundary row), its arena rows only when a view needs them
+  a.views = views;
+  const bool win = (views & LS_VIEW_WINDOW) != 0, sum = (views & LS_VIEW_SUMMARY) != 0;
+  for (int c = 0; c < plan.n_chunks; ++c) {
+    const int lo = c * kChunk, hi = lo + kChunk < p.R ? lo + kChunk : p.R;  // arena rows [lo, hi)
+    const bool need = (win && lo < p.W) || (sum && hi > (lo > p.W ? lo : p.W));
+    if (c == plan.n_chunks - 1) {
+      a.chunk_mask |= 1u << c;
+      a.tail_load = need ? 1 : 0;
+    } else if (need) {
+      a.chunk_mask |= 1u << c;
+    }
+  }
   // at most one CTA per SM, tiles round robin, and no more CTAs than needed for the
   // fewest tiles per CTA: every CTA then gets the same number of tiles (512 tiles on 148
   // SMs: 128 CTAs x 4 instead of 68 x 4 + 80 x 3). The stream is bandwidth-bound, so the

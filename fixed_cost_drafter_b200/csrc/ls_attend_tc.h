@@ -17,8 +17,9 @@ bool tc_supported(const Dev& p);
 int tc_prepare(const Dev& p, TcPlan* plan);
 // after_commit: launched right behind ls_commit_round's kernel on the same stream as its
 // programmatic dependent (the kernel waits on the device for the commit's writes).
+// views: non-zero OR of LS_VIEW_* (the views that take part in the softmax).
 cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
-                             const void* bk, const void* bv, int64_t bstride, float scale,
+                             const void* bk, const void* bv, int64_t bstride, float scale, int views,
                              void* out, int sms, bool after_commit, cudaStream_t stream);
 
 }  // namespace ls

@@ -3,9 +3,9 @@
 // layer, KV head); warp t runs the per-tensor body (ls_commit_body.cuh) for tensor t
 // (0 = K, 1 = V). Every KV head's CTA copies its slice of verify row a's hidden vector into
 // the boundary view, and the last of the (sequence, layer)'s CTAs to arrive (an arrival
-// counter) writes the new counters, after every CTA has read the old ones. The slice's
-// loads and the arrival are issued right after the scan, so their round trips overlap
-// the commit's stores.
+// counter) writes the new counters, after every CTA has read the old ones. The scan needs
+// only the counters and token ids; the bulk inputs, the slice's loads and the arrival are
+// all issued right after it, in one round trip.
 #include "ls_commit_body.cuh"
 
 namespace ls {

@@ -2,10 +2,11 @@
 // verification pass (LongSpark paper page, Figure 2 caption (a)-(b); Figure 3 caption:
 // the summary is updated from only the newly retained rows N, Delta = |N| <= B + 1).
 // One warp handles one tensor (K or V) of one KV head, in two phases:
-//   load_scan  every load that does not depend on the accept scan is issued first
-//              (counters, token ids, all B + 1 verify rows, the fp32 partial / global
-//              sums), so the commit costs one memory round trip; then the greedy accept
-//              scan (two ballots cover B <= 64 drafts): a, Delta = a + 1.
+//   load_scan  the counters and token ids first, then the greedy accept scan (two
+//              ballots cover B <= 64 drafts): a, Delta = a + 1. Only then are the bulk
+//              inputs issued (all B + 1 verify rows, the fp32 partial / global sums), so
+//              the few scan inputs do not queue behind them and the loads that need a
+//              (the boundary slice) join the same round trip.
 //   apply      rows 0..a go to ring slot (len + i) mod W with 16-byte stores, and the same
 //              registers are summed into the rows that close the open segments (i < c) and
 //              the rows that open the next ones (i >= c), reduced across the row groups of
@@ -16,7 +17,7 @@
 //              sit at the single multiple of s_0 in (len, len + Delta], i.e. at
 //              c = s_0 - len mod s_0.
 // Between the phases the caller can issue work that needs a (the boundary slice's loads,
-// the arrival counter), so those round trips overlap the stores.
+// the arrival counter), so those round trips overlap the bulk loads.
 #pragma once
 #include "ls_common.cuh"
 
@@ -69,6 +70,24 @@ __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int 
     const int i = 32 * w + lane;
     mism[w] = i < p.B && draft[int64_t(b) * p.B + i] != target[int64_t(b) * (p.B + 1) + i];
   }
+  // greedy acceptance: first i with draft[i] != target[i], else B
+  const unsigned m0 = __ballot_sync(0xffffffffu, mism[0]);
+  const unsigned m1 = __ballot_sync(0xffffffffu, mism[1]);
+  const int a = m0 ? __ffs(m0) - 1 : (m1 ? 32 + __ffs(m1) - 1 : p.B);
+  // scale k closes a segment this round exactly when its own distance to the next
+  // boundary is <= Delta (then that distance equals the split row)
+  unsigned closes = 0;
+#pragma unroll
+  for (int k = 0; k < NSC; ++k)
+    if (p.scales[k] - (len - nseg[k] * p.scales[k]) <= a + 1) closes |= 1u << k;
+  cs.a = a;
+  cs.len = len;
+  cs.newlen = len + a + 1;
+#pragma unroll
+  for (int k = 0; k < kMaxScales; ++k) cs.nseg[k] = nseg[k];
+  cs.closes = closes;
+  // the rest of the round's inputs: issued once a is known, so they share one round trip
+  // with the loads the caller issues next (the boundary slice at verify row a)
   const T* src = vsrc + int64_t(bl) * (p.B + 1) * row_stride + int64_t(h) * p.D + cb;
 #pragma unroll
   for (int j = 0; j < ROWS; ++j) {
@@ -92,23 +111,6 @@ __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int 
       }
     }
   }
-
-  // greedy acceptance: first i with draft[i] != target[i], else B
-  const unsigned m0 = __ballot_sync(0xffffffffu, mism[0]);
-  const unsigned m1 = __ballot_sync(0xffffffffu, mism[1]);
-  const int a = m0 ? __ffs(m0) - 1 : (m1 ? 32 + __ffs(m1) - 1 : p.B);
-  // scale k closes a segment this round exactly when its own distance to the next
-  // boundary is <= Delta (then that distance equals the split row)
-  unsigned closes = 0;
-#pragma unroll
-  for (int k = 0; k < NSC; ++k)
-    if (p.scales[k] - (len - nseg[k] * p.scales[k]) <= a + 1) closes |= 1u << k;
-  cs.a = a;
-  cs.len = len;
-  cs.newlen = len + a + 1;
-#pragma unroll
-  for (int k = 0; k < kMaxScales; ++k) cs.nseg[k] = nseg[k];
-  cs.closes = closes;
 }
 
 template <typename T, int ROWS, int NSC>

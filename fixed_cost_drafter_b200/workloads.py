@@ -213,15 +213,20 @@ class DeviceRun:
         F.ls_commit_round(self.state, self.draft[r], self.target[r], inputs["vk"][i], inputs["vv"][i],
                           inputs["vh"][i], self.accept_len, self.next_token, self.stream)
 
-    def attend(self, inputs, r, out, layer_begin=0, layer_count=None):
+    def attend(self, inputs, r, out, layer_begin=0, layer_count=None, views=None):
+        """ls_draft_attend (views None) or ls_draft_attend_views with an LS_VIEW_* mask."""
         wl = self.wl
         lc = wl.n_layers if layer_count is None else layer_count
         i = r - inputs["r0"]
         q = inputs["q"][i]
         if lc != wl.n_layers or layer_begin != 0:
             q = q[:, layer_begin:layer_begin + lc].contiguous()
-        F.ls_draft_attend(self.state, layer_begin, lc, q, self.boundary_k, self.boundary_v, wl.hidden,
-                          self.softmax_scale, out, self.stream)
+        if views is None:
+            F.ls_draft_attend(self.state, layer_begin, lc, q, self.boundary_k, self.boundary_v, wl.hidden,
+                              self.softmax_scale, out, self.stream)
+        else:
+            F.ls_draft_attend_views(self.state, layer_begin, lc, q, self.boundary_k, self.boundary_v, wl.hidden,
+                                    self.softmax_scale, views, out, self.stream)
 
     def round(self, inputs, r, out):
         """ls_round: commit and attention over all layers in one call (boundary keys and

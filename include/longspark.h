@@ -72,6 +72,13 @@ extern "C" {
 #define LS_DEVERR_WAIT_TIMEOUT 0x2  /* an mbarrier wait exceeded its iteration limit     */
 #define LS_DEVERR_ORDER        0x4  /* prefill chunk does not continue the state          */
 
+/* ---- views (Figure 2 caption (b); the component ablations of Table 5) -------- */
+#define LS_VIEW_BOUNDARY 0x1        /* the boundary state (one key/value row)          */
+#define LS_VIEW_WINDOW   0x2        /* the recent KV window (W ring rows)              */
+#define LS_VIEW_SUMMARY  0x4        /* the global context summary (segment means per
+                                       scale, partial means, global mean)             */
+#define LS_VIEW_ALL      0x7
+
 /* ---- dtypes and flags -------------------------------------------------------- */
 #define LS_F32  0
 #define LS_BF16 1
@@ -210,6 +217,28 @@ LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t laye
                     const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
                     int64_t boundary_stride, float softmax_scale, void* d_out,
                     cudaStream_t stream);
+
+/* ls_draft_attend over a subset of the views: the drafter of a component ablation
+ * (Table 5: without the global summary, without the boundary state, without the recent
+ * KV window). `views` is a non-zero OR of LS_VIEW_*; the rows of the other views take
+ * no part in the softmax, and the kernels do not read them where whole 128-row chunks
+ * (or the summary rows of the last chunk) belong to left-out views. A query row whose
+ * remaining views hold no valid row (e.g. the window alone before the first commit)
+ * gets an all-zero output. Other arguments and errors as ls_draft_attend;
+ * LS_ERR_INVALID_ARG when `views` is 0 or has bits outside LS_VIEW_ALL.            */
+LS_API int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer_count,
+                                 const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
+                                 int64_t boundary_stride, float softmax_scale, int32_t views,
+                                 void* d_out, cudaStream_t stream);
+
+/* Bytes of the drafting state that a drafter with the given views keeps (the state-size
+ * side of Table 5): the counters always; LS_VIEW_WINDOW the ring rows (b*L*Hkv*W*2*D
+ * elements); LS_VIEW_SUMMARY the fp32 segment means, partial and global sums plus their
+ * attention-dtype copies (b*L*Hkv*2*D*(nsc*(slots+1)+1) of each); LS_VIEW_BOUNDARY the
+ * boundary hidden vectors (b*L*hidden elements). Region sizes without the 256-byte
+ * alignment padding that ls_state_bytes adds between regions. 0 for an invalid config
+ * or `views` outside LS_VIEW_ALL.                                                   */
+LS_API size_t ls_view_state_bytes(const ls_config* cfg, int32_t views);
 
 /* One whole decoding round: ls_commit_round, then ls_draft_attend over all layers, for
  * drafters whose boundary keys/values are slices of the new boundary hidden vector:

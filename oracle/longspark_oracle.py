@@ -52,6 +52,12 @@ import numpy as np
 F32 = "f32"
 BF16 = "bf16"
 
+# the three views (Figure 2 caption (b)); Table 5 ablates each of them
+VIEW_BOUNDARY = 0x1
+VIEW_WINDOW = 0x2
+VIEW_SUMMARY = 0x4
+VIEW_ALL = 0x7
+
 
 # ----------------------------------------------------------------------------------
 # configuration and exact input conversion
@@ -284,26 +290,44 @@ def attention_slots(sh: Shapes, v: Views, l: int, g: int, boundary_k: np.ndarray
     return np.stack(keys), np.stack(vals), np.array(valid, dtype=bool)
 
 
+def view_of_slots(sh: Shapes) -> np.ndarray:
+    """The view (VIEW_*) each of the S attention slots belongs to, in slot order."""
+    n_summary = sh.n_attn_slots - 1 - sh.window
+    return np.array([VIEW_BOUNDARY] + [VIEW_WINDOW] * sh.window + [VIEW_SUMMARY] * n_summary)
+
+
 def draft_attend(sh: Shapes, v: Views, q: np.ndarray, boundary_k: np.ndarray,
-                 boundary_v: np.ndarray, softmax_scale: float) -> np.ndarray:
+                 boundary_v: np.ndarray, softmax_scale: float, views: int = VIEW_ALL,
+                 return_lse: bool = False):
     """Figure 2 (c): block attention of the B drafter queries over the views.
 
     ``q`` is [L][B][Hq][D] fp64; returns [L][B][Hq][D] fp64. Softmax in fp64 with
     masked slots at -inf; the B queries see the same key set (no causal mask).
+
+    ``views`` (OR of VIEW_*): only the slots of these views take part (Table 5's
+    component ablations drop one view each). A row left with no valid slot gets zeros.
+    With ``return_lse`` also returns the natural-log partition function of every row,
+    [L][B][Hq] (-inf for a row with no valid slot).
     """
     out = np.zeros_like(q, dtype=np.float64)
+    lse = np.full(q.shape[:3], -np.inf)
     grp = sh.group
+    keep = (view_of_slots(sh) & views) != 0
     for l in range(sh.n_layers):
         for qh in range(sh.n_q_heads):
             g = qh // grp
             K, V, ok = attention_slots(sh, v, l, g, boundary_k, boundary_v)
+            ok = ok & keep
+            if not ok.any():
+                continue  # nothing to attend to: zero output
             logits = (q[l, :, qh, :] @ K.T) * softmax_scale  # [B][S]
             logits[:, ~ok] = -np.inf
             m = logits.max(axis=1, keepdims=True)
             w = np.exp(logits - m)
-            w /= w.sum(axis=1, keepdims=True)
-            out[l, :, qh, :] = w @ V
-    return out
+            z = w.sum(axis=1, keepdims=True)
+            out[l, :, qh, :] = (w / z) @ V
+            lse[l, :, qh] = (m + np.log(z))[:, 0]
+    return (out, lse) if return_lse else out
 
 
 # ----------------------------------------------------------------------------------

@@ -73,14 +73,15 @@ def tile_views(wl, b, l, h, P, accepts_b, scale=None):
     return sh, O.views_from_scratch(sh, k, v, k.shape[2])
 
 
-def tile_attend(wl, sh, views, b, l, g, r, hidden_vec):
-    """Oracle attention output fp64 [B][grp][D] of tile (b, l, g) with round r's queries."""
+def tile_attend(wl, sh, views, b, l, g, r, hidden_vec, view_set=O.VIEW_ALL):
+    """Oracle attention output fp64 [B][grp][D] of tile (b, l, g) with round r's queries,
+    over the views in view_set (VIEW_*)."""
     D, H = wl.head_dim, wl.n_kv_heads
     hv = O.to_f64(hidden_vec, wl.dtype)
     bk = hv[g * D:(g + 1) * D].reshape(1, 1, D)
     bv = hv[H * D + g * D:H * D + (g + 1) * D].reshape(1, 1, D)
     q = queries(wl, r, b, l, g)
-    return O.draft_attend(sh, views, q, bk, bv, 1.0 / np.sqrt(D))[0]
+    return O.draft_attend(sh, views, q, bk, bv, 1.0 / np.sqrt(D), views=view_set)[0]
 
 
 # ---- comparisons (tolerances as stated for the path) ---------------------------------

@@ -52,6 +52,27 @@ def test_layout_sizes():
     assert 13.2e6 < y.total_bytes / 16 < 13.5e6
 
 
+def test_view_state_bytes():
+    """Per-view state sizes at Qwen3-8B shapes (the state side of Table 5's ablations):
+    per sequence the window is 4 layers x 8 heads x 512 rows x (K, V) x 128 x 2 B
+    = 8.39 MB, the summary 100 rows x (fp32 + the bf16 copy) = 4.92 MB and the boundary
+    4 x 4096 x 2 B = 32 KB; the counters are always kept."""
+    c = _cfg()
+    b, L, H, D = 16, 4, 8, 128
+    counters = b * L * 4 * 8
+    win = b * L * H * 512 * 2 * D * 2
+    summ = b * L * H * 2 * 100 * D * (4 + 2)
+    bnd = b * L * 4096 * 2
+    assert win / b == 8388608 and summ / b == 4915200 and bnd / b == 32768
+    want = {F.LS_VIEW_WINDOW: win, F.LS_VIEW_SUMMARY: summ, F.LS_VIEW_BOUNDARY: bnd}
+    for views in range(1, 8):
+        n = counters + sum(v for bit, v in want.items() if views & bit)
+        assert F.ls_view_state_bytes(c, views) == n, views
+    everything = F.ls_view_state_bytes(c, F.LS_VIEW_ALL)
+    assert everything <= F.ls_state_bytes(c) < everything + 9 * 256  # + alignment padding
+    assert F.ls_view_state_bytes(c, 8) == 0 and F.ls_view_state_bytes(_cfg(batch=0), 1) == 0
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(batch=0), F.LS_ERR_INVALID_ARG),
     (dict(n_q_heads=30), F.LS_ERR_SHAPE),

@@ -36,7 +36,7 @@ def _run_full(wl, rounds=None, prefill_chunk=None, check_every_round=False):
     return run, out, acc_gpu
 
 
-def _sampled_check(run, wl, out, tiles):
+def _sampled_check(run, wl, out, tiles, view_set=None):
     st = run.read_state()
     R = run.rounds
     draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
@@ -54,7 +54,8 @@ def _sampled_check(run, wl, out, tiles):
         OS.check_tile_state(wl, st, b, l, h, views)
         hid = OS.boundary_hidden(wl, b, l, R - 1, int(acc[R - 1, b]))
         assert np.array_equal(st["boundary"][b, l], hid)
-        ref = OS.tile_attend(wl, sh, views, b, l, h, R - 1, hid)
+        ref = OS.tile_attend(wl, sh, views, b, l, h, R - 1, hid,
+                             OS.O.VIEW_ALL if view_set is None else view_set)
         o = out[b, l].view(wl.block, wl.n_q_heads, wl.head_dim)[:, h * wl.group:(h + 1) * wl.group]
         got = o.float().cpu().numpy().astype(np.float64)
         exc = OS.attend_error_excess(got, ref, o.dtype == torch.float32)
@@ -72,6 +73,22 @@ def test_full_config(name):
     run, out, _ = _run_full(wl)
     assert run.error() == (F.LS_OK, 0)
     _sampled_check(run, wl, out, TILES)
+
+
+def test_full_config_view_ablations():
+    """Table 5's three ablations at the bench workload (4 tiles per CTA, W = 512: the four
+    ring chunks skipped without the window, the 100 summary rows not loaded without the
+    summary), on the sampled tiles."""
+    wl = WL.CONFIGS["qwen3_8b_64k"]
+    run, out, _ = _run_full(wl)
+    inp = run.make_round_inputs(run.rounds - 1, 1)
+    for view_set in (F.LS_VIEW_WINDOW | F.LS_VIEW_BOUNDARY, F.LS_VIEW_WINDOW | F.LS_VIEW_SUMMARY,
+                     F.LS_VIEW_SUMMARY | F.LS_VIEW_BOUNDARY):
+        out.fill_(float("nan"))
+        run.attend(inp, run.rounds - 1, out, views=view_set)
+        torch.cuda.synchronize()
+        assert run.error() == (F.LS_OK, 0)
+        _sampled_check(run, wl, out, TILES, view_set)
 
 
 @pytest.mark.parametrize("prefix,batch,mean", [(4096, 1, 2.5), (16384, 4, 4.0), (131072, 64, 6.0)])

@@ -36,8 +36,9 @@ def _out_tile(out, wl, b, l, g):
     return o.float().cpu().numpy().astype(np.float64)
 
 
-def _check_run_against_oracle(run, wl, rounds_done, out, r_last, tiles=None):
-    """Every (or the given) tile's state and attention output vs oracle recompute."""
+def _check_run_against_oracle(run, wl, rounds_done, out, r_last, tiles=None, view_set=None):
+    """Every (or the given) tile's state and attention output vs oracle recompute
+    (attention over the views in view_set, all views when None)."""
     st = run.read_state()
     draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
     acc = (OS.accepts_from_ids(draft[:rounds_done], target[:rounds_done]) if rounds_done
@@ -51,7 +52,8 @@ def _check_run_against_oracle(run, wl, rounds_done, out, r_last, tiles=None):
         hid = OS.boundary_hidden(wl, b, l, rounds_done - 1, int(acc[rounds_done - 1, b]) if rounds_done else 0)
         assert np.array_equal(st["boundary"][b, l], hid), ("boundary", b, l)
         if out is not None:
-            ref = OS.tile_attend(wl, sh, views, b, l, h, r_last, hid)
+            ref = OS.tile_attend(wl, sh, views, b, l, h, r_last, hid,
+                                 O.VIEW_ALL if view_set is None else view_set)
             got = _out_tile(out, wl, b, l, h)
             exc = OS.attend_error_excess(got, ref, out.dtype == torch.float32)
             assert exc <= 0, ("attend", b, l, h, float(np.abs(got - ref).max()), exc)
@@ -121,6 +123,49 @@ def test_mid_ragged_all_tiles(force_simt, out_f32):
         if r in (0, 7, wl.rounds - 1):
             torch.cuda.synchronize()
             _check_run_against_oracle(run, wl, r + 1, out, r)
+    assert run.error() == (F.LS_OK, 0)
+
+
+VIEW_SETS = list(range(1, 8))
+
+
+@pytest.mark.parametrize("force_simt", [False, True], ids=["tensor_cores", "cuda_cores"])
+@pytest.mark.parametrize("view_set", VIEW_SETS, ids=[f"views{v}" for v in VIEW_SETS])
+def test_view_ablations(force_simt, view_set):
+    """ls_draft_attend_views (Table 5's component ablations) on every non-empty subset of the
+    views. W = 128 and R = 144: without the window the kernel skips the ring chunk, without
+    the summary it loads none of the last chunk's arena rows."""
+    wl = _mid(rounds=3, flags=F.LS_FLAG_FORCE_SIMT if force_simt else 0)
+    run = WL.DeviceRun(wl)
+    assert F.ls_attend_uses_tensor_cores(run.state) == (not force_simt)
+    run.prefill()
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    for r in range(wl.rounds):
+        run.commit(inp, r)
+    out.fill_(float("nan"))
+    run.attend(inp, wl.rounds - 1, out, views=view_set)
+    torch.cuda.synchronize()
+    _check_run_against_oracle(run, wl, wl.rounds, out, wl.rounds - 1, view_set=view_set)
+    assert run.error() == (F.LS_OK, 0)
+
+
+@pytest.mark.parametrize("force_simt", [False, True], ids=["tensor_cores", "cuda_cores"])
+def test_view_ablations_empty_state(force_simt):
+    """Before any row is retained the window and the summary have no valid row: zeros."""
+    wl = _mid(rounds=1, flags=F.LS_FLAG_FORCE_SIMT if force_simt else 0)
+    run = WL.DeviceRun(wl)  # initialised, never prefilled: len = 0
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    for view_set in (F.LS_VIEW_WINDOW, F.LS_VIEW_SUMMARY, F.LS_VIEW_WINDOW | F.LS_VIEW_SUMMARY):
+        out.fill_(float("nan"))
+        run.attend(inp, 0, out, views=view_set)
+        torch.cuda.synchronize()
+        assert not out.float().abs().sum().item() and not torch.isnan(out.float()).any().item(), view_set
+    with pytest.raises(F.LsError):
+        run.attend(inp, 0, out, views=0)
+    with pytest.raises(F.LsError):
+        run.attend(inp, 0, out, views=8)
     assert run.error() == (F.LS_OK, 0)
 
 

@@ -93,8 +93,21 @@ def _retain_global_skips(sh, v, k_row, v_row):
         v.glob_v -= v_row
 
 
+def _views_global_in_window(sh):
+    # the global-mean slot (the last one) attributed to the window view
+    vs = ORIG["view_of_slots"](sh).copy()
+    vs[-1] = M.VIEW_WINDOW
+    return vs
+
+
+def _views_boundary_in_summary(sh):
+    vs = ORIG["view_of_slots"](sh).copy()
+    vs[0] = M.VIEW_SUMMARY
+    return vs
+
+
 ORIG = {n: getattr(M, n) for n in ("accept_scan", "retain_row", "views_from_scratch",
-                                   "attention_slots", "draft_attend")}
+                                   "attention_slots", "draft_attend", "view_of_slots")}
 
 CASES = [
     ("accept_scan", _scan_off_by_one, [P.test_scan_golden_examples]),
@@ -104,6 +117,8 @@ CASES = [
     ("draft_attend", _attend_wrong_group, [P.test_attend_matches_torch_sdpa]),
     ("attention_slots", _slots_window_mask_off_by_one, [P.test_mask_counts]),
     ("retain_row", _retain_global_skips, [lambda: P.test_ramp_closed_forms(200)]),
+    ("view_of_slots", _views_global_in_window, [P.test_views_constant_values_per_view]),
+    ("view_of_slots", _views_boundary_in_summary, [P.test_views_boundary_alone_is_its_value]),
 ]
 
 

@@ -316,6 +316,85 @@ def test_attend_special_cases():
     assert ok.sum() == 1 + 4 + (2 + 1) + (2 + 1) + 1
 
 
+# ---------------------------------------------------------------------------------
+# view subsets (Table 5: the component ablations drop one view each)
+# ---------------------------------------------------------------------------------
+def test_view_of_slots_counts():
+    """Slot order [boundary, W window slots, the summary slots]: 1 / W / nsc*(slots+1)+1."""
+    sh = _shapes()
+    vs = O.view_of_slots(sh)
+    assert len(vs) == sh.n_attn_slots
+    assert (vs == O.VIEW_BOUNDARY).sum() == 1 and vs[0] == O.VIEW_BOUNDARY
+    assert (vs == O.VIEW_WINDOW).sum() == sh.window and (vs[1:1 + sh.window] == O.VIEW_WINDOW).all()
+    assert (vs == O.VIEW_SUMMARY).sum() == len(sh.scales) * (sh.slots + 1) + 1
+
+
+def test_views_boundary_alone_is_its_value():
+    """A softmax over the single boundary slot has weight 1: the output is that value row."""
+    sh = _shapes()
+    rng = np.random.default_rng(11)
+    v = _random_views(sh, rng, 37, 6)
+    q = rng.standard_normal((2, 4, 4, 8))
+    bk, bv = rng.standard_normal((2, 2, 8)), rng.standard_normal((2, 2, 8))
+    out, lse = O.draft_attend(sh, v, q, bk, bv, 0.3, views=O.VIEW_BOUNDARY, return_lse=True)
+    for l in range(2):
+        for qh in range(4):
+            g = qh // 2
+            assert np.array_equal(out[l, :, qh], np.broadcast_to(bv[l, g], (4, 8)))
+            np.testing.assert_allclose(lse[l, :, qh], 0.3 * (q[l, :, qh] @ bk[l, g]), rtol=0, atol=1e-14)
+
+
+def test_views_constant_values_per_view():
+    """Window values all 1, summary values all 0, boundary value 2: attending over one view
+    returns that view's constant whatever the keys, and the full attention lies strictly
+    between (every view has a valid slot)."""
+    sh = _shapes()
+    rng = np.random.default_rng(12)
+    v = _random_views(sh, rng, 61, 7)
+    v.ring_v[:] = 1.0
+    for k in range(len(sh.scales)):
+        v.seg_v[k][:] = 0.0
+        v.part_v[k][:] = 0.0
+    v.glob_v[:] = 0.0
+    q = rng.standard_normal((2, 4, 4, 8))
+    bk, bv = rng.standard_normal((2, 2, 8)), np.full((2, 2, 8), 2.0)
+    for views, want in [(O.VIEW_WINDOW, 1.0), (O.VIEW_SUMMARY, 0.0), (O.VIEW_BOUNDARY, 2.0)]:
+        out = O.draft_attend(sh, v, q, bk, bv, 0.5, views=views)
+        np.testing.assert_allclose(out, want, rtol=0, atol=1e-13)
+    out = O.draft_attend(sh, v, q, bk, bv, 0.5)
+    assert (out > 0).all() and (out < 2).all()
+
+
+@pytest.mark.parametrize("split", [(O.VIEW_BOUNDARY, O.VIEW_WINDOW | O.VIEW_SUMMARY),
+                                   (O.VIEW_WINDOW, O.VIEW_BOUNDARY | O.VIEW_SUMMARY),
+                                   (O.VIEW_SUMMARY, O.VIEW_BOUNDARY | O.VIEW_WINDOW)])
+def test_views_partition_identity(split):
+    """Softmax over a disjoint union: Z = Z_A + Z_B and O = (Z_A O_A + Z_B O_B) / Z."""
+    sh = _shapes()
+    rng = np.random.default_rng(13)
+    v = _random_views(sh, rng, 53, 8)
+    q = rng.standard_normal((2, 4, 4, 8))
+    bk, bv = rng.standard_normal((2, 2, 8)), rng.standard_normal((2, 2, 8))
+    oa, la = O.draft_attend(sh, v, q, bk, bv, 0.4, views=split[0], return_lse=True)
+    ob, lb = O.draft_attend(sh, v, q, bk, bv, 0.4, views=split[1], return_lse=True)
+    o, lz = O.draft_attend(sh, v, q, bk, bv, 0.4, return_lse=True)
+    np.testing.assert_allclose(lz, np.logaddexp(la, lb), rtol=1e-13, atol=1e-13)
+    wa, wb = np.exp(la - lz)[..., None], np.exp(lb - lz)[..., None]
+    np.testing.assert_allclose(o, wa * oa + wb * ob, rtol=1e-12, atol=1e-13)
+
+
+def test_views_with_no_valid_slot_give_zeros():
+    """Before any row is retained the window and the summary hold no valid slot."""
+    sh = _shapes()
+    rng = np.random.default_rng(14)
+    v0 = O.empty_views(sh)
+    q = rng.standard_normal((2, 4, 4, 8))
+    bk, bv = rng.standard_normal((2, 2, 8)), rng.standard_normal((2, 2, 8))
+    for views in (O.VIEW_WINDOW, O.VIEW_SUMMARY, O.VIEW_WINDOW | O.VIEW_SUMMARY):
+        out, lse = O.draft_attend(sh, v0, q, bk, bv, 1.0, views=views, return_lse=True)
+        assert not out.any() and np.isneginf(lse).all()
+
+
 def test_mask_counts():
     """Valid slot count = boundary + min(len, W) + per scale min(n_c, slots) + [partial] + [len>0]."""
     sh = _shapes(n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=2, window=16,

@@ -331,6 +331,61 @@ def draft_attend(sh: Shapes, v: Views, q: np.ndarray, boundary_k: np.ndarray,
 
 
 # ----------------------------------------------------------------------------------
+# stochastic acceptance (T > 0)
+# ----------------------------------------------------------------------------------
+# The pages compare greedy decoding (Table 3, T = 0) with sampled decoding (Table 1) but
+# print no acceptance rule for T > 0. The reading taken is standard speculative sampling
+# (Leviathan, Kalman and Matias 2023; Chen et al. 2023), position by position over the
+# block: draft i is kept when u_i * q_i(d_i) < p_i(d_i) (u_i uniform in [0, 1), the test
+# made in fp32 as the GPU makes it: it decides an integer); at the first rejection the
+# next token is drawn from the residual max(0, p_i - q_i), and after B acceptances from
+# p_B. The draws u_0..u_{B-1} and the final draw v are inputs.
+def accept_decisions(draft_ids, q_rows, p_rows, u):
+    """fp32 acceptance tests of one sequence: draft i kept iff u_i * q_i(d_i) < p_i(d_i).
+
+    q_rows [B][V], p_rows [B+1][V] (fp32 probabilities), u [B]. Returns a (leading kept
+    count) and the per-position decisions.
+    """
+    B = len(draft_ids)
+    keep = np.zeros(B, dtype=bool)
+    for i in range(B):
+        d = int(draft_ids[i])
+        qd, pd = np.float32(q_rows[i, d]), np.float32(p_rows[i, d])
+        keep[i] = np.float32(np.float32(u[i]) * qd) < pd
+    a = B
+    for i in range(B):
+        if not keep[i]:
+            a = i
+            break
+    return a, keep
+
+
+def sampling_weights(q_rows, p_rows, a):
+    """The distribution the next token is drawn from (unnormalised, fp64): the residual
+    max(0, p_a - q_a) after a rejection at position a < B, else p_B."""
+    B = q_rows.shape[0]
+    if a < B:
+        return np.maximum(0.0, p_rows[a].astype(np.float64) - q_rows[a].astype(np.float64))
+    return p_rows[B].astype(np.float64)
+
+
+def inverse_cdf(w, v):
+    """Smallest t with sum(w[:t+1]) > v * sum(w); the last index with w > 0 if rounding
+    leaves none (v < 1). w >= 0 with a positive sum."""
+    c = np.cumsum(w)
+    t = int(np.searchsorted(c, v * c[-1], side="right"))
+    if t >= len(w):
+        t = int(np.nonzero(w > 0)[0][-1])
+    return t
+
+
+def accept_sampled(draft_ids, q_rows, p_rows, u, v):
+    """One sequence's stochastic acceptance: (a, next token)."""
+    a, _ = accept_decisions(draft_ids, q_rows, p_rows, u)
+    return a, inverse_cdf(sampling_weights(q_rows, p_rows, a), v)
+
+
+# ----------------------------------------------------------------------------------
 # readout helpers (views in the same terms the device state uses)
 # ----------------------------------------------------------------------------------
 def segment_count(n: int, s: int) -> int:

@@ -106,8 +106,21 @@ def _views_boundary_in_summary(sh):
     return vs
 
 
+def _residual_swapped(q_rows, p_rows, a):
+    # max(0, q - p) instead of max(0, p - q) after a rejection
+    if a < q_rows.shape[0]:
+        return np.maximum(0.0, q_rows[a].astype(np.float64) - p_rows[a].astype(np.float64))
+    return p_rows[-1].astype(np.float64)
+
+
+def _accept_ratio_inverted(draft_ids, q_rows, p_rows, u):
+    # keep when u * p < q
+    return ORIG["accept_decisions"](draft_ids, p_rows[:len(draft_ids)], q_rows, u)
+
+
 ORIG = {n: getattr(M, n) for n in ("accept_scan", "retain_row", "views_from_scratch",
-                                   "attention_slots", "draft_attend", "view_of_slots")}
+                                   "attention_slots", "draft_attend", "view_of_slots",
+                                   "accept_decisions", "sampling_weights")}
 
 CASES = [
     ("accept_scan", _scan_off_by_one, [P.test_scan_golden_examples]),
@@ -119,6 +132,8 @@ CASES = [
     ("retain_row", _retain_global_skips, [lambda: P.test_ramp_closed_forms(200)]),
     ("view_of_slots", _views_global_in_window, [P.test_views_constant_values_per_view]),
     ("view_of_slots", _views_boundary_in_summary, [P.test_views_boundary_alone_is_its_value]),
+    ("sampling_weights", _residual_swapped, [P.test_sampled_emits_target_distribution]),
+    ("accept_decisions", _accept_ratio_inverted, [P.test_sampled_emits_target_distribution]),
 ]
 
 

@@ -395,6 +395,74 @@ def test_views_with_no_valid_slot_give_zeros():
         assert not out.any() and np.isneginf(lse).all()
 
 
+# ---------------------------------------------------------------------------------
+# stochastic acceptance (speculative sampling, T > 0)
+# ---------------------------------------------------------------------------------
+def test_sampled_emits_target_distribution():
+    """The theorem of speculative sampling: with the draft token drawn from q, the token
+    emitted at a position is distributed exactly as the target's p. The oracle's decisions
+    are integrated over the draft token and a midpoint grid of both uniform draws."""
+    rng = np.random.default_rng(21)
+    V, N = 6, 4000
+    grid = (np.arange(N) + 0.5) / N
+    for _ in range(3):
+        q = rng.dirichlet(np.ones(V)).astype(np.float32)
+        p = rng.dirichlet(np.ones(V)).astype(np.float32)
+        p_rows = np.stack([p, rng.dirichlet(np.ones(V)).astype(np.float32)])
+        emitted = np.zeros(V)
+        for d in range(V):
+            rej_next = np.zeros(V)
+            for v in grid:
+                rej_next[O.accept_sampled([d], q[None], p_rows, [0.999999], v)[1]] += 1.0 / N
+            for u in grid:
+                a, _ = O.accept_decisions([d], q[None], p_rows, [u])
+                if a == 1:
+                    emitted[d] += q[d] / N
+                else:
+                    emitted += q[d] / N * rej_next
+        np.testing.assert_allclose(emitted, p.astype(np.float64), rtol=0, atol=2.5 / N)
+
+
+def test_sampled_equal_distributions_accept_everything():
+    rng = np.random.default_rng(22)
+    B, V = 5, 11
+    q = rng.dirichlet(np.ones(V), size=B).astype(np.float32)
+    p_rows = np.concatenate([q, rng.dirichlet(np.ones(V), size=1).astype(np.float32)])
+    for _ in range(50):
+        d = rng.integers(0, V, B)
+        a, nxt = O.accept_sampled(d, q, p_rows, rng.random(B), rng.random())
+        assert a == B and p_rows[B, nxt] > 0
+
+
+def test_sampled_disjoint_support_rejects_first():
+    """A draft token the target gives no mass is always rejected; the residual is p."""
+    q = np.array([[0.5, 0.5, 0.0, 0.0]], dtype=np.float32)
+    p_rows = np.array([[0.0, 0.0, 0.25, 0.75], [0.25, 0.25, 0.25, 0.25]], dtype=np.float32)
+    for d in (0, 1):
+        for v, want in [(0.1, 2), (0.2499, 2), (0.26, 3), (0.99, 3)]:
+            assert O.accept_sampled([d], q, p_rows, [0.0], v) == (0, want)
+
+
+def test_inverse_cdf_boundaries():
+    w = np.array([1.0, 2.0, 3.0, 4.0])
+    assert [O.inverse_cdf(w, v) for v in (0.0, 0.05, 0.1, 0.29, 0.3, 0.95, 0.999)] == [0, 0, 1, 1, 2, 3, 3]
+    assert {O.inverse_cdf(np.array([0.0, 1.0, 0.0, 1.0]), v) for v in np.linspace(0, 0.999, 101)} == {1, 3}
+
+
+def test_sampled_decision_is_fp32():
+    """u * q rounded to fp32 before the comparison: with p set to that rounded product the
+    draft is rejected, although the exact product is below p."""
+    u, q = np.float32(0.1), np.float32(0.7)
+    prod32 = np.float32(u * q)
+    exact = float(u) * float(q)
+    assert exact < float(prod32)  # this pair rounds up
+    p_rows = np.zeros((2, 2), dtype=np.float32)
+    p_rows[0, 0], p_rows[0, 1] = prod32, 1 - prod32
+    q_rows = np.array([[q, 1 - q]], dtype=np.float32)
+    a, keep = O.accept_decisions([0], q_rows, p_rows, [u])
+    assert a == 0 and not keep[0]
+
+
 def test_mask_counts():
     """Valid slot count = boundary + min(len, W) + per scale min(n_c, slots) + [partial] + [len>0]."""
     sh = _shapes(n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=2, window=16,

@@ -428,6 +428,11 @@ def run_gpu(args):
         if status != F.LS_OK:
             raise RuntimeError(f"device error word {word:#x} after the ablation launches")
 
+    # stochastic acceptance (T > 0) at the Qwen3 vocabulary: its own measurement
+    sampled = None
+    if not args.no_sampling:
+        sampled = sampling_measure(F, run, wl, dev, flush, stream, evs, min(K, 200))
+
     # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
     graph_rps = None
     if not args.no_graph:
@@ -494,6 +499,7 @@ def run_gpu(args):
                       "commit_GBps": c_bytes / (float(np.mean(commit_ms)) / 1e3) / 1e9},
             "graph_rounds_per_s": graph_rps,
             "view_ablations": ablations,
+            "sampled_acceptance": sampled,
             "prefill": {"ms": prefill_ms, "bytes": prefill_b, "achieved_GBps": prefill_b / (prefill_ms / 1e3) / 1e9,
                         "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
             "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch,
@@ -510,6 +516,45 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+QWEN3_VOCAB = 151936
+
+
+def sampling_measure(F, run, wl, dev, flush, stream, evs, n):
+    """ls_accept_sampled at batch wl.batch, block wl.block and the Qwen3 vocabulary: fp32
+    probability rows (softmax of seeded normal logits, the target's close to the drafter's),
+    drafts drawn from the drafter's rows, seeded draws. Algorithmic bytes: the gathered test
+    values and the draw's rows (two after a rejection, one for the bonus draw)."""
+    import torch
+    b, B, V = wl.batch, wl.block, QWEN3_VOCAB
+    gen = torch.Generator(device=dev).manual_seed(20260)
+    zq = torch.randn((b, B, V), device=dev, generator=gen) * 2.0
+    q = torch.softmax(zq, -1)
+    zp = torch.cat([zq, zq[:, -1:]], 1) + 0.5 * torch.randn((b, B + 1, V), device=dev, generator=gen)
+    pr = torch.softmax(zp, -1)
+    del zq, zp
+    draft = torch.multinomial(q.view(-1, V), 1, generator=gen).view(b, B).to(torch.int32)
+    u = torch.rand((b, B + 1), device=dev, generator=gen)
+    acc = torch.empty(b, dtype=torch.int32, device=dev)
+    nxt = torch.empty(b, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        F.ls_accept_sampled(run.state, draft, q, pr, V, u, acc, nxt, stream)
+    for i in range(n):
+        flush.zero_()
+        evs[i][0].record(stream)
+        F.ls_accept_sampled(run.state, draft, q, pr, V, u, acc, nxt, stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    status, word = run.error()
+    if status != F.LS_OK:
+        raise RuntimeError(f"device error word {word:#x} after the sampling launches")
+    us = float(np.mean([e[0].elapsed_time(e[1]) for e in evs[:n]])) * 1e3
+    a = acc.cpu().numpy()
+    nbytes = int(b * 2 * B * 4 + b * (B + 1) * 4 + sum((2 if x < B else 1) * V * 4 for x in a))
+    del q, pr
+    return {"vocab": V, "batch": b, "block": B, "us": us, "bytes": nbytes, "GBps": nbytes / us / 1e3,
+            "accept_mean": float(a.mean()), "launches": n}
 
 
 class L2Flush:
@@ -639,6 +684,7 @@ def main(argv=None):
     ap.add_argument("--config", default=WORKLOAD)
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-ablations", action="store_true", help="skip the view-ablation attention timings")
+    ap.add_argument("--no-sampling", action="store_true", help="skip the stochastic-acceptance timing")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

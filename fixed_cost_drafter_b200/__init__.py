@@ -27,6 +27,7 @@ LS_ERR_SCRATCH_LIMIT = -7
 LS_DEVERR_PREFIX_LEN = 0x1
 LS_DEVERR_WAIT_TIMEOUT = 0x2
 LS_DEVERR_ORDER = 0x4
+LS_DEVERR_SAMPLE = 0x8
 LS_F32 = 0
 LS_BF16 = 1
 LS_FLAG_FORCE_SIMT = 0x1
@@ -40,7 +41,7 @@ LS_VIEW_ALL = 0x7
 EXPORTED = (
     "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",
     "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend",
-    "ls_draft_attend_views", "ls_view_state_bytes", "ls_round",
+    "ls_draft_attend_views", "ls_view_state_bytes", "ls_round", "ls_accept_sampled", "ls_commit_accepted",
     "ls_round_overlaps", "ls_attend_uses_tensor_cores",
     "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
 )
@@ -68,7 +69,7 @@ class ls_layout(ctypes.Structure):
         ("off_error", ctypes.c_size_t), ("off_sync", ctypes.c_size_t), ("off_kv", ctypes.c_size_t),
         ("off_seg_mean", ctypes.c_size_t), ("off_part_sum", ctypes.c_size_t),
         ("off_glob_sum", ctypes.c_size_t), ("off_boundary", ctypes.c_size_t),
-        ("kv_rows", ctypes.c_int32), ("elem_bytes", ctypes.c_int32),
+        ("kv_rows", ctypes.c_int32), ("elem_bytes", ctypes.c_int32), ("off_sample", ctypes.c_size_t),
     ]
 
 
@@ -81,6 +82,8 @@ def _load():
     sig = {
         "ls_state_bytes": (sz, [cfgp]),
         "ls_view_state_bytes": (sz, [cfgp, i32]),
+        "ls_accept_sampled": (ctypes.c_int, [vp, vp, vp, vp, i32, vp, vp, vp, vp]),
+        "ls_commit_accepted": (ctypes.c_int, [vp, vp, vp, vp, vp, vp]),
         "ls_get_layout": (ctypes.c_int, [cfgp, ctypes.POINTER(ls_layout)]),
         "ls_init_state": (ctypes.c_int, [cfgp, vp, sz, ctypes.POINTER(vp), vp]),
         "ls_prefill_workspace_bytes": (sz, [cfgp, i64, i64]),
@@ -212,6 +215,18 @@ def ls_draft_attend_views(state, layer_begin, layer_count, q, boundary_k, bounda
     _check("ls_draft_attend_views", _lib.ls_draft_attend_views(
         state, layer_begin, layer_count, _ptr(q), _ptr(boundary_k), _ptr(boundary_v),
         boundary_stride, float(softmax_scale), views, _ptr(out), _stream(stream)))
+
+
+def ls_accept_sampled(state, draft_ids, draft_probs, target_probs, vocab, uniforms, accept_len, next_token,
+                      stream=None) -> None:
+    _check("ls_accept_sampled", _lib.ls_accept_sampled(
+        state, _ptr(draft_ids), _ptr(draft_probs), _ptr(target_probs), vocab, _ptr(uniforms), _ptr(accept_len),
+        _ptr(next_token), _stream(stream)))
+
+
+def ls_commit_accepted(state, accept_len, verify_k, verify_v, verify_hidden, stream=None) -> None:
+    _check("ls_commit_accepted", _lib.ls_commit_accepted(
+        state, _ptr(accept_len), _ptr(verify_k), _ptr(verify_v), _ptr(verify_hidden), _stream(stream)))
 
 
 def ls_round(state, draft_ids, target_ids, verify_k, verify_v, verify_hidden, accept_len, next_token, q,

@@ -10,7 +10,9 @@
 namespace ls {
 cudaError_t launch_commit(const Dev& p, const int32_t* draft, const int32_t* target, const void* vk,
                           const void* vv, const void* vh, int32_t* accept_len, int32_t* next_token,
-                          cudaStream_t stream);
+                          const int32_t* given_a, cudaStream_t stream);
+cudaError_t launch_sample(const Dev& p, const int32_t* draft, const float* q, const float* pr, int vocab,
+                          const float* u, int32_t* accept_len, int32_t* next_token, cudaStream_t stream);
 bool simt_supported(const Dev& p);
 cudaError_t launch_attend_simt(const Dev& p, int lb, int lcount, const void* q, const void* bk,
                                const void* bv, int64_t bstride, float scale, int views, void* out,
@@ -119,6 +121,7 @@ int ls_get_layout(const ls_config* cfg, ls_layout* out) {
   out->off_part_sum = size_t(y.part);
   out->off_glob_sum = size_t(y.glob);
   out->off_boundary = size_t(y.boundary);
+  out->off_sample = size_t(y.sample);
   out->kv_rows = y.R;
   out->elem_bytes = y.elem;
   return LS_OK;
@@ -161,6 +164,8 @@ int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_st
   p.part = reinterpret_cast<float*>(base + y.part);
   p.glob = reinterpret_cast<float*>(base + y.glob);
   p.boundary = base + y.boundary;
+  p.samp_count = reinterpret_cast<int32_t*>(base + y.sample);
+  p.samp_part = reinterpret_cast<float*>(base + y.sample + int64_t(cfg->batch) * 4);
 
   st->use_tc = 0;
   if (!(cfg->flags & LS_FLAG_FORCE_SIMT) && ls::tc_supported(p)) {
@@ -236,7 +241,27 @@ int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_t
   if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden))
     return LS_ERR_INVALID_ARG;
   return cuda_status(ls::launch_commit(st->dev, d_draft_ids, d_target_ids, d_verify_k, d_verify_v,
-                                       d_verify_hidden, d_accept_len, d_next_token, stream));
+                                       d_verify_hidden, d_accept_len, d_next_token, nullptr, stream));
+}
+
+int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const float* d_draft_probs,
+                      const float* d_target_probs, int32_t vocab, const float* d_uniforms, int32_t* d_accept_len,
+                      int32_t* d_next_token, cudaStream_t stream) {
+  if (!st || !d_draft_ids || !d_draft_probs || !d_target_probs || !d_uniforms || !d_accept_len || !d_next_token)
+    return LS_ERR_INVALID_ARG;
+  if (vocab < 4 || vocab % 4 != 0) return LS_ERR_SHAPE;
+  if (vocab > ls::kSampleChunk * ls::kSampleMaxChunks) return LS_ERR_UNSUPPORTED;
+  if (!aligned16(d_draft_probs) || !aligned16(d_target_probs)) return LS_ERR_INVALID_ARG;
+  return cuda_status(ls::launch_sample(st->dev, d_draft_ids, d_draft_probs, d_target_probs, vocab, d_uniforms,
+                                       d_accept_len, d_next_token, stream));
+}
+
+int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const void* d_verify_k, const void* d_verify_v,
+                       const void* d_verify_hidden, cudaStream_t stream) {
+  if (!st || !d_accept_len || !d_verify_k || !d_verify_v || !d_verify_hidden) return LS_ERR_INVALID_ARG;
+  if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
+  return cuda_status(ls::launch_commit(st->dev, nullptr, nullptr, d_verify_k, d_verify_v, d_verify_hidden, nullptr,
+                                       nullptr, d_accept_len, stream));
 }
 
 int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count, const void* d_q,

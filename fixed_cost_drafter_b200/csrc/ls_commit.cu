@@ -15,7 +15,7 @@ __global__ void __launch_bounds__(64)
 commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __restrict__ target,
                     const T* __restrict__ vk, const T* __restrict__ vv,
                     const T* __restrict__ vh, int32_t* __restrict__ accept_len,
-                    int32_t* __restrict__ next_token) {
+                    int32_t* __restrict__ next_token, const int32_t* __restrict__ given_a) {
   // the attention kernel of ls_round may be scheduled now: it waits on the device for
   // this grid's writes before it reads any state
   allow_dependent_launch();
@@ -24,7 +24,7 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   CommitRegs<T, ROWS, NSC> r;
   CommitScan cs;
-  commit_load_scan<T, ROWS, NSC>(p, bl, h, warp, lane, draft, target, warp == 0 ? vk : vv, r, cs);
+  commit_load_scan<T, ROWS, NSC>(p, bl, h, warp, lane, draft, target, warp == 0 ? vk : vv, r, cs, given_a);
   // boundary state: this KV head's slice of the hidden vector at verify row a (loads now,
   // stores after the commit's own)
   BoundarySlice<T, 2> bs;
@@ -42,7 +42,7 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
     ctr[0] = cs.newlen;
 #pragma unroll
     for (int k = 0; k < NSC; ++k) ctr[1 + k] = cs.nseg[k] + ((cs.closes >> k) & 1u);
-    if (l == 0) {
+    if (l == 0 && !given_a) {  // with given counts the caller has the tokens
       accept_len[b] = cs.a;
       next_token[b] = target[int64_t(b) * (p.B + 1) + cs.a];
     }
@@ -52,21 +52,21 @@ commit_round_kernel(Dev p, const int32_t* __restrict__ draft, const int32_t* __r
 template <typename T, int ROWS, int NSC>
 static void launch_commit_t(const Dev& p, const int32_t* draft, const int32_t* target, const void* vk,
                             const void* vv, const void* vh, int32_t* accept_len, int32_t* next_token,
-                            cudaStream_t stream) {
+                            const int32_t* given_a, cudaStream_t stream) {
   commit_round_kernel<T, ROWS, NSC><<<p.b * p.L * p.Hkv, 64, 0, stream>>>(
       p, draft, target, static_cast<const T*>(vk), static_cast<const T*>(vv), static_cast<const T*>(vh),
-      accept_len, next_token);
+      accept_len, next_token, given_a);
 }
 
 template <typename T, int ROWS>
 static void launch_commit_rows(const Dev& p, const int32_t* draft, const int32_t* target, const void* vk,
                                const void* vv, const void* vh, int32_t* accept_len, int32_t* next_token,
-                               cudaStream_t stream) {
+                               const int32_t* given_a, cudaStream_t stream) {
   switch (p.nsc) {  // the scale count is a template argument: only live scale code is compiled
-    case 1: launch_commit_t<T, ROWS, 1>(p, draft, target, vk, vv, vh, accept_len, next_token, stream); break;
-    case 2: launch_commit_t<T, ROWS, 2>(p, draft, target, vk, vv, vh, accept_len, next_token, stream); break;
-    case 3: launch_commit_t<T, ROWS, 3>(p, draft, target, vk, vv, vh, accept_len, next_token, stream); break;
-    default: launch_commit_t<T, ROWS, 4>(p, draft, target, vk, vv, vh, accept_len, next_token, stream); break;
+    case 1: launch_commit_t<T, ROWS, 1>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream); break;
+    case 2: launch_commit_t<T, ROWS, 2>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream); break;
+    case 3: launch_commit_t<T, ROWS, 3>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream); break;
+    default: launch_commit_t<T, ROWS, 4>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream); break;
   }
 }
 
@@ -75,20 +75,20 @@ static void launch_commit_rows(const Dev& p, const int32_t* draft, const int32_t
 template <typename T>
 static void launch_commit_dt(const Dev& p, const int32_t* draft, const int32_t* target, const void* vk,
                              const void* vv, const void* vh, int32_t* accept_len, int32_t* next_token,
-                             cudaStream_t stream) {
+                             const int32_t* given_a, cudaStream_t stream) {
   const int rows = commit_rows_per_lane<T>(p.D, p.B);
-  if (rows <= 9) launch_commit_rows<T, 9>(p, draft, target, vk, vv, vh, accept_len, next_token, stream);
-  else if (rows <= 17) launch_commit_rows<T, 17>(p, draft, target, vk, vv, vh, accept_len, next_token, stream);
-  else launch_commit_rows<T, 33>(p, draft, target, vk, vv, vh, accept_len, next_token, stream);
+  if (rows <= 9) launch_commit_rows<T, 9>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream);
+  else if (rows <= 17) launch_commit_rows<T, 17>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream);
+  else launch_commit_rows<T, 33>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream);
 }
 
 cudaError_t launch_commit(const Dev& p, const int32_t* draft, const int32_t* target, const void* vk,
                           const void* vv, const void* vh, int32_t* accept_len, int32_t* next_token,
-                          cudaStream_t stream) {
+                          const int32_t* given_a, cudaStream_t stream) {
   if (p.dtype == LS_BF16)
-    launch_commit_dt<__nv_bfloat16>(p, draft, target, vk, vv, vh, accept_len, next_token, stream);
+    launch_commit_dt<__nv_bfloat16>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream);
   else
-    launch_commit_dt<float>(p, draft, target, vk, vv, vh, accept_len, next_token, stream);
+    launch_commit_dt<float>(p, draft, target, vk, vv, vh, accept_len, next_token, given_a, stream);
   return cudaGetLastError();
 }
 

@@ -49,7 +49,7 @@ template <typename T, int ROWS, int NSC>
 __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int lane,
                                         const int32_t* __restrict__ draft, const int32_t* __restrict__ target,
                                         const T* __restrict__ vsrc, CommitRegs<T, ROWS, NSC>& r,
-                                        CommitScan& cs) {
+                                        CommitScan& cs, const int32_t* __restrict__ given_a = nullptr) {
   constexpr int VEC = Elem<T>::kVec;
   const int b = bl / p.L;
   const int64_t* ctr = p.counters + int64_t(bl) * (1 + NSC);
@@ -64,16 +64,25 @@ __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int 
   int64_t nseg[kMaxScales];
 #pragma unroll
   for (int k = 0; k < kMaxScales; ++k) nseg[k] = k < NSC ? ctr[1 + k] : 0;
-  bool mism[2];
+  bool mism[2] = {false, false};
+  int a_given = 0;
+  if (given_a) {  // the accepted count comes from the caller (stochastic acceptance)
+    a_given = given_a[b];
+    if (a_given < 0 || a_given > p.B) {
+      if (lane == 0 && t == 0) set_err(p.err, LS_DEVERR_SAMPLE);
+      a_given = a_given < 0 ? 0 : p.B;
+    }
+  } else {
 #pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    const int i = 32 * w + lane;
-    mism[w] = i < p.B && draft[int64_t(b) * p.B + i] != target[int64_t(b) * (p.B + 1) + i];
+    for (int w = 0; w < 2; ++w) {
+      const int i = 32 * w + lane;
+      mism[w] = i < p.B && draft[int64_t(b) * p.B + i] != target[int64_t(b) * (p.B + 1) + i];
+    }
   }
   // greedy acceptance: first i with draft[i] != target[i], else B
   const unsigned m0 = __ballot_sync(0xffffffffu, mism[0]);
   const unsigned m1 = __ballot_sync(0xffffffffu, mism[1]);
-  const int a = m0 ? __ffs(m0) - 1 : (m1 ? 32 + __ffs(m1) - 1 : p.B);
+  const int a = given_a ? a_given : (m0 ? __ffs(m0) - 1 : (m1 ? 32 + __ffs(m1) - 1 : p.B));
   // scale k closes a segment this round exactly when its own distance to the next
   // boundary is <= Delta (then that distance equals the split row)
   unsigned closes = 0;

@@ -26,13 +26,18 @@ struct Dev {
   float* part;        // [b][L][Hkv][nsc][2][D]
   float* glob;        // [b][L][Hkv][2][D]
   char* boundary;     // [b][L][hidden] elements
+  int32_t* samp_count;  // [b] arrivals of a sequence's CTAs in ls_accept_sampled
+  float* samp_part;     // [b][kSampleMaxChunks] vocabulary chunk sums of ls_accept_sampled
 };
+
+constexpr int kSampleChunk = 8192;     // vocabulary entries per CTA of ls_accept_sampled
+constexpr int kSampleMaxChunks = 64;   // vocab <= 524288
 
 __host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
 // Arena layout for a validated config (host and device agree by construction).
 struct Layout {
-  int64_t counters, error, sync, kv, seg, part, glob, boundary, total;
+  int64_t counters, error, sync, kv, seg, part, glob, boundary, sample, total;
   int32_t R, elem;
 };
 
@@ -50,6 +55,7 @@ __host__ inline Layout make_layout(const ls_config& c) {
   y.part = off;     off = align256(off + tiles * c.n_scales * 2 * c.head_dim * 4);
   y.glob = off;     off = align256(off + tiles * 2 * c.head_dim * 4);
   y.boundary = off; off = align256(off + int64_t(c.batch) * c.n_layers * c.hidden * y.elem);
+  y.sample = off;   off = align256(off + int64_t(c.batch) * (1 + kSampleMaxChunks) * 4);
   y.total = off;
   return y;
 }

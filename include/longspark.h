@@ -71,6 +71,9 @@ extern "C" {
 #define LS_DEVERR_PREFIX_LEN   0x1  /* prefix_len[b] < 0 or beyond what the buffers hold */
 #define LS_DEVERR_WAIT_TIMEOUT 0x2  /* an mbarrier wait exceeded its iteration limit     */
 #define LS_DEVERR_ORDER        0x4  /* prefill chunk does not continue the state          */
+#define LS_DEVERR_SAMPLE       0x8  /* ls_accept_sampled: a draft id outside the vocabulary
+                                       or a draw with no probability mass;
+                                       ls_commit_accepted: a count outside [0, B]       */
 
 /* ---- views (Figure 2 caption (b); the component ablations of Table 5) -------- */
 #define LS_VIEW_BOUNDARY 0x1        /* the boundary state (one key/value row)          */
@@ -122,13 +125,16 @@ typedef struct {
  *   seg_mean  fp32  [b][L][Hkv][n_scales][slots][2][D]: segment means in full fp32.
  *   part_sum  fp32  [b][L][Hkv][n_scales][2][D]: sums of the open partial segments.
  *   glob_sum  fp32  [b][L][Hkv][2][D]: sum of all retained rows.
- *   boundary  e     [b][L][hidden]: hidden vectors at the last retained position.     */
+ *   boundary  e     [b][L][hidden]: hidden vectors at the last retained position.
+ *   sample    int32 [b] then fp32 [b][64]: scratch of ls_accept_sampled (zero counts
+ *             between calls), not part of any view.                                 */
 typedef struct {
   size_t total_bytes;
   size_t off_counters, off_error, off_sync, off_kv, off_seg_mean, off_part_sum, off_glob_sum,
          off_boundary;
   int32_t kv_rows;
   int32_t elem_bytes;
+  size_t off_sample;
 } ls_layout;
 
 typedef struct ls_state ls_state; /* opaque host handle */
@@ -203,6 +209,37 @@ LS_API int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32
                     const void* d_verify_k, const void* d_verify_v,
                     const void* d_verify_hidden, int32_t* d_accept_len,
                     int32_t* d_next_token, cudaStream_t stream);
+
+/* Stochastic acceptance for sampled decoding (T > 0; Table 1 against the greedy Table 3).
+ * The pages print no rule for it; this is standard speculative sampling (Leviathan,
+ * Kalman and Matias 2023; Chen et al. 2023), made position by position over the block:
+ *   d_draft_ids    int32 [b][B]          the block's draft tokens
+ *   d_draft_probs  fp32  [b][B][vocab]    the drafter's distribution q_i at block position i
+ *   d_target_probs fp32  [b][B+1][vocab]  the target's distribution p_i after verify row i
+ *   d_uniforms     fp32  [b][B+1]        draws in [0, 1): u_0..u_{B-1} for the tests, u_B for
+ *                                        the final draw
+ *   d_accept_len   int32 [b] out: a = the number of leading drafts kept, draft i kept iff
+ *                  u_i * q_i(d_i) < p_i(d_i) (fp32 product and comparison)
+ *   d_next_token   int32 [b] out: drawn from max(0, p_a - q_a) when a < B, from p_B when
+ *                  a = B: the first token t whose running sum over tokens 0..t exceeds
+ *                  u_B times the total (fp32 sums in the kernel's order); a residual with
+ *                  no mass gives the rejected draft token itself.
+ * vocab a multiple of 4 and <= 524288 (else LS_ERR_SHAPE / LS_ERR_UNSUPPORTED); the
+ * probability pointers 16-byte aligned. Reads 2B gathered values per sequence and the
+ * draw's row(s) once (plus the drawn 8192-entry chunk again). A draft id outside
+ * [0, vocab), or p_B with no mass, sets LS_DEVERR_SAMPLE. The state only lends its
+ * shapes and a scratch region (sequences may not run two of these calls at once). Feed
+ * the accepted counts to ls_commit_accepted.                                          */
+LS_API int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const float* d_draft_probs,
+                             const float* d_target_probs, int32_t vocab, const float* d_uniforms,
+                             int32_t* d_accept_len, int32_t* d_next_token, cudaStream_t stream);
+
+/* ls_commit_round with the accepted counts given (d_accept_len int32 [b], e.g. from
+ * ls_accept_sampled) instead of the greedy scan; the next tokens are the caller's. A
+ * count outside [0, B] sets LS_DEVERR_SAMPLE and is clamped. Other arguments as
+ * ls_commit_round.                                                                     */
+LS_API int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const void* d_verify_k,
+                              const void* d_verify_v, const void* d_verify_hidden, cudaStream_t stream);
 
 /* The drafter's block attention over the three views (Figure 2 (c)).
  *   layers [layer_begin, layer_begin + layer_count)

@@ -380,9 +380,14 @@ def inverse_cdf(w, v):
 
 
 def accept_sampled(draft_ids, q_rows, p_rows, u, v):
-    """One sequence's stochastic acceptance: (a, next token)."""
+    """One sequence's stochastic acceptance: (a, next token). A draw with no mass at all (a
+    residual of rows equal up to rounding) gives the rejected draft token itself (token 0
+    for an empty p_B, an invalid input)."""
     a, _ = accept_decisions(draft_ids, q_rows, p_rows, u)
-    return a, inverse_cdf(sampling_weights(q_rows, p_rows, a), v)
+    w = sampling_weights(q_rows, p_rows, a)
+    if not (w > 0).any():
+        return a, (int(draft_ids[a]) if a < len(draft_ids) else 0)
+    return a, inverse_cdf(w, v)
 
 
 # ----------------------------------------------------------------------------------

@@ -43,9 +43,9 @@ def test_layout_sizes():
     assert y.off_part_sum - y.off_seg_mean >= b * L * H * nsc * sl * 2 * D * 4
     assert y.off_glob_sum - y.off_part_sum >= b * L * H * nsc * 2 * D * 4
     assert y.off_boundary - y.off_glob_sum >= b * L * H * 2 * D * 4
-    assert y.total_bytes - y.off_boundary >= b * L * 4096 * 2
+    assert y.off_sample - y.off_boundary >= b * L * 4096 * 2 and y.total_bytes - y.off_sample >= b * 65 * 4
     for off in (y.off_counters, y.off_error, y.off_sync, y.off_kv, y.off_seg_mean, y.off_part_sum, y.off_glob_sum,
-                y.off_boundary, y.total_bytes):
+                y.off_boundary, y.off_sample, y.total_bytes):
         assert off % 256 == 0
     assert F.ls_state_bytes(c) == y.total_bytes
     # about 13.3 MB per sequence at Qwen3-8B shapes, whatever the prefix
@@ -69,7 +69,10 @@ def test_view_state_bytes():
         n = counters + sum(v for bit, v in want.items() if views & bit)
         assert F.ls_view_state_bytes(c, views) == n, views
     everything = F.ls_view_state_bytes(c, F.LS_VIEW_ALL)
-    assert everything <= F.ls_state_bytes(c) < everything + 9 * 256  # + alignment padding
+    # the arena adds the error word, the commit's arrival counts, the sampler's scratch
+    # (counts + 64 chunk sums per sequence) and the 256-byte alignment of its 10 regions
+    extra = 16 + b * L * 4 + b * 65 * 4
+    assert everything + extra <= F.ls_state_bytes(c) < everything + extra + 10 * 256
     assert F.ls_view_state_bytes(c, 8) == 0 and F.ls_view_state_bytes(_cfg(batch=0), 1) == 0
 
 

@@ -36,9 +36,10 @@ struct SampleArgs {
 // rejection (qrow set), else p; entries past the vocabulary weigh 0.
 __device__ inline float4 weights4(const float* prow, const float* qrow, int j, int V) {
   if (j >= V) return make_float4(0.f, 0.f, 0.f, 0.f);
-  float4 w = __ldcs(reinterpret_cast<const float4*>(prow + j));
+  // (plain loads: the drawn chunk is read again from L2 by the sequence's last CTA)
+  float4 w = *reinterpret_cast<const float4*>(prow + j);
   if (qrow) {
-    const float4 q = __ldcs(reinterpret_cast<const float4*>(qrow + j));
+    const float4 q = *reinterpret_cast<const float4*>(qrow + j);
     w.x = fmaxf(0.f, w.x - q.x);
     w.y = fmaxf(0.f, w.y - q.y);
     w.z = fmaxf(0.f, w.z - q.z);
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float sh[kSampleThreads / 32];
   __shared__ float sub_tot[kSubs];
+  __shared__ float sub_part[kSampleThreads / 32][kSubs];
   __shared__ int a_s, last_s, cstar_s, found_s, lastpos_s;
   __shared__ float rem_s;
 
@@ -129,30 +131,50 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
     if (!last_s) return;
   }
 
-  // the sequence's last CTA: total mass, then the chunk holding u_B * total
+  // the sequence's last CTA: total mass, then the chunk holding u_B * total. The chunk
+  // sums are loaded at once (chunk k by thread k) and scanned by the first two warps.
   __threadfence();
+  if (warp < 2) {
+    const int k = threadIdx.x;
+    const float v = k < s.nchunks ? __ldcg(p.samp_part + b * kSampleMaxChunks + k) : 0.f;
+    float inc = v;  // inclusive prefix within the warp, in chunk order
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) sh[warp] = inc;
+    asm volatile("bar.sync 1, 64;" ::: "memory");  // the two warps' totals
+    if (warp == 1) inc += sh[0];
+    const float z = sh[0] + sh[1];
+    const float t = s.u[b * (p.B + 1) + p.B] * z;
+    // the first chunk whose running sum passes t; the last chunk with mass if rounding
+    // leaves none
+    const unsigned hit = __ballot_sync(0xffffffffu, z > 0.f && k < s.nchunks && inc > t);
+    const unsigned mass = __ballot_sync(0xffffffffu, k < s.nchunks && v > 0.f);
+    if (lane == 0) {
+      sub_tot[warp] = __int_as_float(int(hit));
+      sub_tot[2 + warp] = __int_as_float(int(mass));
+    }
+    asm volatile("bar.sync 1, 64;" ::: "memory");
+    const unsigned h0 = __float_as_int(sub_tot[0]), h1 = __float_as_int(sub_tot[1]);
+    const unsigned m0 = __float_as_int(sub_tot[2]), m1 = __float_as_int(sub_tot[3]);
+    int cstar = h0 ? __ffs(int(h0)) - 1 : (h1 ? 32 + __ffs(int(h1)) - 1 : -1);
+    bool force_last = false;
+    if (cstar < 0 && z > 0.f) {
+      cstar = m1 ? 63 - __clz(int(m1)) : 31 - __clz(int(m0));
+      force_last = true;
+    }
+    if (k == cstar) {
+      cstar_s = cstar;
+      rem_s = force_last ? INFINITY : t - (inc - v);
+    }
+    if (threadIdx.x == 0 && cstar < 0) cstar_s = -1;
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
     p.samp_count[b] = 0;  // zero again for the next call
-    const volatile float* part = p.samp_part + b * kSampleMaxChunks;
-    float z = 0.f;
-    for (int k = 0; k < s.nchunks; ++k) z += part[k];
-    int cstar = -1;
-    float rem = 0.f;
-    if (z > 0.f) {
-      const float t = s.u[b * (p.B + 1) + p.B] * z;
-      float cum = 0.f;
-      for (int k = 0; k < s.nchunks && cstar < 0; ++k) {
-        if (cum + part[k] > t) { cstar = k; rem = t - cum; }
-        cum += part[k];
-      }
-      if (cstar < 0) {  // rounding: the last chunk with mass, and its last entry with mass
-        for (int k = s.nchunks - 1; k >= 0 && cstar < 0; --k)
-          if (part[k] > 0.f) { cstar = k; rem = part[k]; }
-      }
-    }
-    cstar_s = cstar;
-    rem_s = rem;
-    if (cstar < 0) {  // no mass at all: the rejected draft itself, or token 0 (p_B empty)
+    if (cstar_s < 0) {  // no mass at all: the rejected draft itself, or token 0 (p_B empty)
       s.accept_len[b] = a;
       s.next_token[b] = a < p.B ? s.draft[b * p.B + a] : 0;
       if (a == p.B) set_err(p.err, LS_DEVERR_SAMPLE);
@@ -170,16 +192,31 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
     w[m] = weights4(prow, qrow, cbase + m * kSub + 4 * threadIdx.x, s.V);
     ws[m] = sum4(w[m]);
   }
+  {
+    // the 8 sub-block sums in one round: warp trees, then the warps' partials in order
+    float r[kSubs];
 #pragma unroll
-  for (int m = 0; m < kSubs; ++m) {
-    const float t = block_sum(ws[m], sh);
-    if (threadIdx.x == 0) sub_tot[m] = t;
+    for (int m = 0; m < kSubs; ++m) {
+      r[m] = ws[m];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) r[m] += __shfl_xor_sync(0xffffffffu, r[m], o);
+    }
+    if (lane == 0)
+#pragma unroll
+      for (int m = 0; m < kSubs; ++m) sub_part[warp][m] = r[m];
+    if (threadIdx.x == 0) {
+      found_s = 0x7fffffff;
+      lastpos_s = -1;
+    }
+    __syncthreads();
+    if (threadIdx.x < kSubs) {
+      float t = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < kSampleThreads / 32; ++w2) t += sub_part[w2][threadIdx.x];
+      sub_tot[threadIdx.x] = t;
+    }
+    __syncthreads();
   }
-  if (threadIdx.x == 0) {
-    found_s = 0x7fffffff;
-    lastpos_s = -1;
-  }
-  __syncthreads();
   float rem = rem_s;
   int mstar = -1;
   for (int m = 0; m < kSubs && mstar < 0; ++m) {

@@ -391,6 +391,24 @@ def accept_sampled(draft_ids, q_rows, p_rows, u, v):
 
 
 # ----------------------------------------------------------------------------------
+# drafter prologue: projections of the boundary and of the block inputs
+# ----------------------------------------------------------------------------------
+# The pages say only that the drafter uses the views (Figure 2 caption (c)); its learned
+# projections are not described. The reading taken: per tapped layer l, the boundary
+# key/value rows are linear maps of the boundary hidden vector, and the block's queries
+# linear maps of the drafter's block inputs, with no bias or normalisation:
+#   bkv[b][l][n] = sum_k W_kv[l][n][k] h[b][l][k]   (n < Hkv D: key of head n // D, then values)
+#   q[b][l][i][n] = sum_k W_q[l][n][k] x[b][l][i][k]
+def draft_prologue(w_kv, w_q, boundary, x):
+    """fp64 projections: w_kv [L][2 Hkv D][hidden], w_q [L][Hq D][hidden], boundary
+    [b][L][hidden], x [b][L][B][hidden] -> (bkv [b][L][2 Hkv D], q [b][L][B][Hq D])."""
+    w_kv, w_q = np.asarray(w_kv, np.float64), np.asarray(w_q, np.float64)
+    bkv = np.einsum("lnk,blk->bln", w_kv, np.asarray(boundary, np.float64))
+    q = np.einsum("lnk,blik->blin", w_q, np.asarray(x, np.float64))
+    return bkv, q
+
+
+# ----------------------------------------------------------------------------------
 # readout helpers (views in the same terms the device state uses)
 # ----------------------------------------------------------------------------------
 def segment_count(n: int, s: int) -> int:

@@ -118,9 +118,16 @@ def _accept_ratio_inverted(draft_ids, q_rows, p_rows, u):
     return ORIG["accept_decisions"](draft_ids, p_rows[:len(draft_ids)], q_rows, u)
 
 
+def _prologue_layer0_weights(w_kv, w_q, boundary, x):
+    # every layer projected with layer 0's weights
+    w_kv, w_q = np.asarray(w_kv), np.asarray(w_q)
+    return ORIG["draft_prologue"](np.broadcast_to(w_kv[:1], w_kv.shape), np.broadcast_to(w_q[:1], w_q.shape),
+                                  boundary, x)
+
+
 ORIG = {n: getattr(M, n) for n in ("accept_scan", "retain_row", "views_from_scratch",
                                    "attention_slots", "draft_attend", "view_of_slots",
-                                   "accept_decisions", "sampling_weights")}
+                                   "accept_decisions", "sampling_weights", "draft_prologue")}
 
 CASES = [
     ("accept_scan", _scan_off_by_one, [P.test_scan_golden_examples]),
@@ -134,6 +141,7 @@ CASES = [
     ("view_of_slots", _views_boundary_in_summary, [P.test_views_boundary_alone_is_its_value]),
     ("sampling_weights", _residual_swapped, [P.test_sampled_emits_target_distribution]),
     ("accept_decisions", _accept_ratio_inverted, [P.test_sampled_emits_target_distribution]),
+    ("draft_prologue", _prologue_layer0_weights, [P.test_prologue_orientation_and_layers]),
 ]
 
 

@@ -463,6 +463,54 @@ def test_sampled_decision_is_fp32():
     assert a == 0 and not keep[0]
 
 
+# ---------------------------------------------------------------------------------
+# drafter prologue (projections of the boundary and the block inputs)
+# ---------------------------------------------------------------------------------
+def test_prologue_selection_weights_give_the_slices():
+    """Weights that select hidden dimensions reproduce the slice stand-in: boundary keys
+    h[g D:(g+1) D], values h[Hkv D + g D:...], queries the selected input dimensions."""
+    rng = np.random.default_rng(31)
+    b, L, B, H, Hq, D, hid = 2, 3, 4, 2, 4, 5, 40
+    w_kv = np.zeros((L, 2 * H * D, hid))
+    w_kv[:, np.arange(2 * H * D), np.arange(2 * H * D)] = 1.0
+    w_q = np.zeros((L, Hq * D, hid))
+    sel = rng.permutation(hid)[:Hq * D]
+    w_q[:, np.arange(Hq * D), sel] = 1.0
+    h = rng.standard_normal((b, L, hid))
+    x = rng.standard_normal((b, L, B, hid))
+    bkv, q = O.draft_prologue(w_kv, w_q, h, x)
+    assert np.array_equal(bkv, h[:, :, :2 * H * D]) and np.array_equal(q, x[..., sel])
+
+
+def test_prologue_orientation_and_layers():
+    """y[n] = sum_k W[n][k] h[k] per layer, by scalar loops; W is not symmetric and every
+    layer has its own weights."""
+    rng = np.random.default_rng(32)
+    b, L, B, hid, nkv, nq = 2, 2, 3, 7, 4, 6
+    w_kv, w_q = rng.standard_normal((L, nkv, hid)), rng.standard_normal((L, nq, hid))
+    h, x = rng.standard_normal((b, L, hid)), rng.standard_normal((b, L, B, hid))
+    bkv, q = O.draft_prologue(w_kv, w_q, h, x)
+    for bb in range(b):
+        for l in range(L):
+            for n in range(nkv):
+                assert abs(bkv[bb, l, n] - sum(w_kv[l, n, k] * h[bb, l, k] for k in range(hid))) < 1e-12
+            for i in range(B):
+                for n in range(nq):
+                    assert abs(q[bb, l, i, n] - sum(w_q[l, n, k] * x[bb, l, i, k] for k in range(hid))) < 1e-12
+
+
+def test_prologue_is_linear():
+    rng = np.random.default_rng(33)
+    w_kv, w_q = rng.standard_normal((2, 6, 9)), rng.standard_normal((2, 8, 9))
+    h1, h2 = rng.standard_normal((3, 2, 9)), rng.standard_normal((3, 2, 9))
+    x1, x2 = rng.standard_normal((3, 2, 4, 9)), rng.standard_normal((3, 2, 4, 9))
+    a1, q1 = O.draft_prologue(w_kv, w_q, h1, x1)
+    a2, q2 = O.draft_prologue(w_kv, w_q, h2, x2)
+    a3, q3 = O.draft_prologue(w_kv, w_q, 2 * h1 - h2, 2 * x1 - x2)
+    np.testing.assert_allclose(a3, 2 * a1 - a2, atol=1e-12)
+    np.testing.assert_allclose(q3, 2 * q1 - q2, atol=1e-12)
+
+
 def test_mask_counts():
     """Valid slot count = boundary + min(len, W) + per scale min(n_c, slots) + [partial] + [len>0]."""
     sh = _shapes(n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=2, window=16,

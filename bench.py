@@ -433,6 +433,11 @@ def run_gpu(args):
     if not args.no_sampling:
         sampled = sampling_measure(F, run, wl, dev, flush, stream, evs, min(K, 200))
 
+    # the drafter's projections (boundary keys/values, block queries) on the tensor cores
+    prologue = None
+    if not args.no_prologue:
+        prologue = prologue_measure(F, run, wl, dev, flush, stream, evs, min(K, 200))
+
     # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
     graph_rps = None
     if not args.no_graph:
@@ -500,6 +505,7 @@ def run_gpu(args):
             "graph_rounds_per_s": graph_rps,
             "view_ablations": ablations,
             "sampled_acceptance": sampled,
+            "prologue": prologue,
             "prefill": {"ms": prefill_ms, "bytes": prefill_b, "achieved_GBps": prefill_b / (prefill_ms / 1e3) / 1e9,
                         "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
             "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch,
@@ -519,6 +525,38 @@ def run_gpu(args):
 
 
 QWEN3_VOCAB = 151936
+
+
+def prologue_measure(F, run, wl, dev, flush, stream, evs, n):
+    """ls_draft_prologue at the workload's shapes with seeded bf16 weights and block inputs:
+    algorithmic bytes = weights + block inputs + boundary view + outputs, each once."""
+    import torch
+    b, L, H, Hq, D, hid, B = wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.hidden, wl.block
+    gen = torch.Generator(device=dev).manual_seed(20261)
+    w_kv = (torch.randn((L, 2 * H * D, hid), device=dev, generator=gen) * hid ** -0.5).to(torch.bfloat16)
+    w_q = (torch.randn((L, Hq * D, hid), device=dev, generator=gen) * hid ** -0.5).to(torch.bfloat16)
+    x = torch.randn((b, L, B, hid), device=dev, generator=gen).to(torch.bfloat16)
+    bkv = torch.empty((b, L, 2 * H * D), dtype=torch.bfloat16, device=dev)
+    q = torch.empty((b, L, B, Hq * D), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        F.ls_draft_prologue(run.state, w_kv, w_q, x, bkv, q, stream)
+    for i in range(n):
+        flush.zero_()
+        evs[i][0].record(stream)
+        F.ls_draft_prologue(run.state, w_kv, w_q, x, bkv, q, stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    status, word = run.error()
+    if status != F.LS_OK:
+        raise RuntimeError(f"device error word {word:#x} after the prologue launches")
+    us = float(np.mean([e[0].elapsed_time(e[1]) for e in evs[:n]])) * 1e3
+    e = 2
+    nbytes = (w_kv.numel() + w_q.numel() + x.numel() + b * L * hid + bkv.numel() + q.numel()) * e
+    flops = 2.0 * (b * L * 2 * H * D * hid + b * L * B * Hq * D * hid)
+    peak, kind = hbm_peak()
+    del w_kv, w_q, x, bkv, q
+    return {"us": us, "bytes": int(nbytes), "GBps": nbytes / us / 1e3, "TFLOPs": flops / us / 1e6,
+            "hbm_frac": nbytes / us / 1e3 / peak, "peak_kind": kind, "launches": n}
 
 
 def sampling_measure(F, run, wl, dev, flush, stream, evs, n):
@@ -685,6 +723,7 @@ def main(argv=None):
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-ablations", action="store_true", help="skip the view-ablation attention timings")
     ap.add_argument("--no-sampling", action="store_true", help="skip the stochastic-acceptance timing")
+    ap.add_argument("--no-prologue", action="store_true", help="skip the drafter-projection timing")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -42,6 +42,7 @@ EXPORTED = (
     "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",
     "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend",
     "ls_draft_attend_views", "ls_view_state_bytes", "ls_round", "ls_accept_sampled", "ls_commit_accepted",
+    "ls_draft_prologue",
     "ls_round_overlaps", "ls_attend_uses_tensor_cores",
     "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
 )
@@ -84,6 +85,7 @@ def _load():
         "ls_view_state_bytes": (sz, [cfgp, i32]),
         "ls_accept_sampled": (ctypes.c_int, [vp, vp, vp, vp, i32, vp, vp, vp, vp]),
         "ls_commit_accepted": (ctypes.c_int, [vp, vp, vp, vp, vp, vp]),
+        "ls_draft_prologue": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp]),
         "ls_get_layout": (ctypes.c_int, [cfgp, ctypes.POINTER(ls_layout)]),
         "ls_init_state": (ctypes.c_int, [cfgp, vp, sz, ctypes.POINTER(vp), vp]),
         "ls_prefill_workspace_bytes": (sz, [cfgp, i64, i64]),
@@ -222,6 +224,11 @@ def ls_accept_sampled(state, draft_ids, draft_probs, target_probs, vocab, unifor
     _check("ls_accept_sampled", _lib.ls_accept_sampled(
         state, _ptr(draft_ids), _ptr(draft_probs), _ptr(target_probs), vocab, _ptr(uniforms), _ptr(accept_len),
         _ptr(next_token), _stream(stream)))
+
+
+def ls_draft_prologue(state, w_kv, w_q, x, bkv, q, stream=None) -> None:
+    _check("ls_draft_prologue", _lib.ls_draft_prologue(
+        state, _ptr(w_kv), _ptr(w_q), _ptr(x), _ptr(bkv), _ptr(q), _stream(stream)))
 
 
 def ls_commit_accepted(state, accept_len, verify_k, verify_v, verify_hidden, stream=None) -> None:

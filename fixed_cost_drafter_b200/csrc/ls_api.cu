@@ -11,6 +11,9 @@ namespace ls {
 cudaError_t launch_commit(const Dev& p, const int32_t* draft, const int32_t* target, const void* vk,
                           const void* vv, const void* vh, int32_t* accept_len, int32_t* next_token,
                           const int32_t* given_a, cudaStream_t stream);
+bool prologue_supported(const Dev& p);
+cudaError_t launch_prologue(const Dev& p, const void* w_kv, const void* w_q, const void* x, void* bkv, void* q,
+                            int sms, cudaStream_t stream);
 cudaError_t launch_sample(const Dev& p, const int32_t* draft, const float* q, const float* pr, int vocab,
                           const float* u, int32_t* accept_len, int32_t* next_token, cudaStream_t stream);
 bool simt_supported(const Dev& p);
@@ -254,6 +257,16 @@ int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const float* d_d
   if (!aligned16(d_draft_probs) || !aligned16(d_target_probs)) return LS_ERR_INVALID_ARG;
   return cuda_status(ls::launch_sample(st->dev, d_draft_ids, d_draft_probs, d_target_probs, vocab, d_uniforms,
                                        d_accept_len, d_next_token, stream));
+}
+
+int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q, const void* d_x, void* d_bkv,
+                      void* d_q, cudaStream_t stream) {
+  if (!st || !d_w_kv || !d_w_q || !d_x || !d_bkv || !d_q) return LS_ERR_INVALID_ARG;
+  if (!ls::prologue_supported(st->dev)) return LS_ERR_UNSUPPORTED;
+  if (!aligned16(d_w_kv) || !aligned16(d_w_q) || !aligned16(d_x) || !aligned16(d_bkv) || !aligned16(d_q))
+    return LS_ERR_INVALID_ARG;
+  const cudaError_t e = ls::launch_prologue(st->dev, d_w_kv, d_w_q, d_x, d_bkv, d_q, st->sms, stream);
+  return e == cudaErrorNotSupported ? LS_ERR_UNSUPPORTED : cuda_status(e);
 }
 
 int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const void* d_verify_k, const void* d_verify_v,

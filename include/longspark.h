@@ -234,6 +234,23 @@ LS_API int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const flo
                              const float* d_target_probs, int32_t vocab, const float* d_uniforms,
                              int32_t* d_accept_len, int32_t* d_next_token, cudaStream_t stream);
 
+/* The drafter's projections ahead of its attention: boundary keys/values from the
+ * boundary view and block queries from the drafter's block inputs (Figure 2 caption (c):
+ * the drafter uses the views; the pages do not describe its learned projections, so this
+ * is a plain linear map per tapped layer, no bias, fp32 accumulation):
+ *   d_w_kv  bf16 [L][2 Hkv D][hidden]  rows g D + d: key of KV head g; Hkv D + g D + d: value
+ *   d_w_q   bf16 [L][Hq D][hidden]     rows qh D + d: query head qh
+ *   d_x     bf16 [b][L][B][hidden]     the drafter's block inputs
+ *   d_bkv   bf16 [b][L][2 Hkv D] out   bkv[b][l][n] = sum_k W_kv[l][n][k] boundary[b][l][k]
+ *   d_q     bf16 [b][L][B][Hq D] out   q[b][l][i][n] = sum_k W_q[l][n][k] x[b][l][i][k]
+ * The boundary hidden vectors are the state's boundary view. The outputs feed
+ * ls_draft_attend: d_q as its queries, boundary_k = d_bkv, boundary_v = d_bkv + Hkv D,
+ * boundary_stride = 2 Hkv D. Runs on the tcgen05 tensor cores: needs a bf16 state,
+ * hidden a multiple of 64, Hq D and 2 Hkv D multiples of 128 (else LS_ERR_UNSUPPORTED);
+ * pointers 16-byte aligned.                                                              */
+LS_API int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q, const void* d_x,
+                             void* d_bkv, void* d_q, cudaStream_t stream);
+
 /* ls_commit_round with the accepted counts given (d_accept_len int32 [b], e.g. from
  * ls_accept_sampled) instead of the greedy scan; the next tokens are the caller's. A
  * count outside [0, B] sets LS_DEVERR_SAMPLE and is clamped. Other arguments as

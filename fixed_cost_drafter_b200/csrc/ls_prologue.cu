@@ -8,27 +8,31 @@
 // activations as its B operand (N = up to 256 activation rows, K-major): the weights
 // stream through once, the few activation rows come from L2.
 //
-// Persistent kernel, 6 warps: warp 0 TMA producer (a ring of 4 stages, each 64 hidden
-// entries of the unit's 128 weight rows and of its activation rows, 128-byte swizzle),
-// warp 1 TMEM allocator and MMA issuer (double-buffered accumulator, 2 x 256 columns),
-// warps 2-5 epilogue (one TMEM subpartition each: a thread owns one weight row n and
-// writes its column of outputs). Units: (problem, layer, 128-row weight tile, activation
-// tile), queries first; CTA c takes units c, c + grid, ... Every wait is bounded.
+// Persistent kernel, 7 warps: warp 0 TMA producer of the weights (a ring of 6 stages of 64
+// hidden entries of the unit's 128 weight rows, from HBM), warp 6 TMA producer of the
+// activations (3 stages of up to 256 rows, mostly from L2), both 128-byte swizzled; warp 1
+// TMEM allocator and MMA issuer (double-buffered accumulator, 2 x 256 columns); warps 2-5
+// epilogue (one TMEM subpartition each: a thread owns one weight row, its outputs go
+// through a shared-memory tile so that whole 256-byte output rows leave as 16-byte
+// stores). Units: (problem, layer, 128-row weight tile, activation tile), queries first;
+// CTA c takes units c, c + grid, ... Every wait is bounded.
 #include "ls_tc.cuh"
 
 namespace ls {
 
 namespace {
 
-constexpr int kPThreads = 192;
-constexpr int kPStages = 4;
+constexpr int kPThreads = 224;                       // 7 warps
 constexpr int kPKStep = 64;                          // hidden entries per stage
 constexpr int kPTileN = 128;                         // weight rows per unit (MMA M)
 constexpr int kPMaxAct = 256;                        // activation rows per unit (MMA N)
+constexpr int kPAStages = 6;                         // weight ring (read from HBM: deeper)
+constexpr int kPBStages = 3;                         // activation ring (read from L2)
 constexpr int kPABytes = kPTileN * kPKStep * 2;      // 16 KB
 constexpr int kPBBytes = kPMaxAct * kPKStep * 2;     // 32 KB
-constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr int kPSmemBytes = kPStages * kPStageBytes + 1024;
+constexpr int kPOutRows = 128;                       // activation rows per epilogue pass
+constexpr int kPOutBytes = kPOutRows * kPTileN * 2;  // 32 KB: [128 rows][128 weight rows] bf16
+constexpr int kPSmemBytes = kPAStages * kPABytes + kPBStages * kPBBytes + kPOutBytes + 1024;
 constexpr uint32_t kPTmemCols = 512;
 
 struct PProblem {
@@ -52,9 +56,11 @@ struct PArgs {
 };
 
 struct PBars {
-  uint64_t full[kPStages], empty[kPStages];
+  uint64_t afull[kPAStages], aempty[kPAStages];
+  uint64_t bfull[kPBStages], bempty[kPBStages];
   uint64_t acc_full[2], acc_empty[2];
-  uint64_t drain;  // after an abort: the MMAs issued so far have completed
+  uint64_t out_full, out_free;  // epilogue pass: staged by all 128 threads / copied out
+  uint64_t drain;               // after an abort: the MMAs issued so far have completed
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -93,12 +99,18 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   __shared__ PBars s;
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* a_ring = smem;                              // [kPAStages][16 KB]
+  unsigned char* b_ring = a_ring + kPAStages * kPABytes;     // [kPBStages][32 KB]
+  unsigned char* out_st = b_ring + kPBStages * kPBBytes;     // [128][128] bf16
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_mine = int(blockIdx.x) < a.n_units ? (a.n_units - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPStages; ++i) { mbar_init(&s.full[i], 1); mbar_init(&s.empty[i], 1); }
+    for (int i = 0; i < kPAStages; ++i) { mbar_init(&s.afull[i], 1); mbar_init(&s.aempty[i], 1); }
+    for (int i = 0; i < kPBStages; ++i) { mbar_init(&s.bfull[i], 1); mbar_init(&s.bempty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&s.acc_full[i], 1); mbar_init(&s.acc_empty[i], 128); }
+    mbar_init(&s.out_full, 128);
+    mbar_init(&s.out_free, 128);
     mbar_init(&s.drain, 1);
     s.abort = 0;
     fence_mbar_init();
@@ -113,34 +125,40 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  int issued = 0;  // producer: copies issued (for the drain after an abort)
+  int issued = 0;  // producers: copies issued into their ring (for the drain after an abort)
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 6) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0: the weights (A) of every k-step; warp 6: the activations (B)
     if (lane == 0) {
-      prefetch_map(&w0);
-      prefetch_map(&x0);
-      prefetch_map(&w1);
-      prefetch_map(&x1);
+      const bool is_a = warp == 0;
+      const int nst = is_a ? kPAStages : kPBStages;
+      uint64_t* fullb = is_a ? s.afull : s.bfull;
+      uint64_t* emptyb = is_a ? s.aempty : s.bempty;
+      prefetch_map(is_a ? &w0 : &x0);
+      prefetch_map(is_a ? &w1 : &x1);
+      const uint64_t pol = is_a ? l2_evict_first() : l2_evict_last();
       bool ok = true;
       int k = 0;
       for (int i = 0; i < n_mine && ok; ++i) {
         const PUnit u = unit_of(a, int(blockIdx.x) + i * int(gridDim.x));
         const PProblem& P = a.pr[u.p];
-        const CUtensorMap* wm = u.p ? &w1 : &w0;
-        const CUtensorMap* xm = u.p ? &x1 : &x0;
-        const uint32_t bytes = uint32_t(kPABytes + P.load_rows * kPKStep * 2);
+        const CUtensorMap* m = is_a ? (u.p ? &w1 : &w0) : (u.p ? &x1 : &x0);
+        const uint32_t bytes = is_a ? uint32_t(kPABytes) : uint32_t(P.load_rows * kPKStep * 2);
+        // the weights are read once: they must not push the activations (read again by
+        // every weight tile of the layer) out of L2
         for (int ks = 0; ks < a.k_steps; ++ks, ++k) {
-          const int st = k % kPStages;
-          if (!pwait(s, &s.empty[st], ((k / kPStages) & 1) ^ 1, a.err)) { ok = false; break; }
-          unsigned char* A = smem + st * kPStageBytes;
-          unsigned char* Bt = A + kPABytes;
-          mbar_arrive_expect_tx(&s.full[st], bytes);
-          tma_load_2d(A, wm, ks * kPKStep, u.l * P.n_out + u.nt * kPTileN, &s.full[st]);
-          if (P.is_4d)
-            tma_load_4d(Bt, xm, ks * kPKStep, 0, u.l, u.mt * P.seq_per_unit, &s.full[st]);
+          const int st = k % nst;
+          if (!pwait(s, &emptyb[st], ((k / nst) & 1) ^ 1, a.err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&fullb[st], bytes);
+          if (is_a)
+            tma_load_2d_hint(a_ring + st * kPABytes, m, ks * kPKStep, u.l * P.n_out + u.nt * kPTileN, &fullb[st],
+                             pol);
+          else if (P.is_4d)
+            tma_load_4d_hint(b_ring + st * kPBBytes, m, ks * kPKStep, 0, u.l, u.mt * P.seq_per_unit, &fullb[st],
+                             pol);
           else
-            tma_load_3d(Bt, xm, ks * kPKStep, u.l, u.mt * P.seq_per_unit, &s.full[st]);
+            tma_load_3d_hint(b_ring + st * kPBBytes, m, ks * kPKStep, u.l, u.mt * P.seq_per_unit, &fullb[st], pol);
           ++issued;
         }
       }
@@ -159,44 +177,62 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
         const uint32_t id = idesc_bf16(P.act_rows, false, kPTileN);
         const uint32_t d = tmem + uint32_t(ab * kPMaxAct);
         for (int ks = 0; ks < a.k_steps; ++ks, ++k) {
-          const int st = k % kPStages;
-          if (!pwait(s, &s.full[st], (k / kPStages) & 1, a.err)) { ok = false; break; }
+          const int sa = k % kPAStages, sb = k % kPBStages;
+          if (!pwait(s, &s.afull[sa], (k / kPAStages) & 1, a.err)) { ok = false; break; }
+          if (!pwait(s, &s.bfull[sb], (k / kPBStages) & 1, a.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t A = smem_u32(smem + st * kPStageBytes);
-          const uint64_t da = sdesc(A, 16, 1024), db = sdesc(A + kPABytes, 16, 1024);
+          const uint64_t da = sdesc(smem_u32(a_ring + sa * kPABytes), 16, 1024);
+          const uint64_t db = sdesc(smem_u32(b_ring + sb * kPBBytes), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kPKStep / 16; ++kk)  // K = 16 per MMA: 32 bytes along the row
             mma_bf16(d, da + uint32_t(kk * 2), db + uint32_t(kk * 2), id, (ks > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&s.empty[st]);
+          mma_commit(&s.aempty[sa]);
+          mma_commit(&s.bempty[sb]);
         }
         if (ok) mma_commit(&s.acc_full[ab]);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-5)
+    // Per 128 activation rows: each thread writes its weight row's outputs (a column of the
+    // staging tile [row][128 weight rows]), then all 128 threads copy the tile's valid rows
+    // out as 16-byte pieces of 256-byte output rows.
     const int sub = warp & 3;
+    const int ecol = 32 * sub + lane;  // this thread's weight row within the unit
+    const int etid = threadIdx.x - 64;  // 0..127
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
-    for (int i = 0; i < n_mine; ++i) {
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(out_st);
+    int pass = 0;  // epilogue passes so far (phases of out_full / out_free)
+    bool ok = true;
+    for (int i = 0; i < n_mine && ok; ++i) {
       const PUnit u = unit_of(a, int(blockIdx.x) + i * int(gridDim.x));
       const PProblem& P = a.pr[u.p];
       const int ab = i & 1;
       if (!__all_sync(0xffffffffu, pwait(s, &s.acc_full[ab], (i >> 1) & 1, a.err))) break;
       tc_fence_after();
-      const int n = u.nt * kPTileN + 32 * sub + lane;  // this thread's weight row
       const int seq0 = u.mt * P.seq_per_unit;
-      const int seqs = min(P.seq_per_unit, a.b - seq0);
-      const int rows = seqs * P.rows_per_seq;  // valid activation rows of the tile
-      for (int c0 = 0; c0 < P.act_rows; c0 += 32) {
-        float v[32];
-        tmem_ld32(trow + uint32_t(ab * kPMaxAct + c0), v);
+      const int rows = min(P.seq_per_unit, a.b - seq0) * P.rows_per_seq;  // valid activation rows
+      for (int r0 = 0; r0 < rows && ok; r0 += kPOutRows, ++pass) {
+        // the staging tile is free once every thread has copied the previous pass out
+        if (pass > 0 && !__all_sync(0xffffffffu, pwait(s, &s.out_free, (pass - 1) & 1, a.err))) { ok = false; break; }
+        const int nr = min(kPOutRows, P.act_rows - r0);
+        for (int c0 = 0; c0 < nr; c0 += 32) {
+          float v[32];
+          tmem_ld32(trow + uint32_t(ab * kPMaxAct + r0 + c0), v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = c0 + j;
-          if (m < rows) {
-            const int sq = seq0 + m / P.rows_per_seq, r = m % P.rows_per_seq;
-            P.y[((int64_t(sq) * a.L + u.l) * P.rows_per_seq + r) * P.n_out + n] = __float2bfloat16_rn(v[j]);
-          }
+          for (int j = 0; j < 32; ++j) stage[(c0 + j) * kPTileN + ecol] = __float2bfloat16_rn(v[j]);
         }
+        mbar_arrive(&s.out_full);
+        if (!__all_sync(0xffffffffu, pwait(s, &s.out_full, pass & 1, a.err))) { ok = false; break; }
+        const int vr = min(kPOutRows, rows - r0);
+        for (int c = etid; c < vr * 16; c += 128) {  // 16 pieces of 16 bytes per row
+          const int m = r0 + (c >> 4);
+          const int sq = seq0 + m / P.rows_per_seq, r = m % P.rows_per_seq;
+          uint4* dst = reinterpret_cast<uint4*>(P.y + ((int64_t(sq) * a.L + u.l) * P.rows_per_seq + r) * P.n_out +
+                                                u.nt * kPTileN) + (c & 15);
+          *dst = reinterpret_cast<const uint4*>(stage + (c >> 4) * kPTileN)[c & 15];
+        }
+        mbar_arrive(&s.out_free);
       }
       tc_fence_before();
       mbar_arrive(&s.acc_empty[ab]);
@@ -204,10 +240,12 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   }
 
   __syncthreads();
-  if (warp == 0 && lane == 0 && s.abort) {
+  if ((warp == 0 || warp == 6) && lane == 0 && s.abort) {
     // let the copies still in flight land before the shared memory is released
-    for (int n = issued > kPStages ? issued - kPStages : 0; n < issued; ++n)
-      mbar_wait_bounded(&s.full[n % kPStages], (n / kPStages) & 1, kWaitLimit);
+    const int nst = warp == 0 ? kPAStages : kPBStages;
+    uint64_t* fullb = warp == 0 ? s.afull : s.bfull;
+    for (int n = issued > nst ? issued - nst : 0; n < issued; ++n)
+      mbar_wait_bounded(&fullb[n % nst], (n / nst) & 1, kWaitLimit);
   }
   if (warp == 1 && lane == 0 && s.abort) {
     // and the MMAs issued so far, before TMEM is released

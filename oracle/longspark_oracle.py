@@ -257,6 +257,46 @@ def commit_round(sh: Shapes, v: Views, draft_ids, target_ids, verify_k: np.ndarr
 
 
 # ----------------------------------------------------------------------------------
+# (b') the same extraction reading the target's paged KV cache
+# ----------------------------------------------------------------------------------
+# The views come from the target's state (Figure 2 caption (b)); an inference engine keeps
+# that state's K/V rows in fixed-size pages. The reading taken: every tapped layer has
+# pages of its own, [num_pages][page_size][Hkv][D]; position p of sequence b sits in page
+# block_table[b][p // page_size] at offset p % page_size. Prefill reads positions
+# 0 .. P - 1; a round's verify row i is the target's position len + i (the bonus token
+# of verify row 0 follows the last retained row), so the retained rows N of Figure 3 are
+# positions len .. len + a.
+def paged_rows(pages, block_table, page_size: int, b: int, positions) -> np.ndarray:
+    """Rows of sequence ``b`` at ``positions`` from ``pages`` [L][num_pages][page_size]
+    [Hkv][D]: returns [L][len(positions)][Hkv][D] fp64 (position-major, as ``prefill``
+    and ``commit_round`` take them)."""
+    pages = np.asarray(pages)
+    L, _, _, H, D = pages.shape
+    out = np.zeros((L, len(positions), H, D), dtype=np.float64)
+    for i, pos in enumerate(positions):
+        page = int(block_table[b][pos // page_size])
+        out[:, i] = pages[:, page, pos % page_size]
+    return out
+
+
+def prefill_paged(sh: Shapes, k_pages, v_pages, block_table, page_size: int, b: int, n: int,
+                  last_hidden: np.ndarray) -> Views:
+    """``prefill`` of sequence ``b`` over its first ``n`` positions read from the pages."""
+    pos = range(n)
+    return prefill(sh, paged_rows(k_pages, block_table, page_size, b, pos),
+                   paged_rows(v_pages, block_table, page_size, b, pos), n, last_hidden)
+
+
+def commit_round_paged(sh: Shapes, v: Views, draft_ids, target_ids, k_pages, v_pages, block_table,
+                       page_size: int, b: int, verify_hidden: np.ndarray):
+    """``commit_round`` of sequence ``b`` with verify row i read from the pages at
+    position ``v.length + i``. Returns ``(a, next_token)``."""
+    pos = range(v.length, v.length + sh.block + 1)
+    return commit_round(sh, v, draft_ids, target_ids, paged_rows(k_pages, block_table, page_size, b, pos),
+                        paged_rows(v_pages, block_table, page_size, b, pos), verify_hidden)
+
+
+# ----------------------------------------------------------------------------------
 # (c) the drafter's block attention over the views
 # ----------------------------------------------------------------------------------
 def attention_slots(sh: Shapes, v: Views, l: int, g: int, boundary_k: np.ndarray,

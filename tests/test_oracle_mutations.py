@@ -118,6 +118,23 @@ def _accept_ratio_inverted(draft_ids, q_rows, p_rows, u):
     return ORIG["accept_decisions"](draft_ids, p_rows[:len(draft_ids)], q_rows, u)
 
 
+def _paged_offset_from_page_end(pages, block_table, page_size, b, positions):
+    # offset counted from the end of the page instead of its start
+    pages = np.asarray(pages)
+    out = ORIG["paged_rows"](pages, block_table, page_size, b, positions)
+    for i, pos in enumerate(positions):
+        out[:, i] = pages[:, int(block_table[b][pos // page_size]), page_size - 1 - pos % page_size]
+    return out
+
+
+def _paged_commit_from_position_zero(sh, v, draft_ids, target_ids, k_pages, v_pages, block_table, page_size, b,
+                                     verify_hidden):
+    # verify rows read from the start of the sequence instead of its current length
+    pos = range(sh.block + 1)
+    return M.commit_round(sh, v, draft_ids, target_ids, M.paged_rows(k_pages, block_table, page_size, b, pos),
+                          M.paged_rows(v_pages, block_table, page_size, b, pos), verify_hidden)
+
+
 def _prologue_layer0_weights(w_kv, w_q, boundary, x):
     # every layer projected with layer 0's weights
     w_kv, w_q = np.asarray(w_kv), np.asarray(w_q)
@@ -127,7 +144,7 @@ def _prologue_layer0_weights(w_kv, w_q, boundary, x):
 
 ORIG = {n: getattr(M, n) for n in ("accept_scan", "retain_row", "views_from_scratch",
                                    "attention_slots", "draft_attend", "view_of_slots",
-                                   "accept_decisions", "sampling_weights", "draft_prologue")}
+                                   "accept_decisions", "sampling_weights", "draft_prologue", "paged_rows")}
 
 CASES = [
     ("accept_scan", _scan_off_by_one, [P.test_scan_golden_examples]),
@@ -142,6 +159,8 @@ CASES = [
     ("sampling_weights", _residual_swapped, [P.test_sampled_emits_target_distribution]),
     ("accept_decisions", _accept_ratio_inverted, [P.test_sampled_emits_target_distribution]),
     ("draft_prologue", _prologue_layer0_weights, [P.test_prologue_orientation_and_layers]),
+    ("paged_rows", _paged_offset_from_page_end, [P.test_paged_rows_hand_worked]),
+    ("commit_round_paged", _paged_commit_from_position_zero, [lambda: P.test_paged_commit_equals_dense(3)]),
 ]
 
 

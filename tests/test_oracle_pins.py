@@ -511,6 +511,95 @@ def test_prologue_is_linear():
     np.testing.assert_allclose(q3, 2 * q1 - q2, atol=1e-12)
 
 
+# ---------------------------------------------------------------------------------
+# paged KV cache (position p in page block_table[b][p // page_size], offset p % page_size)
+# ---------------------------------------------------------------------------------
+def test_paged_rows_hand_worked():
+    """Page size 2, sequence 1's pages 3, 0, 2: positions 0..5 sit in pages 3 3 0 0 2 2
+    at offsets 0 1 0 1 0 1 (worked out by hand, stored values name their page/offset)."""
+    L, NP, PS, H, D = 2, 4, 2, 1, 1
+    pages = np.zeros((L, NP, PS, H, D))
+    for l in range(L):
+        for pg in range(NP):
+            for off in range(PS):
+                pages[l, pg, off] = 100 * l + 10 * pg + off
+    table = [[1, 2, 3], [3, 0, 2]]
+    got = O.paged_rows(pages, table, PS, 1, range(6))
+    assert got.shape == (L, 6, H, D)
+    assert got[0, :, 0, 0].tolist() == [30, 31, 0, 1, 20, 21]
+    assert got[1, :, 0, 0].tolist() == [130, 131, 100, 101, 120, 121]
+    assert O.paged_rows(pages, table, PS, 0, [5, 0]).ravel().tolist() == [31, 10, 131, 110]
+    assert O.paged_rows(pages, table, PS, 0, []).shape == (L, 0, H, D)
+
+
+def _scatter_pages(rng, dense, page_size, n_pages_total):
+    """Cut [L][P][H][D] rows into pages placed at random page ids; return (pages, table row).
+    Positions past P in the last page hold noise, pages nobody owns hold noise too."""
+    L, P, H, D = dense.shape
+    n_pages = -(-P // page_size)
+    ids = rng.permutation(n_pages_total)[:n_pages]
+    pages = rng.standard_normal((L, n_pages_total, page_size, H, D))
+    for j in range(n_pages):
+        chunk = dense[:, j * page_size:(j + 1) * page_size]
+        pages[:, ids[j], :chunk.shape[1]] = chunk
+    return pages, ids
+
+
+@pytest.mark.parametrize("P,page_size", [(0, 4), (37, 1), (37, 4), (100, 16), (40, 64)])
+def test_paged_prefill_equals_dense(P, page_size):
+    sh = _shapes()
+    rng = np.random.default_rng(P * 7 + page_size)
+    L, H, D = sh.n_layers, sh.n_kv_heads, sh.head_dim
+    pk, pv = rng.standard_normal((L, P, H, D)), rng.standard_normal((L, P, H, D))
+    hid = rng.standard_normal((L, sh.hidden))
+    kp, ids = _scatter_pages(rng, pk, page_size, -(-P // page_size) + 3)
+    vp = rng.standard_normal(kp.shape)
+    for j, pg in enumerate(ids):
+        chunk = pv[:, j * page_size:(j + 1) * page_size]
+        vp[:, pg, :chunk.shape[1]] = chunk
+    table = [list(ids) + [0] * 2, [0]]  # sequence 0 owns the pages; row 1 is another sequence's
+    got = O.prefill_paged(sh, kp, vp, table, page_size, 0, P, hid)
+    _assert_views_close(sh, got, O.prefill(sh, pk, pv, P, hid), rtol=0)
+
+
+@pytest.mark.parametrize("page_size", [1, 3, 16])
+def test_paged_commit_equals_dense(page_size):
+    """Rounds whose verify rows the target wrote into its pages at positions len .. len + B
+    (crossing page boundaries) give the views of the dense rounds."""
+    sh = _shapes()
+    rng = np.random.default_rng(page_size)
+    L, H, D, B = sh.n_layers, sh.n_kv_heads, sh.head_dim, sh.block
+    P, accepts = 23, [4, 0, 2, 4, 1, 3]
+    total = P + sum(a + 1 for a in accepts[:-1]) + B + 1
+    n_pages = -(-total // page_size)
+    ids = rng.permutation(n_pages + 5)[:n_pages]
+    kp = rng.standard_normal((L, n_pages + 5, page_size, H, D))
+    vp = rng.standard_normal(kp.shape)
+    pk, pv = rng.standard_normal((L, P, H, D)), rng.standard_normal((L, P, H, D))
+    for p in range(P):
+        kp[:, ids[p // page_size], p % page_size] = pk[:, p]
+        vp[:, ids[p // page_size], p % page_size] = pv[:, p]
+    hid = rng.standard_normal((L, sh.hidden))
+    dense = O.prefill(sh, pk, pv, P, hid)
+    paged = O.prefill_paged(sh, kp, vp, [ids], page_size, 0, P, hid)
+    for a in accepts:
+        draft = rng.integers(0, 50, B)
+        target = np.concatenate([draft, [0]])
+        if a < B:
+            target[a] = draft[a] + 1
+        vk, vv = rng.standard_normal((L, B + 1, H, D)), rng.standard_normal((L, B + 1, H, D))
+        vh = rng.standard_normal((L, B + 1, sh.hidden))
+        for i in range(B + 1):  # the verify pass writes all B + 1 rows at len + i
+            p = dense.length + i
+            kp[:, ids[p // page_size], p % page_size] = vk[:, i]
+            vp[:, ids[p // page_size], p % page_size] = vv[:, i]
+        ra = O.commit_round(sh, dense, draft, target, vk, vv, vh)
+        rb = O.commit_round_paged(sh, paged, draft, target, kp, vp, [ids], page_size, 0, vh)
+        assert ra == rb and ra[0] == a
+        _assert_views_close(sh, paged, dense, rtol=0)
+        np.testing.assert_array_equal(paged.boundary, dense.boundary)
+
+
 def test_mask_counts():
     """Valid slot count = boundary + min(len, W) + per scale min(n_c, slots) + [partial] + [len>0]."""
     sh = _shapes(n_layers=1, n_kv_heads=1, n_q_heads=1, head_dim=2, window=16,

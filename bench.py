@@ -438,6 +438,11 @@ def run_gpu(args):
     if not args.no_prologue:
         prologue = prologue_measure(F, run, wl, dev, flush, stream, evs, min(K, 200))
 
+    # prefill and rounds reading the target's paged KV cache in place (page size 16)
+    paged = None
+    if not args.no_paged:
+        paged = paged_measure(WLM, wl, dev, flush, evs, min(K, 200), rank)
+
     # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
     graph_rps = None
     if not args.no_graph:
@@ -506,6 +511,7 @@ def run_gpu(args):
             "view_ablations": ablations,
             "sampled_acceptance": sampled,
             "prologue": prologue,
+            "paged": paged,
             "prefill": {"ms": prefill_ms, "bytes": prefill_b, "achieved_GBps": prefill_b / (prefill_ms / 1e3) / 1e9,
                         "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
             "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch,
@@ -525,6 +531,68 @@ def run_gpu(args):
 
 
 QWEN3_VOCAB = 151936
+PAGE_SIZE = 16
+LARGE_PAGE_SIZE = 256
+
+
+def paged_measure(WLM, wl, dev, flush, evs, n, rank):
+    """ls_prefill_paged and ls_round_paged on the workload with its prefix and verify rows in
+    a paged cache (page size 16, each sequence's pages scattered over the pool; the prefill
+    also with 256-row pages). The
+    verify pass's writes into the pages happen before the timed region (the target's work);
+    every timed round is preceded by an L2 flush. Returns the timings and their HBM rates."""
+    import torch
+    import fixed_cost_drafter_b200 as F
+    peak, _ = hbm_peak()
+    # prefill with large pages first (locality of each copy), then the rounds' page size
+    by_ps = {}
+    for ps in (LARGE_PAGE_SIZE, PAGE_SIZE):
+        run = WLM.DeviceRun(wl, device=dev, rounds=n, seq_offset=sequence_offset(rank, wl.batch))
+        cache = WLM.PagedCache(run, ps, run.prefix_len + (n + 1) * (wl.block + 1), seed=1)
+        run.fill_pages(cache)
+        torch.cuda.synchronize()
+        pre = []
+        run.prefill_paged(cache, timer=lambda e0, e1, nbytes: pre.append((e0, e1, nbytes)))
+        torch.cuda.synchronize()
+        pre_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in pre)
+        pre_b = sum(nb for _, _, nb in pre)
+        by_ps[ps] = {"ms": pre_ms, "bytes": pre_b, "achieved_GBps": pre_b / (pre_ms / 1e3) / 1e9,
+                     "frac": pre_b / (pre_ms / 1e3) / 1e9 / peak}
+        if ps != PAGE_SIZE:
+            run.close()
+            del cache
+            torch.cuda.empty_cache()
+    inp = run.make_round_inputs(0, n)
+    for r in range(n):
+        run.write_verify_pages(cache, inp, r)
+    torch.cuda.synchronize()
+    out = run.new_out()
+    stream = run.stream
+    kv = cache.descriptor()
+    span = wl.n_kv_heads * wl.head_dim
+    warm = 3  # the first rounds load the kernels; rounds run in order (the pages hold them)
+    for i in range(n):
+        flush.zero_()
+        evs[i][0].record(stream)
+        F.ls_round_paged(run.state, run.draft[i], run.target[i], kv, inp["vh"][i], run.accept_len, run.next_token,
+                         inp["q"][i], 0, span, run.softmax_scale, out, stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = [e[0].elapsed_time(e[1]) for e in evs[warm:n]]
+    status, word = run.error()
+    if status != F.LS_OK:
+        raise RuntimeError(f"device error word {word:#x} after the paged rounds")
+    deltas = run.accept_host[warm:n] + 1
+    r_bytes = attend_bytes(wl) + commit_bytes(wl, float(deltas.mean()))
+    us = float(np.mean(ms)) * 1e3
+    res = {"page_size": PAGE_SIZE, "num_pages": cache.num_pages, "prefill": by_ps[PAGE_SIZE],
+           "prefill_page_size_%d" % LARGE_PAGE_SIZE: by_ps[LARGE_PAGE_SIZE],
+           "round_us": {"mean": us, "median": float(np.median(ms)) * 1e3}, "round_bytes": r_bytes,
+           "round_GBps": r_bytes / us / 1e3, "rounds": n - warm}
+    run.close()
+    del cache
+    torch.cuda.empty_cache()
+    return res
 
 
 def prologue_measure(F, run, wl, dev, flush, stream, evs, n):
@@ -724,6 +792,7 @@ def main(argv=None):
     ap.add_argument("--no-ablations", action="store_true", help="skip the view-ablation attention timings")
     ap.add_argument("--no-sampling", action="store_true", help="skip the stochastic-acceptance timing")
     ap.add_argument("--no-prologue", action="store_true", help="skip the drafter-projection timing")
+    ap.add_argument("--no-paged", action="store_true", help="skip the paged-KV prefill and round timings")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

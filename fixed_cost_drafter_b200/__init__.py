@@ -28,6 +28,8 @@ LS_DEVERR_PREFIX_LEN = 0x1
 LS_DEVERR_WAIT_TIMEOUT = 0x2
 LS_DEVERR_ORDER = 0x4
 LS_DEVERR_SAMPLE = 0x8
+LS_DEVERR_PAGE = 0x10
+LS_MAX_PAGED_LAYERS = 64
 LS_F32 = 0
 LS_BF16 = 1
 LS_FLAG_FORCE_SIMT = 0x1
@@ -42,7 +44,7 @@ EXPORTED = (
     "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",
     "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend",
     "ls_draft_attend_views", "ls_view_state_bytes", "ls_round", "ls_accept_sampled", "ls_commit_accepted",
-    "ls_draft_prologue",
+    "ls_draft_prologue", "ls_prefill_paged", "ls_commit_round_paged", "ls_commit_accepted_paged", "ls_round_paged",
     "ls_round_overlaps", "ls_attend_uses_tensor_cores",
     "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
 )
@@ -74,13 +76,44 @@ class ls_layout(ctypes.Structure):
     ]
 
 
+class ls_paged_kv(ctypes.Structure):
+    """A target's paged KV cache: per tapped layer the base of its key and value pages;
+    element (page, offset, h, d) at base[page * page_stride + offset * slot_stride + h * D + d];
+    position p of sequence b in page block_table[b][p // page_size] at offset p % page_size."""
+    _fields_ = [
+        ("k_layers", ctypes.c_void_p * LS_MAX_PAGED_LAYERS), ("v_layers", ctypes.c_void_p * LS_MAX_PAGED_LAYERS),
+        ("page_stride", ctypes.c_int64), ("slot_stride", ctypes.c_int64), ("block_table", ctypes.c_void_p),
+        ("max_blocks", ctypes.c_int32), ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int64),
+    ]
+
+
+def make_paged_kv(k_layers, v_layers, page_stride, slot_stride, block_table, max_blocks, page_size,
+                  num_pages) -> ls_paged_kv:
+    """Descriptor from per-layer page buffers (tensors or addresses) and an int32 block table."""
+    if len(k_layers) != len(v_layers) or len(k_layers) > LS_MAX_PAGED_LAYERS:
+        raise ValueError("one key and one value page buffer per tapped layer, at most LS_MAX_PAGED_LAYERS")
+    kv = ls_paged_kv()
+    for l, (k, v) in enumerate(zip(k_layers, v_layers)):
+        kv.k_layers[l] = _ptr(k)
+        kv.v_layers[l] = _ptr(v)
+    kv.page_stride, kv.slot_stride = page_stride, slot_stride
+    kv.block_table = _ptr(block_table)
+    kv.max_blocks, kv.page_size, kv.num_pages = max_blocks, page_size, num_pages
+    return kv
+
+
 def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(f"{_LIB_PATH} is missing: build it with __graft_entry__.build()")
     lib = ctypes.CDLL(_LIB_PATH)
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     cfgp = ctypes.POINTER(ls_config)
+    pkvp = ctypes.POINTER(ls_paged_kv)
     sig = {
+        "ls_prefill_paged": (ctypes.c_int, [vp, pkvp, vp, i64, i64, vp, vp, sz, vp]),
+        "ls_commit_round_paged": (ctypes.c_int, [vp, vp, vp, pkvp, vp, vp, vp, vp]),
+        "ls_commit_accepted_paged": (ctypes.c_int, [vp, vp, pkvp, vp, vp]),
+        "ls_round_paged": (ctypes.c_int, [vp, vp, vp, pkvp, vp, vp, vp, vp, i64, i64, ctypes.c_float, vp, vp]),
         "ls_state_bytes": (sz, [cfgp]),
         "ls_view_state_bytes": (sz, [cfgp, i32]),
         "ls_accept_sampled": (ctypes.c_int, [vp, vp, vp, vp, i32, vp, vp, vp, vp]),
@@ -242,6 +275,34 @@ def ls_round(state, draft_ids, target_ids, verify_k, verify_v, verify_hidden, ac
         state, _ptr(draft_ids), _ptr(target_ids), _ptr(verify_k), _ptr(verify_v), _ptr(verify_hidden),
         _ptr(accept_len), _ptr(next_token), _ptr(q), boundary_k_offset, boundary_v_offset,
         float(softmax_scale), _ptr(out), _stream(stream)))
+
+
+def ls_prefill_paged(state, kv: ls_paged_kv, prefix_len, row_begin, row_end, last_hidden, workspace=None,
+                     workspace_bytes=0, stream=None) -> None:
+    """Prefill reading the prefix from the paged cache; workspace None uses the library's fixed scratch."""
+    _check("ls_prefill_paged", _lib.ls_prefill_paged(
+        state, ctypes.byref(kv), _ptr(prefix_len), row_begin, row_end, _ptr(last_hidden), _ptr(workspace),
+        workspace_bytes, _stream(stream)))
+
+
+def ls_commit_round_paged(state, draft_ids, target_ids, kv: ls_paged_kv, verify_hidden, accept_len, next_token,
+                          stream=None) -> None:
+    _check("ls_commit_round_paged", _lib.ls_commit_round_paged(
+        state, _ptr(draft_ids), _ptr(target_ids), ctypes.byref(kv), _ptr(verify_hidden), _ptr(accept_len),
+        _ptr(next_token), _stream(stream)))
+
+
+def ls_commit_accepted_paged(state, accept_len, kv: ls_paged_kv, verify_hidden, stream=None) -> None:
+    _check("ls_commit_accepted_paged", _lib.ls_commit_accepted_paged(
+        state, _ptr(accept_len), ctypes.byref(kv), _ptr(verify_hidden), _stream(stream)))
+
+
+def ls_round_paged(state, draft_ids, target_ids, kv: ls_paged_kv, verify_hidden, accept_len, next_token, q,
+                   boundary_k_offset, boundary_v_offset, softmax_scale, out, stream=None) -> None:
+    _check("ls_round_paged", _lib.ls_round_paged(
+        state, _ptr(draft_ids), _ptr(target_ids), ctypes.byref(kv), _ptr(verify_hidden), _ptr(accept_len),
+        _ptr(next_token), _ptr(q), boundary_k_offset, boundary_v_offset, float(softmax_scale), _ptr(out),
+        _stream(stream)))
 
 
 def ls_round_overlaps(state) -> bool:

@@ -25,6 +25,12 @@ cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, cons
                            int64_t plane_stride, int64_t row_stride, const int64_t* prefix_len,
                            int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws,
                            int sms, cudaStream_t stream);
+cudaError_t launch_commit_paged(const Dev& p, const int32_t* draft, const int32_t* target, const ls_paged_kv& kv,
+                                const void* vh, int32_t* accept_len, int32_t* next_token, const int32_t* given_a,
+                                cudaStream_t stream);
+cudaError_t launch_prefill_paged(const Dev& p, const ls_config& c, const ls_paged_kv& kv, const int64_t* prefix_len,
+                                 int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws, int sms,
+                                 cudaStream_t stream);
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** out);
 }  // namespace ls
@@ -73,6 +79,40 @@ int validate(const ls_config* c) {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? LS_OK : LS_ERR_CUDA; }
+
+// A paged-cache descriptor usable by the kernels for this config: every tapped layer's
+// pages given and 16-byte aligned, packed rows of all KV heads, strides in whole
+// 16-byte steps (8 elements), a block table and at least one page.
+int validate_paged(const ls_config& c, const ls_paged_kv* kv) {
+  if (!kv) return LS_ERR_INVALID_ARG;
+  if (c.n_layers > LS_MAX_PAGED_LAYERS) return LS_ERR_UNSUPPORTED;
+  for (int l = 0; l < c.n_layers; ++l) {
+    if (!kv->k_layers[l] || !kv->v_layers[l]) return LS_ERR_INVALID_ARG;
+    if (!aligned16(kv->k_layers[l]) || !aligned16(kv->v_layers[l])) return LS_ERR_INVALID_ARG;
+  }
+  if (!kv->block_table || kv->page_size < 1 || kv->max_blocks < 1 || kv->num_pages < 1) return LS_ERR_INVALID_ARG;
+  if (kv->slot_stride < int64_t(c.n_kv_heads) * c.head_dim || kv->slot_stride % 8 != 0 ||
+      kv->page_stride < 0 || kv->page_stride % 8 != 0)
+    return LS_ERR_SHAPE;
+  return LS_OK;
+}
+
+// Argument checks of the whole-round calls beyond those of the commit they make.
+int round_checks(const ls_state* st, int64_t boundary_k_offset, int64_t boundary_v_offset, float softmax_scale,
+                 const void* d_q, const void* d_out) {
+  const ls_config& c = st->cfg;
+  const int64_t span = int64_t(c.n_kv_heads) * c.head_dim;
+  if (boundary_k_offset < 0 || boundary_v_offset < 0 || boundary_k_offset % 8 != 0 ||
+      boundary_v_offset % 8 != 0 || boundary_k_offset + span > c.hidden || boundary_v_offset + span > c.hidden)
+    return LS_ERR_SHAPE;
+  if (!(softmax_scale > 0.0f) || softmax_scale == INFINITY) return LS_ERR_INVALID_ARG;
+  if (!aligned16(d_q) || !aligned16(d_out)) return LS_ERR_INVALID_ARG;
+  return LS_OK;
+}
+
+// The attention half of a whole round (after its commit was enqueued).
+int round_attend(ls_state* st, const void* d_q, int64_t boundary_k_offset, int64_t boundary_v_offset,
+                 float softmax_scale, void* d_out, cudaStream_t stream);
 
 }  // namespace
 
@@ -235,6 +275,54 @@ int ls_prefill_summary_noalloc(ls_state* st, const void* d_k, const void* d_v, i
                                         row_begin, row_end, d_last_hidden, ws, st->sms, stream));
 }
 
+int ls_prefill_paged(ls_state* st, const ls_paged_kv* h_kv, const int64_t* d_prefix_len, int64_t row_begin,
+                     int64_t row_end, const void* d_last_hidden, void* d_workspace, size_t workspace_bytes,
+                     cudaStream_t stream) {
+  if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
+  const ls_config& c = st->cfg;
+  if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
+  if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
+  if (row_end > row_begin) {
+    const int v = validate_paged(c, h_kv);
+    if (v != LS_OK) return v;
+  }
+  if (d_last_hidden && !aligned16(d_last_hidden)) return LS_ERR_INVALID_ARG;
+  const size_t need = ls::prefill_workspace_bytes(c, row_begin, row_end);
+  void* ws = d_workspace;
+  if (ws) {
+    if (!aligned16(ws)) return LS_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return LS_ERR_SHAPE;
+  } else {  // the library's fixed scratch
+    if (need > ls::noalloc_scratch_bytes()) return LS_ERR_SCRATCH_LIMIT;
+    if (ls::noalloc_scratch(&ws) != cudaSuccess) return LS_ERR_CUDA;
+  }
+  static const ls_paged_kv kNone{};
+  return cuda_status(ls::launch_prefill_paged(st->dev, c, row_end > row_begin ? *h_kv : kNone, d_prefix_len,
+                                              row_begin, row_end, d_last_hidden, ws, st->sms, stream));
+}
+
+int ls_commit_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
+                          const ls_paged_kv* h_kv, const void* d_verify_hidden, int32_t* d_accept_len,
+                          int32_t* d_next_token, cudaStream_t stream) {
+  if (!st || !d_draft_ids || !d_target_ids || !d_verify_hidden || !d_accept_len || !d_next_token)
+    return LS_ERR_INVALID_ARG;
+  const int v = validate_paged(st->cfg, h_kv);
+  if (v != LS_OK) return v;
+  if (!aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
+  return cuda_status(ls::launch_commit_paged(st->dev, d_draft_ids, d_target_ids, *h_kv, d_verify_hidden,
+                                             d_accept_len, d_next_token, nullptr, stream));
+}
+
+int ls_commit_accepted_paged(ls_state* st, const int32_t* d_accept_len, const ls_paged_kv* h_kv,
+                             const void* d_verify_hidden, cudaStream_t stream) {
+  if (!st || !d_accept_len || !d_verify_hidden) return LS_ERR_INVALID_ARG;
+  const int v = validate_paged(st->cfg, h_kv);
+  if (v != LS_OK) return v;
+  if (!aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
+  return cuda_status(ls::launch_commit_paged(st->dev, nullptr, nullptr, *h_kv, d_verify_hidden, nullptr, nullptr,
+                                             d_accept_len, stream));
+}
+
 int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
                     const void* d_verify_k, const void* d_verify_v, const void* d_verify_hidden,
                     int32_t* d_accept_len, int32_t* d_next_token, cudaStream_t stream) {
@@ -313,18 +401,32 @@ int ls_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_i
   if (!st || !d_draft_ids || !d_target_ids || !d_verify_k || !d_verify_v || !d_verify_hidden || !d_accept_len ||
       !d_next_token || !d_q || !d_out)
     return LS_ERR_INVALID_ARG;
-  const ls_config& c = st->cfg;
-  const int64_t span = int64_t(c.n_kv_heads) * c.head_dim;
-  if (boundary_k_offset < 0 || boundary_v_offset < 0 || boundary_k_offset % 8 != 0 ||
-      boundary_v_offset % 8 != 0 || boundary_k_offset + span > c.hidden || boundary_v_offset + span > c.hidden)
-    return LS_ERR_SHAPE;
-  if (!(softmax_scale > 0.0f) || softmax_scale == INFINITY) return LS_ERR_INVALID_ARG;
-  if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden) || !aligned16(d_q) ||
-      !aligned16(d_out))
-    return LS_ERR_INVALID_ARG;
+  const int rc = round_checks(st, boundary_k_offset, boundary_v_offset, softmax_scale, d_q, d_out);
+  if (rc != LS_OK) return rc;
   int r = ls_commit_round(st, d_draft_ids, d_target_ids, d_verify_k, d_verify_v, d_verify_hidden, d_accept_len,
                           d_next_token, stream);
   if (r != LS_OK) return r;
+  return round_attend(st, d_q, boundary_k_offset, boundary_v_offset, softmax_scale, d_out, stream);
+}
+
+int ls_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids, const ls_paged_kv* h_kv,
+                   const void* d_verify_hidden, int32_t* d_accept_len, int32_t* d_next_token, const void* d_q,
+                   int64_t boundary_k_offset, int64_t boundary_v_offset, float softmax_scale, void* d_out,
+                   cudaStream_t stream) {
+  if (!st || !d_q || !d_out) return LS_ERR_INVALID_ARG;
+  int r = round_checks(st, boundary_k_offset, boundary_v_offset, softmax_scale, d_q, d_out);
+  if (r != LS_OK) return r;
+  r = ls_commit_round_paged(st, d_draft_ids, d_target_ids, h_kv, d_verify_hidden, d_accept_len, d_next_token, stream);
+  if (r != LS_OK) return r;
+  return round_attend(st, d_q, boundary_k_offset, boundary_v_offset, softmax_scale, d_out, stream);
+}
+
+}  // extern "C"
+
+namespace {
+int round_attend(ls_state* st, const void* d_q, int64_t boundary_k_offset, int64_t boundary_v_offset,
+                 float softmax_scale, void* d_out, cudaStream_t stream) {
+  const ls_config& c = st->cfg;
   const char* bnd = static_cast<const char*>(st->dev.boundary);
   const int64_t e = st->lay.elem;
   if (st->use_tc)  // the attention kernel is scheduled while the commit runs
@@ -334,6 +436,9 @@ int ls_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_i
   return ls_draft_attend(st, 0, c.n_layers, d_q, bnd + boundary_k_offset * e, bnd + boundary_v_offset * e, c.hidden,
                          softmax_scale, d_out, stream);
 }
+}  // namespace
+
+extern "C" {
 
 int ls_round_overlaps(const ls_state* st) { return st && st->use_tc ? 1 : 0; }
 

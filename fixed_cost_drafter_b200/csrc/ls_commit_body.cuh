@@ -4,7 +4,8 @@
 // One warp handles one tensor (K or V) of one KV head, in two phases:
 //   load_scan  the counters and token ids first, then the greedy accept scan (two
 //              ballots cover B <= 64 drafts): a, Delta = a + 1. Only then are the bulk
-//              inputs issued (all B + 1 verify rows, the fp32 partial / global sums), so
+//              inputs issued (the retained verify rows 0..a, from the dense verify block
+//              or the target's paged cache, and the fp32 partial / global sums), so
 //              the few scan inputs do not queue behind them and the loads that need a
 //              (the boundary slice) join the same round trip.
 //   apply      rows 0..a go to ring slot (len + i) mod W with 16-byte stores, and the same
@@ -45,10 +46,52 @@ struct CommitRegs {
   float pr[NSC][Elem<T>::kVec];   // partial sums per scale (lanes of row group 0)
 };
 
-template <typename T, int ROWS, int NSC>
+// Where the verify rows come from: the dense verify block [b][L][B+1][Hkv][D] ...
+struct DenseVerify {
+  const void* k;
+  const void* v;
+};
+// ... or the target's paged KV cache, verify row i at the target's position len + i.
+struct PagedVerify {
+  ls_paged_kv kv;
+};
+
+// This lane's 16-byte pieces of the retained verify rows 0..a (rows rg + j * rpi).
+template <typename T, int ROWS>
+__device__ inline void load_verify_rows(const Dev& p, const DenseVerify& s, int bl, int h, int t, int64_t, int a,
+                                        int rg, int rpi, int cb, uint4 (&raw)[ROWS]) {
+  const int64_t row_stride = int64_t(p.Hkv) * p.D;
+  const T* src = static_cast<const T*>(t == 0 ? s.k : s.v) + int64_t(bl) * (p.B + 1) * row_stride +
+                 int64_t(h) * p.D + cb;
+#pragma unroll
+  for (int j = 0; j < ROWS; ++j) {
+    const int i = rg + j * rpi;
+    if (i <= a) raw[j] = ld_nc_v4(src + int64_t(i) * row_stride);
+  }
+}
+
+template <typename T, int ROWS>
+__device__ inline void load_verify_rows(const Dev& p, const PagedVerify& s, int bl, int h, int t, int64_t len,
+                                        int a, int rg, int rpi, int cb, uint4 (&raw)[ROWS]) {
+  const int b = bl / p.L, l = bl - b * p.L;
+  const char* base = static_cast<const char*>(t == 0 ? s.kv.k_layers[l] : s.kv.v_layers[l]);
+  const int64_t col = (int64_t(h) * p.D + cb) * int64_t(sizeof(T));
+  // every page lookup first, so the row loads leave in one round trip after them
+  const char* rp[ROWS];
+#pragma unroll
+  for (int j = 0; j < ROWS; ++j) {
+    const int i = rg + j * rpi;
+    rp[j] = i <= a ? paged_row(s.kv, base, b, len + i, int(sizeof(T)), p.err) : nullptr;
+  }
+#pragma unroll
+  for (int j = 0; j < ROWS; ++j)
+    if (rg + j * rpi <= a) raw[j] = ld_nc_v4(rp[j] + col);
+}
+
+template <typename T, int ROWS, int NSC, typename Src>
 __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int lane,
                                         const int32_t* __restrict__ draft, const int32_t* __restrict__ target,
-                                        const T* __restrict__ vsrc, CommitRegs<T, ROWS, NSC>& r,
+                                        const Src& vsrc, CommitRegs<T, ROWS, NSC>& r,
                                         CommitScan& cs, const int32_t* __restrict__ given_a = nullptr) {
   constexpr int VEC = Elem<T>::kVec;
   const int b = bl / p.L;
@@ -58,7 +101,6 @@ __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int 
   const int c = lane & (lpr - 1), rg = lane / lpr;
   const int cb = c * VEC;
   const int64_t tile = int64_t(bl) * p.Hkv + h;
-  const int64_t row_stride = int64_t(p.Hkv) * p.D;
 
   const int64_t len = ctr[0];
   int64_t nseg[kMaxScales];
@@ -95,14 +137,10 @@ __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int 
 #pragma unroll
   for (int k = 0; k < kMaxScales; ++k) cs.nseg[k] = nseg[k];
   cs.closes = closes;
-  // the rest of the round's inputs: issued once a is known, so they share one round trip
-  // with the loads the caller issues next (the boundary slice at verify row a)
-  const T* src = vsrc + int64_t(bl) * (p.B + 1) * row_stride + int64_t(h) * p.D + cb;
-#pragma unroll
-  for (int j = 0; j < ROWS; ++j) {
-    const int i = rg + j * rpi;
-    if (i <= p.B) r.raw[j] = ld_nc_v4(src + int64_t(i) * row_stride);
-  }
+  // the rest of the round's inputs: issued once a is known (only the retained rows are
+  // read), so they share one round trip with the loads the caller issues next (the
+  // boundary slice at verify row a)
+  load_verify_rows<T, ROWS>(p, vsrc, bl, h, t, len, a, rg, rpi, cb, r.raw);
   if (rg == 0) {
     const float* gp = p.glob + (tile * 2 + t) * p.D + cb;
 #pragma unroll

@@ -192,4 +192,34 @@ __device__ inline uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
+// ---- paged KV cache ---------------------------------------------------------------
+// Byte address of the row (all KV heads) at position `pos` of sequence b in the layer
+// whose pages start at `base`: page block_table[b][pos / page_size], offset
+// pos mod page_size. A position past the block table or a page id outside
+// [0, num_pages) sets LS_DEVERR_PAGE and gives the same offset in page 0, so no access
+// leaves the caller's pages.
+__device__ inline const char* paged_row(const ls_paged_kv& kv, const char* base, int b, int64_t pos, int elem,
+                                        int32_t* err) {
+  int64_t pi;
+  int off;
+  const int ps = kv.page_size;
+  if ((ps & (ps - 1)) == 0) {  // the usual page sizes: shift and mask
+    pi = pos >> (__ffs(ps) - 1);
+    off = int(pos & (ps - 1));
+  } else if (pos < (int64_t(1) << 32)) {
+    const uint32_t q = uint32_t(pos) / uint32_t(ps);
+    pi = q;
+    off = int(uint32_t(pos) - q * uint32_t(ps));
+  } else {
+    pi = pos / ps;
+    off = int(pos - pi * ps);
+  }
+  int64_t page = pi < kv.max_blocks ? int64_t(__ldg(kv.block_table + int64_t(b) * kv.max_blocks + pi)) : -1;
+  if (page < 0 || page >= kv.num_pages) {
+    set_err(err, LS_DEVERR_PAGE);
+    page = 0;
+  }
+  return base + (page * kv.page_stride + int64_t(off) * kv.slot_stride) * elem;
+}
+
 }  // namespace ls

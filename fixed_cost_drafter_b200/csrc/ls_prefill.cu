@@ -3,7 +3,8 @@
 //
 // Pass 1 (prefill_units_kernel, persistent, one CTA per SM): the work items are units
 // of U prefix rows of one (sequence, layer); U is the largest scale <= 512. A producer
-// warp streams each unit's K and V rows (all KV heads of a row are contiguous) through
+// warp streams each unit's K and V rows (all KV heads of a row are contiguous; from a
+// dense input, or in place from the target's paged cache, one copy per page run) through
 // the TMA engine into a ring of shared-memory stages (cp.async.bulk + mbarrier
 // transaction counts; the consumers release a stage through an "empty" mbarrier, no
 // block-wide barrier); every consumer thread owns one 16-byte column vector and keeps
@@ -78,9 +79,52 @@ __device__ inline void cursor_next(const PrefillArgs& a, const Dev& p, Cursor& c
   cursor_settle(a, p, c);
 }
 
-template <typename T, int CVT>
+// Where the prefix rows come from: the dense [b*L planes][rows][Hkv][D] input (a.k, a.v)
+// or the target's paged KV cache read in place.
+struct DensePrefix {};
+
+// Issues the bulk copies of rows [g0, g0 + nrows) of tensor t (0 = K, 1 = V) of (sequence,
+// layer) bl into dst (rows of rowBytes bytes, back to back), completing on `bar`.
+template <typename T>
+__device__ inline void issue_prefix_rows(const Dev&, const PrefillArgs& a, const DensePrefix&, int t, int bl,
+                                         int64_t g0, int nrows, char* dst, int rowBytes, uint64_t* bar) {
+  const char* base = (t == 0 ? a.k : a.v) +
+                     (int64_t(bl) * a.plane_stride + (g0 - a.row_begin) * a.row_stride) * int64_t(sizeof(T));
+  if (a.row_stride * int64_t(sizeof(T)) == rowBytes) {
+    bulk_g2s(dst, base, uint32_t(nrows * rowBytes), bar);
+  } else {
+    for (int r = 0; r < nrows; ++r)
+      bulk_g2s(dst + r * rowBytes, base + int64_t(r) * a.row_stride * int64_t(sizeof(T)), uint32_t(rowBytes), bar);
+  }
+}
+
+// Paged: one copy per run of rows inside a page (per row when the slots are not packed).
+template <typename T>
+__device__ inline void issue_prefix_rows(const Dev& p, const PrefillArgs&, const ls_paged_kv& kv, int t, int bl,
+                                         int64_t g0, int nrows, char* dst, int rowBytes, uint64_t* bar) {
+  const int b = bl / p.L, l = bl - b * p.L;
+  const char* base = static_cast<const char*>(t == 0 ? kv.k_layers[l] : kv.v_layers[l]);
+  const bool packed = kv.slot_stride * int64_t(sizeof(T)) == rowBytes;
+  int r = 0;
+  while (r < nrows) {
+    const int64_t pos = g0 + r;
+    const int off = int(pos % kv.page_size);
+    const int run = min(nrows - r, kv.page_size - off);
+    const char* src = paged_row(kv, base, b, pos, int(sizeof(T)), p.err);
+    if (packed) {
+      bulk_g2s(dst + r * rowBytes, src, uint32_t(run * rowBytes), bar);
+    } else {
+      for (int i = 0; i < run; ++i)
+        bulk_g2s(dst + (r + i) * rowBytes, src + int64_t(i) * kv.slot_stride * int64_t(sizeof(T)),
+                 uint32_t(rowBytes), bar);
+    }
+    r += run;
+  }
+}
+
+template <typename T, int CVT, typename Src>
 __global__ void __launch_bounds__(kPrefillBlock, 1)
-prefill_units_kernel(Dev p, PrefillArgs a) {
+prefill_units_kernel(Dev p, PrefillArgs a, const Src src) {
   using E = Elem<T>;
   constexpr int VEC = E::kVec;
   extern __shared__ __align__(128) char smem[];
@@ -132,18 +176,8 @@ prefill_units_kernel(Dev p, PrefillArgs a) {
         const int nrows = int(min(int64_t(a.G), r1 - g0));
         char* dst = smem + buf * stageBytes;
         mbar_arrive_expect_tx(&full[buf], uint32_t(2 * nrows * rowBytes));
-        for (int t = 0; t < 2; ++t) {
-          const char* base = (t == 0 ? a.k : a.v) +
-                             (int64_t(bl) * a.plane_stride + (g0 - a.row_begin) * a.row_stride) * int64_t(sizeof(T));
-          char* d = dst + t * a.G * rowBytes;
-          if (a.row_stride == rowElems) {
-            bulk_g2s(d, base, uint32_t(nrows * rowBytes), &full[buf]);
-          } else {
-            for (int r = 0; r < nrows; ++r)
-              bulk_g2s(d + r * rowBytes, base + int64_t(r) * a.row_stride * int64_t(sizeof(T)), uint32_t(rowBytes),
-                       &full[buf]);
-          }
-        }
+        for (int t = 0; t < 2; ++t)
+          issue_prefix_rows<T>(p, a, src, t, bl, g0, nrows, dst + t * a.G * rowBytes, rowBytes, &full[buf]);
         last_issue[buf] = n;
         cursor_next(a, p, prod);
       }
@@ -490,22 +524,23 @@ size_t prefill_workspace_bytes(const ls_config& c, int64_t row_begin, int64_t ro
   return size_t(c.batch) * c.n_layers * size_t(pl.n_units) * 2 * c.n_kv_heads * c.head_dim * 4 + 256;
 }
 
-template <typename T, int CVT>
-static cudaError_t launch_units(const Dev& p, const PrefillArgs& a, int sms, cudaStream_t stream) {
+template <typename T, int CVT, typename Src>
+static cudaError_t launch_units(const Dev& p, const PrefillArgs& a, const Src& src, int sms, cudaStream_t stream) {
   const int rowBytes = p.Hkv * p.D * int(sizeof(T));
   const size_t smem = size_t(kPrefillStages) * 2 * a.G * rowBytes;
-  auto kern = prefill_units_kernel<T, CVT>;
+  auto kern = prefill_units_kernel<T, CVT, Src>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int grid = max(1, min(a.n_items, sms));
-  kern<<<grid, kPrefillBlock, smem, stream>>>(p, a);
+  kern<<<grid, kPrefillBlock, smem, stream>>>(p, a, src);
   return cudaGetLastError();
 }
 
-cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, const void* v,
-                           int64_t plane_stride, int64_t row_stride, const int64_t* prefix_len,
-                           int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws,
-                           int sms, cudaStream_t stream) {
+template <typename Src>
+static cudaError_t launch_prefill_src(const Dev& p, const ls_config& c, const void* k, const void* v,
+                                      int64_t plane_stride, int64_t row_stride, const Src& src,
+                                      const int64_t* prefix_len, int64_t row_begin, int64_t row_end,
+                                      const void* last_hidden, void* ws, int sms, cudaStream_t stream) {
   const PrefillPlan pl = prefill_plan(c, row_begin, row_end);
   PrefillArgs a{};
   a.k = static_cast<const char*>(k);
@@ -527,13 +562,13 @@ cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, cons
   cudaError_t e = cudaSuccess;
   if (a.n_items > 0) {
     if (p.dtype == LS_BF16) {
-      if (cvt <= 1) e = launch_units<__nv_bfloat16, 1>(p, a, sms, stream);
-      else if (cvt <= 2) e = launch_units<__nv_bfloat16, 2>(p, a, sms, stream);
-      else e = launch_units<__nv_bfloat16, 4>(p, a, sms, stream);
+      if (cvt <= 1) e = launch_units<__nv_bfloat16, 1>(p, a, src, sms, stream);
+      else if (cvt <= 2) e = launch_units<__nv_bfloat16, 2>(p, a, src, sms, stream);
+      else e = launch_units<__nv_bfloat16, 4>(p, a, src, sms, stream);
     } else {
-      if (cvt <= 1) e = launch_units<float, 1>(p, a, sms, stream);
-      else if (cvt <= 2) e = launch_units<float, 2>(p, a, sms, stream);
-      else e = launch_units<float, 4>(p, a, sms, stream);
+      if (cvt <= 1) e = launch_units<float, 1>(p, a, src, sms, stream);
+      else if (cvt <= 2) e = launch_units<float, 2>(p, a, src, sms, stream);
+      else e = launch_units<float, 4>(p, a, src, sms, stream);
     }
     if (e != cudaSuccess) return e;
   }
@@ -544,6 +579,21 @@ cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, cons
   else
     prefill_finalize_kernel<float><<<grid, 64, 0, stream>>>(p, a, static_cast<const float*>(last_hidden));
   return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const Dev& p, const ls_config& c, const void* k, const void* v,
+                           int64_t plane_stride, int64_t row_stride, const int64_t* prefix_len,
+                           int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws,
+                           int sms, cudaStream_t stream) {
+  return launch_prefill_src(p, c, k, v, plane_stride, row_stride, DensePrefix{}, prefix_len, row_begin, row_end,
+                            last_hidden, ws, sms, stream);
+}
+
+cudaError_t launch_prefill_paged(const Dev& p, const ls_config& c, const ls_paged_kv& kv, const int64_t* prefix_len,
+                                 int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws, int sms,
+                                 cudaStream_t stream) {
+  return launch_prefill_src(p, c, nullptr, nullptr, 0, 0, kv, prefix_len, row_begin, row_end, last_hidden, ws,
+                            sms, stream);
 }
 
 // ---- fixed scratch for callers that cannot allocate ----------------------------------

@@ -147,31 +147,59 @@ class DeviceRun:
             scale_ptr=self.scale_dev.data_ptr() if (scaled and self.scale_dev is not None) else None,
             scale_heads=self.wl.n_kv_heads, dtype=self.wl.dtype, stream=self.stream.cuda_stream)
 
-    def prefill(self, timer=None):
-        """Generates the prefix (in chunks when asked) and runs ls_prefill_summary over it.
-
-        ``timer``, if given, is called as ``timer(start_event, end_event, bytes)`` around each
-        library call (generation excluded)."""
-        torch, wl = self.torch, self.wl
-        S = self.synth
+    def chunk_bounds(self):
+        """[(row_begin, row_end)]: the prefill chunks, whole largest-scale segments each."""
         P = self.prefix_len
         pmax = int(P.max()) if len(P) else 0
         chunk = self.prefill_chunk or max(pmax, 1)
-        smax = wl.scales[-1]
+        smax = self.wl.scales[-1]
         chunk = max(smax, (chunk // smax) * smax) if pmax > chunk else chunk
-        plen = torch.from_numpy(P).to(self.dev)
-        last_hidden = torch.empty((wl.batch, wl.n_layers, wl.hidden), dtype=self.tdtype, device=self.dev)
-        self._fill(last_hidden, S.LAST_HIDDEN, (1, wl.batch, wl.n_layers, 1, wl.hidden), 0)
-        rowel = wl.n_kv_heads * wl.head_dim
-        rb = 0
+        out, rb = [], 0
         while True:
             re_ = min(rb + chunk, pmax)
+            out.append((rb, re_))
+            if re_ >= pmax:
+                return out
+            rb = re_
+
+    def prefix_chunks(self):
+        """Yields (row_begin, row_end, k, v): the generated prefix chunk by chunk,
+        k/v [b][L][rows][Hkv*D]."""
+        torch, wl, S = self.torch, self.wl, self.synth
+        rowel = wl.n_kv_heads * wl.head_dim
+        for rb, re_ in self.chunk_bounds():
             n = max(re_ - rb, 0)
             k = torch.empty((wl.batch, wl.n_layers, max(n, 1), rowel), dtype=self.tdtype, device=self.dev)
             v = torch.empty_like(k)
             if n:
                 self._fill(k, S.PREFIX_K, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True)
                 self._fill(v, S.PREFIX_V, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True)
+            yield rb, re_, k, v
+            del k, v
+
+    def _last_hidden(self):
+        wl = self.wl
+        last_hidden = self.torch.empty((wl.batch, wl.n_layers, wl.hidden), dtype=self.tdtype, device=self.dev)
+        self._fill(last_hidden, self.synth.LAST_HIDDEN, (1, wl.batch, wl.n_layers, 1, wl.hidden), 0)
+        return last_hidden
+
+    def _prefill_bytes(self, rb, re_):
+        wl = self.wl
+        rows = int(np.maximum(np.minimum(self.prefix_len, re_) - rb, 0).sum())
+        return rows * wl.n_layers * wl.n_kv_heads * wl.head_dim * 2 * wl.elem()
+
+    def prefill(self, timer=None):
+        """Generates the prefix (in chunks when asked) and runs ls_prefill_summary over it.
+
+        ``timer``, if given, is called as ``timer(start_event, end_event, bytes)`` around each
+        library call (generation excluded)."""
+        torch, wl = self.torch, self.wl
+        pmax = int(self.prefix_len.max()) if len(self.prefix_len) else 0
+        plen = torch.from_numpy(self.prefix_len).to(self.dev)
+        last_hidden = self._last_hidden()
+        rowel = wl.n_kv_heads * wl.head_dim
+        for rb, re_, k, v in self.prefix_chunks():
+            n = max(re_ - rb, 0)
             wsb = F.ls_prefill_workspace_bytes(self.cfg, rb, re_)
             ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=self.dev)
             last = re_ >= pmax
@@ -182,13 +210,40 @@ class DeviceRun:
                                  last_hidden if last else None, ws, wsb, self.stream)
             if timer is not None:
                 e1.record(self.stream)
-                rows = int(np.maximum(np.minimum(P, re_) - rb, 0).sum())
-                timer(e0, e1, rows * wl.n_layers * rowel * 2 * wl.elem())
-            del k, v, ws
-            if last:
-                break
-            rb = re_
+                timer(e0, e1, self._prefill_bytes(rb, re_))
+            del ws
         self.last_hidden = last_hidden
+
+    def fill_pages(self, cache):
+        """Writes the generated prefix into a PagedCache (what the target's prefill leaves)."""
+        for rb, re_, k, v in self.prefix_chunks():
+            for b in range(self.wl.batch):
+                hi = min(re_, int(self.prefix_len[b]))
+                if hi > rb:
+                    cache.write(b, rb, k[b, :, :hi - rb], v[b, :, :hi - rb])
+
+    def prefill_paged(self, cache, timer=None, workspace=True):
+        """ls_prefill_paged over the prefix already in ``cache`` (same chunks as ``prefill``;
+        ``workspace`` False uses the library's fixed scratch)."""
+        torch = self.torch
+        pmax = int(self.prefix_len.max()) if len(self.prefix_len) else 0
+        plen = torch.from_numpy(self.prefix_len).to(self.dev)
+        last_hidden = self._last_hidden()
+        kv = cache.descriptor()
+        for rb, re_ in self.chunk_bounds():
+            wsb = F.ls_prefill_workspace_bytes(self.cfg, rb, re_)
+            ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=self.dev) if workspace else None
+            last = re_ >= pmax
+            if timer is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+            F.ls_prefill_paged(self.state, kv, plen, rb, re_, last_hidden if last else None, ws,
+                               wsb if workspace else 0, self.stream)
+            if timer is not None:
+                e1.record(self.stream)
+                timer(e0, e1, self._prefill_bytes(rb, re_))
+        self.last_hidden = last_hidden
+        self.paged_len = self.prefix_len.copy()
 
     def make_round_inputs(self, r0=0, n=None):
         """All inputs of rounds [r0, r0+n): verify K/V/hidden and drafter queries."""
@@ -207,6 +262,20 @@ class DeviceRun:
         self._fill(q, S.QUERY, (n, wl.batch, wl.n_layers, wl.block, wl.n_q_heads * wl.head_dim),
                    wl.head_dim, r0=r0)
         return dict(vk=vk, vv=vv, vh=vh, q=q, r0=r0)
+
+    def write_verify_pages(self, cache, inputs, r):
+        """The target's verify pass of round r into ``cache``: its B + 1 K/V rows at the
+        sequences' positions len .. len + B; len then advances by the round's a + 1."""
+        i = r - inputs["r0"]
+        for b in range(self.wl.batch):
+            cache.write(b, int(self.paged_len[b]), inputs["vk"][i][b], inputs["vv"][i][b])
+        self.paged_len = self.paged_len + self.accept_host[r] + 1
+
+    def commit_paged(self, cache, inputs, r):
+        """ls_commit_round_paged of round r (its verify rows already written to ``cache``)."""
+        i = r - inputs["r0"]
+        F.ls_commit_round_paged(self.state, self.draft[r], self.target[r], cache.descriptor(), inputs["vh"][i],
+                                self.accept_len, self.next_token, self.stream)
 
     def commit(self, inputs, r):
         i = r - inputs["r0"]
@@ -279,3 +348,73 @@ class DeviceRun:
             self.close()
         except Exception:
             pass
+
+
+class PagedCache:
+    """A target's paged KV cache of the tapped layers, as an inference engine keeps it.
+
+    Pages are handed out to the sequences from a seeded permutation of the pool, so a
+    sequence's pages are scattered and interleaved with other sequences' pages. Layouts:
+    ``packed``      per layer K and V tensors [num_pages][page_size][Hkv*D];
+    ``interleaved`` per layer one tensor [num_pages][2][page_size][Hkv*D] (K then V per page);
+    ``padded``      packed with each slot padded to Hkv*D + 64 elements (rows not back to back).
+    Positions 0 .. capacity[b] - 1 of sequence b have pages; other block-table entries are -1.
+    """
+
+    def __init__(self, run: DeviceRun, page_size: int, capacity, layout: str = "packed", spare_pages: int = 3,
+                 seed: int = 0):
+        torch, wl = run.torch, run.wl
+        self.torch, self.page_size, self.layout = torch, int(page_size), layout
+        rowel = wl.n_kv_heads * wl.head_dim
+        self.rowel = rowel
+        cap = np.asarray(capacity, dtype=np.int64)
+        n_b = -(-cap // page_size)
+        self.max_blocks = max(int(n_b.max()), 1)
+        self.num_pages = int(n_b.sum()) + spare_pages
+        perm = np.random.default_rng(seed).permutation(self.num_pages)
+        table = np.full((wl.batch, self.max_blocks), -1, dtype=np.int32)
+        o = 0
+        for b in range(wl.batch):
+            table[b, :n_b[b]] = perm[o:o + n_b[b]]
+            o += n_b[b]
+        self.table_host = table
+        self.block_table = torch.from_numpy(table).to(run.dev)
+        NP, PS = self.num_pages, self.page_size
+        self.k, self.v, self.bufs = [], [], []
+        for _ in range(wl.n_layers):
+            if layout == "interleaved":
+                t = torch.zeros((NP, 2, PS, rowel), dtype=run.tdtype, device=run.dev)
+                self.bufs.append(t)
+                self.k.append(t[:, 0])
+                self.v.append(t[:, 1])
+            else:
+                slot = rowel + (64 if layout == "padded" else 0)
+                tk = torch.zeros((NP, PS, slot), dtype=run.tdtype, device=run.dev)
+                tv = torch.zeros_like(tk)
+                self.bufs += [tk, tv]
+                self.k.append(tk[..., :rowel])
+                self.v.append(tv[..., :rowel])
+        self.slot_stride = self.k[0].stride(1)
+        self.page_stride = self.k[0].stride(0)
+        self._desc = F.make_paged_kv([t.data_ptr() for t in self.k], [t.data_ptr() for t in self.v],
+                                     self.page_stride, self.slot_stride, self.block_table, self.max_blocks,
+                                     self.page_size, self.num_pages)
+
+    def descriptor(self):
+        return self._desc
+
+    def locate(self, b: int, p0: int, n: int):
+        """(pages, offsets) of positions p0 .. p0 + n - 1 of sequence b (host arrays)."""
+        pos = np.arange(p0, p0 + n)
+        return self.table_host[b, pos // self.page_size].astype(np.int64), pos % self.page_size
+
+    def write(self, b: int, p0: int, k_rows, v_rows):
+        """Rows [L][n][Hkv*D] of sequence b at positions p0 .. p0 + n - 1, every layer."""
+        n = k_rows.shape[1]
+        pg, off = self.locate(b, p0, n)
+        assert (pg >= 0).all(), "position beyond the sequence's pages"
+        pg = self.torch.from_numpy(pg).to(k_rows.device)
+        off = self.torch.from_numpy(off).to(k_rows.device)
+        for l in range(len(self.k)):
+            self.k[l][pg, off] = k_rows[l]
+            self.v[l][pg, off] = v_rows[l]

@@ -74,6 +74,9 @@ extern "C" {
 #define LS_DEVERR_SAMPLE       0x8  /* ls_accept_sampled: a draft id outside the vocabulary
                                        or a draw with no probability mass;
                                        ls_commit_accepted: a count outside [0, B]       */
+#define LS_DEVERR_PAGE        0x10  /* paged calls: a position past the block table's
+                                       max_blocks pages or a page id outside
+                                       [0, num_pages) (the rows are read from page 0)  */
 
 /* ---- views (Figure 2 caption (b); the component ablations of Table 5) -------- */
 #define LS_VIEW_BOUNDARY 0x1        /* the boundary state (one key/value row)          */
@@ -138,6 +141,33 @@ typedef struct {
 } ls_layout;
 
 typedef struct ls_state ls_state; /* opaque host handle */
+
+/* A target's paged KV cache, read in place (an inference engine keeps K/V in fixed-size
+ * pages; the views are extracted from that state, Figure 2 caption (b)). Host struct,
+ * passed by pointer; the pointers in it are DEVICE memory owned by the caller.
+ *   k_layers[l], v_layers[l]  base of tapped layer l's key / value pages (`dtype`), for
+ *               l < n_layers (<= LS_MAX_PAGED_LAYERS); 16-byte aligned.
+ *   Element (page, offset, h, d) of a layer sits at
+ *               base[page * page_stride + offset * slot_stride + h * D + d]
+ *               (e.g. pages [num_pages][page_size][Hkv][D]: slot_stride = Hkv*D,
+ *               page_stride = page_size*Hkv*D; keys and values interleaved per page as
+ *               [num_pages][2][page_size][Hkv][D]: page_stride = 2*page_size*Hkv*D and
+ *               v_layers[l] = k_layers[l] + page_size*Hkv*D). Both strides are multiples
+ *               of 8 elements, slot_stride >= Hkv*D.
+ *   block_table int32 [b][max_blocks]: position p of sequence b is in page
+ *               block_table[b][p / page_size] at offset p mod page_size.
+ *   num_pages   page ids outside [0, num_pages) set LS_DEVERR_PAGE.                  */
+#define LS_MAX_PAGED_LAYERS 64
+typedef struct {
+  const void* k_layers[LS_MAX_PAGED_LAYERS];
+  const void* v_layers[LS_MAX_PAGED_LAYERS];
+  int64_t page_stride;
+  int64_t slot_stride;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int32_t page_size;
+  int64_t num_pages;
+} ls_paged_kv;
 
 /* Bytes of the state arena for `cfg`. Depends on the shapes only, never on a prefix
  * length (the views are fixed-size: Figure 1 caption, abstract). 0 if cfg is invalid. */
@@ -293,6 +323,34 @@ LS_API int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_
  * alignment padding that ls_state_bytes adds between regions. 0 for an invalid config
  * or `views` outside LS_VIEW_ALL.                                                   */
 LS_API size_t ls_view_state_bytes(const ls_config* cfg, int32_t views);
+
+/* ---- the same calls reading the target's paged KV cache (no dense staging) -------
+ * Prefill: ls_prefill_summary with the prefix rows of sequence b at positions
+ * 0 .. P_b - 1 read from `kv` (h_kv: host pointer to the descriptor, read during the call
+ * only). d_workspace may be NULL: the unit sums then live in the library's fixed 16 MiB
+ * array (the rules of ls_prefill_summary_noalloc apply, LS_ERR_SCRATCH_LIMIT included).
+ * Positions past max_blocks * page_size, or pages outside [0, num_pages), set
+ * LS_DEVERR_PAGE.                                                                     */
+LS_API int ls_prefill_paged(ls_state* st, const ls_paged_kv* h_kv, const int64_t* d_prefix_len,
+                            int64_t row_begin, int64_t row_end, const void* d_last_hidden, void* d_workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+/* ls_commit_round with verify row i's keys/values read from `kv` at the target's position
+ * len_b + i (len_b: the rows the state holds; the verify pass wrote rows 0..B there).
+ * Only the retained rows 0..a are read. The hidden vectors stay a dense input.        */
+LS_API int ls_commit_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
+                                 const ls_paged_kv* h_kv, const void* d_verify_hidden, int32_t* d_accept_len,
+                                 int32_t* d_next_token, cudaStream_t stream);
+
+/* ls_commit_accepted (given counts) reading the verify rows from `kv` as above.        */
+LS_API int ls_commit_accepted_paged(ls_state* st, const int32_t* d_accept_len, const ls_paged_kv* h_kv,
+                                    const void* d_verify_hidden, cudaStream_t stream);
+
+/* ls_round with the commit reading `kv` (ls_commit_round_paged, then the attention).    */
+LS_API int ls_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_ids,
+                          const ls_paged_kv* h_kv, const void* d_verify_hidden, int32_t* d_accept_len,
+                          int32_t* d_next_token, const void* d_q, int64_t boundary_k_offset,
+                          int64_t boundary_v_offset, float softmax_scale, void* d_out, cudaStream_t stream);
 
 /* One whole decoding round: ls_commit_round, then ls_draft_attend over all layers, for
  * drafters whose boundary keys/values are slices of the new boundary hidden vector:

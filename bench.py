@@ -571,24 +571,29 @@ def paged_measure(WLM, wl, dev, flush, evs, n, rank):
     kv = cache.descriptor()
     span = wl.n_kv_heads * wl.head_dim
     warm = 3  # the first rounds load the kernels; rounds run in order (the pages hold them)
+    half = n // 2  # rounds [0, half): block-table lookups; [half, n): the engine's slot mapping
     for i in range(n):
+        d = kv if i < half else run.paged_descriptor(cache, i, with_slots=True)
         flush.zero_()
         evs[i][0].record(stream)
-        F.ls_round_paged(run.state, run.draft[i], run.target[i], kv, inp["vh"][i], run.accept_len, run.next_token,
+        F.ls_round_paged(run.state, run.draft[i], run.target[i], d, inp["vh"][i], run.accept_len, run.next_token,
                          inp["q"][i], 0, span, run.softmax_scale, out, stream)
         evs[i][1].record(stream)
     torch.cuda.synchronize()
-    ms = [e[0].elapsed_time(e[1]) for e in evs[warm:n]]
+    ms = [e[0].elapsed_time(e[1]) for e in evs[warm:half]]
+    ms_slots = [e[0].elapsed_time(e[1]) for e in evs[half + warm:n]]
     status, word = run.error()
     if status != F.LS_OK:
         raise RuntimeError(f"device error word {word:#x} after the paged rounds")
-    deltas = run.accept_host[warm:n] + 1
+    deltas = run.accept_host[warm:half] + 1
     r_bytes = attend_bytes(wl) + commit_bytes(wl, float(deltas.mean()))
     us = float(np.mean(ms)) * 1e3
     res = {"page_size": PAGE_SIZE, "num_pages": cache.num_pages, "prefill": by_ps[PAGE_SIZE],
            "prefill_page_size_%d" % LARGE_PAGE_SIZE: by_ps[LARGE_PAGE_SIZE],
            "round_us": {"mean": us, "median": float(np.median(ms)) * 1e3}, "round_bytes": r_bytes,
-           "round_GBps": r_bytes / us / 1e3, "rounds": n - warm}
+           "round_GBps": r_bytes / us / 1e3, "rounds": half - warm,
+           "round_slots_us": {"mean": float(np.mean(ms_slots)) * 1e3, "median": float(np.median(ms_slots)) * 1e3,
+                              "rounds": len(ms_slots)}}
     run.close()
     del cache
     torch.cuda.empty_cache()

@@ -84,12 +84,14 @@ class ls_paged_kv(ctypes.Structure):
         ("k_layers", ctypes.c_void_p * LS_MAX_PAGED_LAYERS), ("v_layers", ctypes.c_void_p * LS_MAX_PAGED_LAYERS),
         ("page_stride", ctypes.c_int64), ("slot_stride", ctypes.c_int64), ("block_table", ctypes.c_void_p),
         ("max_blocks", ctypes.c_int32), ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int64),
+        ("verify_slots", ctypes.c_void_p),
     ]
 
 
 def make_paged_kv(k_layers, v_layers, page_stride, slot_stride, block_table, max_blocks, page_size,
-                  num_pages) -> ls_paged_kv:
-    """Descriptor from per-layer page buffers (tensors or addresses) and an int32 block table."""
+                  num_pages, verify_slots=None) -> ls_paged_kv:
+    """Descriptor from per-layer page buffers (tensors or addresses), an int32 block table and,
+    optionally, the verify rows' int64 slots [b][B+1]."""
     if len(k_layers) != len(v_layers) or len(k_layers) > LS_MAX_PAGED_LAYERS:
         raise ValueError("one key and one value page buffer per tapped layer, at most LS_MAX_PAGED_LAYERS")
     kv = ls_paged_kv()
@@ -99,6 +101,7 @@ def make_paged_kv(k_layers, v_layers, page_stride, slot_stride, block_table, max
     kv.page_stride, kv.slot_stride = page_stride, slot_stride
     kv.block_table = _ptr(block_table)
     kv.max_blocks, kv.page_size, kv.num_pages = max_blocks, page_size, num_pages
+    kv.verify_slots = _ptr(verify_slots)
     return kv
 
 

@@ -91,6 +91,7 @@ int validate_paged(const ls_config& c, const ls_paged_kv* kv) {
     if (!aligned16(kv->k_layers[l]) || !aligned16(kv->v_layers[l])) return LS_ERR_INVALID_ARG;
   }
   if (!kv->block_table || kv->page_size < 1 || kv->max_blocks < 1 || kv->num_pages < 1) return LS_ERR_INVALID_ARG;
+  if (kv->verify_slots && (reinterpret_cast<uintptr_t>(kv->verify_slots) & 7) != 0) return LS_ERR_INVALID_ARG;
   if (kv->slot_stride < int64_t(c.n_kv_heads) * c.head_dim || kv->slot_stride % 8 != 0 ||
       kv->page_stride < 0 || kv->page_stride % 8 != 0)
     return LS_ERR_SHAPE;

@@ -56,10 +56,27 @@ struct PagedVerify {
   ls_paged_kv kv;
 };
 
+// Loads a source needs before the scan (issued with the counters and token ids): the
+// verify rows' slots when the caller passes an engine's slot mapping.
+template <int ROWS>
+__device__ inline void early_verify(const Dev&, const DenseVerify&, int, int, int, int64_t (&)[ROWS]) {}
+
+template <int ROWS>
+__device__ inline void early_verify(const Dev& p, const PagedVerify& s, int b, int rg, int rpi,
+                                    int64_t (&slot)[ROWS]) {
+  if (!s.kv.verify_slots) return;
+  const int64_t* src = s.kv.verify_slots + int64_t(b) * (p.B + 1);
+#pragma unroll
+  for (int j = 0; j < ROWS; ++j) {
+    const int i = rg + j * rpi;
+    if (i <= p.B) slot[j] = __ldg(src + i);
+  }
+}
+
 // This lane's 16-byte pieces of the retained verify rows 0..a (rows rg + j * rpi).
 template <typename T, int ROWS>
 __device__ inline void load_verify_rows(const Dev& p, const DenseVerify& s, int bl, int h, int t, int64_t, int a,
-                                        int rg, int rpi, int cb, uint4 (&raw)[ROWS]) {
+                                        int rg, int rpi, int cb, const int64_t (&)[ROWS], uint4 (&raw)[ROWS]) {
   const int64_t row_stride = int64_t(p.Hkv) * p.D;
   const T* src = static_cast<const T*>(t == 0 ? s.k : s.v) + int64_t(bl) * (p.B + 1) * row_stride +
                  int64_t(h) * p.D + cb;
@@ -72,16 +89,20 @@ __device__ inline void load_verify_rows(const Dev& p, const DenseVerify& s, int 
 
 template <typename T, int ROWS>
 __device__ inline void load_verify_rows(const Dev& p, const PagedVerify& s, int bl, int h, int t, int64_t len,
-                                        int a, int rg, int rpi, int cb, uint4 (&raw)[ROWS]) {
+                                        int a, int rg, int rpi, int cb, const int64_t (&slot)[ROWS],
+                                        uint4 (&raw)[ROWS]) {
   const int b = bl / p.L, l = bl - b * p.L;
   const char* base = static_cast<const char*>(t == 0 ? s.kv.k_layers[l] : s.kv.v_layers[l]);
   const int64_t col = (int64_t(h) * p.D + cb) * int64_t(sizeof(T));
-  // every page lookup first, so the row loads leave in one round trip after them
+  // the slots given, else every page lookup first, so the row loads leave in one round trip
   const char* rp[ROWS];
+  const bool given = s.kv.verify_slots != nullptr;
 #pragma unroll
   for (int j = 0; j < ROWS; ++j) {
     const int i = rg + j * rpi;
-    rp[j] = i <= a ? paged_row(s.kv, base, b, len + i, int(sizeof(T)), p.err) : nullptr;
+    rp[j] = i > a ? nullptr
+                  : (given ? paged_slot(s.kv, base, slot[j], int(sizeof(T)), p.err)
+                           : paged_row(s.kv, base, b, len + i, int(sizeof(T)), p.err));
   }
 #pragma unroll
   for (int j = 0; j < ROWS; ++j)
@@ -102,6 +123,8 @@ __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int 
   const int cb = c * VEC;
   const int64_t tile = int64_t(bl) * p.Hkv + h;
 
+  int64_t early[ROWS];
+  early_verify<ROWS>(p, vsrc, b, rg, rpi, early);
   const int64_t len = ctr[0];
   int64_t nseg[kMaxScales];
 #pragma unroll
@@ -140,7 +163,7 @@ __device__ inline void commit_load_scan(const Dev& p, int bl, int h, int t, int 
   // the rest of the round's inputs: issued once a is known (only the retained rows are
   // read), so they share one round trip with the loads the caller issues next (the
   // boundary slice at verify row a)
-  load_verify_rows<T, ROWS>(p, vsrc, bl, h, t, len, a, rg, rpi, cb, r.raw);
+  load_verify_rows<T, ROWS>(p, vsrc, bl, h, t, len, a, rg, rpi, cb, early, r.raw);
   if (rg == 0) {
     const float* gp = p.glob + (tile * 2 + t) * p.D + cb;
 #pragma unroll

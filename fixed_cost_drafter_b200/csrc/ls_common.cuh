@@ -222,4 +222,26 @@ __device__ inline const char* paged_row(const ls_paged_kv& kv, const char* base,
   return base + (page * kv.page_stride + int64_t(off) * kv.slot_stride) * elem;
 }
 
+// Byte address of slot `slot` (page * page_size + offset) in the layer at `base`; a slot
+// outside the pool sets LS_DEVERR_PAGE and gives slot 0.
+__device__ inline const char* paged_slot(const ls_paged_kv& kv, const char* base, int64_t slot, int elem,
+                                         int32_t* err) {
+  const int ps = kv.page_size;
+  int64_t page;
+  int off;
+  if ((ps & (ps - 1)) == 0) {
+    page = slot >> (__ffs(ps) - 1);
+    off = int(slot & (ps - 1));
+  } else {
+    page = slot / ps;
+    off = int(slot - page * ps);
+  }
+  if (slot < 0 || page >= kv.num_pages) {
+    set_err(err, LS_DEVERR_PAGE);
+    page = 0;
+    off = 0;
+  }
+  return base + (page * kv.page_stride + int64_t(off) * kv.slot_stride) * elem;
+}
+
 }  // namespace ls

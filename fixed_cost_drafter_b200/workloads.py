@@ -269,13 +269,21 @@ class DeviceRun:
         i = r - inputs["r0"]
         for b in range(self.wl.batch):
             cache.write(b, int(self.paged_len[b]), inputs["vk"][i][b], inputs["vv"][i][b])
+        if not hasattr(self, "verify_slots"):
+            self.verify_slots = {}
+        self.verify_slots[r] = cache.slots(self.paged_len, self.wl.block + 1)
         self.paged_len = self.paged_len + self.accept_host[r] + 1
 
-    def commit_paged(self, cache, inputs, r):
-        """ls_commit_round_paged of round r (its verify rows already written to ``cache``)."""
+    def paged_descriptor(self, cache, r, with_slots=False):
+        """The cache's descriptor, with round r's verify slots when asked."""
+        return cache.descriptor(self.verify_slots[r] if with_slots else None)
+
+    def commit_paged(self, cache, inputs, r, with_slots=False):
+        """ls_commit_round_paged of round r (its verify rows already written to ``cache``),
+        reading them through the block table or, with_slots, at the slots the write used."""
         i = r - inputs["r0"]
-        F.ls_commit_round_paged(self.state, self.draft[r], self.target[r], cache.descriptor(), inputs["vh"][i],
-                                self.accept_len, self.next_token, self.stream)
+        F.ls_commit_round_paged(self.state, self.draft[r], self.target[r], self.paged_descriptor(cache, r, with_slots),
+                                inputs["vh"][i], self.accept_len, self.next_token, self.stream)
 
     def commit(self, inputs, r):
         i = r - inputs["r0"]
@@ -400,8 +408,22 @@ class PagedCache:
                                      self.page_stride, self.slot_stride, self.block_table, self.max_blocks,
                                      self.page_size, self.num_pages)
 
-    def descriptor(self):
-        return self._desc
+    def descriptor(self, verify_slots=None):
+        """The ls_paged_kv descriptor; with ``verify_slots`` (int64 [b][B+1]) set in a copy."""
+        if verify_slots is None:
+            return self._desc
+        d = F.ls_paged_kv.from_buffer_copy(self._desc)
+        d.verify_slots = verify_slots.data_ptr()
+        return d
+
+    def slots(self, lens, n):
+        """int64 [b][n] device tensor: slots (page * page_size + offset) of positions
+        lens[b] .. lens[b] + n - 1, as an engine's slot mapping holds them."""
+        out = np.zeros((len(lens), n), dtype=np.int64)
+        for b, p0 in enumerate(lens):
+            pg, off = self.locate(b, int(p0), n)
+            out[b] = pg * self.page_size + off
+        return self.torch.from_numpy(out).to(self.block_table.device)
 
     def locate(self, b: int, p0: int, n: int):
         """(pages, offsets) of positions p0 .. p0 + n - 1 of sequence b (host arrays)."""

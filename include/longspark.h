@@ -156,7 +156,12 @@ typedef struct ls_state ls_state; /* opaque host handle */
  *               of 8 elements, slot_stride >= Hkv*D.
  *   block_table int32 [b][max_blocks]: position p of sequence b is in page
  *               block_table[b][p / page_size] at offset p mod page_size.
- *   num_pages   page ids outside [0, num_pages) set LS_DEVERR_PAGE.                  */
+ *   num_pages   page ids outside [0, num_pages) set LS_DEVERR_PAGE.
+ *   verify_slots  NULL, or int64 [b][B+1]: the slot (page * page_size + offset) where the
+ *               verify pass wrote verify row i of sequence b (an engine's slot mapping).
+ *               The commit then reads the rows there instead of looking position len + i
+ *               up in the block table, so its row loads no longer wait for that lookup.
+ *               Prefill ignores it.                                                    */
 #define LS_MAX_PAGED_LAYERS 64
 typedef struct {
   const void* k_layers[LS_MAX_PAGED_LAYERS];
@@ -167,6 +172,7 @@ typedef struct {
   int32_t max_blocks;
   int32_t page_size;
   int64_t num_pages;
+  const int64_t* verify_slots;
 } ls_paged_kv;
 
 /* Bytes of the state arena for `cfg`. Depends on the shapes only, never on a prefix

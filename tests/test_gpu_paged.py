@@ -76,6 +76,37 @@ def test_paged_prefill_and_commits_match_dense(page_size, layout, chunk):
     assert paged.error() == (F.LS_OK, 0) and dense.error() == (F.LS_OK, 0)
 
 
+@pytest.mark.parametrize("page_size,layout", [(16, "packed"), (48, "interleaved")])
+def test_paged_commit_with_slot_mapping(page_size, layout):
+    """The commit reading the verify rows at the slots the verify pass wrote (an engine's
+    slot mapping) instead of through the block table: same state as the dense path."""
+    wl = _wl()
+    dense, paged, cache = _pair(wl, page_size, layout, seed=page_size + 1)
+    inp = dense.make_round_inputs()
+    for r in range(dense.rounds):
+        paged.write_verify_pages(cache, inp, r)
+        dense.commit(inp, r)
+        paged.commit_paged(cache, inp, r, with_slots=True)
+        torch.cuda.synchronize()
+        assert torch.equal(dense.accept_len, paged.accept_len) and torch.equal(dense.next_token, paged.next_token)
+    _same_state(dense, paged)
+    assert paged.error() == (F.LS_OK, 0)
+
+
+def test_paged_bad_slot_is_flagged():
+    wl = _wl(rounds=1)
+    run = WL.DeviceRun(wl)
+    cache = WL.PagedCache(run, 16, _capacity(run), seed=12)
+    run.fill_pages(cache)
+    run.prefill_paged(cache)
+    inp = run.make_round_inputs()
+    run.write_verify_pages(cache, inp, 0)
+    run.verify_slots[0][1, 0] = cache.num_pages * cache.page_size  # one slot past the pool
+    run.commit_paged(cache, inp, 0, with_slots=True)
+    status, word = run.error()
+    assert status == F.LS_ERR_DEVICE and word & F.LS_DEVERR_PAGE
+
+
 def _pages_f64(t, H, D):
     bits = t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
     return O.to_f64(bits, "bf16").reshape(t.shape[0], t.shape[1], H, D)
@@ -199,6 +230,7 @@ def test_paged_host_checks():
         return kv
 
     bad = [variant(slot_stride=wl.n_kv_heads * wl.head_dim - 8), variant(slot_stride=good.slot_stride + 4),
+           variant(verify_slots=cache.block_table.data_ptr() + 4),
            variant(page_size=0), variant(num_pages=0), variant(max_blocks=0), variant(block_table=None)]
     k1 = variant()
     k1.k_layers[1] = None

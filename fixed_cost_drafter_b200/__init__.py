@@ -73,6 +73,7 @@ class ls_layout(ctypes.Structure):
         ("off_seg_mean", ctypes.c_size_t), ("off_part_sum", ctypes.c_size_t),
         ("off_glob_sum", ctypes.c_size_t), ("off_boundary", ctypes.c_size_t),
         ("kv_rows", ctypes.c_int32), ("elem_bytes", ctypes.c_int32), ("off_sample", ctypes.c_size_t),
+        ("off_prologue", ctypes.c_size_t),
     ]
 
 

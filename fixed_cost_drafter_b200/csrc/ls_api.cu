@@ -166,6 +166,7 @@ int ls_get_layout(const ls_config* cfg, ls_layout* out) {
   out->off_glob_sum = size_t(y.glob);
   out->off_boundary = size_t(y.boundary);
   out->off_sample = size_t(y.sample);
+  out->off_prologue = size_t(y.prologue);
   out->kv_rows = y.R;
   out->elem_bytes = y.elem;
   return LS_OK;
@@ -210,6 +211,9 @@ int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_st
   p.boundary = base + y.boundary;
   p.samp_count = reinterpret_cast<int32_t*>(base + y.sample);
   p.samp_part = reinterpret_cast<float*>(base + y.sample + int64_t(cfg->batch) * 4);
+  p.pro_part = reinterpret_cast<float*>(base + y.prologue);
+  p.pro_count = reinterpret_cast<int32_t*>(base + y.prologue + int64_t(ls::kProMaxSlots) * ls::kProTileN *
+                                                                       ls::prologue_boundary_rows(cfg->batch) * 4);
 
   st->use_tc = 0;
   if (!(cfg->flags & LS_FLAG_FORCE_SIMT) && ls::tc_supported(p)) {

@@ -28,16 +28,38 @@ struct Dev {
   char* boundary;     // [b][L][hidden] elements
   int32_t* samp_count;  // [b] arrivals of a sequence's CTAs in ls_accept_sampled
   float* samp_part;     // [b][kSampleMaxChunks] vocabulary chunk sums of ls_accept_sampled
+  float* pro_part;      // [kProMaxSlots][128][boundary rows] split-tile partial sums of ls_draft_prologue
+  int32_t* pro_count;   // [kProMaxGrid] arrivals of a split tile's pieces
 };
 
 constexpr int kSampleChunk = 8192;     // vocabulary entries per CTA of ls_accept_sampled
 constexpr int kSampleMaxChunks = 64;   // vocab <= 524288
 
+// ls_draft_prologue: at most this many CTAs (one per SM), tiles of 128 weight rows, 64
+// hidden entries per k-step, at most 256 activation rows per tile.
+constexpr int kProMaxGrid = 160;
+constexpr int kProTileN = 128;
+constexpr int kProKStep = 64;
+constexpr int kProMaxAct = 256;
+
+__host__ __device__ inline bool prologue_shapes_ok(int dtype, int hidden, int Hq, int Hkv, int D, int B) {
+  return dtype == LS_BF16 && hidden % kProKStep == 0 && (Hq * D) % kProTileN == 0 && (2 * Hkv * D) % kProTileN == 0 &&
+         B <= kProMaxAct;
+}
+// MMA N of the boundary projection: the batch (at most 256 per tile) rounded up to 16.
+__host__ __device__ inline int prologue_boundary_rows(int batch) {
+  const int r = batch < kProMaxAct ? batch : kProMaxAct;
+  return (r + 15) & ~15;
+}
+// Split pieces of boundary tiles at most in flight (a CTA's range of k-steps touches at
+// most one more tile than it finishes): 2 per CTA.
+constexpr int kProMaxSlots = 2 * kProMaxGrid;
+
 __host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
 // Arena layout for a validated config (host and device agree by construction).
 struct Layout {
-  int64_t counters, error, sync, kv, seg, part, glob, boundary, sample, total;
+  int64_t counters, error, sync, kv, seg, part, glob, boundary, sample, prologue, total;
   int32_t R, elem;
 };
 
@@ -56,6 +78,9 @@ __host__ inline Layout make_layout(const ls_config& c) {
   y.glob = off;     off = align256(off + tiles * 2 * c.head_dim * 4);
   y.boundary = off; off = align256(off + int64_t(c.batch) * c.n_layers * c.hidden * y.elem);
   y.sample = off;   off = align256(off + int64_t(c.batch) * (1 + kSampleMaxChunks) * 4);
+  y.prologue = off;
+  if (prologue_shapes_ok(c.dtype, c.hidden, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block))
+    off = align256(off + int64_t(kProMaxSlots) * kProTileN * prologue_boundary_rows(c.batch) * 4 + kProMaxGrid * 4);
   y.total = off;
   return y;
 }

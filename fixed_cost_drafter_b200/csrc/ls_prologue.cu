@@ -14,8 +14,14 @@
 // TMEM allocator and MMA issuer (double-buffered accumulator, 2 x 256 columns); warps 2-5
 // epilogue (one TMEM subpartition each: a thread owns one weight row, its outputs go
 // through a shared-memory tile so that whole 256-byte output rows leave as 16-byte
-// stores). Units: (problem, layer, 128-row weight tile, activation tile), queries first;
-// CTA c takes units c, c + grid, ... Every wait is bounded.
+// stores). Units: (problem, layer, 128-row weight tile, activation tile), queries first.
+// CTA c runs units c, c + grid, ... whole as long as every CTA has one; the k-steps of the
+// units left over (boundary tiles, whose outputs are few) are spread evenly over all CTAs,
+// so that every SM streams the same weight bytes, and run first. A piece of such a split
+// tile leaves its fp32 partial sums in the state's scratch; the last piece of a tile to
+// arrive adds them up in piece order (the same sum whatever the arrival order) and stores
+// the tile.
+// Every wait is bounded.
 #include "ls_tc.cuh"
 
 namespace ls {
@@ -23,9 +29,9 @@ namespace ls {
 namespace {
 
 constexpr int kPThreads = 224;                       // 7 warps
-constexpr int kPKStep = 64;                          // hidden entries per stage
-constexpr int kPTileN = 128;                         // weight rows per unit (MMA M)
-constexpr int kPMaxAct = 256;                        // activation rows per unit (MMA N)
+constexpr int kPKStep = kProKStep;                   // hidden entries per stage
+constexpr int kPTileN = kProTileN;                   // weight rows per unit (MMA M)
+constexpr int kPMaxAct = kProMaxAct;                 // activation rows per unit (MMA N)
 constexpr int kPAStages = 6;                         // weight ring (read from HBM: deeper)
 constexpr int kPBStages = 3;                         // activation ring (read from L2)
 constexpr int kPABytes = kPTileN * kPKStep * 2;      // 16 KB
@@ -52,6 +58,10 @@ struct PArgs {
   PProblem pr[2];
   int32_t b, L, k_steps;
   int32_t n_units;
+  int32_t n_full;     // units [0, n_full) run whole, round robin over the CTAs
+  int32_t rem_steps;  // k-steps of the split units [n_full, n_units) (all boundary tiles), 0 if none
+  float* part;        // [slot][128][pr[1].act_rows] partial sums of the split tiles' pieces
+  int32_t* count;     // [unit - n_full] arrivals of a split tile's pieces (zero between calls)
   int32_t* err;
 };
 
@@ -61,8 +71,10 @@ struct PBars {
   uint64_t acc_full[2], acc_empty[2];
   uint64_t out_full, out_free;  // epilogue pass: staged by all 128 threads / copied out
   uint64_t drain;               // after an abort: the MMAs issued so far have completed
+  uint64_t epi;                 // the 128 epilogue threads meet (split tiles' arrivals)
   uint32_t tmem_base;
   uint32_t abort;
+  uint32_t last;                // the epilogue's piece was its tile's last to arrive
 };
 
 struct PUnit {
@@ -79,6 +91,58 @@ __device__ inline PUnit unit_of(const PArgs& a, int u) {
   r.l = u % a.L;
   r.mt = u / a.L;
   return r;
+}
+
+// This CTA's work: pieces of the split units first (a contiguous range of their flattened
+// k-steps, [g0, g1) = [c T / grid, (c + 1) T / grid)), then its whole units. With the
+// pieces first, the sum of a split tile (by its last piece to arrive) runs in the epilogue
+// warps while the CTA's whole units stream, instead of after them.
+struct PWork {
+  int n_pieces, n_items;
+  int64_t g0, g1;
+};
+
+struct PItem {
+  int u;       // unit
+  int k0, k1;  // its k-steps [k0, k1)
+  int slot;    // -1: the whole unit; else the piece's partial-sum slot
+  int r;       // split unit index (u - n_full)
+};
+
+__device__ inline int64_t range_begin(int c, int64_t T, int grid) { return int64_t(c) * T / grid; }
+
+// the CTA whose range holds split k-step g: the largest c with c T / grid <= g (rounded down)
+__device__ inline int range_cta(int64_t g, int64_t T, int grid) { return int(((g + 1) * grid + T - 1) / T) - 1; }
+
+__device__ inline PWork work_of(const PArgs& a) {
+  PWork w;
+  const int c = int(blockIdx.x), G = int(gridDim.x);
+  const int n_whole = c < a.n_full ? (a.n_full - 1 - c) / G + 1 : 0;
+  w.g0 = range_begin(c, a.rem_steps, G);
+  w.g1 = range_begin(c + 1, a.rem_steps, G);
+  w.n_pieces = w.g1 > w.g0 ? int((w.g1 - 1) / a.k_steps - w.g0 / a.k_steps + 1) : 0;
+  w.n_items = w.n_pieces + n_whole;
+  return w;
+}
+
+__device__ inline PItem item_of(const PArgs& a, const PWork& w, int i) {
+  PItem it;
+  if (i >= w.n_pieces) {
+    it.u = int(blockIdx.x) + (i - w.n_pieces) * int(gridDim.x);
+    it.k0 = 0;
+    it.k1 = a.k_steps;
+    it.slot = -1;
+    it.r = -1;
+    return it;
+  }
+  it.r = int(w.g0 / a.k_steps) + i;
+  const int64_t lo = int64_t(it.r) * a.k_steps;
+  it.u = a.n_full + it.r;
+  it.k0 = int((w.g0 > lo ? w.g0 : lo) - lo);
+  it.k1 = int((w.g1 < lo + a.k_steps ? w.g1 : lo + a.k_steps) - lo);
+  // (CTA, split unit) pairs are ordered the same way in both: c + r is unique per piece
+  it.slot = int(blockIdx.x) + it.r;
+  return it;
 }
 
 __device__ inline bool pwait(PBars& s, uint64_t* bar, uint32_t parity, int32_t* err) {
@@ -103,7 +167,7 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   unsigned char* b_ring = a_ring + kPAStages * kPABytes;     // [kPBStages][32 KB]
   unsigned char* out_st = b_ring + kPBStages * kPBBytes;     // [128][128] bf16
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_mine = int(blockIdx.x) < a.n_units ? (a.n_units - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+  const PWork w = work_of(a);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPAStages; ++i) { mbar_init(&s.afull[i], 1); mbar_init(&s.aempty[i], 1); }
@@ -112,6 +176,7 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
     mbar_init(&s.out_full, 128);
     mbar_init(&s.out_free, 128);
     mbar_init(&s.drain, 1);
+    mbar_init(&s.epi, 128);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -140,14 +205,15 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
       const uint64_t pol = is_a ? l2_evict_first() : l2_evict_last();
       bool ok = true;
       int k = 0;
-      for (int i = 0; i < n_mine && ok; ++i) {
-        const PUnit u = unit_of(a, int(blockIdx.x) + i * int(gridDim.x));
+      for (int i = 0; i < w.n_items && ok; ++i) {
+        const PItem it = item_of(a, w, i);
+        const PUnit u = unit_of(a, it.u);
         const PProblem& P = a.pr[u.p];
         const CUtensorMap* m = is_a ? (u.p ? &w1 : &w0) : (u.p ? &x1 : &x0);
         const uint32_t bytes = is_a ? uint32_t(kPABytes) : uint32_t(P.load_rows * kPKStep * 2);
         // the weights are read once: they must not push the activations (read again by
         // every weight tile of the layer) out of L2
-        for (int ks = 0; ks < a.k_steps; ++ks, ++k) {
+        for (int ks = it.k0; ks < it.k1; ++ks, ++k) {
           const int st = k % nst;
           if (!pwait(s, &emptyb[st], ((k / nst) & 1) ^ 1, a.err)) { ok = false; break; }
           mbar_arrive_expect_tx(&fullb[st], bytes);
@@ -168,15 +234,16 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
     if (lane == 0) {
       bool ok = true;
       int k = 0;
-      for (int i = 0; i < n_mine && ok; ++i) {
-        const PUnit u = unit_of(a, int(blockIdx.x) + i * int(gridDim.x));
+      for (int i = 0; i < w.n_items && ok; ++i) {
+        const PItem it = item_of(a, w, i);
+        const PUnit u = unit_of(a, it.u);
         const PProblem& P = a.pr[u.p];
         const int ab = i & 1;
         if (!pwait(s, &s.acc_empty[ab], ((i >> 1) & 1) ^ 1, a.err)) break;
         tc_fence_after();
         const uint32_t id = idesc_bf16(P.act_rows, false, kPTileN);
         const uint32_t d = tmem + uint32_t(ab * kPMaxAct);
-        for (int ks = 0; ks < a.k_steps; ++ks, ++k) {
+        for (int ks = it.k0; ks < it.k1; ++ks, ++k) {
           const int sa = k % kPAStages, sb = k % kPBStages;
           if (!pwait(s, &s.afull[sa], (k / kPAStages) & 1, a.err)) { ok = false; break; }
           if (!pwait(s, &s.bfull[sb], (k / kPBStages) & 1, a.err)) { ok = false; break; }
@@ -185,7 +252,7 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
           const uint64_t db = sdesc(smem_u32(b_ring + sb * kPBBytes), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kPKStep / 16; ++kk)  // K = 16 per MMA: 32 bytes along the row
-            mma_bf16(d, da + uint32_t(kk * 2), db + uint32_t(kk * 2), id, (ks > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(d, da + uint32_t(kk * 2), db + uint32_t(kk * 2), id, (ks > it.k0 || kk > 0) ? 1u : 0u);
           mma_commit(&s.aempty[sa]);
           mma_commit(&s.bempty[sb]);
         }
@@ -196,34 +263,36 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
     // ------------------------------------------------------------ epilogue (warps 2-5)
     // Per 128 activation rows: each thread writes its weight row's outputs (a column of the
     // staging tile [row][128 weight rows]), then all 128 threads copy the tile's valid rows
-    // out as 16-byte pieces of 256-byte output rows.
+    // out as 16-byte pieces of 256-byte output rows. fetch(col, v) gives the thread's 32
+    // accumulator values of activation rows col .. col + 31 (TMEM, or summed partials).
     const int sub = warp & 3;
     const int ecol = 32 * sub + lane;  // this thread's weight row within the unit
     const int etid = threadIdx.x - 64;  // 0..127
     const uint32_t trow = tmem + (uint32_t(32 * sub) << 16);
     __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(out_st);
     int pass = 0;  // epilogue passes so far (phases of out_full / out_free)
+    int meets = 0;  // phases of `epi` so far
     bool ok = true;
-    for (int i = 0; i < n_mine && ok; ++i) {
-      const PUnit u = unit_of(a, int(blockIdx.x) + i * int(gridDim.x));
-      const PProblem& P = a.pr[u.p];
-      const int ab = i & 1;
-      if (!__all_sync(0xffffffffu, pwait(s, &s.acc_full[ab], (i >> 1) & 1, a.err))) break;
-      tc_fence_after();
+    // all 128 epilogue threads meet here (bounded: a thread that gave up makes the rest give up)
+    auto epi_meet = [&]() -> bool {
+      mbar_arrive(&s.epi);
+      return __all_sync(0xffffffffu, pwait(s, &s.epi, uint32_t(meets++) & 1, a.err));
+    };
+    auto store_tile = [&](const PUnit& u, const PProblem& P, auto&& fetch) -> bool {
       const int seq0 = u.mt * P.seq_per_unit;
       const int rows = min(P.seq_per_unit, a.b - seq0) * P.rows_per_seq;  // valid activation rows
-      for (int r0 = 0; r0 < rows && ok; r0 += kPOutRows, ++pass) {
+      for (int r0 = 0; r0 < rows; r0 += kPOutRows, ++pass) {
         // the staging tile is free once every thread has copied the previous pass out
-        if (pass > 0 && !__all_sync(0xffffffffu, pwait(s, &s.out_free, (pass - 1) & 1, a.err))) { ok = false; break; }
+        if (pass > 0 && !__all_sync(0xffffffffu, pwait(s, &s.out_free, (pass - 1) & 1, a.err))) return false;
         const int nr = min(kPOutRows, P.act_rows - r0);
         for (int c0 = 0; c0 < nr; c0 += 32) {
           float v[32];
-          tmem_ld32(trow + uint32_t(ab * kPMaxAct + r0 + c0), v);
+          fetch(r0 + c0, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) stage[(c0 + j) * kPTileN + ecol] = __float2bfloat16_rn(v[j]);
         }
         mbar_arrive(&s.out_full);
-        if (!__all_sync(0xffffffffu, pwait(s, &s.out_full, pass & 1, a.err))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, pwait(s, &s.out_full, pass & 1, a.err))) return false;
         const int vr = min(kPOutRows, rows - r0);
         for (int c = etid; c < vr * 16; c += 128) {  // 16 pieces of 16 bytes per row
           const int m = r0 + (c >> 4);
@@ -234,8 +303,59 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
         }
         mbar_arrive(&s.out_free);
       }
+      return true;
+    };
+    for (int i = 0; i < w.n_items && ok; ++i) {
+      const PItem it = item_of(a, w, i);
+      const PUnit u = unit_of(a, it.u);
+      const PProblem& P = a.pr[u.p];
+      const int ab = i & 1;
+      if (!__all_sync(0xffffffffu, pwait(s, &s.acc_full[ab], (i >> 1) & 1, a.err))) break;
+      tc_fence_after();
+      if (it.slot < 0) {
+        ok = store_tile(u, P, [&](int col, float (&v)[32]) { tmem_ld32(trow + uint32_t(ab * kPMaxAct + col), v); });
+        tc_fence_before();
+        mbar_arrive(&s.acc_empty[ab]);
+        continue;
+      }
+      // a piece of a split tile: its partial sums (this thread's weight row, all activation
+      // rows) go to its slot, and the accumulator is released at once
+      const int na = P.act_rows;  // a multiple of 16
+      float* mine = a.part + (int64_t(it.slot) * kPTileN + ecol) * na;
+      for (int c0 = 0; c0 < na; c0 += 32) {
+        float v[32];
+        tmem_ld32(trow + uint32_t(ab * kPMaxAct + c0), v);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          if (c0 + j < na) *reinterpret_cast<float4*>(mine + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
       tc_fence_before();
       mbar_arrive(&s.acc_empty[ab]);
+      __threadfence();  // this thread's partials are visible before the arrival below
+      if (!epi_meet()) { ok = false; break; }
+      const int64_t T = a.rem_steps;
+      const int G = int(gridDim.x);
+      const int c_first = range_cta(int64_t(it.r) * a.k_steps, T, G);
+      const int c_last = range_cta(int64_t(it.r + 1) * a.k_steps - 1, T, G);
+      if (etid == 0) s.last = atomicAdd(a.count + it.r, 1) == c_last - c_first ? 1u : 0u;
+      if (!epi_meet()) { ok = false; break; }
+      if (!s.last) continue;
+      __threadfence();  // every piece's partials are visible from here on
+      ok = store_tile(u, P, [&](int col, float (&v)[32]) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        for (int c = c_first; c <= c_last; ++c) {  // slot order: the same sum for every arrival order
+          const float* src = a.part + (int64_t(c + it.r) * kPTileN + ecol) * na + col;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            if (col + j < na) {
+              const float4 x = __ldcg(reinterpret_cast<const float4*>(src + j));
+              v[j] += x.x; v[j + 1] += x.y; v[j + 2] += x.z; v[j + 3] += x.w;
+            }
+          }
+        }
+      });
+      if (etid == 0) a.count[it.r] = 0;  // ready for the next call
     }
   }
 
@@ -272,10 +392,7 @@ bool encode_bf16(void* base, int rank, const cuuint64_t* dims, const cuuint64_t*
 
 }  // namespace
 
-bool prologue_supported(const Dev& p) {
-  return p.dtype == LS_BF16 && p.hidden % kPKStep == 0 && (p.Hq * p.D) % kPTileN == 0 &&
-         (2 * p.Hkv * p.D) % kPTileN == 0 && p.B <= kPMaxAct;
-}
+bool prologue_supported(const Dev& p) { return prologue_shapes_ok(p.dtype, p.hidden, p.Hq, p.Hkv, p.D, p.B); }
 
 cudaError_t launch_prologue(const Dev& p, const void* w_kv, const void* w_q, const void* x, void* bkv, void* q,
                             int sms, cudaStream_t stream) {
@@ -341,7 +458,16 @@ cudaError_t launch_prologue(const Dev& p, const void* w_kv, const void* w_q, con
     const cuuint32_t box[3] = {kPKStep, 1, cuuint32_t(K.load_rows)};
     if (!encode_bf16(p.boundary, 3, dims, str, box, &mx1)) return cudaErrorInvalidValue;
   }
-  const int grid = a.n_units < sms ? a.n_units : sms;
+  int grid = sms < kProMaxGrid ? sms : kProMaxGrid;
+  if (a.n_units < grid) grid = a.n_units;
+  // units left over after whole waves: split their k-steps over every CTA when they are all
+  // boundary tiles (their partial sums fit the state's scratch: 128 x K.act_rows fp32 each)
+  const int rem = a.n_units % grid;
+  const bool split = rem > 0 && rem <= K.n_units && K.act_rows == prologue_boundary_rows(p.b);
+  a.n_full = split ? a.n_units - rem : a.n_units;
+  a.rem_steps = split ? rem * a.k_steps : 0;
+  a.part = p.pro_part;
+  a.count = p.pro_count;
   prologue_kernel<<<grid, kPThreads, kPSmemBytes, stream>>>(a, mw0, mx0, mw1, mx1);
   return cudaGetLastError();
 }

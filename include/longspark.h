@@ -130,7 +130,10 @@ typedef struct {
  *   glob_sum  fp32  [b][L][Hkv][2][D]: sum of all retained rows.
  *   boundary  e     [b][L][hidden]: hidden vectors at the last retained position.
  *   sample    int32 [b] then fp32 [b][64]: scratch of ls_accept_sampled (zero counts
- *             between calls), not part of any view.                                 */
+ *             between calls), not part of any view.
+ *   prologue  scratch of ls_draft_prologue (bf16 states whose shapes it supports; else
+ *             empty): fp32 partial sums of the boundary projection's split tiles, then
+ *             int32 arrival counts (zero between calls); not part of any view.         */
 typedef struct {
   size_t total_bytes;
   size_t off_counters, off_error, off_sync, off_kv, off_seg_mean, off_part_sum, off_glob_sum,
@@ -138,6 +141,7 @@ typedef struct {
   int32_t kv_rows;
   int32_t elem_bytes;
   size_t off_sample;
+  size_t off_prologue;
 } ls_layout;
 
 typedef struct ls_state ls_state; /* opaque host handle */

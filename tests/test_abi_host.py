@@ -43,13 +43,19 @@ def test_layout_sizes():
     assert y.off_part_sum - y.off_seg_mean >= b * L * H * nsc * sl * 2 * D * 4
     assert y.off_glob_sum - y.off_part_sum >= b * L * H * nsc * 2 * D * 4
     assert y.off_boundary - y.off_glob_sum >= b * L * H * 2 * D * 4
-    assert y.off_sample - y.off_boundary >= b * L * 4096 * 2 and y.total_bytes - y.off_sample >= b * 65 * 4
+    assert y.off_sample - y.off_boundary >= b * L * 4096 * 2 and y.off_prologue - y.off_sample >= b * 65 * 4
+    # the projections' scratch: 320 split-tile slots of 128 x 16 fp32 partial sums, 160 counts
+    assert y.total_bytes - y.off_prologue == 320 * 128 * 16 * 4 + 160 * 4 + 256 - (320 * 128 * 16 * 4 + 160 * 4) % 256
     for off in (y.off_counters, y.off_error, y.off_sync, y.off_kv, y.off_seg_mean, y.off_part_sum, y.off_glob_sum,
-                y.off_boundary, y.off_sample, y.total_bytes):
+                y.off_boundary, y.off_sample, y.off_prologue, y.total_bytes):
         assert off % 256 == 0
     assert F.ls_state_bytes(c) == y.total_bytes
-    # about 13.3 MB per sequence at Qwen3-8B shapes, whatever the prefix
-    assert 13.2e6 < y.total_bytes / 16 < 13.5e6
+    # about 13.3 MB per sequence of views at Qwen3-8B shapes, whatever the prefix, plus the
+    # 2.6 MB scratch of the projections for the whole batch
+    assert 13.2e6 < y.off_prologue / 16 < 13.4e6 and y.total_bytes - y.off_prologue < 2.7e6
+    # no scratch where the projections do not run (fp32 state)
+    y32 = F.ls_get_layout(_cfg(dtype=F.LS_F32))
+    assert y32.total_bytes == y32.off_prologue
 
 
 def test_view_state_bytes():
@@ -70,9 +76,10 @@ def test_view_state_bytes():
         assert F.ls_view_state_bytes(c, views) == n, views
     everything = F.ls_view_state_bytes(c, F.LS_VIEW_ALL)
     # the arena adds the error word, the commit's arrival counts, the sampler's scratch
-    # (counts + 64 chunk sums per sequence) and the 256-byte alignment of its 10 regions
-    extra = 16 + b * L * 4 + b * 65 * 4
-    assert everything + extra <= F.ls_state_bytes(c) < everything + extra + 10 * 256
+    # (counts + 64 chunk sums per sequence), the projections' scratch and the 256-byte
+    # alignment of its 11 regions
+    extra = 16 + b * L * 4 + b * 65 * 4 + 320 * 128 * 16 * 4 + 160 * 4
+    assert everything + extra <= F.ls_state_bytes(c) < everything + extra + 11 * 256
     assert F.ls_view_state_bytes(c, 8) == 0 and F.ls_view_state_bytes(_cfg(batch=0), 1) == 0
 
 

@@ -6,6 +6,10 @@ the result (an 8-bit significand: within 2^-8 |y| when rounded to nearest):
     |gpu - ref| <= 2^-8 |ref| + hidden * 2^-24 * sum_k |w_nk x_mk|
 Selection weights (ones that pick hidden dimensions) make every sum exact, so the
 boundary keys/values then equal the slice stand-in bit for bit.
+
+Where the tiles do not fill whole waves of CTAs, the boundary tiles left over are split
+along the hidden size and their fp32 partial sums added in a fixed order: the bound above
+holds for any association, and repeated calls give the same bits.
 """
 
 import numpy as np
@@ -162,4 +166,46 @@ def test_prologue_qwen_shapes():
         rows = [(0, 0), (7, 5), (15, 15)]
         Xs = np.stack([_f64(x[b, l, i]) for b, i in rows])
         _check(np.stack([Q[b, l, i] for b, i in rows]), Xs @ Wq.T, _bound_terms(Wq, Xs, hid))
+    assert run.error() == (F.LS_OK, 0)
+
+
+def test_prologue_split_tiles_match_the_oracle():
+    """384 tiles on the GPU's CTAs (256 query tiles, 128 boundary tiles over 8 layers): the
+    boundary tiles past the last whole wave run split along the hidden size. Every output
+    against the oracle; a second call gives the same bits (pieces summed in a fixed order)."""
+    wl = _wl(batch=16, n_layers=8, n_kv_heads=8, n_q_heads=32, hidden=512, prefix=(300, 300))
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    dev = run.dev
+    L, H, Hq, D, hid, B = wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.hidden, wl.block
+    w_kv = _gen((L, 2 * H * D, hid), 21, dev, hid ** -0.5)
+    w_q = _gen((L, Hq * D, hid), 22, dev, hid ** -0.5)
+    x = _gen((wl.batch, L, B, hid), 23, dev, 1.0)
+    bkv, q = _run_prologue(run, wl, w_kv, w_q, x)
+    bkv2, q2 = _run_prologue(run, wl, w_kv, w_q, x)
+    assert torch.equal(bkv, bkv2) and torch.equal(q, q2)
+    h = O.to_f64(run.read_state()["boundary"], "bf16")
+    Wkv, Wq, X = _f64(w_kv), _f64(w_q), _f64(x)
+    ref_bkv, ref_q = O.draft_prologue(Wkv, Wq, h, X)
+    for l in range(L):
+        _check(_f64(bkv)[:, l], ref_bkv[:, l], _bound_terms(Wkv[l], h[:, l], hid))
+        _check(_f64(q)[:, l].reshape(-1, Hq * D), ref_q[:, l].reshape(-1, Hq * D),
+               _bound_terms(Wq[l], X[:, l].reshape(-1, hid), hid))
+    assert run.error() == (F.LS_OK, 0)
+
+
+def test_prologue_split_tiles_selection_exact():
+    """The split boundary tiles with selection weights: every partial sum is exact, so the
+    keys/values equal the boundary slices bit for bit however the pieces are cut."""
+    wl = _wl(batch=16, n_layers=8, n_kv_heads=8, n_q_heads=32, hidden=2048, prefix=(300, 300))
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    dev = run.dev
+    L, H, Hq, D, hid, B = wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.hidden, wl.block
+    w_kv = torch.zeros((L, 2 * H * D, hid), dtype=torch.bfloat16, device=dev)
+    w_kv[:, torch.arange(2 * H * D), torch.arange(2 * H * D)] = 1.0
+    w_q = _gen((L, Hq * D, hid), 24, dev, hid ** -0.5)
+    x = _gen((wl.batch, L, B, hid), 25, dev, 1.0)
+    bkv, _ = _run_prologue(run, wl, w_kv, w_q, x)
+    assert np.array_equal(_bits(bkv), run.read_state()["boundary"][:, :, :2 * H * D])
     assert run.error() == (F.LS_OK, 0)

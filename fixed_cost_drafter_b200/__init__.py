@@ -45,7 +45,7 @@ EXPORTED = (
     "ls_prefill_summary", "ls_prefill_summary_noalloc", "ls_commit_round", "ls_draft_attend",
     "ls_draft_attend_views", "ls_view_state_bytes", "ls_round", "ls_accept_sampled", "ls_commit_accepted",
     "ls_draft_prologue", "ls_prefill_paged", "ls_commit_round_paged", "ls_commit_accepted_paged", "ls_round_paged",
-    "ls_round_overlaps", "ls_attend_uses_tensor_cores",
+    "ls_clear_error", "ls_check_wait_timeout", "ls_round_overlaps", "ls_attend_uses_tensor_cores",
     "ls_read_state", "ls_get_error", "ls_destroy_state", "ls_status_string",
 )
 
@@ -133,6 +133,8 @@ def _load():
         "ls_draft_attend_views": (ctypes.c_int, [vp, i32, i32, vp, vp, vp, i64, ctypes.c_float, i32, vp, vp]),
         "ls_round": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, ctypes.c_float, vp, vp]),
         "ls_round_overlaps": (ctypes.c_int, [vp]),
+        "ls_clear_error": (ctypes.c_int, [vp, vp]),
+        "ls_check_wait_timeout": (ctypes.c_int, [vp, ctypes.c_uint32, vp]),
         "ls_attend_uses_tensor_cores": (ctypes.c_int, [vp]),
         "ls_read_state": (ctypes.c_int, [vp, vp, sz, vp]),
         "ls_get_error": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
@@ -326,6 +328,15 @@ def ls_get_error(state) -> tuple[int, int]:
     code = ctypes.c_int32(0)
     st = _lib.ls_get_error(state, ctypes.byref(code))
     return st, code.value
+
+
+def ls_clear_error(state, stream=None) -> None:
+    _check("ls_clear_error", _lib.ls_clear_error(state, _stream(stream)))
+
+
+def ls_check_wait_timeout(state, polls, stream=None) -> None:
+    """One bounded wait that nothing signals: sets LS_DEVERR_WAIT_TIMEOUT (see the header)."""
+    _check("ls_check_wait_timeout", _lib.ls_check_wait_timeout(state, polls, _stream(stream)))
 
 
 def ls_destroy_state(state) -> None:

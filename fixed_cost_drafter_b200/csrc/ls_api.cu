@@ -33,6 +33,7 @@ cudaError_t launch_prefill_paged(const Dev& p, const ls_config& c, const ls_page
                                  cudaStream_t stream);
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** out);
+cudaError_t launch_wait_timeout(const Dev& p, uint32_t polls, cudaStream_t stream);
 }  // namespace ls
 
 struct ls_state {
@@ -464,6 +465,16 @@ int ls_get_error(const ls_state* st, int32_t* h_code) {
     return LS_ERR_CUDA;
   if (*h_code & LS_DEVERR_WAIT_TIMEOUT) return LS_ERR_DEVICE_TIMEOUT;
   return *h_code ? LS_ERR_DEVICE : LS_OK;
+}
+
+int ls_clear_error(ls_state* st, cudaStream_t stream) {
+  if (!st) return LS_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(st->dev.err, 0, sizeof(int32_t), stream));
+}
+
+int ls_check_wait_timeout(ls_state* st, uint32_t polls, cudaStream_t stream) {
+  if (!st || polls == 0 || polls > ls::kWaitLimit) return LS_ERR_INVALID_ARG;
+  return cuda_status(ls::launch_wait_timeout(st->dev, polls, stream));
 }
 
 void ls_destroy_state(ls_state* st) { delete st; }

@@ -396,12 +396,9 @@ bool prologue_supported(const Dev& p) { return prologue_shapes_ok(p.dtype, p.hid
 
 cudaError_t launch_prologue(const Dev& p, const void* w_kv, const void* w_q, const void* x, void* bkv, void* q,
                             int sms, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // per launch: the attribute belongs to the current device's copy of the kernel
+  cudaError_t e = cudaFuncSetAttribute(prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
+  if (e != cudaSuccess) return e;
   PArgs a{};
   a.b = p.b;
   a.L = p.L;

@@ -393,6 +393,18 @@ LS_API int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStre
  * LS_ERR_DEVICE_TIMEOUT when it is non-zero, LS_OK otherwise.                      */
 LS_API int ls_get_error(const ls_state* st, int32_t* h_code);
 
+/* Clears the device error word (enqueued on `stream`). The word is sticky otherwise: a
+ * bit once set stays until this call or a fresh ls_init_state.                        */
+LS_API int ls_clear_error(ls_state* st, cudaStream_t stream);
+
+/* Check of the device-side failure detection: one kernel polls an mbarrier that nothing
+ * signals, gives up after `polls` polls (1 .. 2^22; each poll suspends for at most a
+ * hardware-chosen interval), sets LS_DEVERR_WAIT_TIMEOUT in the error word and returns,
+ * as every bounded wait of the path kernels does when a partner never arrives. The next
+ * ls_get_error reports LS_ERR_DEVICE_TIMEOUT; the context stays usable (ls_clear_error,
+ * then carry on).                                                                      */
+LS_API int ls_check_wait_timeout(ls_state* st, uint32_t polls, cudaStream_t stream);
+
 /* Frees the host handle only; the arena stays the caller's. */
 LS_API void ls_destroy_state(ls_state* st);
 

@@ -66,3 +66,27 @@ def test_host_validation_rejects_bad_calls():
         F.ls_prefill_summary(run.state, run.arena, run.arena, 0, 128, run.accept_len, 5, 10, None,
                              run.arena, 1 << 20)
     assert e.value.status == F.LS_ERR_SHAPE  # row_begin not a multiple of the largest scale
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    """Failure detection on the device, without a fault: a wait that nothing signals gives
+    up after its poll limit, the host reads LS_ERR_DEVICE_TIMEOUT, and after clearing the
+    error word the same state runs prefill and rounds normally."""
+    wl = WL.Workload("waitcheck", 41, 2, 2, 2, 8, 128, 512, 16, 128, (32, 64, 256), 4, "bf16", (300, 700), 3, None,
+                     1000, head_scale=True)
+    run = WL.DeviceRun(wl)
+    F.ls_check_wait_timeout(run.state, 1000, run.stream)
+    status, word = run.error()
+    assert status == F.LS_ERR_DEVICE_TIMEOUT and word == F.LS_DEVERR_WAIT_TIMEOUT
+    F.ls_clear_error(run.state, run.stream)
+    assert run.error() == (F.LS_OK, 0)
+    run.prefill()
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    for r in range(wl.rounds):
+        run.round(inp, r, out)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    assert run.error() == (F.LS_OK, 0)
+    with pytest.raises(F.LsError):
+        F.ls_check_wait_timeout(run.state, 0, run.stream)

@@ -105,3 +105,27 @@ def test_state_bytes_fixed_across_sweep():
     for batch in WL.SWEEP_BATCHES:
         sizes = {F.ls_state_bytes(WL.sweep_point(p, batch, 4.0).config()) for p in WL.SWEEP_PREFIXES}
         assert len(sizes) == 1
+
+
+def test_full_config_paged():
+    """The bench workload with the prefix and every round's verify rows in a paged cache
+    (page size 16, pages scattered over a 70K-page pool, 18 GB): ls_prefill_paged, then
+    commits reading the pages in place (block table on even rounds, the engine's slot
+    mapping on odd ones) and the attention; sampled tiles against the oracle."""
+    wl = WL.CONFIGS["qwen3_8b_64k"]
+    run = WL.DeviceRun(wl)
+    cache = WL.PagedCache(run, 16, run.prefix_len + (run.rounds + 1) * (wl.block + 1), seed=2)
+    run.fill_pages(cache)
+    run.prefill_paged(cache)
+    inp = run.make_round_inputs()
+    for r in range(run.rounds):
+        run.write_verify_pages(cache, inp, r)
+    out = run.new_out()
+    for r in range(run.rounds):
+        run.commit_paged(cache, inp, r, with_slots=bool(r & 1))
+        run.attend(inp, r, out)
+    torch.cuda.synchronize()
+    assert run.error() == (F.LS_OK, 0)
+    del cache
+    torch.cuda.empty_cache()
+    _sampled_check(run, wl, out, TILES)

@@ -444,6 +444,28 @@ def run_gpu(args):
         paged = paged_measure(WLM, wl, dev, flush, evs, min(K, 200), rank)
 
     # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
+    # the attention as a drafter calls it layer by layer (one launch per tapped layer)
+    per_layer = None
+    if not args.no_ablations:
+        KP = min(K, 200)
+        pl_out = run.new_out(layer_count=1)
+        rs = sorted({(W + i) % n_rounds for i in range(KP)})
+        q_l = {r: [inp["q"][r - inp["r0"]][:, l:l + 1].contiguous() for l in range(wl.n_layers)] for r in rs}
+        ms = []
+        for i in range(KP):
+            r = (W + i) % n_rounds
+            flush.zero_()
+            evs[i][0].record(stream)
+            for l in range(wl.n_layers):
+                F.ls_draft_attend(run.state, l, 1, q_l[r][l], run.boundary_k, run.boundary_v, wl.hidden,
+                                  run.softmax_scale, pl_out, stream)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms = [e[0].elapsed_time(e[1]) for e in evs[:KP]]
+        per_layer = {"launches_per_round": wl.n_layers, "us_per_round": float(np.mean(ms)) * 1e3,
+                     "GBps": attend_bytes(wl) / (float(np.mean(ms)) * 1e3) / 1e3, "rounds": KP}
+        del q_l
+
     graph_rps = None
     if not args.no_graph:
         g = torch.cuda.CUDAGraph()
@@ -496,7 +518,8 @@ def run_gpu(args):
             "roofline": {"bound": "hbm",
                          "kernel": "ls_draft_attend (" + ("tcgen05" if tc else "CUDA cores") + ")",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": a_bytes,
+                         "frac": achieved / peak, "frac_of_nominal_8TBps": achieved / 8000.0,
+                         "traffic": traffic, "algorithmic_bytes": a_bytes,
                          "us": att_s * 1e6, "timed_launches": KS},
             "round_roofline": {"kernels": "ls_round: commit + attention" + (
                                    " (programmatic dependent launch)" if overlapped else " (two launches)"),
@@ -508,6 +531,7 @@ def run_gpu(args):
                       "attend_us": att_s * 1e6, "commit_bytes": c_bytes,
                       "commit_GBps": c_bytes / (float(np.mean(commit_ms)) / 1e3) / 1e9},
             "graph_rounds_per_s": graph_rps,
+            "attend_per_layer": per_layer,
             "view_ablations": ablations,
             "sampled_acceptance": sampled,
             "prologue": prologue,

@@ -287,7 +287,10 @@ LS_API int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const flo
  * ls_draft_attend: d_q as its queries, boundary_k = d_bkv, boundary_v = d_bkv + Hkv D,
  * boundary_stride = 2 Hkv D. Runs on the tcgen05 tensor cores: needs a bf16 state,
  * hidden a multiple of 64, Hq D and 2 Hkv D multiples of 128 (else LS_ERR_UNSUPPORTED);
- * pointers 16-byte aligned.                                                              */
+ * pointers 16-byte aligned. Boundary tiles left over after whole waves of CTAs are split
+ * along the hidden size; their fp32 partial sums use the state's prologue scratch
+ * (ls_layout.off_prologue), so two calls on one state must not overlap on the GPU (order
+ * them on one stream). Repeated calls give the same bits.                               */
 LS_API int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q, const void* d_x,
                              void* d_bkv, void* d_q, cudaStream_t stream);
 

@@ -373,8 +373,7 @@ def run_gpu(args):
     stream = run.stream
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
 
-    clock_path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else "_build",
-                              f"clocks_rank{rank}.csv")
+    clock_path = (args.clock_log or os.path.join(ROOT, "_build", "clocks_rank{rank}.csv")).format(rank=rank)
     os.makedirs(os.path.dirname(clock_path), exist_ok=True)
     overlapped = F.ls_round_overlaps(run.state)
     # the sampler starts with the warm-up rounds so that its samples cover a loaded GPU
@@ -848,6 +847,8 @@ def main(argv=None):
     ap.add_argument("--no-paged", action="store_true", help="skip the paged-KV prefill and round timings")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None,
+                    help="CSV of the nvidia-smi clock samples ('{rank}' is replaced; default _build/clocks_rank{rank}.csv)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--sweep-rounds", type=int, default=40)
     ap.add_argument("--prefix", type=int, default=0, help="override the workload's prefix length")

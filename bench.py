@@ -59,6 +59,16 @@ def sequence_offset(rank: int, batch_per_rank: int) -> int:
     return rank * batch_per_rank
 
 
+def kv_head_range(rank: int, world: int, n_kv_heads: int):
+    """KV heads (h0, h1) owned by `rank` when the ranks split every sequence's KV heads
+    (the natural split for a tensor-parallel target: heads are independent in the commit
+    and the attention, so there is no exchange)."""
+    if n_kv_heads % world:
+        raise ValueError(f"{n_kv_heads} KV heads do not split evenly over {world} ranks")
+    per = n_kv_heads // world
+    return rank * per, (rank + 1) * per
+
+
 def max_over_ranks(x: float, world: int, device=None) -> float:
     if world == 1:
         return x
@@ -358,7 +368,13 @@ def run_gpu(args):
     # distinct rounds of generated inputs; the timed loop cycles through them (the state
     # keeps growing, every round re-reads its inputs from HBM after the L2 flush)
     n_rounds = min(K + W, args.distinct_rounds)
-    run = WLM.DeviceRun(wl, device=dev, rounds=n_rounds, seq_offset=sequence_offset(rank, wl.batch))
+    if args.shard == "kv-heads":  # every rank: all sequences, its share of the KV heads
+        run = WLM.DeviceRun(wl, device=dev, rounds=n_rounds, kv_heads=kv_head_range(rank, world, wl.n_kv_heads))
+    else:  # every rank: its own batch of sequences
+        run = WLM.DeviceRun(wl, device=dev, rounds=n_rounds, seq_offset=sequence_offset(rank, wl.batch))
+    # from here on `wl` is this rank's part (its KV heads under kv-heads sharding)
+    full_wl, wl = wl, run.wl
+    strong = args.shard == "kv-heads"
 
     # prefill (timed separately)
     pre = []
@@ -512,7 +528,7 @@ def run_gpu(args):
         del g
 
     # end to end through the public API with host buffers (pinned), copies inside the region
-    e2e = e2e_measure(run, wl, dev, flush, K, world, inp)
+    e2e = e2e_measure(run, wl, dev, flush, K, world, inp, strong)
 
     # flatness over the prefix (b = 16) on a short sweep
     flat = None
@@ -532,10 +548,11 @@ def run_gpu(args):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": world * K / total_max, "unit": "rounds/s", "n_gpus": world,
-            "steps": K, "warmup": W, "ms_per_step": total_max * 1e3 / K, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(wl),
+            "metric": METRIC, "value": (1 if strong else world) * K / total_max, "unit": "rounds/s",
+            "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": total_max * 1e3 / K, "higher_is_better": True,
+            "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(full_wl),
+                           parallelism=(f"kv-heads x {world}" if strong else f"batch x {world}")),
             "roofline": {"bound": "hbm",
                          "kernel": "ls_draft_attend (" + ("tcgen05" if tc else "CUDA cores") + ")",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
@@ -728,7 +745,7 @@ class L2Flush:
         self.r.sum()
 
 
-def e2e_measure(run, wl, dev, flush, steps, world, inp):
+def e2e_measure(run, wl, dev, flush, steps, world, inp, strong=False):
     """Rounds/s through the public entry point with every step's inputs in pinned host memory
     and its results read back to pinned host memory, inside one timed region.
 
@@ -800,7 +817,7 @@ def e2e_measure(run, wl, dev, flush, steps, world, inp):
     e1.record(cout)
     e1.synchronize()
     tot = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
-    return {"value": world * steps / tot, "unit": "rounds/s", "h2d_bytes_per_step": int(h2d),
+    return {"value": (1 if strong else world) * steps / tot, "unit": "rounds/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "pipelined": "2 buffer slots, copy streams in and out"}
 
 
@@ -847,6 +864,9 @@ def main(argv=None):
     ap.add_argument("--no-paged", action="store_true", help="skip the paged-KV prefill and round timings")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="batch", choices=["batch", "kv-heads"],
+                    help="N > 1: each rank owns a batch of sequences (weak scaling) or a share of every "
+                         "sequence's KV heads (strong scaling)")
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples ('{rank}' is replaced; default _build/clocks_rank{rank}.csv)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

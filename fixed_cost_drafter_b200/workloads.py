@@ -98,10 +98,21 @@ class DeviceRun:
 
     def __init__(self, wl: Workload, device="cuda", rounds: int | None = None,
                  prefill_chunk: int | None = None, prefix_override=None, accepts_override=None,
-                 seq_offset: int = 0):
+                 seq_offset: int = 0, kv_heads=None):
+        """``kv_heads`` = (h0, h1): this run holds KV heads h0 .. h1 - 1 of every sequence (and
+        their query heads), a KV-head shard of the workload; inputs are the same generated
+        values as the whole run's, sliced by head."""
         import torch
         import synth
         self.torch, self.synth = torch, synth
+        self.full_wl = wl
+        self.h0 = 0
+        if kv_heads is not None:
+            h0, h1 = kv_heads
+            if not 0 <= h0 < h1 <= wl.n_kv_heads:
+                raise ValueError(f"KV heads {kv_heads} outside 0..{wl.n_kv_heads}")
+            wl = replace(wl, n_kv_heads=h1 - h0, n_q_heads=(h1 - h0) * wl.group)
+            self.h0 = h0
         self.wl = wl
         self.dev = torch.device(device)
         self.cfg = wl.config()
@@ -116,7 +127,9 @@ class DeviceRun:
         self.prefix_len = (np.asarray(prefix_override, dtype=np.int64) if prefix_override is not None
                            else replace(wl, batch=self.b0 + wl.batch).prefix_lengths()[self.b0:])
         self.prefill_chunk = prefill_chunk
-        self.scale_host = synth.head_scales(wl.seed, wl.n_layers, wl.n_kv_heads) if wl.head_scale else None
+        # per-head scales of every KV head of the workload (a shard indexes them from h0)
+        self.scale_host = (synth.head_scales(wl.seed, wl.n_layers, self.full_wl.n_kv_heads) if wl.head_scale
+                           else None)
         self.scale_dev = (torch.from_numpy(self.scale_host).to(self.dev) if self.scale_host is not None
                           else None)
         nb = self.b0 + wl.batch
@@ -135,17 +148,32 @@ class DeviceRun:
         self.accept_len = torch.zeros(wl.batch, dtype=torch.int32, device=self.dev)
         self.next_token = torch.zeros(wl.batch, dtype=torch.int32, device=self.dev)
         e = wl.elem()
-        self.boundary_k = self.arena.data_ptr() + self.layout.off_boundary
-        self.boundary_v = self.boundary_k + wl.n_kv_heads * wl.head_dim * e
+        # boundary keys/values: this run's heads' slices [h0 D, ...) and [Hkv D + h0 D, ...)
+        # of the (replicated) boundary hidden vector
+        self.bk_off = self.h0 * wl.head_dim
+        self.bv_off = (self.full_wl.n_kv_heads + self.h0) * wl.head_dim
+        self.boundary_k = self.arena.data_ptr() + self.layout.off_boundary + self.bk_off * e
+        self.boundary_v = self.arena.data_ptr() + self.layout.off_boundary + self.bv_off * e
         self.softmax_scale = 1.0 / math.sqrt(wl.head_dim)
 
     # ---- generated inputs -------------------------------------------------------
-    def _fill(self, t, tensor_id, shape, head_dim, r0=0, b0=0, l0=0, p0=0, scaled=False):
+    def _fill(self, t, tensor_id, shape, head_dim, r0=0, b0=0, l0=0, p0=0, scaled=False, x0=0):
         self.synth.device_fill_normal(
             t.data_ptr(), self.wl.seed, tensor_id, shape, r0=r0, b0=self.b0 + b0, l0=l0, p0=p0,
             head_dim=head_dim,
             scale_ptr=self.scale_dev.data_ptr() if (scaled and self.scale_dev is not None) else None,
-            scale_heads=self.wl.n_kv_heads, dtype=self.wl.dtype, stream=self.stream.cuda_stream)
+            scale_heads=self.full_wl.n_kv_heads, dtype=self.wl.dtype, stream=self.stream.cuda_stream, x0=x0,
+            scale_layers=self.wl.n_layers)
+
+    @property
+    def kv_x0(self):
+        """First K/V row column of this run's heads in the workload's rows."""
+        return self.h0 * self.wl.head_dim
+
+    @property
+    def q_x0(self):
+        """First query column of this run's query heads."""
+        return self.h0 * self.wl.group * self.wl.head_dim
 
     def chunk_bounds(self):
         """[(row_begin, row_end)]: the prefill chunks, whole largest-scale segments each."""
@@ -172,8 +200,10 @@ class DeviceRun:
             k = torch.empty((wl.batch, wl.n_layers, max(n, 1), rowel), dtype=self.tdtype, device=self.dev)
             v = torch.empty_like(k)
             if n:
-                self._fill(k, S.PREFIX_K, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True)
-                self._fill(v, S.PREFIX_V, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True)
+                self._fill(k, S.PREFIX_K, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True,
+                           x0=self.kv_x0)
+                self._fill(v, S.PREFIX_V, (1, wl.batch, wl.n_layers, n, rowel), wl.head_dim, p0=rb, scaled=True,
+                           x0=self.kv_x0)
             yield rb, re_, k, v
             del k, v
 
@@ -256,11 +286,13 @@ class DeviceRun:
         vh = torch.empty((n, wl.batch, wl.n_layers, B1, wl.hidden), dtype=self.tdtype, device=self.dev)
         q = torch.empty((n, wl.batch, wl.n_layers, wl.block, wl.n_q_heads * wl.head_dim),
                         dtype=self.tdtype, device=self.dev)
-        self._fill(vk, S.VERIFY_K, (n, wl.batch, wl.n_layers, B1, rowel), wl.head_dim, r0=r0, scaled=True)
-        self._fill(vv, S.VERIFY_V, (n, wl.batch, wl.n_layers, B1, rowel), wl.head_dim, r0=r0, scaled=True)
+        self._fill(vk, S.VERIFY_K, (n, wl.batch, wl.n_layers, B1, rowel), wl.head_dim, r0=r0, scaled=True,
+                   x0=self.kv_x0)
+        self._fill(vv, S.VERIFY_V, (n, wl.batch, wl.n_layers, B1, rowel), wl.head_dim, r0=r0, scaled=True,
+                   x0=self.kv_x0)
         self._fill(vh, S.VERIFY_HIDDEN, (n, wl.batch, wl.n_layers, B1, wl.hidden), 0, r0=r0)
         self._fill(q, S.QUERY, (n, wl.batch, wl.n_layers, wl.block, wl.n_q_heads * wl.head_dim),
-                   wl.head_dim, r0=r0)
+                   wl.head_dim, r0=r0, x0=self.q_x0)
         return dict(vk=vk, vv=vv, vh=vh, q=q, r0=r0)
 
     def write_verify_pages(self, cache, inputs, r):
@@ -307,11 +339,11 @@ class DeviceRun:
 
     def round(self, inputs, r, out):
         """ls_round: commit and attention over all layers in one call (boundary keys and
-        values are the slices [0, Hkv*D) and [Hkv*D, 2*Hkv*D) of the boundary hidden)."""
-        wl = self.wl
+        values are this run's heads' slices of [0, Hkv*D) and [Hkv*D, 2*Hkv*D) of the
+        boundary hidden)."""
         i = r - inputs["r0"]
         F.ls_round(self.state, self.draft[r], self.target[r], inputs["vk"][i], inputs["vv"][i], inputs["vh"][i],
-                   self.accept_len, self.next_token, inputs["q"][i], 0, wl.n_kv_heads * wl.head_dim,
+                   self.accept_len, self.next_token, inputs["q"][i], self.bk_off, self.bv_off,
                    self.softmax_scale, out, self.stream)
 
     def new_out(self, layer_count=None):

@@ -201,24 +201,31 @@ def device_lib():
         lib.lss_fill_normal.argtypes = [
             ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64,
             ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
-            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
             ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p]
         _LIB = lib
     return _LIB
 
 
 def device_fill_normal(out_ptr, seed, tensor_id, shape, r0=0, b0=0, l0=0, p0=0, head_dim=0,
-                       scale_ptr=None, scale_heads=0, dtype="bf16", stream=0):
-    """Same values as :func:`fill_normal` (with x0 = 0) written to device memory.
+                       scale_ptr=None, scale_heads=0, dtype="bf16", stream=0, x0=0, scale_layers=None):
+    """Same values as :func:`fill_normal` written to device memory.
 
     ``out_ptr`` is a device pointer to a contiguous (nr, nb, nl, np, nx) array;
     ``scale_ptr`` a device fp32 [L][scale_heads] array or None.
     """
     nr, nb, nl, npos, nx = shape
+    if scale_ptr:
+        # the kernel reads scale[l][h] for l < l0 + nl and h < (x0 + nx) / head_dim: the
+        # [L][scale_heads] array the caller passes must cover them
+        if head_dim <= 0 or (x0 + nx + head_dim - 1) // head_dim > scale_heads:
+            raise ValueError("per-head scales need head_dim > 0 and columns within scale_heads heads")
+        if scale_layers is not None and l0 + nl > scale_layers:
+            raise ValueError(f"layers {l0}..{l0 + nl - 1} past the {scale_layers}-layer scale array")
     rc = device_lib().lss_fill_normal(
         ctypes.c_void_p(out_ptr), 1 if dtype == "bf16" else 0,
         ctypes.c_uint64(stream_key(seed, tensor_id)),
-        nr, nb, nl, npos, nx, r0, b0, l0, p0, head_dim,
+        nr, nb, nl, npos, nx, r0, b0, l0, p0, x0, head_dim,
         ctypes.c_void_p(scale_ptr or 0), scale_heads, float(INV_STD), ctypes.c_void_p(stream))
     if rc != 0:
         raise RuntimeError(f"lss_fill_normal failed with {rc}")

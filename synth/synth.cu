@@ -23,10 +23,10 @@ __device__ __forceinline__ uint16_t bf16_rne(float x) {
   return uint16_t(u);
 }
 
-// out[((((r*nb + b)*nl + l)*np + p)*nx + x] for the element at (r0+r, b0+b, l0+l, p0+p, x)
+// out[((((r*nb + b)*nl + l)*np + p)*nx + x] for the element at (r0+r, b0+b, l0+l, p0+p, x0+x)
 __global__ void fill_normal_kernel(void* out, int bf16, uint64_t key, int64_t nb, int64_t nl,
                                    int64_t np, int64_t nx, int64_t total, int64_t r0, int64_t b0,
-                                   int64_t l0, int64_t p0, int head_dim, const float* scale,
+                                   int64_t l0, int64_t p0, int64_t x0, int head_dim, const float* scale,
                                    int scale_heads, float inv_std) {
   for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
        idx += int64_t(gridDim.x) * blockDim.x) {
@@ -36,9 +36,10 @@ __global__ void fill_normal_kernel(void* out, int bf16, uint64_t key, int64_t nb
     const int64_t l = t % nl; t /= nl;
     const int64_t b = t % nb; t /= nb;
     const int64_t r = t;
+    const int64_t xg = x0 + x;
     int64_t h, d;
-    if (head_dim > 0) { h = x / head_dim; d = x - h * head_dim; }
-    else { h = x >> 9; d = x & 511; }
+    if (head_dim > 0) { h = xg / head_dim; d = xg - h * head_dim; }
+    else { h = xg >> 9; d = xg & 511; }
     const uint64_t ctr = (uint64_t(r0 + r) << 52) | (uint64_t(b0 + b) << 44) |
                          (uint64_t(l0 + l) << 38) | (uint64_t(p0 + p) << 16) |
                          (uint64_t(h) << 9) | uint64_t(d);
@@ -56,7 +57,7 @@ __global__ void fill_normal_kernel(void* out, int bf16, uint64_t key, int64_t nb
 
 extern "C" __attribute__((visibility("default"))) int lss_fill_normal(void* out, int bf16, uint64_t key, int64_t nr, int64_t nb,
                                int64_t nl, int64_t np, int64_t nx, int64_t r0, int64_t b0,
-                               int64_t l0, int64_t p0, int32_t head_dim, const float* scale,
+                               int64_t l0, int64_t p0, int64_t x0, int32_t head_dim, const float* scale,
                                int32_t scale_heads, float inv_std, cudaStream_t stream) {
   const int64_t total = nr * nb * nl * np * nx;
   if (total <= 0) return 0;
@@ -65,7 +66,7 @@ extern "C" __attribute__((visibility("default"))) int lss_fill_normal(void* out,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (total + 255) / 256;
   const int grid = int(want < int64_t(sms) * 16 ? want : int64_t(sms) * 16);
-  fill_normal_kernel<<<grid, 256, 0, stream>>>(out, bf16, key, nb, nl, np, nx, total, r0, b0, l0, p0,
+  fill_normal_kernel<<<grid, 256, 0, stream>>>(out, bf16, key, nb, nl, np, nx, total, r0, b0, l0, p0, x0,
                                                head_dim, scale, scale_heads, inv_std);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }

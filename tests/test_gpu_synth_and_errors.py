@@ -21,12 +21,14 @@ def test_device_generator_matches_host(dtype):
     sdev = torch.from_numpy(scale).cuda()
     for tid, hd, use_scale, off in [(S.PREFIX_K, 128, True, dict(r0=0, b0=3, l0=1, p0=1000)),
                                     (S.VERIFY_V, 128, False, dict(r0=17, b0=0, l0=2, p0=0)),
-                                    (S.VERIFY_HIDDEN, 0, False, dict(r0=5, b0=1, l0=0, p0=3))]:
+                                    (S.VERIFY_HIDDEN, 0, False, dict(r0=5, b0=1, l0=0, p0=3)),
+                                    # a column block starting at KV head 6 (a KV-head shard)
+                                    (S.PREFIX_V, 128, True, dict(r0=0, b0=2, l0=2, p0=77, x0=768))]:
         t = torch.empty(int(np.prod(shape)), dtype=torch.bfloat16 if dtype == "bf16" else torch.float32,
                         device="cuda")
         S.device_fill_normal(t.data_ptr(), 9, tid, shape, head_dim=hd,
                              scale_ptr=sdev.data_ptr() if use_scale else None, scale_heads=8, dtype=dtype,
-                             stream=torch.cuda.current_stream().cuda_stream, **off)
+                             stream=torch.cuda.current_stream().cuda_stream, scale_layers=4, **off)
         torch.cuda.synchronize()
         host = S.fill_normal(9, tid, shape, head_dim=hd, scale=scale if use_scale else None, dtype=dtype,
                              **off).reshape(-1)

@@ -1,7 +1,8 @@
 """World-size-2 gloo run of the bench's multi-rank host logic on CPU.
 
-The path shards by sequence with no data-path collective: every rank owns a disjoint
-batch (weak scaling) and the only collective is the max over ranks of the timed region.
+The path shards with no data-path collective: every rank owns a disjoint batch (weak
+scaling) or a disjoint share of every sequence's KV heads (strong scaling); the only
+collective is the max over ranks of the timed region.
 """
 
 import os
@@ -29,9 +30,10 @@ def _worker(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     r, w, _ = bench.dist_env()
     off = bench.sequence_offset(r, 16)
+    heads = bench.kv_head_range(r, w, 8)
     t = bench.max_over_ranks(1.0 + r, w, torch.device("cpu"))
     bench.barrier(w)
-    q.put((r, off, t))
+    q.put((r, off, heads, t))
     dist.destroy_process_group()
 
 
@@ -46,8 +48,18 @@ def test_two_ranks_shard_and_max():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert [o for _, o, _ in res] == [0, 16]       # disjoint sequence ranges
-    assert all(t == 2.0 for _, _, t in res)         # every rank sees the slowest rank's time
+    assert [o for _, o, _, _ in res] == [0, 16]            # disjoint sequence ranges
+    assert [h for _, _, h, _ in res] == [(0, 4), (4, 8)]   # or disjoint KV-head ranges covering all
+    assert all(t == 2.0 for _, _, _, t in res)              # every rank sees the slowest rank's time
+
+
+def test_kv_head_ranges():
+    for world in (1, 2, 4, 8):
+        got = [bench.kv_head_range(r, world, 8) for r in range(world)]
+        assert got[0][0] == 0 and got[-1][1] == 8
+        assert all(a[1] == b[0] for a, b in zip(got, got[1:]))
+    with pytest.raises(ValueError):
+        bench.kv_head_range(0, 3, 8)
 
 
 def test_reference_arm_other_ranks_exit(monkeypatch):

@@ -1,5 +1,6 @@
 """Host-side checks of the seeded input generator (no method arithmetic involved)."""
 
+import pytest
 import numpy as np
 import torch
 
@@ -64,3 +65,15 @@ def test_token_ids_yield_the_drawn_accepts():
 def test_prefix_lengths_range():
     p = S.prefix_lengths(3, 1000, 98304, 131072)
     assert p.min() >= 98304 and p.max() <= 131072 and len(np.unique(p)) > 900
+
+
+def test_device_fill_refuses_scale_reads_past_the_array():
+    """The device generator's wrapper checks, before any launch, that the per-head scale
+    array covers every (layer, head) the block reads."""
+    import synth as S
+    with pytest.raises(ValueError):
+        S.device_fill_normal(1, 0, S.PREFIX_K, (1, 1, 2, 4, 256), l0=3, head_dim=128, scale_ptr=1, scale_heads=8,
+                             scale_layers=4)
+    with pytest.raises(ValueError):
+        S.device_fill_normal(1, 0, S.PREFIX_K, (1, 1, 1, 4, 256), x0=7 * 128, head_dim=128, scale_ptr=1,
+                             scale_heads=8, scale_layers=4)

@@ -1,0 +1,60 @@
+"""The boundary from C: a C11 program (not C++) includes include/longspark.h with every
+warning as an error, links liblongspark.so and calls the host-side queries, which need no
+GPU. Its answers must equal the Python binding's."""
+
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import fixed_cost_drafter_b200 as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+C_SRC = r"""
+#include <stdio.h>
+#include "longspark.h"
+
+int main(void) {
+  ls_config c = {0};
+  c.batch = 16; c.n_layers = 4; c.n_kv_heads = 8; c.n_q_heads = 32; c.head_dim = 128;
+  c.hidden = 4096; c.block = 16; c.window = 512; c.n_scales = 3;
+  c.scales[0] = 64; c.scales[1] = 512; c.scales[2] = 4096;
+  c.slots_per_scale = 32; c.dtype = LS_BF16; c.flags = 0;
+  ls_layout y;
+  const int st = ls_get_layout(&c, &y);
+  ls_config bad = c;
+  bad.window = 4;  /* < B + 1 */
+  ls_layout y2;
+  printf("%d %zu %zu %zu %zu %d %d %zu %d %s\n", st, ls_state_bytes(&c), y.total_bytes, y.off_kv,
+         y.off_prologue, y.kv_rows, ls_get_layout(&bad, &y2), ls_view_state_bytes(&c, LS_VIEW_WINDOW),
+         ls_get_layout(NULL, &y2), ls_status_string(LS_ERR_SHAPE));
+  return 0;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(tmp_path):
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    src = tmp_path / "abi.c"
+    src.write_text(C_SRC)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(F.library_path())
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    "-I", cuda_inc, str(src), "-o", str(exe), "-L", libdir, "-llongspark",
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    cfg = F.make_config(batch=16, n_layers=4, n_kv_heads=8, n_q_heads=32, head_dim=128, hidden=4096, block=16,
+                        window=512, scales=[64, 512, 4096], slots_per_scale=32, dtype=F.LS_BF16)
+    y = F.ls_get_layout(cfg)
+    assert int(out[0]) == F.LS_OK
+    assert int(out[1]) == int(out[2]) == F.ls_state_bytes(cfg) == y.total_bytes
+    assert int(out[3]) == y.off_kv and int(out[4]) == y.off_prologue and int(out[5]) == y.kv_rows
+    assert int(out[6]) == F.LS_ERR_SHAPE
+    assert int(out[7]) == F.ls_view_state_bytes(cfg, F.LS_VIEW_WINDOW)
+    assert int(out[8]) == F.LS_ERR_INVALID_ARG
+    assert " ".join(out[9:]) == F.ls_status_string(F.LS_ERR_SHAPE)

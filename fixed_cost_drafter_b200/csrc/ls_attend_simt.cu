@@ -137,11 +137,10 @@ static cudaError_t launch_simt_t(const Dev& p, int lb, int lcount, const void* q
   const int M = (p.Hq / p.Hkv) * p.B;
   const size_t smem = size_t(M * D + 32 * (D + 1) + 32 * D) * sizeof(float);
   auto kern = attend_simt_kernel<T, DV>;
-  static size_t configured = 0;  // opt-in shared memory set once per size (not per launch)
-  if (smem > configured) {
+  // per launch: the opt-in belongs to the current device's copy of the kernel
+  if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    configured = smem;
   }
   const dim3 grid(p.Hkv, lcount, p.b);
   kern<<<grid, kSimtWarps * 32, smem, stream>>>(p, lb, lcount, static_cast<const T*>(q),

@@ -209,3 +209,30 @@ def test_prologue_split_tiles_selection_exact():
     bkv, _ = _run_prologue(run, wl, w_kv, w_q, x)
     assert np.array_equal(_bits(bkv), run.read_state()["boundary"][:, :, :2 * H * D])
     assert run.error() == (F.LS_OK, 0)
+
+
+def test_prologue_batch_past_one_activation_tile():
+    """Batch 300: both problems run two activation tiles (the second ragged: 44 rows, the
+    rest of its box zero-filled), and the 88 boundary tiles left after whole waves (all of
+    the ragged tile) are split with 256-row partial sums. Every boundary key/value and the
+    queries of sequences on both sides of the tile edge against the oracle."""
+    wl = _wl(batch=300, n_layers=8, n_kv_heads=8, n_q_heads=32, hidden=512, prefix=(300, 300))
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    dev = run.dev
+    L, H, Hq, D, hid, B = wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.hidden, wl.block
+    w_kv = _gen((L, 2 * H * D, hid), 31, dev, hid ** -0.5)
+    w_q = _gen((L, Hq * D, hid), 32, dev, hid ** -0.5)
+    x = _gen((wl.batch, L, B, hid), 33, dev, 1.0)
+    bkv, q = _run_prologue(run, wl, w_kv, w_q, x)
+    h = O.to_f64(run.read_state()["boundary"], "bf16")
+    BKV, Q = _f64(bkv), _f64(q)
+    for l in range(L):
+        Wkv = _f64(w_kv[l])
+        _check(BKV[:, l], h[:, l] @ Wkv.T, _bound_terms(Wkv, h[:, l], hid))
+    seqs = [0, 15, 16, 255, 256, 299]
+    for l in (0, L - 1):
+        Wq = _f64(w_q[l])
+        Xs = _f64(x[seqs, l]).reshape(-1, hid)
+        _check(Q[seqs, l].reshape(-1, Hq * D), Xs @ Wq.T, _bound_terms(Wq, Xs, hid))
+    assert run.error() == (F.LS_OK, 0)

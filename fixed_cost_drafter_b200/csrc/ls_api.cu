@@ -469,7 +469,18 @@ int ls_get_error(const ls_state* st, int32_t* h_code) {
 
 int ls_clear_error(ls_state* st, cudaStream_t stream) {
   if (!st) return LS_ERR_INVALID_ARG;
-  return cuda_status(cudaMemsetAsync(st->dev.err, 0, sizeof(int32_t), stream));
+  // the error word, and the arrival counts a call that gave up part-way may have left
+  // (they are zero between completed calls): the commit's, the sampler's, the projections'
+  const ls::Layout& y = st->lay;
+  const ls_config& c = st->cfg;
+  char* base = static_cast<char*>(st->arena);
+  if (cudaMemsetAsync(base + y.error, 0, 16, stream) != cudaSuccess) return LS_ERR_CUDA;
+  if (cudaMemsetAsync(base + y.sync, 0, size_t(c.batch) * c.n_layers * 4, stream) != cudaSuccess) return LS_ERR_CUDA;
+  if (cudaMemsetAsync(base + y.sample, 0, size_t(c.batch) * 4, stream) != cudaSuccess) return LS_ERR_CUDA;
+  if (y.total > y.prologue &&
+      cudaMemsetAsync(st->dev.pro_count, 0, size_t(ls::kProMaxGrid) * 4, stream) != cudaSuccess)
+    return LS_ERR_CUDA;
+  return LS_OK;
 }
 
 int ls_check_wait_timeout(ls_state* st, uint32_t polls, cudaStream_t stream) {

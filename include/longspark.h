@@ -397,7 +397,10 @@ LS_API int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStre
 LS_API int ls_get_error(const ls_state* st, int32_t* h_code);
 
 /* Clears the device error word (enqueued on `stream`). The word is sticky otherwise: a
- * bit once set stays until this call or a fresh ls_init_state.                        */
+ * bit once set stays until this call or a fresh ls_init_state. Also zeroes the arrival
+ * counts that a call which gave up part-way (LS_DEVERR_WAIT_TIMEOUT) may have left in the
+ * arena (commit, ls_accept_sampled, ls_draft_prologue), so that later calls count right;
+ * the views themselves are whatever that call left (restore a checkpoint if needed).    */
 LS_API int ls_clear_error(ls_state* st, cudaStream_t stream);
 
 /* Check of the device-side failure detection: one kernel polls an mbarrier that nothing

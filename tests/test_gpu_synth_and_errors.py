@@ -92,3 +92,44 @@ def test_bounded_wait_gives_up_and_the_context_stays_usable():
     assert run.error() == (F.LS_OK, 0)
     with pytest.raises(F.LsError):
         F.ls_check_wait_timeout(run.state, 0, run.stream)
+
+
+def test_clear_error_resets_left_over_arrival_counts():
+    """Arrival counts a call that gave up part-way could leave (planted here by hand in the
+    arena) are zeroed by ls_clear_error: rounds and the projections then give exactly what
+    a clean state gives."""
+    wl = WL.Workload("clear", 43, 3, 2, 2, 8, 128, 512, 16, 128, (32, 64, 256), 4, "bf16", (300, 900), 4, None,
+                     1000, head_scale=True)
+    clean, dirty = WL.DeviceRun(wl), WL.DeviceRun(wl)
+    for run in (clean, dirty):
+        run.prefill()
+    y = dirty.layout
+    b, L = wl.batch, wl.n_layers
+    dirty.arena[y.off_sync:y.off_sync + b * L * 4] = 1                      # commit arrivals
+    dirty.arena[y.off_sample:y.off_sample + b * 4] = 2                      # sampler arrivals
+    cnt = y.off_prologue + 320 * 128 * 16 * 4                               # after the partial-sum slots
+    dirty.arena[cnt:cnt + 160 * 4] = 3                                      # projections' tile arrivals
+    F.ls_clear_error(dirty.state, dirty.stream)
+    inp = clean.make_round_inputs()
+    outs = [clean.new_out(), dirty.new_out()]
+    for r in range(wl.rounds):
+        for run, out in zip((clean, dirty), outs):
+            run.round(inp, r, out)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1]) and torch.equal(clean.accept_len, dirty.accept_len)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    w_kv = (torch.randn((L, 2 * 2 * 128, 512), device="cuda", generator=g) * 0.05).to(torch.bfloat16)
+    w_q = (torch.randn((L, 8 * 128, 512), device="cuda", generator=g) * 0.05).to(torch.bfloat16)
+    x = torch.randn((b, L, 16, 512), device="cuda", generator=g).to(torch.bfloat16)
+    res = []
+    for run in (clean, dirty):
+        bkv = torch.empty((b, L, 512), dtype=torch.bfloat16, device="cuda")
+        q = torch.empty((b, L, 16, 1024), dtype=torch.bfloat16, device="cuda")
+        F.ls_draft_prologue(run.state, w_kv, w_q, x, bkv, q, run.stream)
+        res.append((bkv, q))
+    torch.cuda.synchronize()
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    sc, sd = clean.read_state(), dirty.read_state()
+    for k in sc:
+        assert np.array_equal(sc[k], sd[k]), k
+    assert clean.error() == (F.LS_OK, 0) and dirty.error() == (F.LS_OK, 0)

@@ -99,6 +99,75 @@ __device__ inline void issue_prefix_rows(const Dev&, const PrefillArgs& a, const
 }
 
 // Paged: one copy per run of rows inside a page (per row when the slots are not packed).
+// The runs (their page lookups included) are planned before the producer waits for a free
+// stage, so the lookups' latency overlaps that wait instead of delaying the refill.
+struct PrefixPlan {
+  static constexpr int kMaxRuns = 2;  // a stage of G rows spans at most 2 pages when page_size >= G
+  const char* src[2][kMaxRuns];
+  int r0[2][kMaxRuns], n[2][kMaxRuns], nrun[2];
+  bool ok;  // false: the stage needs more runs, issue_prefix_rows plans it after the wait
+};
+
+__device__ inline int page_offset(int64_t pos, int ps) {
+  if ((ps & (ps - 1)) == 0) return int(pos & (ps - 1));
+  if (pos < (int64_t(1) << 32)) return int(uint32_t(pos) % uint32_t(ps));
+  return int(pos % ps);
+}
+
+template <typename T>
+__device__ inline void plan_prefix_rows(const Dev&, const DensePrefix&, int, int64_t, int, PrefixPlan& pl) {
+  pl.ok = false;  // dense: addresses are plain arithmetic, nothing to plan
+}
+
+template <typename T>
+__device__ inline void plan_prefix_rows(const Dev& p, const ls_paged_kv& kv, int bl, int64_t g0, int nrows,
+                                        PrefixPlan& pl) {
+  const int b = bl / p.L, l = bl - b * p.L;
+  pl.ok = true;
+  // (fixed trip counts: the plan stays in registers)
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const char* base = static_cast<const char*>(t == 0 ? kv.k_layers[l] : kv.v_layers[l]);
+    int r = 0;
+    pl.nrun[t] = 0;
+#pragma unroll
+    for (int k = 0; k < PrefixPlan::kMaxRuns; ++k) {
+      pl.src[t][k] = nullptr;
+      pl.r0[t][k] = r;
+      pl.n[t][k] = 0;
+      if (r < nrows) {
+        const int64_t pos = g0 + r;
+        const int run = min(nrows - r, kv.page_size - page_offset(pos, kv.page_size));
+        pl.src[t][k] = paged_row(kv, base, b, pos, int(sizeof(T)), p.err);
+        pl.n[t][k] = run;
+        pl.nrun[t] = k + 1;
+        r += run;
+      }
+    }
+    if (r < nrows) pl.ok = false;
+  }
+}
+
+template <typename T>
+__device__ inline void issue_plan(const ls_paged_kv& kv, const PrefixPlan& pl, int t, char* dst, int rowBytes,
+                                  uint64_t* bar) {
+  const bool packed = kv.slot_stride * int64_t(sizeof(T)) == rowBytes;
+#pragma unroll
+  for (int k = 0; k < PrefixPlan::kMaxRuns; ++k) {
+    if (k >= pl.nrun[t]) break;
+    if (packed) {
+      bulk_g2s(dst + pl.r0[t][k] * rowBytes, pl.src[t][k], uint32_t(pl.n[t][k] * rowBytes), bar);
+    } else {
+      for (int i = 0; i < pl.n[t][k]; ++i)
+        bulk_g2s(dst + (pl.r0[t][k] + i) * rowBytes, pl.src[t][k] + int64_t(i) * kv.slot_stride * int64_t(sizeof(T)),
+                 uint32_t(rowBytes), bar);
+    }
+  }
+}
+template <typename T>
+__device__ inline void issue_plan(const DensePrefix&, const PrefixPlan&, int, char*, int, uint64_t*) {}
+
+// Paged, unplanned (a stage spanning more than 2 pages): lookups after the wait.
 template <typename T>
 __device__ inline void issue_prefix_rows(const Dev& p, const PrefillArgs&, const ls_paged_kv& kv, int t, int bl,
                                          int64_t g0, int nrows, char* dst, int rowBytes, uint64_t* bar) {
@@ -108,8 +177,7 @@ __device__ inline void issue_prefix_rows(const Dev& p, const PrefillArgs&, const
   int r = 0;
   while (r < nrows) {
     const int64_t pos = g0 + r;
-    const int off = int(pos % kv.page_size);
-    const int run = min(nrows - r, kv.page_size - off);
+    const int run = min(nrows - r, kv.page_size - page_offset(pos, kv.page_size));
     const char* src = paged_row(kv, base, b, pos, int(sizeof(T)), p.err);
     if (packed) {
       bulk_g2s(dst + r * rowBytes, src, uint32_t(run * rowBytes), bar);
@@ -167,17 +235,25 @@ prefill_units_kernel(Dev p, PrefillArgs a, const Src src) {
       for (int s = 0; s < kPrefillStages; ++s) last_issue[s] = -1;
       for (; prod.valid; ++n) {
         const int buf = n % kPrefillStages;
-        if (!wait(&empty[buf], ((n / kPrefillStages) & 1) ^ 1)) break;
-        fence_proxy_async_smem();  // the consumers' reads of the buffer come before its refill
+        // the stage's rows (and, paged, their page lookups) before waiting for the buffer
         const int it = blockIdx.x + prod.j * gridDim.x;
         int bl, u; int64_t r0, r1;
         item_rows(a, p, it, bl, u, r0, r1);
         const int64_t g0 = r0 + int64_t(prod.grp) * a.G;
         const int nrows = int(min(int64_t(a.G), r1 - g0));
+        PrefixPlan plan;
+        plan_prefix_rows<T>(p, src, bl, g0, nrows, plan);
+        if (!wait(&empty[buf], ((n / kPrefillStages) & 1) ^ 1)) break;
+        fence_proxy_async_smem();  // the consumers' reads of the buffer come before its refill
         char* dst = smem + buf * stageBytes;
         mbar_arrive_expect_tx(&full[buf], uint32_t(2 * nrows * rowBytes));
-        for (int t = 0; t < 2; ++t)
-          issue_prefix_rows<T>(p, a, src, t, bl, g0, nrows, dst + t * a.G * rowBytes, rowBytes, &full[buf]);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (plan.ok)
+            issue_plan<T>(src, plan, t, dst + t * a.G * rowBytes, rowBytes, &full[buf]);
+          else
+            issue_prefix_rows<T>(p, a, src, t, bl, g0, nrows, dst + t * a.G * rowBytes, rowBytes, &full[buf]);
+        }
         last_issue[buf] = n;
         cursor_next(a, p, prod);
       }

@@ -376,7 +376,9 @@ def run_gpu(args):
     full_wl, wl = wl, run.wl
     strong = args.shard == "kv-heads"
 
-    # prefill (timed separately)
+    # prefill (timed separately, after one untimed prefill into a state then reset)
+    run.prefill()
+    run.reset_state()
     pre = []
     run.prefill(timer=lambda e0, e1, nbytes: pre.append((e0, e1, nbytes)))
     torch.cuda.synchronize()
@@ -615,6 +617,8 @@ def paged_measure(WLM, wl, dev, flush, evs, n, rank):
         run = WLM.DeviceRun(wl, device=dev, rounds=n, seq_offset=sequence_offset(rank, wl.batch))
         cache = WLM.PagedCache(run, ps, run.prefix_len + (n + 1) * (wl.block + 1), seed=1)
         run.fill_pages(cache)
+        run.prefill_paged(cache)  # untimed, then a fresh state
+        run.reset_state()
         torch.cuda.synchronize()
         pre = []
         run.prefill_paged(cache, timer=lambda e0, e1, nbytes: pre.append((e0, e1, nbytes)))

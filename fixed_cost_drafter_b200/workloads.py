@@ -375,6 +375,11 @@ class DeviceRun:
             boundary=view(y.off_boundary, ed, (b, L, wl.hidden)).copy(),
         )
 
+    def reset_state(self):
+        """A fresh state in the same arena (ls_init_state zeroes it): nothing retained."""
+        F.ls_destroy_state(self.state)
+        self.state = F.ls_init_state(self.cfg, self.arena, self.nbytes, self.stream)
+
     def error(self):
         return F.ls_get_error(self.state)
 

@@ -481,7 +481,8 @@ def run_gpu(args):
     # prefill and rounds reading the target's paged KV cache in place (page size 16)
     paged = None
     if not args.no_paged:
-        paged = paged_measure(WLM, wl, dev, flush, evs, min(K, 200), rank)
+        # its own round count (two halves of 3 warm-up rounds and at least 5 timed ones)
+        paged = paged_measure(WLM, wl, dev, flush, max(16, min(K, 200)), rank)
 
     # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
     # the attention as a drafter calls it layer by layer (one launch per tapped layer)
@@ -602,7 +603,7 @@ PAGE_SIZE = 16
 LARGE_PAGE_SIZE = 256
 
 
-def paged_measure(WLM, wl, dev, flush, evs, n, rank):
+def paged_measure(WLM, wl, dev, flush, n, rank):
     """ls_prefill_paged and ls_round_paged on the workload with its prefix and verify rows in
     a paged cache (page size 16, each sequence's pages scattered over the pool; the prefill
     also with 256-row pages). The
@@ -639,6 +640,7 @@ def paged_measure(WLM, wl, dev, flush, evs, n, rank):
     stream = run.stream
     kv = cache.descriptor()
     span = wl.n_kv_heads * wl.head_dim
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
     warm = 3  # the first rounds load the kernels; rounds run in order (the pages hold them)
     half = n // 2  # rounds [0, half): block-table lookups; [half, n): the engine's slot mapping
     for i in range(n):

@@ -246,3 +246,33 @@ def test_paged_host_checks():
             F.ls_commit_round_paged(run.state, run.draft[0], run.target[0], kv, vh, run.accept_len, run.next_token,
                                     run.stream)
     assert run.error() == (F.LS_OK, 0)
+
+
+def test_paged_fp32_tiny_round_matches_dense():
+    """The fp32 instantiations (4-byte rows) and ls_round_paged on the CUDA-core attention:
+    the tiny fp32 config with a page size of 5 (not a power of two) and keys and values
+    interleaved per page, against ls_round on the dense rows, bit for bit."""
+    wl = WL.CONFIGS["tiny"]
+    dense = WL.DeviceRun(wl)
+    paged = WL.DeviceRun(wl)
+    cache = WL.PagedCache(paged, 5, _capacity(paged), layout="interleaved", seed=13)
+    paged.fill_pages(cache)
+    dense.prefill()
+    paged.prefill_paged(cache)
+    torch.cuda.synchronize()
+    _same_state(dense, paged)
+    inp = dense.make_round_inputs()
+    out_d, out_p = dense.new_out(), paged.new_out()
+    for r in range(dense.rounds):
+        paged.write_verify_pages(cache, inp, r)
+        dense.round(inp, r, out_d)
+        F.ls_round_paged(paged.state, paged.draft[r], paged.target[r],
+                         paged.paged_descriptor(cache, r, with_slots=bool(r & 1)), inp["vh"][r],
+                         paged.accept_len, paged.next_token, inp["q"][r], paged.bk_off, paged.bv_off,
+                         paged.softmax_scale, out_p, paged.stream)
+        torch.cuda.synchronize()
+        assert torch.equal(out_d, out_p), r
+        assert torch.equal(dense.accept_len, paged.accept_len) and torch.equal(dense.next_token, paged.next_token)
+    _same_state(dense, paged)
+    assert not F.ls_attend_uses_tensor_cores(paged.state)
+    assert paged.error() == (F.LS_OK, 0) and dense.error() == (F.LS_OK, 0)

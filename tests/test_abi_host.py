@@ -125,3 +125,19 @@ def test_prefill_workspace_bytes():
 def test_status_strings():
     for s in (0, -1, -2, -3, -4, -5, -6):
         assert F.ls_status_string(s) != "unknown status"
+
+
+def test_make_paged_kv_descriptor():
+    """The binding's paged-cache descriptor: per-layer bases in order, the rest of the
+    fields as given; more layers than LS_MAX_PAGED_LAYERS, or unequal key/value lists, are
+    refused before any call."""
+    kv = F.make_paged_kv([0x1000, 0x2000], [0x3000, 0x4000], 4096, 256, 0x5000, 7, 16, 99, verify_slots=0x6000)
+    assert list(kv.k_layers[:2]) == [0x1000, 0x2000] and list(kv.v_layers[:2]) == [0x3000, 0x4000]
+    assert kv.k_layers[2] is None and kv.v_layers[2] is None
+    assert (kv.page_stride, kv.slot_stride, kv.block_table) == (4096, 256, 0x5000)
+    assert (kv.max_blocks, kv.page_size, kv.num_pages, kv.verify_slots) == (7, 16, 99, 0x6000)
+    assert F.make_paged_kv([0x1000], [0x2000], 256, 256, 0x5000, 1, 1, 1).verify_slots is None
+    with pytest.raises(ValueError):
+        F.make_paged_kv([0x10] * (F.LS_MAX_PAGED_LAYERS + 1), [0x10] * (F.LS_MAX_PAGED_LAYERS + 1), 0, 256, 1, 1, 1, 1)
+    with pytest.raises(ValueError):
+        F.make_paged_kv([0x10, 0x20], [0x10], 0, 256, 1, 1, 1, 1)

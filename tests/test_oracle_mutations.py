@@ -135,6 +135,26 @@ def _paged_commit_from_position_zero(sh, v, draft_ids, target_ids, k_pages, v_pa
                           M.paged_rows(v_pages, block_table, page_size, b, pos), verify_hidden)
 
 
+def _inverse_cdf_side_left(w, v):
+    # the first token whose running sum reaches (instead of passes) the threshold
+    c = np.cumsum(w)
+    t = int(np.searchsorted(c, v * c[-1], side="left"))
+    return min(t, len(w) - 1)
+
+
+def _paged_rows_first_sequence(pages, block_table, page_size, b, positions):
+    # every sequence read through sequence 0's row of the block table
+    return ORIG["paged_rows"](pages, block_table, page_size, 0, positions)
+
+
+def _residual_from_next_position(q_rows, p_rows, a):
+    # the residual built from the target's row after the rejected position
+    B = q_rows.shape[0]
+    if a < B:
+        return np.maximum(0.0, p_rows[a + 1].astype(np.float64) - q_rows[a].astype(np.float64))
+    return p_rows[B].astype(np.float64)
+
+
 def _prologue_layer0_weights(w_kv, w_q, boundary, x):
     # every layer projected with layer 0's weights
     w_kv, w_q = np.asarray(w_kv), np.asarray(w_q)
@@ -144,7 +164,8 @@ def _prologue_layer0_weights(w_kv, w_q, boundary, x):
 
 ORIG = {n: getattr(M, n) for n in ("accept_scan", "retain_row", "views_from_scratch",
                                    "attention_slots", "draft_attend", "view_of_slots",
-                                   "accept_decisions", "sampling_weights", "draft_prologue", "paged_rows")}
+                                   "accept_decisions", "sampling_weights", "draft_prologue", "paged_rows",
+                                   "inverse_cdf")}
 
 CASES = [
     ("accept_scan", _scan_off_by_one, [P.test_scan_golden_examples]),
@@ -160,6 +181,9 @@ CASES = [
     ("accept_decisions", _accept_ratio_inverted, [P.test_sampled_emits_target_distribution]),
     ("draft_prologue", _prologue_layer0_weights, [P.test_prologue_orientation_and_layers]),
     ("paged_rows", _paged_offset_from_page_end, [P.test_paged_rows_hand_worked]),
+    ("paged_rows", _paged_rows_first_sequence, [P.test_paged_rows_hand_worked]),
+    ("inverse_cdf", _inverse_cdf_side_left, [P.test_inverse_cdf_boundaries]),
+    ("sampling_weights", _residual_from_next_position, [P.test_sampled_emits_target_distribution]),
     ("commit_round_paged", _paged_commit_from_position_zero, [lambda: P.test_paged_commit_equals_dense(3)]),
 ]
 

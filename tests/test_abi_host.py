@@ -93,6 +93,10 @@ def test_view_state_bytes():
     (dict(head_dim=96), F.LS_ERR_UNSUPPORTED),
     (dict(dtype=7), F.LS_ERR_INVALID_ARG),
     (dict(n_kv_heads=16, n_q_heads=64), F.LS_ERR_UNSUPPORTED),
+    (dict(block=33, window=64), F.LS_ERR_UNSUPPORTED),        # more drafts than two ballots
+    (dict(hidden=4100), F.LS_ERR_UNSUPPORTED),                # hidden not whole 16-byte pieces
+    (dict(slots_per_scale=0), F.LS_ERR_INVALID_ARG),
+    (dict(flags=0x100), F.LS_ERR_INVALID_ARG),                # unknown flag bit
 ])
 def test_config_validation(kw, status):
     c = _cfg(**kw)

@@ -165,7 +165,10 @@ typedef struct ls_state ls_state; /* opaque host handle */
  *               verify pass wrote verify row i of sequence b (an engine's slot mapping).
  *               The commit then reads the rows there instead of looking position len + i
  *               up in the block table, so its row loads no longer wait for that lookup.
- *               Prefill ignores it.                                                    */
+ *               8-byte aligned; a slot outside the pool sets LS_DEVERR_PAGE. Prefill
+ *               ignores it.
+ * Each slot holds one row of all KV heads (a head-major page, [Hkv][page_size][D],
+ * is not read).                                                                        */
 #define LS_MAX_PAGED_LAYERS 64
 typedef struct {
   const void* k_layers[LS_MAX_PAGED_LAYERS];

@@ -195,7 +195,7 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 __device__ inline void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ inline void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Bulk asynchronous global->shared copy on the TMA engine (no tensor map, no multicast).
+// Bulk asynchronous global->shared copy on the TMA engine (no tensor map, into this CTA only).
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ inline void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

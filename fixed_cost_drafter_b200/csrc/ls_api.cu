@@ -32,7 +32,7 @@ cudaError_t launch_prefill_paged(const Dev& p, const ls_config& c, const ls_page
                                  int64_t row_begin, int64_t row_end, const void* last_hidden, void* ws, int sms,
                                  cudaStream_t stream);
 size_t noalloc_scratch_bytes();
-cudaError_t noalloc_scratch(void** out);
+cudaError_t noalloc_scratch(int device, void** out);
 cudaError_t launch_wait_timeout(const Dev& p, uint32_t polls, cudaStream_t stream);
 }  // namespace ls
 
@@ -50,6 +50,14 @@ struct ls_state {
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// A state belongs to the device that was current at ls_init_state: its arena, tensor maps
+// and the library's fixed scratch are that device's. Calls made while another device is
+// current are refused.
+bool on_state_device(const ls_state* st) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == st->device;
+}
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 int validate(const ls_config* c) {
@@ -239,6 +247,7 @@ int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t p
                        int64_t row_end, const void* d_last_hidden, void* d_workspace,
                        size_t workspace_bytes, cudaStream_t stream) {
   if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   const ls_config& c = st->cfg;
   if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
   if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
@@ -261,6 +270,7 @@ int ls_prefill_summary_noalloc(ls_state* st, const void* d_k, const void* d_v, i
                                int64_t row_stride, const int64_t* d_prefix_len, int64_t row_begin,
                                int64_t row_end, const void* d_last_hidden, cudaStream_t stream) {
   if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   const ls_config& c = st->cfg;
   if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
   if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
@@ -276,7 +286,7 @@ int ls_prefill_summary_noalloc(ls_state* st, const void* d_k, const void* d_v, i
   if (ls::prefill_workspace_bytes(c, row_begin, row_end) > ls::noalloc_scratch_bytes())
     return LS_ERR_SCRATCH_LIMIT;
   void* ws = nullptr;
-  if (ls::noalloc_scratch(&ws) != cudaSuccess) return LS_ERR_CUDA;
+  if (ls::noalloc_scratch(st->device, &ws) != cudaSuccess) return LS_ERR_CUDA;
   return cuda_status(ls::launch_prefill(st->dev, c, d_k, d_v, plane_stride, row_stride, d_prefix_len,
                                         row_begin, row_end, d_last_hidden, ws, st->sms, stream));
 }
@@ -285,6 +295,7 @@ int ls_prefill_paged(ls_state* st, const ls_paged_kv* h_kv, const int64_t* d_pre
                      int64_t row_end, const void* d_last_hidden, void* d_workspace, size_t workspace_bytes,
                      cudaStream_t stream) {
   if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   const ls_config& c = st->cfg;
   if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
   if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
@@ -300,7 +311,7 @@ int ls_prefill_paged(ls_state* st, const ls_paged_kv* h_kv, const int64_t* d_pre
     if (workspace_bytes < need) return LS_ERR_SHAPE;
   } else {  // the library's fixed scratch
     if (need > ls::noalloc_scratch_bytes()) return LS_ERR_SCRATCH_LIMIT;
-    if (ls::noalloc_scratch(&ws) != cudaSuccess) return LS_ERR_CUDA;
+    if (ls::noalloc_scratch(st->device, &ws) != cudaSuccess) return LS_ERR_CUDA;
   }
   static const ls_paged_kv kNone{};
   return cuda_status(ls::launch_prefill_paged(st->dev, c, row_end > row_begin ? *h_kv : kNone, d_prefix_len,
@@ -312,6 +323,7 @@ int ls_commit_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_
                           int32_t* d_next_token, cudaStream_t stream) {
   if (!st || !d_draft_ids || !d_target_ids || !d_verify_hidden || !d_accept_len || !d_next_token)
     return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   const int v = validate_paged(st->cfg, h_kv);
   if (v != LS_OK) return v;
   if (!aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
@@ -322,6 +334,7 @@ int ls_commit_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_
 int ls_commit_accepted_paged(ls_state* st, const int32_t* d_accept_len, const ls_paged_kv* h_kv,
                              const void* d_verify_hidden, cudaStream_t stream) {
   if (!st || !d_accept_len || !d_verify_hidden) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   const int v = validate_paged(st->cfg, h_kv);
   if (v != LS_OK) return v;
   if (!aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
@@ -335,6 +348,7 @@ int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_t
   if (!st || !d_draft_ids || !d_target_ids || !d_verify_k || !d_verify_v || !d_verify_hidden ||
       !d_accept_len || !d_next_token)
     return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden))
     return LS_ERR_INVALID_ARG;
   return cuda_status(ls::launch_commit(st->dev, d_draft_ids, d_target_ids, d_verify_k, d_verify_v,
@@ -346,6 +360,7 @@ int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const float* d_d
                       int32_t* d_next_token, cudaStream_t stream) {
   if (!st || !d_draft_ids || !d_draft_probs || !d_target_probs || !d_uniforms || !d_accept_len || !d_next_token)
     return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   if (vocab < 4 || vocab % 4 != 0) return LS_ERR_SHAPE;
   if (vocab > ls::kSampleChunk * ls::kSampleMaxChunks) return LS_ERR_UNSUPPORTED;
   if (!aligned16(d_draft_probs) || !aligned16(d_target_probs)) return LS_ERR_INVALID_ARG;
@@ -356,6 +371,7 @@ int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const float* d_d
 int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q, const void* d_x, void* d_bkv,
                       void* d_q, cudaStream_t stream) {
   if (!st || !d_w_kv || !d_w_q || !d_x || !d_bkv || !d_q) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   if (!ls::prologue_supported(st->dev)) return LS_ERR_UNSUPPORTED;
   if (!aligned16(d_w_kv) || !aligned16(d_w_q) || !aligned16(d_x) || !aligned16(d_bkv) || !aligned16(d_q))
     return LS_ERR_INVALID_ARG;
@@ -366,6 +382,7 @@ int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q,
 int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const void* d_verify_k, const void* d_verify_v,
                        const void* d_verify_hidden, cudaStream_t stream) {
   if (!st || !d_accept_len || !d_verify_k || !d_verify_v || !d_verify_hidden) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
   return cuda_status(ls::launch_commit(st->dev, nullptr, nullptr, d_verify_k, d_verify_v, d_verify_hidden, nullptr,
                                        nullptr, d_accept_len, stream));
@@ -382,6 +399,7 @@ int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer
                           const void* d_boundary_k, const void* d_boundary_v, int64_t boundary_stride,
                           float softmax_scale, int32_t views, void* d_out, cudaStream_t stream) {
   if (!st || !d_q || !d_boundary_k || !d_boundary_v || !d_out) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   if (views == 0 || (views & ~LS_VIEW_ALL)) return LS_ERR_INVALID_ARG;
   const ls_config& c = st->cfg;
   if (layer_begin < 0 || layer_count < 1 || layer_begin + layer_count > c.n_layers)
@@ -407,6 +425,7 @@ int ls_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_target_i
   if (!st || !d_draft_ids || !d_target_ids || !d_verify_k || !d_verify_v || !d_verify_hidden || !d_accept_len ||
       !d_next_token || !d_q || !d_out)
     return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   const int rc = round_checks(st, boundary_k_offset, boundary_v_offset, softmax_scale, d_q, d_out);
   if (rc != LS_OK) return rc;
   int r = ls_commit_round(st, d_draft_ids, d_target_ids, d_verify_k, d_verify_v, d_verify_hidden, d_accept_len,
@@ -420,6 +439,7 @@ int ls_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_ta
                    int64_t boundary_k_offset, int64_t boundary_v_offset, float softmax_scale, void* d_out,
                    cudaStream_t stream) {
   if (!st || !d_q || !d_out) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   int r = round_checks(st, boundary_k_offset, boundary_v_offset, softmax_scale, d_q, d_out);
   if (r != LS_OK) return r;
   r = ls_commit_round_paged(st, d_draft_ids, d_target_ids, h_kv, d_verify_hidden, d_accept_len, d_next_token, stream);
@@ -452,6 +472,7 @@ int ls_attend_uses_tensor_cores(const ls_state* st) { return st && st->use_tc ? 
 
 int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStream_t stream) {
   if (!st || !h_dst) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   if (bytes > size_t(st->lay.total)) return LS_ERR_SHAPE;
   if (cudaMemcpyAsync(h_dst, st->arena, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return LS_ERR_CUDA;
@@ -460,6 +481,7 @@ int ls_read_state(const ls_state* st, void* h_dst, size_t bytes, cudaStream_t st
 
 int ls_get_error(const ls_state* st, int32_t* h_code) {
   if (!st || !h_code) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return LS_ERR_CUDA;
   if (cudaMemcpy(h_code, st->dev.err, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
     return LS_ERR_CUDA;
@@ -469,6 +491,7 @@ int ls_get_error(const ls_state* st, int32_t* h_code) {
 
 int ls_clear_error(ls_state* st, cudaStream_t stream) {
   if (!st) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   // the error word, and the arrival counts a call that gave up part-way may have left
   // (they are zero between completed calls): the commit's, the sampler's, the projections'
   const ls::Layout& y = st->lay;
@@ -485,6 +508,7 @@ int ls_clear_error(ls_state* st, cudaStream_t stream) {
 
 int ls_check_wait_timeout(ls_state* st, uint32_t polls, cudaStream_t stream) {
   if (!st || polls == 0 || polls > ls::kWaitLimit) return LS_ERR_INVALID_ARG;
+  if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
   return cuda_status(ls::launch_wait_timeout(st->dev, polls, stream));
 }
 

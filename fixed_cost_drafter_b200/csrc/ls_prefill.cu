@@ -682,24 +682,25 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
-// Device address of the array on the current device, looked up once per device (the
-// host-side name of the array is not a device address).
-cudaError_t noalloc_scratch(void** out) {
+// Device address of the array on `device`, which must be the current device (the entry
+// points check that the state's device is current), looked up once per device: the
+// host-side name of the array is not a device address.
+cudaError_t noalloc_scratch(int device, void** out) {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (device != cur || device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[device]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    addr[dev] = p;
+    addr[device] = p;
   }
-  *out = addr[dev];
+  *out = addr[device];
   return cudaSuccess;
 }
 

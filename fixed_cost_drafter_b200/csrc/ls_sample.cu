@@ -2,8 +2,10 @@
 // (Table 3, T = 0) with sampled decoding (Table 1) but print no acceptance rule, so this
 // is standard speculative sampling (Leviathan, Kalman and Matias 2023; Chen et al. 2023):
 // draft i of a block is kept while u_i * q_i(d_i) < p_i(d_i) (fp32 product and compare),
-// and the next token is drawn from max(0, p_a - q_a) after a rejection at position a, or
-// from p_B after B acceptances, by inverse CDF in vocabulary order with the draw u_B.
+// and the next token is drawn from max(0, p_a - q_a) after a rejection at position a (from
+// p_a itself when that residual has no mass: speculative sampling emits samples of the
+// target's distribution), or from p_B after B acceptances, by inverse CDF in vocabulary
+// order with the draw u_B. A row drawn from that has no mass sets LS_DEVERR_SAMPLE.
 //
 // Grid (vocabulary chunks of 8192, sequences), 256 threads. Every CTA of a sequence makes
 // the B acceptance tests itself (2 B gathers) and sums the draw's weights over its chunk
@@ -84,12 +86,58 @@ __device__ inline float block_exclusive(float x, float* sh, float* total) {
   return before + inc - x;
 }
 
+// The chunk holding the draw: the first chunk whose running sum (chunks in order) passes
+// t = u * total, or the last chunk with mass when rounding leaves none. The first two warps
+// scan the nchunks <= 64 sums in csum; *cstar gets the chunk (-1: no mass at all) and *rem
+// the part of t left inside it (infinity in the rounding case). Every thread calls it.
+__device__ inline void find_chunk(const float* csum, int nchunks, float u, float* sh, float* scratch, int* cstar_out,
+                                  float* rem_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < 2) {
+    const int k = threadIdx.x;
+    const float v = k < nchunks ? csum[k] : 0.f;
+    float inc = v;  // inclusive prefix within the warp, in chunk order
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) sh[warp] = inc;
+    asm volatile("bar.sync 1, 64;" ::: "memory");  // the two warps' totals
+    if (warp == 1) inc += sh[0];
+    const float z = sh[0] + sh[1];
+    const float t = u * z;
+    const unsigned hit = __ballot_sync(0xffffffffu, z > 0.f && k < nchunks && inc > t);
+    const unsigned mass = __ballot_sync(0xffffffffu, k < nchunks && v > 0.f);
+    if (lane == 0) {
+      scratch[warp] = __int_as_float(int(hit));
+      scratch[2 + warp] = __int_as_float(int(mass));
+    }
+    asm volatile("bar.sync 1, 64;" ::: "memory");
+    const unsigned h0 = __float_as_int(scratch[0]), h1 = __float_as_int(scratch[1]);
+    const unsigned m0 = __float_as_int(scratch[2]), m1 = __float_as_int(scratch[3]);
+    int cstar = h0 ? __ffs(int(h0)) - 1 : (h1 ? 32 + __ffs(int(h1)) - 1 : -1);
+    bool force_last = false;
+    if (cstar < 0 && z > 0.f) {
+      cstar = m1 ? 63 - __clz(int(m1)) : 31 - __clz(int(m0));
+      force_last = true;
+    }
+    if (k == cstar) {
+      *cstar_out = cstar;
+      *rem_out = force_last ? INFINITY : t - (inc - v);
+    }
+    if (threadIdx.x == 0 && cstar < 0) *cstar_out = -1;
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, const SampleArgs s) {
   const int c = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float sh[kSampleThreads / 32];
   __shared__ float sub_tot[kSubs];
   __shared__ float sub_part[kSampleThreads / 32][kSubs];
+  __shared__ float csum_s[kSampleMaxChunks];
   __shared__ int a_s, last_s, cstar_s, found_s, lastpos_s;
   __shared__ float rem_s;
 
@@ -113,7 +161,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
   __syncthreads();
   const int a = a_s;
   const float* prow = s.p + (int64_t(b) * (p.B + 1) + a) * s.V;
-  const float* qrow = a < p.B ? s.q + (int64_t(b) * p.B + a) * s.V : nullptr;
+  const float* qrow = a < p.B ? s.q + (int64_t(b) * p.B + a) * s.V : nullptr;  // null: draw from p
 
   // this chunk's share of the draw's mass
   {
@@ -131,57 +179,40 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
     if (!last_s) return;
   }
 
-  // the sequence's last CTA: total mass, then the chunk holding u_B * total. The chunk
-  // sums are loaded at once (chunk k by thread k) and scanned by the first two warps.
+  // the sequence's last CTA: the chunk sums (loaded at once, chunk k by thread k), then
+  // the chunk holding u_B * total
   __threadfence();
-  if (warp < 2) {
-    const int k = threadIdx.x;
-    const float v = k < s.nchunks ? __ldcg(p.samp_part + b * kSampleMaxChunks + k) : 0.f;
-    float inc = v;  // inclusive prefix within the warp, in chunk order
+  if (threadIdx.x < kSampleMaxChunks)
+    csum_s[threadIdx.x] =
+        int(threadIdx.x) < s.nchunks ? __ldcg(p.samp_part + b * kSampleMaxChunks + threadIdx.x) : 0.f;
+  if (threadIdx.x == 0) p.samp_count[b] = 0;  // zero again for the next call
+  __syncthreads();
+  const float ub = s.u[b * (p.B + 1) + p.B];
+  find_chunk(csum_s, s.nchunks, ub, sh, sub_tot, &cstar_s, &rem_s);
+  if (cstar_s < 0 && qrow != nullptr) {
+    // The residual has no mass (p_a <= q_a everywhere: equal rows up to rounding, or a
+    // draft neither row gives mass): the token is drawn from the target's row p_a itself,
+    // whose chunk sums this CTA makes in the order the chunk CTAs use.
+    qrow = nullptr;
+    for (int c2 = 0; c2 < s.nchunks; ++c2) {
+      const int base = c2 * kSampleChunk + 4 * threadIdx.x;
+      float acc = 0.f;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
+      for (int m = 0; m < kSubs; ++m) acc += sum4(weights4(prow, nullptr, base + m * kSub, s.V));
+      const float tot = block_sum(acc, sh);
+      if (threadIdx.x == 0) csum_s[c2] = tot;
     }
-    if (lane == 31) sh[warp] = inc;
-    asm volatile("bar.sync 1, 64;" ::: "memory");  // the two warps' totals
-    if (warp == 1) inc += sh[0];
-    const float z = sh[0] + sh[1];
-    const float t = s.u[b * (p.B + 1) + p.B] * z;
-    // the first chunk whose running sum passes t; the last chunk with mass if rounding
-    // leaves none
-    const unsigned hit = __ballot_sync(0xffffffffu, z > 0.f && k < s.nchunks && inc > t);
-    const unsigned mass = __ballot_sync(0xffffffffu, k < s.nchunks && v > 0.f);
-    if (lane == 0) {
-      sub_tot[warp] = __int_as_float(int(hit));
-      sub_tot[2 + warp] = __int_as_float(int(mass));
-    }
-    asm volatile("bar.sync 1, 64;" ::: "memory");
-    const unsigned h0 = __float_as_int(sub_tot[0]), h1 = __float_as_int(sub_tot[1]);
-    const unsigned m0 = __float_as_int(sub_tot[2]), m1 = __float_as_int(sub_tot[3]);
-    int cstar = h0 ? __ffs(int(h0)) - 1 : (h1 ? 32 + __ffs(int(h1)) - 1 : -1);
-    bool force_last = false;
-    if (cstar < 0 && z > 0.f) {
-      cstar = m1 ? 63 - __clz(int(m1)) : 31 - __clz(int(m0));
-      force_last = true;
-    }
-    if (k == cstar) {
-      cstar_s = cstar;
-      rem_s = force_last ? INFINITY : t - (inc - v);
-    }
-    if (threadIdx.x == 0 && cstar < 0) cstar_s = -1;
+    __syncthreads();
+    find_chunk(csum_s, s.nchunks, ub, sh, sub_tot, &cstar_s, &rem_s);
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    p.samp_count[b] = 0;  // zero again for the next call
-    if (cstar_s < 0) {  // no mass at all: the rejected draft itself, or token 0 (p_B empty)
+  if (cstar_s < 0) {  // the row drawn from has no mass: not a distribution
+    if (threadIdx.x == 0) {
       s.accept_len[b] = a;
-      s.next_token[b] = a < p.B ? s.draft[b * p.B + a] : 0;
-      if (a == p.B) set_err(p.err, LS_DEVERR_SAMPLE);
+      s.next_token[b] = 0;
+      set_err(p.err, LS_DEVERR_SAMPLE);
     }
+    return;
   }
-  __syncthreads();
-  if (cstar_s < 0) return;
 
   // sub-block and entry: the first entry whose running sum in the chunk passes rem
   const int cbase = cstar_s * kSampleChunk;

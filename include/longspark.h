@@ -38,6 +38,9 @@
  *     the window and mirror rows in the arena. Summary sums and segment means are fp32.
  *   - Kernels never trap. Conditions found on the device (bad prefix length, bounded
  *     waits that ran out) set bits in the device error word; read it with ls_get_error.
+ *   - A state belongs to the device that was current at ls_init_state. Every call that
+ *     takes a state returns LS_ERR_INVALID_ARG, and does nothing, while another device
+ *     is current.
  */
 #ifndef LONGSPARK_H_
 #define LONGSPARK_H_
@@ -92,7 +95,7 @@ extern "C" {
                                        tcgen05 tensor-core kernel applies              */
 #define LS_FLAG_OUT_F32    0x2      /* ls_draft_attend writes fp32 outputs (otherwise
                                        `dtype`); a bf16 output adds its own rounding of
-                                       up to 2^-9 |out| to the attention's error       */
+                                       up to 2^-8 |out| to the attention's error       */
 
 #define LS_MAX_SCALES 4
 
@@ -228,9 +231,9 @@ LS_API int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, in
  * library holds it until the process exits. Each call needs
  * ls_prefill_workspace_bytes(cfg, row_begin, row_end) <= 16 MiB, otherwise it returns
  * LS_ERR_SCRATCH_LIMIT and does nothing: split the prefix into chunks (row_begin a
- * multiple of the largest scale) that each fit. The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress); make that first call before any stream
- * capture. Every call uses the same array, which keeps the last call's contents (nothing
+ * multiple of the largest scale) that each fit. The first call for a state's device
+ * looks up that device's copy of the array (cudaGetSymbolAddress, with the state's
+ * device current); make that first call before any stream capture. Every call uses the same array, which keeps the last call's contents (nothing
  * in it has to start at zero), so calls that overlap on the GPU race: order them on one
  * stream or with events. Calls no cudaMalloc/cudaFree and no allocating routine.      */
 LS_API int ls_prefill_summary_noalloc(ls_state* st, const void* d_k, const void* d_v,
@@ -265,12 +268,14 @@ LS_API int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32
  *                  u_i * q_i(d_i) < p_i(d_i) (fp32 product and comparison)
  *   d_next_token   int32 [b] out: drawn from max(0, p_a - q_a) when a < B, from p_B when
  *                  a = B: the first token t whose running sum over tokens 0..t exceeds
- *                  u_B times the total (fp32 sums in the kernel's order); a residual with
- *                  no mass gives the rejected draft token itself.
+ *                  u_B times the total (fp32 sums in the kernel's order). A residual
+ *                  with no mass (p_a <= q_a everywhere) is replaced by p_a itself, so
+ *                  the token is always one the target gives mass.
  * vocab a multiple of 4 and <= 524288 (else LS_ERR_SHAPE / LS_ERR_UNSUPPORTED); the
  * probability pointers 16-byte aligned. Reads 2B gathered values per sequence and the
  * draw's row(s) once (plus the drawn 8192-entry chunk again). A draft id outside
- * [0, vocab), or p_B with no mass, sets LS_DEVERR_SAMPLE. The state only lends its
+ * [0, vocab), or a target row drawn from with no mass (next token 0), sets
+ * LS_DEVERR_SAMPLE. The state only lends its
  * shapes and a scratch region (sequences may not run two of these calls at once). Feed
  * the accepted counts to ls_commit_accepted.                                          */
 LS_API int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const float* d_draft_probs,

@@ -378,8 +378,9 @@ def draft_attend(sh: Shapes, v: Views, q: np.ndarray, boundary_k: np.ndarray,
 # (Leviathan, Kalman and Matias 2023; Chen et al. 2023), position by position over the
 # block: draft i is kept when u_i * q_i(d_i) < p_i(d_i) (u_i uniform in [0, 1), the test
 # made in fp32 as the GPU makes it: it decides an integer); at the first rejection the
-# next token is drawn from the residual max(0, p_i - q_i), and after B acceptances from
-# p_B. The draws u_0..u_{B-1} and the final draw v are inputs.
+# next token is drawn from the residual max(0, p_i - q_i) (from p_i itself when that
+# residual has no mass), and after B acceptances from p_B. The draws u_0..u_{B-1} and the
+# final draw v are inputs.
 def accept_decisions(draft_ids, q_rows, p_rows, u):
     """fp32 acceptance tests of one sequence: draft i kept iff u_i * q_i(d_i) < p_i(d_i).
 
@@ -409,25 +410,42 @@ def sampling_weights(q_rows, p_rows, a):
     return p_rows[B].astype(np.float64)
 
 
+def draw_weights(q_rows, p_rows, a):
+    """The weights the next token is actually drawn from: ``sampling_weights``, except that
+    a residual with no mass (p_a <= q_a everywhere, which exact arithmetic only reaches when
+    the two rows are equal, so a rejection there comes from rounding or from a draft that q
+    gives no mass) is replaced by the target's own row p_a. Speculative sampling emits
+    samples of the target's distribution; p_a is that distribution at the rejected
+    position, so the emitted token always lies in the target's support there.
+
+    Raises ValueError when the row drawn from has no mass at all (not a probability row).
+    """
+    w = sampling_weights(q_rows, p_rows, a)
+    if not (w > 0).any() and a < q_rows.shape[0]:
+        w = p_rows[a].astype(np.float64)
+    if not (w > 0).any():
+        raise ValueError("the target's probability row has no mass")
+    return w
+
+
 def inverse_cdf(w, v):
-    """Smallest t with sum(w[:t+1]) > v * sum(w); the last index with w > 0 if rounding
-    leaves none (v < 1). w >= 0 with a positive sum."""
+    """Smallest t with sum(w[:t+1]) > v * sum(w), for weights w >= 0 with a positive sum
+    and a draw 0 <= v < 1. The threshold is then below the total, so some running sum
+    passes it, and the first that does ends on an entry with mass."""
+    w = np.asarray(w, np.float64)
+    if not (0.0 <= v < 1.0):
+        raise ValueError("the draw must lie in [0, 1)")
     c = np.cumsum(w)
-    t = int(np.searchsorted(c, v * c[-1], side="right"))
-    if t >= len(w):
-        t = int(np.nonzero(w > 0)[0][-1])
-    return t
+    if not c[-1] > 0:
+        raise ValueError("weights without mass")
+    return int(np.searchsorted(c, v * c[-1], side="right"))
 
 
 def accept_sampled(draft_ids, q_rows, p_rows, u, v):
-    """One sequence's stochastic acceptance: (a, next token). A draw with no mass at all (a
-    residual of rows equal up to rounding) gives the rejected draft token itself (token 0
-    for an empty p_B, an invalid input)."""
+    """One sequence's stochastic acceptance: (a, next token), the next token drawn from
+    ``draw_weights`` with the draw v."""
     a, _ = accept_decisions(draft_ids, q_rows, p_rows, u)
-    w = sampling_weights(q_rows, p_rows, a)
-    if not (w > 0).any():
-        return a, (int(draft_ids[a]) if a < len(draft_ids) else 0)
-    return a, inverse_cdf(w, v)
+    return a, inverse_cdf(draw_weights(q_rows, p_rows, a), v)
 
 
 # ----------------------------------------------------------------------------------

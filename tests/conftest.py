@@ -18,3 +18,13 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def repo_root():
     return ROOT
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The largest attention error against the oracle per test (the bound is 1e-2)."""
+    side = sys.modules.get("tests.oracle_side")
+    if side is None or not side.ATTEND_MAX_ERR:
+        return
+    terminalreporter.write_sep("-", "attention: max |gpu - oracle| per test (bound 1e-2)")
+    for key, err in sorted(side.ATTEND_MAX_ERR.items()):
+        terminalreporter.write_line(f"{err:.3e}  {key}")

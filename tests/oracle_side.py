@@ -6,6 +6,8 @@ inputs come from ``synth`` (the same draws the device runner writes on the GPU).
 
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 import oracle as O
@@ -86,18 +88,19 @@ def tile_attend(wl, sh, views, b, l, g, r, hidden_vec, view_set=O.VIEW_ALL):
 
 # ---- comparisons (tolerances as stated for the path) ---------------------------------
 SUMMARY_RTOL = 1e-3  # normwise per slot vector
-ATTEND_ATOL = 1e-2   # max absolute
-BF16_OUT_RTOL = 2.0 ** -8  # rounding of a bf16 output (8-bit significand, nearest even): at most 2^-8 |x|
+ATTEND_ATOL = 1e-2   # max absolute, for every output dtype (a bf16 output's rounding included)
+
+# largest max |gpu - oracle| of the attention seen per test (printed at the end of a run)
+ATTEND_MAX_ERR: dict = {}
 
 
-def attend_error_excess(got, ref, out_is_f32):
-    """max(|got - ref| - bound): <= 0 when within tolerance.
-
-    fp32 outputs: bound 1e-2. bf16 outputs: 1e-2 plus the output's own rounding,
-    2^-8 |ref| (the attention value itself cannot be stored closer than that).
-    """
-    bound = ATTEND_ATOL + (0.0 if out_is_f32 else BF16_OUT_RTOL * np.abs(ref))
-    return float(np.max(np.abs(got - ref) - bound))
+def attend_error_excess(got, ref):
+    """max |got - ref| - 1e-2: <= 0 when the attention output is within tolerance. The
+    bound is flat: a bf16 output's own rounding (at most 2^-8 |out|) has to fit in it."""
+    err = float(np.max(np.abs(np.asarray(got, np.float64) - ref))) if np.size(ref) else 0.0
+    key = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0] or "?"
+    ATTEND_MAX_ERR[key] = max(ATTEND_MAX_ERR.get(key, 0.0), err)
+    return err - ATTEND_ATOL
 
 
 def gpu_f64(x, dtype):

@@ -21,26 +21,47 @@ if torch.cuda.is_available():
     from fixed_cost_drafter_b200 import workloads as WL
 
 
-def _run_full(wl, rounds=None, prefill_chunk=None, check_every_round=False):
+EARLY_ROUND = 3  # an early round whose attention output is kept and checked as well
+
+
+def _run_full(wl, rounds=None, prefill_chunk=None):
+    """Prefill, then every round's commit and attention; returns the run, the last round's
+    output and a copy of round EARLY_ROUND's output."""
     run = WL.DeviceRun(wl, rounds=rounds, prefill_chunk=prefill_chunk)
     run.prefill()
     inp = run.make_round_inputs()
     out = run.new_out()
-    acc_gpu = []
+    early = None
     for r in range(run.rounds):
         run.commit(inp, r)
         run.attend(inp, r, out)
-        if check_every_round:
-            acc_gpu.append(run.accept_len.clone())
+        if r == EARLY_ROUND:
+            early = out.clone()
     torch.cuda.synchronize()
-    return run, out, acc_gpu
+    return run, out, early
 
 
-def _sampled_check(run, wl, out, tiles, view_set=None):
+def _check_attend_at(run, wl, out, tiles, r, acc, view_set=None):
+    """Attention output of round r on the sampled tiles against the oracle's attention over
+    the views as they stood after round r's commit."""
+    P = run.prefix_len
+    for b, l, h in tiles:
+        sh, views = OS.tile_views(wl, b, l, h, int(P[b]), acc[:r + 1, b], run.scale_host)
+        hid = OS.boundary_hidden(wl, b, l, r, int(acc[r, b]))
+        ref = OS.tile_attend(wl, sh, views, b, l, h, r, hid, OS.O.VIEW_ALL if view_set is None else view_set)
+        o = out[b, l].view(wl.block, wl.n_q_heads, wl.head_dim)[:, h * wl.group:(h + 1) * wl.group]
+        got = o.float().cpu().numpy().astype(np.float64)
+        exc = OS.attend_error_excess(got, ref)
+        assert exc <= 0, ("attend", r, b, l, h, float(np.abs(got - ref).max()), exc)
+
+
+def _sampled_check(run, wl, out, tiles, view_set=None, early=None):
     st = run.read_state()
     R = run.rounds
     draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
     acc = OS.accepts_from_ids(draft, target)
+    if early is not None:
+        _check_attend_at(run, wl, early, tiles, EARLY_ROUND, acc, view_set)
     assert np.array_equal(acc, run.accept_host), "generator accepts vs oracle scan"
     # any-size properties on every tile: len and counters consistent, all layers equal
     P = run.prefix_len
@@ -58,11 +79,14 @@ def _sampled_check(run, wl, out, tiles, view_set=None):
                              OS.O.VIEW_ALL if view_set is None else view_set)
         o = out[b, l].view(wl.block, wl.n_q_heads, wl.head_dim)[:, h * wl.group:(h + 1) * wl.group]
         got = o.float().cpu().numpy().astype(np.float64)
-        exc = OS.attend_error_excess(got, ref, o.dtype == torch.float32)
+        exc = OS.attend_error_excess(got, ref)
         assert exc <= 0, ("attend", b, l, h, float(np.abs(got - ref).max()), exc)
 
 
-TILES = [(0, 0, 0), (7, 2, 5), (15, 3, 7)]
+# At batch 16 the attention runs 512 tiles t = (b L + l) Hkv + h on 128 CTAs, tiles
+# c, c + 128, c + 256, c + 384 on CTA c: these tiles (t = 0, 245, 331, 511) sit in each of
+# the four places of a CTA's schedule.
+TILES = [(0, 0, 0), (7, 2, 5), (10, 1, 3), (15, 3, 7)]
 
 
 @pytest.mark.parametrize("name", ["qwen3_4b_32k", "qwen3_8b_64k", "qwen3_8b_64k_f32out", "qwen3_8b_128k_ragged"])
@@ -70,9 +94,9 @@ def test_full_config(name):
     from dataclasses import replace
     wl = (replace(WL.CONFIGS["qwen3_8b_64k"], flags=F.LS_FLAG_OUT_F32) if name.endswith("_f32out")
           else WL.CONFIGS[name])
-    run, out, _ = _run_full(wl)
+    run, out, early = _run_full(wl)
     assert run.error() == (F.LS_OK, 0)
-    _sampled_check(run, wl, out, TILES)
+    _sampled_check(run, wl, out, TILES, early=early)
 
 
 def test_full_config_view_ablations():

@@ -140,7 +140,7 @@ def test_prologue_feeds_the_attention():
         bv = BKV[b, l, H * D + g * D:H * D + (g + 1) * D].reshape(1, 1, D)
         ref = O.draft_attend(sh, views, qt, bk, bv, 1.0 / np.sqrt(D))[0]
         got = out[b, l].view(B, Hq, D)[:, g * wl.group:(g + 1) * wl.group].double().cpu().numpy()
-        assert OS.attend_error_excess(got, ref, False) <= 0
+        assert OS.attend_error_excess(got, ref) <= 0
     assert run.error() == (F.LS_OK, 0)
 
 

@@ -72,7 +72,7 @@ def test_round_matches_oracle():
                 ref = OS.tile_attend(wl, sh, views, b, l, h, wl.rounds - 1, hid)
                 o = out[b, l].view(wl.block, wl.n_q_heads, wl.head_dim)[:, h * wl.group:(h + 1) * wl.group]
                 got = o.float().cpu().numpy().astype(np.float64)
-                assert OS.attend_error_excess(got, ref, True) <= 0
+                assert OS.attend_error_excess(got, ref) <= 0
 
 
 def test_round_fallback_equals_two_calls():

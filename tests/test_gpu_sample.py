@@ -54,10 +54,7 @@ def _check(draft, q, p, u, acc, nxt):
     for b in range(draft.shape[0]):
         a, _ = O.accept_decisions(draft[b], q[b], p[b], u[b, :B])
         assert acc[b] == a, (b, acc[b], a)
-        w = O.sampling_weights(q[b], p[b], a)
-        if not (w > 0).any():
-            assert nxt[b] == (draft[b, a] if a < B else 0)
-            continue
+        w = O.draw_weights(q[b], p[b], a)
         t = int(nxt[b])
         cdf = np.cumsum(w)
         z = cdf[-1]
@@ -86,7 +83,7 @@ def test_sampled_random(vocab):
 
 def test_sampled_edge_cases():
     rng = np.random.default_rng(7)
-    b, B, V = 4, 8, 4096
+    b, B, V = 6, 8, 4096
     run = _state(b, B)
     q, _ = _probs(rng, (b, B, V))
     p = np.concatenate([q, _probs(rng, (b, 1, V))[0]], axis=1)
@@ -99,9 +96,24 @@ def test_sampled_edge_cases():
     u[2, B] = 0.999999
     u[3, B] = 0.0
     p[3, 2, draft[3, 2]] = 0.0  # sequence 3 rejects at position 2
+    # sequence 4: p_0 = q_0 and a first draft both give no mass: rejected, the residual has
+    # no mass, the token comes from p_0 (draws in three different chunks of the row)
+    q[4, 0, draft[4, 0]] = 0.0
+    p[4, 0] = q[4, 0]
+    u[4, B] = 0.73
+    # sequence 5: rows equal up to rounding: p_0 one fp32 step below q_0 at the draft, whose
+    # test fails only because u_0 * q_0(d) rounds to p_0(d)
+    d5 = int(draft[5, 0])
+    q[5, 0, d5] = np.float32(0.75)
+    p[5, 0] = q[5, 0]
+    p[5, 0, d5] = np.nextafter(np.float32(0.75), np.float32(0))
+    u[5, 0] = 1 - 2.0 ** -24
     acc, nxt = _run(run, draft, q, p, u)
     _check(draft, q, p, u, acc, nxt)
-    assert acc[0] == B and acc[1] == 0 and acc[3] == 2
+    assert acc[0] == B and acc[1] == 0 and acc[3] == 2 and acc[4] == 0 and acc[5] == 0
+    for i in (4, 5):
+        assert not (O.sampling_weights(q[i], p[i], 0) > 0).any()  # the branch is taken
+        assert p[i, 0, nxt[i]] > 0
     assert run.error() == (F.LS_OK, 0)
 
 
@@ -136,6 +148,14 @@ def test_sampled_errors():
     draft[1, 0] = V + 5  # outside the vocabulary: error bit, treated as rejected
     acc, nxt = _run(run, draft, q, p, u)
     assert acc[1] == 0
+    status, word = run.error()
+    assert status == F.LS_ERR_DEVICE and word & F.LS_DEVERR_SAMPLE
+    # a target row without mass to draw from: error bit, token 0
+    F.ls_clear_error(run.state, run.stream)
+    draft = rng.integers(0, V, (b, B)).astype(np.int32)
+    p[0, 0] = 0.0  # the first draft is rejected (no target mass) and p_0 has none either
+    acc, nxt = _run(run, draft, q, p, u)
+    assert acc[0] == 0 and nxt[0] == 0
     status, word = run.error()
     assert status == F.LS_ERR_DEVICE and word & F.LS_DEVERR_SAMPLE
 

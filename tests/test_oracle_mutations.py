@@ -155,6 +155,20 @@ def _residual_from_next_position(q_rows, p_rows, a):
     return p_rows[B].astype(np.float64)
 
 
+def _zero_mass_emits_rejected_draft(draft_ids, q_rows, p_rows, u, v):
+    # a residual without mass answered with the rejected draft token itself
+    a, _ = M.accept_decisions(draft_ids, q_rows, p_rows, u)
+    w = M.sampling_weights(q_rows, p_rows, a)
+    if not (w > 0).any():
+        return a, int(draft_ids[a]) if a < len(draft_ids) else 0
+    return a, M.inverse_cdf(w, v)
+
+
+def _inverse_cdf_one_past(w, v):
+    # the index after the one whose running sum passes the threshold (clamped)
+    return min(ORIG["inverse_cdf"](w, v) + 1, len(w) - 1)
+
+
 def _prologue_layer0_weights(w_kv, w_q, boundary, x):
     # every layer projected with layer 0's weights
     w_kv, w_q = np.asarray(w_kv), np.asarray(w_q)
@@ -165,7 +179,7 @@ def _prologue_layer0_weights(w_kv, w_q, boundary, x):
 ORIG = {n: getattr(M, n) for n in ("accept_scan", "retain_row", "views_from_scratch",
                                    "attention_slots", "draft_attend", "view_of_slots",
                                    "accept_decisions", "sampling_weights", "draft_prologue", "paged_rows",
-                                   "inverse_cdf")}
+                                   "inverse_cdf", "accept_sampled")}
 
 CASES = [
     ("accept_scan", _scan_off_by_one, [P.test_scan_golden_examples]),
@@ -185,6 +199,8 @@ CASES = [
     ("inverse_cdf", _inverse_cdf_side_left, [P.test_inverse_cdf_boundaries]),
     ("sampling_weights", _residual_from_next_position, [P.test_sampled_emits_target_distribution]),
     ("commit_round_paged", _paged_commit_from_position_zero, [lambda: P.test_paged_commit_equals_dense(3)]),
+    ("accept_sampled", _zero_mass_emits_rejected_draft, [P.test_sampled_residual_without_mass_draws_from_target_row]),
+    ("inverse_cdf", _inverse_cdf_one_past, [P.test_inverse_cdf_exact_brute_force]),
 ]
 
 

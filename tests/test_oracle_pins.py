@@ -449,6 +449,64 @@ def test_inverse_cdf_boundaries():
     assert {O.inverse_cdf(np.array([0.0, 1.0, 0.0, 1.0]), v) for v in np.linspace(0, 0.999, 101)} == {1, 3}
 
 
+def test_sampled_residual_without_mass_draws_from_target_row():
+    """A rejection whose residual max(0, p_a - q_a) has no mass (p_a <= q_a everywhere).
+    Speculative sampling emits samples of the target's distribution, so the token must
+    lie in p_a's support, and with p_a = q_a its distribution over the draw v must be p_a
+    itself. Hand-worked: p_0 = q_0 = (1/4, 3/4, 0, 0) and a draft (token 2) that both rows
+    give no mass: 0 * 0 < 0 fails, a = 0, the residual is all zero, and the inverse CDF of
+    p_0 gives token 0 for v < 1/4 and token 1 for 1/4 <= v < 1 (never the draft)."""
+    q = np.array([[0.25, 0.75, 0.0, 0.0]], dtype=np.float32)
+    p_rows = np.array([[0.25, 0.75, 0.0, 0.0], [0.0, 0.0, 0.0, 1.0]], dtype=np.float32)
+    for v, want in [(0.0, 0), (0.1, 0), (0.2499, 0), (0.25, 1), (0.6, 1), (1 - 2.0 ** -24, 1)]:
+        assert O.accept_sampled([2], q, p_rows, [0.5], v) == (0, want)
+    # the emitted distribution over a midpoint grid of v is p_0 exactly (grid of 4: 1 and 3)
+    grid = (np.arange(4) + 0.5) / 4
+    assert [O.accept_sampled([2], q, p_rows, [0.5], v)[1] for v in grid] == [0, 1, 1, 1]
+    # rows equal up to rounding: p_0(1) is one fp32 step below q_0(1); u = 1 - 2^-24 makes
+    # u * q_0(1) round to p_0(1), so the test fails; the residual is zero everywhere and
+    # the token comes from p_0 (token 0 for v < 1/4 of its total)
+    q2 = np.array([[0.25, 0.75]], dtype=np.float32)
+    p2 = np.array([[0.25, np.nextafter(np.float32(0.75), np.float32(0))], [0.5, 0.5]], dtype=np.float32)
+    u = np.float32(1 - 2.0 ** -24)
+    assert np.float32(u * q2[0, 1]) == p2[0, 1]
+    assert not (O.sampling_weights(q2, p2, 0) > 0).any()
+    assert O.accept_sampled([1], q2, p2, [u], 0.1) == (0, 0)
+    assert O.accept_sampled([1], q2, p2, [u], 0.9) == (0, 1)
+    # a target row without any mass is not a distribution: refused
+    with pytest.raises(ValueError):
+        O.accept_sampled([0], q2, np.zeros((2, 2), np.float32), [0.5], 0.5)
+
+
+def test_inverse_cdf_exact_brute_force():
+    """The draw against its definition in exact rational arithmetic: small integer weights
+    (zeros included, leading and trailing) and draws on a dyadic grid of [0, 1) with its
+    ends 0 and 1 - 2^-24. The index is the smallest t whose running sum exceeds v times
+    the total, and it always carries mass."""
+    from fractions import Fraction
+    rng = np.random.default_rng(23)
+    vs = [0.0, 1 - 2.0 ** -24] + [k / 64 for k in range(64)]
+    for _ in range(200):
+        n = int(rng.integers(1, 7))
+        w = rng.integers(0, 4, n)
+        if w.sum() == 0:
+            w[int(rng.integers(0, n))] = 1
+        tot = int(w.sum())
+        for v in vs:
+            thr = Fraction(v) * tot
+            run, want = 0, None
+            for t in range(n):
+                run += int(w[t])
+                if run > thr:
+                    want = t
+                    break
+            got = O.inverse_cdf(w.astype(np.float64), v)
+            assert got == want and w[got] > 0, (w, v, got, want)
+    for bad in (1.0, -0.1):
+        with pytest.raises(ValueError):
+            O.inverse_cdf(np.ones(3), bad)
+
+
 def test_sampled_decision_is_fp32():
     """u * q rounded to fp32 before the comparison: with p set to that rounded product the
     draft is rejected, although the exact product is below p."""

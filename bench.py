@@ -236,98 +236,179 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline and --impl reference)
 # ---------------------------------------------------------------------------------------
-class OracleSample:
-    """The CPU oracle on a bounded slice of the workload: one tapped layer of sequence 0.
+class OracleSlices:
+    """The CPU oracle's drafting state for some (sequence, layer) slices of a workload.
 
     The oracle's views are fixed-size, so its per-round work does not depend on the
-    prefix: the views are initialised (untimed) from the first ``prefix_rows`` prefix rows.
-    One step = the oracle's round for that (sequence, layer): commit of the retained rows
-    and the attention of all query heads; a full round is batch x layers such steps.
+    prefix: each slice's views are initialised (untimed) from its first ``prefix_rows``
+    prefix rows. ``step(r)`` runs one round on every slice it holds: the commit of the
+    retained rows and the attention of all query heads, with the round's own synthetic
+    inputs (``n_inputs`` distinct rounds, cycled). A whole round of the workload is every
+    (sequence, layer) slice once.
     """
 
-    def __init__(self, wl, prefix_rows: int = 4096, n_inputs: int = 16):
+    def __init__(self, wl_name, slices, prefix_rows=4096, n_inputs=4):
         import oracle as O
         import synth as S
-        self.O, self.wl = O, wl
+        from synth.workloads import CONFIGS
+        wl = CONFIGS[wl_name]
+        self.O, self.wl, self.slices = O, wl, list(slices)
         H, Hq, D, B = wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.block
         self.sh = O.Shapes(n_layers=1, n_kv_heads=H, n_q_heads=Hq, head_dim=D, hidden=wl.hidden, block=B,
                            window=wl.window, scales=tuple(wl.scales), slots=wl.slots)
         scale = S.head_scales(wl.seed, wl.n_layers, H) if wl.head_scale else None
         P = prefix_rows
         f = lambda tid, shape, **kw: O.to_f64(S.fill_normal(wl.seed, tid, shape, **kw), wl.dtype)  # noqa: E731
-        pk = f(S.PREFIX_K, (1, 1, 1, P, H * D), head_dim=D, scale=scale)[0, 0]
-        pv = f(S.PREFIX_V, (1, 1, 1, P, H * D), head_dim=D, scale=scale)[0, 0]
-        hid = f(S.LAST_HIDDEN, (1, 1, 1, 1, wl.hidden))[0, 0, :, 0]
-        self.views = O.prefill(self.sh, pk.reshape(1, P, H, D), pv.reshape(1, P, H, D), P, hid)
-        acc = S.accept_lengths(wl.seed, n_inputs, 1, B, wl.accept_mean)
-        self.draft, self.target = S.token_ids(wl.seed, n_inputs, 1, B, acc, wl.vocab)
-        self.inputs = []
-        for r in range(n_inputs):
-            vk = f(S.VERIFY_K, (1, 1, 1, B + 1, H * D), r0=r, head_dim=D, scale=scale)[0, 0].reshape(1, B + 1, H, D)
-            vv = f(S.VERIFY_V, (1, 1, 1, B + 1, H * D), r0=r, head_dim=D, scale=scale)[0, 0].reshape(1, B + 1, H, D)
-            vh = f(S.VERIFY_HIDDEN, (1, 1, 1, B + 1, wl.hidden), r0=r)[0, 0]
-            q = f(S.QUERY, (1, 1, 1, B, Hq * D), r0=r, head_dim=D)[0, 0].reshape(1, B, Hq, D)
-            self.inputs.append((vk, vv, vh, q))
-        self.step_no = 0
+        acc = S.accept_lengths(wl.seed, n_inputs, wl.batch, B, wl.accept_mean)
+        self.draft, self.target = S.token_ids(wl.seed, n_inputs, wl.batch, B, acc, wl.vocab)
+        self.views, self.inputs = [], []
+        for b, l in self.slices:
+            pk = f(S.PREFIX_K, (1, 1, 1, P, H * D), b0=b, l0=l, head_dim=D, scale=scale)[0, 0]
+            pv = f(S.PREFIX_V, (1, 1, 1, P, H * D), b0=b, l0=l, head_dim=D, scale=scale)[0, 0]
+            hid = f(S.LAST_HIDDEN, (1, 1, 1, 1, wl.hidden), b0=b, l0=l)[0, 0, :, 0]
+            self.views.append(O.prefill(self.sh, pk.reshape(1, P, H, D), pv.reshape(1, P, H, D), P, hid))
+            ins = []
+            for r in range(n_inputs):
+                kw = dict(r0=r, b0=b, l0=l)
+                vk = f(S.VERIFY_K, (1, 1, 1, B + 1, H * D), head_dim=D, scale=scale, **kw)[0, 0]
+                vv = f(S.VERIFY_V, (1, 1, 1, B + 1, H * D), head_dim=D, scale=scale, **kw)[0, 0]
+                vh = f(S.VERIFY_HIDDEN, (1, 1, 1, B + 1, wl.hidden), **kw)[0, 0]
+                q = f(S.QUERY, (1, 1, 1, B, Hq * D), head_dim=D, **kw)[0, 0]
+                ins.append((vk.reshape(1, B + 1, H, D), vv.reshape(1, B + 1, H, D), vh, q.reshape(1, B, Hq, D)))
+            self.inputs.append(ins)
         self.sm = 1.0 / math.sqrt(D)
 
-    def step(self) -> float:
-        """Seconds for one oracle (sequence, layer) round slice."""
-        O, wl = self.O, self.wl
-        H, D = wl.n_kv_heads, wl.head_dim
-        r = self.step_no % len(self.inputs)
-        self.step_no += 1
-        vk, vv, vh, q = self.inputs[r]
+    def step(self, r: int) -> float:
+        """Seconds for round r on every slice held."""
+        O, H, D = self.O, self.wl.n_kv_heads, self.wl.head_dim
         t0 = time.perf_counter()
-        O.commit_round(self.sh, self.views, self.draft[r, 0], self.target[r, 0], vk, vv, vh)
-        bk = self.views.boundary[:, :H * D].reshape(1, H, D)
-        bv = self.views.boundary[:, H * D:2 * H * D].reshape(1, H, D)
-        O.draft_attend(self.sh, self.views, q, bk, bv, self.sm)
+        for (b, _), views, ins in zip(self.slices, self.views, self.inputs):
+            k = r % len(ins)
+            vk, vv, vh, q = ins[k]
+            O.commit_round(self.sh, views, self.draft[k, b], self.target[k, b], vk, vv, vh)
+            bk = views.boundary[:, :H * D].reshape(1, H, D)
+            bv = views.boundary[:, H * D:2 * H * D].reshape(1, H, D)
+            O.draft_attend(self.sh, views, q, bk, bv, self.sm)
         return time.perf_counter() - t0
 
-    def slices_per_round(self) -> int:
-        return self.wl.batch * self.wl.n_layers
+
+def _oracle_worker(conn, wl_name, slices, prefix_rows):
+    """A worker process: one BLAS thread, its slices' state; steps on request."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        st = OracleSlices(wl_name, slices, prefix_rows)
+        conn.send("ready")
+        while True:
+            r = conn.recv()
+            if r is None:
+                break
+            conn.send(st.step(r))
+    conn.close()
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class OracleRounds:
+    """Whole rounds of the CPU oracle on ``workers`` processes (spawned, one thread each),
+    the workload's (sequence, layer) slices dealt round-robin over them. ``round(r)``
+    returns the wall time of one whole round, from the request to the last worker's
+    answer."""
+
+    def __init__(self, wl_name, workers, prefix_rows=4096):
+        import multiprocessing as mp
+        from synth.workloads import CONFIGS
+        wl = CONFIGS[wl_name]
+        all_slices = [(b, l) for b in range(wl.batch) for l in range(wl.n_layers)]
+        self.workers = max(1, min(int(workers), len(all_slices)))
+        self.n_slices = len(all_slices)
+        ctx = mp.get_context("spawn")
+        self.conns, self.procs = [], []
+        for w in range(self.workers):
+            a, b = ctx.Pipe()
+            proc = ctx.Process(target=_oracle_worker, args=(b, wl_name, all_slices[w::self.workers], prefix_rows),
+                               daemon=True)
+            proc.start()
+            self.conns.append(a)
+            self.procs.append(proc)
+        for c in self.conns:
+            if c.recv() != "ready":
+                raise RuntimeError("oracle worker failed to start")
+
+    def round(self, r: int):
+        """(wall seconds of the whole round, its compute seconds summed over the workers)."""
+        t0 = time.perf_counter()
+        for c in self.conns:
+            c.send(r)
+        busy = sum(c.recv() for c in self.conns)
+        return time.perf_counter() - t0, busy
+
+    def close(self):
+        for c in self.conns:
+            c.send(None)
+        for p in self.procs:
+            p.join(timeout=30)
+
+
+def oracle_sample_text(wl, workers, rounds, prefix_rows=4096):
+    return (f"{rounds} whole rounds of the oracle (commit + attention of all {wl.n_q_heads} query heads for "
+            f"every one of the {wl.batch} sequences x {wl.n_layers} tapped layers) on {workers} worker "
+            f"processes of one thread each; views initialised from a {prefix_rows}-row prefix (the oracle's "
+            f"per-round work does not depend on the prefix)")
+
+
+def oracle_timing(wl_name, warmup, steps=None, budget_s=None):
+    """Whole oracle rounds on every host core: ``warmup`` untimed rounds, then ``steps``
+    rounds (or rounds until ``budget_s`` has passed). Returns (wall seconds per round,
+    summed worker seconds per round, rounds timed, workers)."""
+    pool = OracleRounds(wl_name, host_cores())
+    try:
+        for i in range(warmup):
+            pool.round(i)
+        walls, busy = [], []
+        t_end = time.perf_counter() + (budget_s or 0.0)
+        while (steps is not None and len(walls) < steps) or (steps is None and (time.perf_counter() < t_end
+                                                                                  or len(walls) < 2)):
+            w, b = pool.round(warmup + len(walls))
+            walls.append(w)
+            busy.append(b)
+    finally:
+        pool.close()
+    return float(np.mean(walls)), float(np.mean(busy)), len(walls), pool.workers
+
+
+def cpu_record(wl, per_round, busy, rounds, workers):
+    return {"value": 1.0 / per_round, "unit": "rounds/s", "cores": workers, "kind": "oracle",
+            "sample": oracle_sample_text(wl, workers, rounds),
+            "one_core": {"value": 1.0 / busy, "unit": "rounds/s", "cores": 1,
+                         "sample": "the same rounds' compute time summed over the worker processes (each "
+                                   "worker times its own slices on its own core, all running at once): "
+                                   "a whole round's work at one core's speed"}}
 
 
 def cpu_baseline(wl, budget_s: float = 15.0):
-    from threadpoolctl import threadpool_limits
-    smp = OracleSample(wl)
-    with threadpool_limits(limits=1):
-        smp.step()
-        times = []
-        t_end = time.perf_counter() + budget_s
-        while time.perf_counter() < t_end or len(times) < 3:
-            times.append(smp.step())
-    per_round = float(np.mean(times)) * smp.slices_per_round()
-    return {"value": 1.0 / per_round, "unit": "rounds/s", "cores": 1, "kind": "oracle",
-            "sample": f"{len(times)} oracle round slices (commit + attention of all {wl.n_q_heads} query "
-                      f"heads for one tapped layer of sequence 0), mean x {smp.slices_per_round()} "
-                      f"(= {wl.batch} sequences x {wl.n_layers} layers); views initialised from a 4096-row "
-                      f"prefix (the oracle's per-round work does not depend on the prefix)"}
+    """The oracle on the host cores: one untimed round, then whole rounds for about budget_s."""
+    per_round, busy, n, workers = oracle_timing(wl.name, 1, budget_s=budget_s)
+    return cpu_record(wl, per_round, busy, n, workers)
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    from threadpoolctl import threadpool_limits
-    from fixed_cost_drafter_b200 import workloads as WLM
-    wl = WLM.CONFIGS[args.config]
-    smp = OracleSample(wl)
-    with threadpool_limits(limits=1):
-        for _ in range(args.warmup):
-            smp.step()
-        times = [smp.step() for _ in range(args.steps)]
-    per_round = float(np.mean(times)) * smp.slices_per_round()
+    from synth.workloads import CONFIGS
+    wl = CONFIGS[args.config]
+    per_round, busy, n, workers = oracle_timing(wl.name, args.warmup, steps=args.steps)
     v = 1.0 / per_round
-    sample = (f"each step: the oracle's round for one tapped layer of sequence 0 (commit + attention of "
-              f"all {wl.n_q_heads} query heads); a round of the workload = {smp.slices_per_round()} such "
-              f"slices ({wl.batch} sequences x {wl.n_layers} layers); 1 thread")
     line = {"metric": METRIC, "value": v, "unit": "rounds/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": per_round * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": workload_config(wl),
-            "cpu_baseline": {"value": v, "unit": "rounds/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "config": workload_config(wl), "parallelism": f"{workers} host processes",
+            "cpu_baseline": cpu_record(wl, per_round, busy, n, workers),
             "e2e": {"value": v, "unit": "rounds/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
@@ -534,10 +615,25 @@ def run_gpu(args):
     # end to end through the public API with host buffers (pinned), copies inside the region
     e2e = e2e_measure(run, wl, dev, flush, K, world, inp, strong)
 
-    # flatness over the prefix (b = 16) on a short sweep
-    flat = None
+    # the drafting round with sampled acceptance and the projections (4 launches)
+    drafting = None
+    if not args.no_drafting_round:
+        drafting = drafting_round_measure(WLM, wl, dev, flush, max(16, min(K, 200)),
+                                          WLM.SWEEP_PREFIXES if rank == 0 and not args.no_sweep else None)
+
+    # the other workload configurations, end to end (prefill and every round)
+    configs = None
+    if not args.no_configs and rank == 0 and not strong:
+        configs = {name: config_record(WLM, name, dev, flush, 0) for name in ("qwen3_4b_32k", "qwen3_8b_128k_ragged")}
+
+    # the prefix x concurrency x accept-mean sweep; flatness over the prefixes
+    grid, flat = None, None
     if not args.no_sweep and rank == 0:
-        flat = flatness_sweep(WLM, dev, flush, args.sweep_rounds)
+        grid = sweep_grid(WLM, dev, flush, args.sweep_rounds)
+        b16 = {str(p["prefix"]): p["us_per_round"] for p in grid["points"] if p["batch"] == 16
+               and p["accept_mean"] == 4.0}
+        flat = {"us_per_round": b16, "flatness": grid["flatness"]["batch16_mean4.0"], "batch": 16,
+                "accept_mean": 4.0, "rounds": grid["rounds_per_point"]}
 
     peak, peak_kind = hbm_peak()
     a_bytes = attend_bytes(wl)
@@ -555,8 +651,8 @@ def run_gpu(args):
             "metric": METRIC, "value": (1 if strong else world) * K / total_max, "unit": "rounds/s",
             "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": total_max * 1e3 / K, "higher_is_better": True,
             "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(workload_config(full_wl),
-                           parallelism=(f"kv-heads x {world}" if strong else f"batch x {world}")),
+            "config": workload_config(full_wl),
+            "parallelism": f"kv-heads x {world}" if strong else f"batch x {world}",
             "roofline": {"bound": "hbm",
                          "kernel": "ls_draft_attend (" + ("tcgen05" if tc else "CUDA cores") + ")",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
@@ -584,6 +680,9 @@ def run_gpu(args):
                         "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
             "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch,
             "flatness": flat,
+            "configs": configs,
+            "sweep": grid,
+            "drafting_round": drafting,
             "gpu_launches": 2 * K,
             "e2e": e2e,
             "clocks": clk.summary(),
@@ -828,32 +927,206 @@ def e2e_measure(run, wl, dev, flush, steps, world, inp, strong=False):
             "d2h_bytes_per_step": int(d2h), "steps": steps, "pipelined": "2 buffer slots, copy streams in and out"}
 
 
-def flatness_sweep(WLM, dev, flush, rounds):
-    """Per-round time at batch 16 over prefixes 4K..128K (accept mean 4.0)."""
+def time_rounds(run, inp, out, flush, n, warm=3):
+    """CUDA-event times (ms) of rounds warm .. n - 1 of ``run`` (``ls_round``), each after an
+    untimed L2 flush; rounds 0 .. warm - 1 run untimed first (they load the kernels)."""
     import torch
-    res = {}
-    for P in WLM.SWEEP_PREFIXES:
-        wl = WLM.sweep_point(P, 16, 4.0)
-        run = WLM.DeviceRun(wl, device=dev, rounds=rounds)
+    stream = run.stream
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for r in range(n):
+        flush.zero_()
+        evs[r][0].record(stream)
+        run.round(inp, r, out)
+        evs[r][1].record(stream)
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in evs[warm:]]
+
+
+def us_stats(ms):
+    return {"mean": float(np.mean(ms)) * 1e3, "median": float(np.median(ms)) * 1e3,
+            "p90": float(np.percentile(ms, 90)) * 1e3}
+
+
+def config_record(WLM, name, dev, flush, rank):
+    """One of the workload configurations end to end: its prefill (after one untimed
+    prefill into a state then reset) and all of its rounds (3 untimed), an L2 flush before
+    each round."""
+    import torch
+    import fixed_cost_drafter_b200 as F
+    peak, _ = hbm_peak()
+    wl = WLM.CONFIGS[name]
+    run = WLM.DeviceRun(wl, device=dev, seq_offset=sequence_offset(rank, wl.batch))
+    run.prefill()
+    run.reset_state()
+    pre = []
+    run.prefill(timer=lambda e0, e1, nbytes: pre.append((e0, e1, nbytes)))
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    pre_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in pre)
+    pre_b = sum(nb for _, _, nb in pre)
+    inp = run.make_round_inputs()
+    out = run.new_out()
+    warm = 3
+    ms = time_rounds(run, inp, out, flush, run.rounds, warm)
+    status, word = run.error()
+    if status != F.LS_OK:
+        raise RuntimeError(f"device error word {word:#x} in {name}")
+    deltas = run.accept_host[warm:] + 1
+    r_bytes = attend_bytes(wl) + commit_bytes(wl, float(deltas.mean()))
+    st = us_stats(ms)
+    rec = {"workload": workload_config(wl)["workload"],
+           "prefix_rows": int(np.sum(run.prefix_len)),
+           "prefill": {"ms": pre_ms, "bytes": pre_b, "achieved_GBps": pre_b / (pre_ms / 1e3) / 1e9,
+                       "frac": pre_b / (pre_ms / 1e3) / 1e9 / peak, "calls": len(pre)},
+           "rounds": len(ms), "us_per_round": st, "rounds_per_s": 1e6 / st["mean"],
+           "realised_accept_mean": float(deltas.mean() - 1), "round_bytes": r_bytes,
+           "round_frac": r_bytes / st["mean"] / 1e3 / peak,
+           "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch}
+    run.close()
+    del run, inp, out
+    torch.cuda.empty_cache()
+    return rec
+
+
+def sweep_grid(WLM, dev, flush, rounds):
+    """The prefix x concurrency x accept-mean sweep (Qwen3-8B shapes): per point the
+    per-round time (median over the rounds after 3 untimed ones, an L2 flush before each)
+    and the drafter state bytes; flatness of the per-round time over the prefixes for
+    every (batch, accept mean). Prefixes of more than 4M rows in total run the chunked
+    prefill (32K rows per call)."""
+    import torch
+    import fixed_cost_drafter_b200 as F
+    peak, _ = hbm_peak()
+    points, flat = [], {}
+    for b in WLM.SWEEP_BATCHES:
+        for m in WLM.SWEEP_MEANS:
+            row = {}
+            for P in WLM.SWEEP_PREFIXES:
+                wl = WLM.sweep_point(P, b, m)
+                chunk = 32768 if P * b > 4 * 1024 * 1024 else None
+                run = WLM.DeviceRun(wl, device=dev, rounds=rounds, prefill_chunk=chunk)
+                run.prefill()
+                torch.cuda.synchronize()
+                torch.cuda.empty_cache()
+                inp = run.make_round_inputs(0, rounds)
+                out = run.new_out()
+                ms = time_rounds(run, inp, out, flush, rounds)
+                status, word = run.error()
+                if status != F.LS_OK:
+                    raise RuntimeError(f"device error word {word:#x} at sweep point {wl.name}")
+                deltas = run.accept_host[3:] + 1
+                st = us_stats(ms)
+                r_bytes = attend_bytes(wl) + commit_bytes(wl, float(deltas.mean()))
+                sb = F.ls_state_bytes(run.cfg)
+                points.append({"prefix": P, "batch": b, "accept_mean": m, "us_per_round": st["median"],
+                               "us_mean": st["mean"], "rounds": len(ms),
+                               "realised_accept_mean": float(deltas.mean() - 1),
+                               "round_frac": r_bytes / st["median"] / 1e3 / peak,
+                               "state_bytes": sb, "state_bytes_per_sequence": sb / b})
+                row[P] = st["median"]
+                run.close()
+                del run, inp, out
+                torch.cuda.empty_cache()
+            v = list(row.values())
+            flat[f"batch{b}_mean{m}"] = (max(v) - min(v)) / min(v)
+    return {"points": points, "flatness": flat, "rounds_per_point": rounds - 3,
+            "state_bytes_identical_across_prefixes": all(
+                len({p["state_bytes"] for p in points if p["batch"] == b}) == 1 for b in WLM.SWEEP_BATCHES)}
+
+
+def drafting_round_measure(WLM, wl, dev, flush, n, prefixes=None):
+    """The round a drafter runs with sampled decoding (T > 0): the stochastic acceptance of
+    the verified block (``ls_accept_sampled`` at the Qwen3 vocabulary), the commit of the
+    accepted rows (``ls_commit_accepted``), the drafter's projections of the new boundary
+    and of its block inputs (``ls_draft_prologue``, seeded weights) and the attention over
+    the views with those projections (``ls_draft_attend``), an L2 flush before each round.
+    Timed at the workload's prefix and, with ``prefixes``, at batch 16 over those prefixes
+    (flatness)."""
+    import torch
+    import fixed_cost_drafter_b200 as F
+    from dataclasses import replace
+    peak, _ = hbm_peak()
+    b, L, H, Hq, D, hid, B, V = (wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.hidden,
+                                 wl.block, QWEN3_VOCAB)
+    gen = torch.Generator(device=dev).manual_seed(20262)
+    zq = torch.randn((b, B, V), device=dev, generator=gen) * 2.0
+    qp = torch.softmax(zq, -1)
+    zp = torch.cat([zq, zq[:, -1:]], 1) + 0.5 * torch.randn((b, B + 1, V), device=dev, generator=gen)
+    pp = torch.softmax(zp, -1)
+    del zq, zp
+    draft = torch.multinomial(qp.view(-1, V), 1, generator=gen).view(b, B).to(torch.int32)
+    n_u = 8
+    us_draws = torch.rand((n_u, b, B + 1), device=dev, generator=gen)
+    w_kv = (torch.randn((L, 2 * H * D, hid), device=dev, generator=gen) * hid ** -0.5).to(torch.bfloat16)
+    w_q = (torch.randn((L, Hq * D, hid), device=dev, generator=gen) * hid ** -0.5).to(torch.bfloat16)
+    x = torch.randn((b, L, B, hid), device=dev, generator=gen).to(torch.bfloat16)
+    bkv = torch.empty((b, L, 2 * H * D), dtype=torch.bfloat16, device=dev)
+    qd = torch.empty((b, L, B, Hq * D), dtype=torch.bfloat16, device=dev)
+    acc = torch.empty(b, dtype=torch.int32, device=dev)
+    nxt = torch.empty(b, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+
+    def series(w, rounds):
+        run = WLM.DeviceRun(w, device=dev, rounds=rounds,
+                            prefill_chunk=32768 if int(np.max(w.prefix_lengths())) * w.batch > 4 * 1024 * 1024
+                            else None)
         run.prefill()
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
         inp = run.make_round_inputs(0, rounds)
         out = run.new_out()
-        ms = []
+        st = run.stream
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(rounds)]
+        a_seen = []
         for r in range(rounds):
             flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(run.stream)
-            run.round(inp, r, out)
-            e1.record(run.stream)
-            e1.synchronize()
-            if r >= 3:
-                ms.append(e0.elapsed_time(e1))
-        res[str(P)] = float(np.median(ms)) * 1e3
+            e = evs[r]
+            e[0].record(st)
+            F.ls_accept_sampled(run.state, draft, qp, pp, V, us_draws[r % n_u], acc, nxt, st)
+            e[1].record(st)
+            F.ls_commit_accepted(run.state, acc, inp["vk"][r], inp["vv"][r], inp["vh"][r], st)
+            e[2].record(st)
+            F.ls_draft_prologue(run.state, w_kv, w_q, x, bkv, qd, st)
+            e[3].record(st)
+            F.ls_draft_attend(run.state, 0, L, qd, bkv, bkv[..., H * D:], 2 * H * D, scale, out, st)
+            e[4].record(st)
+            if r < n_u:
+                a_seen.append(acc.clone())
+        torch.cuda.synchronize()
+        status, word = run.error()
+        if status != F.LS_OK:
+            raise RuntimeError(f"device error word {word:#x} in the drafting round")
+        warm = 3
+        tot = [e[0].elapsed_time(e[4]) for e in evs[warm:]]
+        parts = {k: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs[warm:]])) * 1e3
+                 for i, k in enumerate(("accept_sampled_us", "commit_accepted_us", "prologue_us", "attend_us"))}
+        a_all = torch.stack(a_seen).cpu().numpy()
+        rows = float(np.mean(np.where(a_all < B, 2, 1).sum(axis=1)))  # probability rows the draw reads
         run.close()
         del run, inp, out
         torch.cuda.empty_cache()
-    v = list(res.values())
-    return {"us_per_round": res, "flatness": (max(v) - min(v)) / min(v), "batch": 16, "accept_mean": 4.0}
+        return tot, parts, float(a_all.mean()), rows
+
+    tot, parts, a_mean, rows = series(wl, n)
+    nbytes = (int(b * 2 * B * 4 + b * (B + 1) * 4 + rows * V * 4)  # sampling: tests, draws, the drawn rows
+              + commit_bytes(wl, a_mean + 1)
+              + (w_kv.numel() + w_q.numel() + x.numel() + b * L * hid + bkv.numel() + qd.numel()) * 2
+              + attend_bytes(wl))
+    st = us_stats(tot)
+    res = {"kernels": "ls_accept_sampled -> ls_commit_accepted -> ls_draft_prologue -> ls_draft_attend",
+           "vocab": V, "us_per_round": st, "rounds_per_s": 1e6 / st["mean"], "rounds": len(tot), "split": parts,
+           "accept_mean": a_mean, "bytes": nbytes, "frac": nbytes / st["mean"] / 1e3 / peak, "launches_per_round": 4}
+    if prefixes:
+        by_p = {}
+        for P in prefixes:
+            t, _, _, _ = series(replace(wl, name=f"{wl.name}_p{P}", prefix=P), max(16, n // 4))
+            by_p[str(P)] = float(np.median(t)) * 1e3
+        v = list(by_p.values())
+        res["over_prefix"] = {"us_per_round_median": by_p, "flatness": (max(v) - min(v)) / min(v),
+                              "batch": wl.batch}
+    del qp, pp, w_kv, w_q, x
+    torch.cuda.empty_cache()
+    return res
 
 
 def main(argv=None):
@@ -877,7 +1150,10 @@ def main(argv=None):
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples ('{rank}' is replaced; default _build/clocks_rank{rank}.csv)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--sweep-rounds", type=int, default=40)
+    ap.add_argument("--sweep-rounds", type=int, default=128, help="rounds per sweep point (3 of them untimed)")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workload configurations")
+    ap.add_argument("--no-drafting-round", action="store_true",
+                    help="skip the drafting round with sampled acceptance and projections")
     ap.add_argument("--prefix", type=int, default=0, help="override the workload's prefix length")
     args = ap.parse_args(argv)
     if args.warmup < 3:

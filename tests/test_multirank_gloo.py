@@ -15,6 +15,8 @@ import torch.multiprocessing as mp
 
 import bench
 
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
 
 def _free_port():
     s = socket.socket()
@@ -83,3 +85,20 @@ def test_reference_arm_line(monkeypatch, capsys):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["metric"] == bench.METRIC
+    # whole rounds on every host core, and the same config dict the GPU arm prints
+    assert d["cpu_baseline"]["cores"] == min(bench.host_cores(), 64)
+    assert d["cpu_baseline"]["one_core"]["cores"] == 1 and d["cpu_baseline"]["one_core"]["value"] > 0
+    from synth.workloads import CONFIGS
+    assert d["config"] == bench.workload_config(CONFIGS[bench.WORKLOAD])
+
+
+def test_reference_arm_does_not_load_the_library():
+    """The oracle's timing runs in processes that never map the CUDA library."""
+    import subprocess
+    import sys
+    code = ("import sys; sys.argv = ['bench.py']; import bench; "
+            "assert bench.main(['--impl', 'reference', '--steps', '1', '--warmup', '3']) == 0; "
+            "maps = open('/proc/self/maps').read(); "
+            "assert 'liblongspark' not in maps and 'fixed_cost_drafter_b200' not in sys.modules, 'library loaded'")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]

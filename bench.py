@@ -89,6 +89,7 @@ def barrier(world):
 # algorithmic bytes (the layout built: bf16 window and mean rows, fp32 summary sums)
 # ---------------------------------------------------------------------------------------
 VIEW_BOUNDARY, VIEW_WINDOW, VIEW_SUMMARY, VIEW_ALL = 0x1, 0x2, 0x4, 0x7  # LS_VIEW_*
+LS_FLAG_OUT_F32 = 0x2
 
 # Table 5's component ablations: the views each variant keeps
 ABLATIONS = {"full": VIEW_ALL, "without_global_summary": VIEW_BOUNDARY | VIEW_WINDOW,
@@ -99,9 +100,10 @@ ABLATIONS = {"full": VIEW_ALL, "without_global_summary": VIEW_BOUNDARY | VIEW_WI
 def attend_bytes(wl, views: int = VIEW_ALL) -> int:
     """Algorithmic bytes of one attention launch over the given views."""
     e = wl.elem()
+    e_out = 4 if wl.flags & LS_FLAG_OUT_F32 else e
     b, L, H, Hq, D, B = wl.batch, wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.block
     summary_rows = len(wl.scales) * (wl.slots + 1) + 1
-    return (2 * b * L * B * Hq * D * e                                        # Q in, O out
+    return (b * L * B * Hq * D * (e + e_out)                                  # Q in, O out
             + (b * L * H * wl.window * 2 * D * e if views & VIEW_WINDOW else 0)  # ring window K/V
             + (b * L * H * summary_rows * 2 * D * e if views & VIEW_SUMMARY else 0)  # summary mean rows
             + (b * L * H * 2 * D * e if views & VIEW_BOUNDARY else 0)          # boundary K/V
@@ -400,8 +402,11 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
+    from dataclasses import replace
     from synth.workloads import CONFIGS
     wl = CONFIGS[args.config]
+    if args.out == "f32":  # (the oracle computes in fp64 either way; the config names the GPU's output)
+        wl = replace(wl, flags=wl.flags | LS_FLAG_OUT_F32)
     per_round, busy, n, workers = oracle_timing(wl.name, args.warmup, steps=args.steps)
     v = 1.0 / per_round
     line = {"metric": METRIC, "value": v, "unit": "rounds/s", "n_gpus": world, "steps": args.steps,
@@ -421,6 +426,7 @@ def workload_config(wl):
                         f"partials + global mean, prefix {wl.prefix}",
             "batch": wl.batch, "prefix": wl.prefix if not isinstance(wl.prefix, tuple) else list(wl.prefix),
             "accept_mean": wl.accept_mean,
+            "attention_output": "f32" if wl.flags & LS_FLAG_OUT_F32 else wl.dtype,
             "l2": "flushed before every timed round: 256 MB written then 256 MB read (untimed), "
                   "so the round starts cold with no dirty flush lines to write back"}
 
@@ -441,9 +447,11 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
+    from dataclasses import replace
     wl = WLM.CONFIGS[args.config]
+    if args.out == "f32":
+        wl = replace(wl, flags=wl.flags | F.LS_FLAG_OUT_F32)
     if args.prefix:  # profiling runs: same per-round work, smaller prefix to generate
-        from dataclasses import replace
         wl = replace(wl, prefix=args.prefix)
     K, W = args.steps, args.warmup
     # distinct rounds of generated inputs; the timed loop cycles through them (the state
@@ -566,27 +574,36 @@ def run_gpu(args):
         paged = paged_measure(WLM, wl, dev, flush, max(16, min(K, 200)), rank)
 
     # back-to-back rounds in one CUDA graph (no flush; L2 warm between rounds)
-    # the attention as a drafter calls it layer by layer (one launch per tapped layer)
+    # the attention as a drafter calls it layer by layer (one launch per tapped layer), with
+    # every layer's queries computed before the calls (as ls_draft_prologue computes them):
+    # LS_ATTEND_INPUTS_READY; and without the hint (inputs as if written just before each call)
     per_layer = None
     if not args.no_ablations:
         KP = min(K, 200)
-        pl_out = run.new_out(layer_count=1)
+        pl_outs = [run.new_out(layer_count=1) for _ in range(wl.n_layers)]
         rs = sorted({(W + i) % n_rounds for i in range(KP)})
         q_l = {r: [inp["q"][r - inp["r0"]][:, l:l + 1].contiguous() for l in range(wl.n_layers)] for r in rs}
-        ms = []
-        for i in range(KP):
-            r = (W + i) % n_rounds
-            flush.zero_()
-            evs[i][0].record(stream)
-            for l in range(wl.n_layers):
-                F.ls_draft_attend(run.state, l, 1, q_l[r][l], run.boundary_k, run.boundary_v, wl.hidden,
-                                  run.softmax_scale, pl_out, stream)
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-        ms = [e[0].elapsed_time(e[1]) for e in evs[:KP]]
-        per_layer = {"launches_per_round": wl.n_layers, "us_per_round": float(np.mean(ms)) * 1e3,
-                     "GBps": attend_bytes(wl) / (float(np.mean(ms)) * 1e3) / 1e3, "rounds": KP}
-        del q_l
+        peak, _ = hbm_peak()
+        per_layer = {"launches_per_round": wl.n_layers, "rounds": KP}
+        for key, views in (("inputs_ready", VIEW_ALL | F.LS_ATTEND_INPUTS_READY), ("inputs_written_before", VIEW_ALL)):
+            for i in range(KP):
+                r = (W + i) % n_rounds
+                flush.zero_()
+                evs[i][0].record(stream)
+                for l in range(wl.n_layers):
+                    F.ls_draft_attend_views(run.state, l, 1, q_l[r][l], run.boundary_k, run.boundary_v, wl.hidden,
+                                            run.softmax_scale, views, pl_outs[l], stream)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize()
+            us = float(np.mean([e[0].elapsed_time(e[1]) for e in evs[:KP]])) * 1e3
+            per_layer[key] = {"us_per_round": us, "GBps": attend_bytes(wl) / us / 1e3,
+                              "frac": attend_bytes(wl) / us / 1e3 / peak}
+        per_layer["us_per_round"] = per_layer["inputs_ready"]["us_per_round"]
+        per_layer["GBps"] = per_layer["inputs_ready"]["GBps"]
+        status, word = run.error()
+        if status != F.LS_OK:
+            raise RuntimeError(f"device error word {word:#x} after the per-layer launches")
+        del q_l, pl_outs
 
     graph_rps = None
     if not args.no_graph:
@@ -621,15 +638,21 @@ def run_gpu(args):
         drafting = drafting_round_measure(WLM, wl, dev, flush, max(16, min(K, 200)),
                                           WLM.SWEEP_PREFIXES if rank == 0 and not args.no_sweep else None)
 
+    # the same round with the attention output in the other dtype
+    other_out = None
+    if not args.no_configs and rank == 0 and not strong:
+        other_out = out_dtype_measure(WLM, wl, dev, flush, max(16, min(K, 200)), wl.flags ^ F.LS_FLAG_OUT_F32)
+
     # the other workload configurations, end to end (prefill and every round)
     configs = None
     if not args.no_configs and rank == 0 and not strong:
-        configs = {name: config_record(WLM, name, dev, flush, 0) for name in ("qwen3_4b_32k", "qwen3_8b_128k_ragged")}
+        configs = {name: config_record(WLM, name, dev, flush, 0, wl.flags & F.LS_FLAG_OUT_F32)
+                   for name in ("qwen3_4b_32k", "qwen3_8b_128k_ragged")}
 
     # the prefix x concurrency x accept-mean sweep; flatness over the prefixes
     grid, flat = None, None
     if not args.no_sweep and rank == 0:
-        grid = sweep_grid(WLM, dev, flush, args.sweep_rounds)
+        grid = sweep_grid(WLM, dev, flush, args.sweep_rounds, wl.flags & F.LS_FLAG_OUT_F32)
         b16 = {str(p["prefix"]): p["us_per_round"] for p in grid["points"] if p["batch"] == 16
                and p["accept_mean"] == 4.0}
         flat = {"us_per_round": b16, "flatness": grid["flatness"]["batch16_mean4.0"], "batch": 16,
@@ -680,6 +703,7 @@ def run_gpu(args):
                         "frac": prefill_b / (prefill_ms / 1e3) / 1e9 / peak},
             "state_bytes_per_sequence": F.ls_state_bytes(run.cfg) / wl.batch,
             "flatness": flat,
+            "other_output_dtype": other_out,
             "configs": configs,
             "sweep": grid,
             "drafting_round": drafting,
@@ -927,6 +951,46 @@ def e2e_measure(run, wl, dev, flush, steps, world, inp, strong=False):
             "d2h_bytes_per_step": int(d2h), "steps": steps, "pipelined": "2 buffer slots, copy streams in and out"}
 
 
+def out_dtype_measure(WLM, wl, dev, flush, n, flags):
+    """The workload's round (``ls_round``) and attention alone with the attention output in
+    the other dtype (``flags`` the state's flags for it), L2 flushed before each."""
+    import torch
+    import fixed_cost_drafter_b200 as F
+    from dataclasses import replace
+    peak, _ = hbm_peak()
+    w = replace(wl, flags=flags)
+    run = WLM.DeviceRun(w, device=dev, rounds=n)
+    run.prefill()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    inp = run.make_round_inputs(0, n)
+    out = run.new_out()
+    ms = time_rounds(run, inp, out, flush, n)
+    stream = run.stream
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for r in range(n):
+        flush.zero_()
+        evs[r][0].record(stream)
+        run.attend(inp, r, out)
+        evs[r][1].record(stream)
+    torch.cuda.synchronize()
+    status, word = run.error()
+    if status != F.LS_OK:
+        raise RuntimeError(f"device error word {word:#x} in the output-dtype measurement")
+    att = [e0.elapsed_time(e1) for e0, e1 in evs[3:]]
+    deltas = run.accept_host[3:] + 1
+    a_b = attend_bytes(w)
+    r_b = a_b + commit_bytes(w, float(deltas.mean()))
+    st, at = us_stats(ms), us_stats(att)
+    res = {"out_dtype": "f32" if flags & LS_FLAG_OUT_F32 else w.dtype, "us_per_round": st,
+           "round_frac": r_b / st["mean"] / 1e3 / peak, "attend_us": at,
+           "attend_frac": a_b / at["mean"] / 1e3 / peak, "attend_bytes": a_b, "rounds": len(ms)}
+    run.close()
+    del run, inp, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def time_rounds(run, inp, out, flush, n, warm=3):
     """CUDA-event times (ms) of rounds warm .. n - 1 of ``run`` (``ls_round``), each after an
     untimed L2 flush; rounds 0 .. warm - 1 run untimed first (they load the kernels)."""
@@ -947,14 +1011,16 @@ def us_stats(ms):
             "p90": float(np.percentile(ms, 90)) * 1e3}
 
 
-def config_record(WLM, name, dev, flush, rank):
+def config_record(WLM, name, dev, flush, rank, flags=0):
     """One of the workload configurations end to end: its prefill (after one untimed
     prefill into a state then reset) and all of its rounds (3 untimed), an L2 flush before
     each round."""
     import torch
     import fixed_cost_drafter_b200 as F
+    from dataclasses import replace
     peak, _ = hbm_peak()
     wl = WLM.CONFIGS[name]
+    wl = replace(wl, flags=wl.flags | flags)
     run = WLM.DeviceRun(wl, device=dev, seq_offset=sequence_offset(rank, wl.batch))
     run.prefill()
     run.reset_state()
@@ -988,7 +1054,7 @@ def config_record(WLM, name, dev, flush, rank):
     return rec
 
 
-def sweep_grid(WLM, dev, flush, rounds):
+def sweep_grid(WLM, dev, flush, rounds, flags=0):
     """The prefix x concurrency x accept-mean sweep (Qwen3-8B shapes): per point the
     per-round time (median over the rounds after 3 untimed ones, an L2 flush before each)
     and the drafter state bytes; flatness of the per-round time over the prefixes for
@@ -996,6 +1062,7 @@ def sweep_grid(WLM, dev, flush, rounds):
     prefill (32K rows per call)."""
     import torch
     import fixed_cost_drafter_b200 as F
+    from dataclasses import replace
     peak, _ = hbm_peak()
     points, flat = [], {}
     for b in WLM.SWEEP_BATCHES:
@@ -1003,6 +1070,7 @@ def sweep_grid(WLM, dev, flush, rounds):
             row = {}
             for P in WLM.SWEEP_PREFIXES:
                 wl = WLM.sweep_point(P, b, m)
+                wl = replace(wl, flags=wl.flags | flags)
                 chunk = 32768 if P * b > 4 * 1024 * 1024 else None
                 run = WLM.DeviceRun(wl, device=dev, rounds=rounds, prefill_chunk=chunk)
                 run.prefill()
@@ -1117,13 +1185,14 @@ def drafting_round_measure(WLM, wl, dev, flush, n, prefixes=None):
            "vocab": V, "us_per_round": st, "rounds_per_s": 1e6 / st["mean"], "rounds": len(tot), "split": parts,
            "accept_mean": a_mean, "bytes": nbytes, "frac": nbytes / st["mean"] / 1e3 / peak, "launches_per_round": 4}
     if prefixes:
-        by_p = {}
+        by_p, split_p = {}, {}
         for P in prefixes:
-            t, _, _, _ = series(replace(wl, name=f"{wl.name}_p{P}", prefix=P), max(16, n // 4))
+            t, parts_p, _, _ = series(replace(wl, name=f"{wl.name}_p{P}", prefix=P), max(16, n // 4))
             by_p[str(P)] = float(np.median(t)) * 1e3
+            split_p[str(P)] = parts_p
         v = list(by_p.values())
         res["over_prefix"] = {"us_per_round_median": by_p, "flatness": (max(v) - min(v)) / min(v),
-                              "batch": wl.batch}
+                              "batch": wl.batch, "split": split_p}
     del qp, pp, w_kv, w_q, x
     torch.cuda.empty_cache()
     return res
@@ -1155,6 +1224,7 @@ def main(argv=None):
     ap.add_argument("--no-drafting-round", action="store_true",
                     help="skip the drafting round with sampled acceptance and projections")
     ap.add_argument("--prefix", type=int, default=0, help="override the workload's prefix length")
+    ap.add_argument("--out", default="bf16", choices=["bf16", "f32"], help="dtype of the attention output")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

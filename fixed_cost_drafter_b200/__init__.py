@@ -39,6 +39,7 @@ LS_VIEW_BOUNDARY = 0x1
 LS_VIEW_WINDOW = 0x2
 LS_VIEW_SUMMARY = 0x4
 LS_VIEW_ALL = 0x7
+LS_ATTEND_INPUTS_READY = 0x100
 
 EXPORTED = (
     "ls_state_bytes", "ls_get_layout", "ls_init_state", "ls_prefill_workspace_bytes",

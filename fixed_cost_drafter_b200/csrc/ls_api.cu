@@ -45,6 +45,12 @@ struct ls_state {
   int sms;
   int use_tc;
   ls::TcPlan tc;
+  // No call has written the views since a tensor-core attention was launched on
+  // settled_stream: an attention launched next on that stream may load its first K/V
+  // chunks before its grid dependency wait (ls::kAttendViewsSettled).
+  // (kept by the calls that only read the state too: mutable)
+  mutable int views_settled;
+  mutable cudaStream_t settled_stream;
 };
 
 namespace {
@@ -248,6 +254,7 @@ int ls_prefill_summary(ls_state* st, const void* d_k, const void* d_v, int64_t p
                        size_t workspace_bytes, cudaStream_t stream) {
   if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   const ls_config& c = st->cfg;
   if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
   if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
@@ -271,6 +278,7 @@ int ls_prefill_summary_noalloc(ls_state* st, const void* d_k, const void* d_v, i
                                int64_t row_end, const void* d_last_hidden, cudaStream_t stream) {
   if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   const ls_config& c = st->cfg;
   if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
   if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
@@ -296,6 +304,7 @@ int ls_prefill_paged(ls_state* st, const ls_paged_kv* h_kv, const int64_t* d_pre
                      cudaStream_t stream) {
   if (!st || !d_prefix_len) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   const ls_config& c = st->cfg;
   if (row_begin < 0 || row_end < row_begin) return LS_ERR_INVALID_ARG;
   if (row_begin % c.scales[c.n_scales - 1] != 0) return LS_ERR_SHAPE;
@@ -324,6 +333,7 @@ int ls_commit_round_paged(ls_state* st, const int32_t* d_draft_ids, const int32_
   if (!st || !d_draft_ids || !d_target_ids || !d_verify_hidden || !d_accept_len || !d_next_token)
     return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   const int v = validate_paged(st->cfg, h_kv);
   if (v != LS_OK) return v;
   if (!aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
@@ -335,6 +345,7 @@ int ls_commit_accepted_paged(ls_state* st, const int32_t* d_accept_len, const ls
                              const void* d_verify_hidden, cudaStream_t stream) {
   if (!st || !d_accept_len || !d_verify_hidden) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   const int v = validate_paged(st->cfg, h_kv);
   if (v != LS_OK) return v;
   if (!aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
@@ -349,6 +360,7 @@ int ls_commit_round(ls_state* st, const int32_t* d_draft_ids, const int32_t* d_t
       !d_accept_len || !d_next_token)
     return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden))
     return LS_ERR_INVALID_ARG;
   return cuda_status(ls::launch_commit(st->dev, d_draft_ids, d_target_ids, d_verify_k, d_verify_v,
@@ -383,6 +395,7 @@ int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const void* d_
                        const void* d_verify_hidden, cudaStream_t stream) {
   if (!st || !d_accept_len || !d_verify_k || !d_verify_v || !d_verify_hidden) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   if (!aligned16(d_verify_k) || !aligned16(d_verify_v) || !aligned16(d_verify_hidden)) return LS_ERR_INVALID_ARG;
   return cuda_status(ls::launch_commit(st->dev, nullptr, nullptr, d_verify_k, d_verify_v, d_verify_hidden, nullptr,
                                        nullptr, d_accept_len, stream));
@@ -400,6 +413,8 @@ int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer
                           float softmax_scale, int32_t views, void* d_out, cudaStream_t stream) {
   if (!st || !d_q || !d_boundary_k || !d_boundary_v || !d_out) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  const bool inputs_ready = (views & LS_ATTEND_INPUTS_READY) != 0;
+  views &= ~LS_ATTEND_INPUTS_READY;
   if (views == 0 || (views & ~LS_VIEW_ALL)) return LS_ERR_INVALID_ARG;
   const ls_config& c = st->cfg;
   if (layer_begin < 0 || layer_count < 1 || layer_begin + layer_count > c.n_layers)
@@ -409,10 +424,22 @@ int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer
   if (!(softmax_scale > 0.0f) || softmax_scale == INFINITY) return LS_ERR_INVALID_ARG;
   if (!aligned16(d_q) || !aligned16(d_out) || !aligned16(d_boundary_k) || !aligned16(d_boundary_v))
     return LS_ERR_INVALID_ARG;
-  if (st->use_tc)
-    return cuda_status(ls::launch_attend_tc(st->dev, st->tc, layer_begin, layer_count, d_q,
-                                            d_boundary_k, d_boundary_v, boundary_stride,
-                                            softmax_scale, views, d_out, st->sms, false, stream));
+  if (st->use_tc) {
+    // inside a stream capture the order of later replays is not known: no early loads
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return LS_ERR_CUDA;
+    const bool settled = st->views_settled && st->settled_stream == stream && cap == cudaStreamCaptureStatusNone;
+    const ls::AttendLaunch mode = settled ? (inputs_ready ? ls::kAttendFree : ls::kAttendViewsSettled)
+                                          : (inputs_ready ? ls::kAttendAfterCommit : ls::kAttendPlain);
+    const int r = cuda_status(ls::launch_attend_tc(st->dev, st->tc, layer_begin, layer_count, d_q, d_boundary_k,
+                                                   d_boundary_v, boundary_stride, softmax_scale, views, d_out,
+                                                   st->sms, mode, stream));
+    if (r == LS_OK) {
+      st->views_settled = 1;
+      st->settled_stream = stream;
+    }
+    return r;
+  }
   return cuda_status(ls::launch_attend_simt(st->dev, layer_begin, layer_count, d_q, d_boundary_k,
                                             d_boundary_v, boundary_stride, softmax_scale, views, d_out,
                                             stream));
@@ -455,10 +482,16 @@ int round_attend(ls_state* st, const void* d_q, int64_t boundary_k_offset, int64
   const ls_config& c = st->cfg;
   const char* bnd = static_cast<const char*>(st->dev.boundary);
   const int64_t e = st->lay.elem;
-  if (st->use_tc)  // the attention kernel is scheduled while the commit runs
-    return cuda_status(ls::launch_attend_tc(st->dev, st->tc, 0, c.n_layers, d_q, bnd + boundary_k_offset * e,
-                                            bnd + boundary_v_offset * e, c.hidden, softmax_scale, LS_VIEW_ALL,
-                                            d_out, st->sms, true, stream));
+  if (st->use_tc) {  // the attention kernel is scheduled while the commit runs
+    const int r = cuda_status(ls::launch_attend_tc(st->dev, st->tc, 0, c.n_layers, d_q, bnd + boundary_k_offset * e,
+                                                   bnd + boundary_v_offset * e, c.hidden, softmax_scale, LS_VIEW_ALL,
+                                                   d_out, st->sms, ls::kAttendAfterCommit, stream));
+    if (r == LS_OK) {
+      st->views_settled = 1;
+      st->settled_stream = stream;
+    }
+    return r;
+  }
   return ls_draft_attend(st, 0, c.n_layers, d_q, bnd + boundary_k_offset * e, bnd + boundary_v_offset * e, c.hidden,
                          softmax_scale, d_out, stream);
 }
@@ -492,6 +525,7 @@ int ls_get_error(const ls_state* st, int32_t* h_code) {
 int ls_clear_error(ls_state* st, cudaStream_t stream) {
   if (!st) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
+  st->views_settled = 0;  // this call writes the views
   // the error word, and the arrival counts a call that gave up part-way may have left
   // (they are zero between completed calls): the commit's, the sampler's, the projections'
   const ls::Layout& y = st->lay;

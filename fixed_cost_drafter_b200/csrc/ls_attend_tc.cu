@@ -43,10 +43,16 @@
 //             TMA tensor store, so no global store instruction competes with the softmax's
 //             exp2 for the SM sub-partitions' shared-function queue. Warp 8 also turns the
 //             counters of the tile two ahead into the key masks of its chunks.
-// ls_round launches this kernel programmatically dependent on the commit kernel: it is
-// scheduled while the commit runs, allocates TMEM, sets up its barriers and issues the
-// first tile's Q (complete before the commit started), then waits on the device
-// (griddepcontrol.wait) for the commit's writes before it reads any state.
+// Every launch is programmatically dependent on the kernel before it on the stream: the
+// kernel allocates TMEM and sets up its barriers, then every thread waits on the device
+// (griddepcontrol.wait) before it reads what that kernel may have written, and triggers
+// its own dependents right after the wait (so a kernel launched behind this one starts
+// only once the kernel before this one has completed). ls_round launches it behind the
+// commit kernel, whose trigger comes once its loads are in flight: the first tile's Q
+// (complete before the commit started) is loaded before the wait. When no call has
+// written the views since an attention launched on the same stream (a drafter's
+// per-layer calls), the producers issue the first tile's first K/V chunks before the
+// wait, so one launch's pipeline fills while the launch before it drains.
 // Every wait is bounded and warp-uniform; a wait that runs out sets
 // LS_DEVERR_WAIT_TIMEOUT, all roles stop, the copies in flight land, TMEM is freed.
 #include <cuda.h>
@@ -84,6 +90,7 @@ struct TcArgs {
   int32_t views;         // LS_VIEW_* taking part in the softmax
   uint32_t chunk_mask;   // bit c: chunk c is streamed (the last chunk always is)
   int32_t tail_load;     // the last chunk's arena rows are loaded (else only its boundary row)
+  int32_t mode;          // AttendLaunch: what may be read before the grid dependency wait
 };
 
 // Chunks streamed after chunk c (c = -1: the first one): nC or more when none is left.
@@ -251,6 +258,14 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  // Every thread passes the grid dependency wait before it triggers this grid's dependents;
+  // the producers (warps 0, 6) and the mask warp (8) do both in their roles, after what
+  // they may read before the wait. The other roles need data only those roles bring.
+  const bool no_wait = a.mode == kAttendFree;  // nothing this kernel reads is the kernel before's
+  if (warp != 0 && warp != 6 && warp != 8) {
+    if (!no_wait) grid_dependency_wait();
+    allow_dependent_launch();
+  }
   int issued = 0;  // producers: loads issued into their ring (for the drain after an abort)
   auto chunk_rows = [&](int c) { return c == nC - 1 ? last_rows : kChunk; };
 
@@ -270,25 +285,64 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       if (tail > 0) prefetch_map(&kv_tail_map);
       if (is_k) prefetch_map(&q_map);
     }
-    if (!is_k) grid_dependency_wait();
     const int grp = p.Hq / p.Hkv;
+    // Q of item i into its buffer (the K producer's job)
+    auto load_q = [&](int i, int b, int lc, int g) -> bool {
+      const int qb = i & 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_empty[qb], ((i >> 1) & 1) ^ 1, p.err))) return false;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&s.q_full[qb], kQBytes);
+        const int zrow = (b * a.lcount + lc) * p.B;
+        tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
+        tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
+      }
+      return true;
+    };
+    // one chunk's arena rows into stage st (lane 0 issues)
+    auto load_chunk = [&](int64_t tile, int c, int st) {
+      if (lane == 0) {
+        const bool last = c == nC - 1;
+        const int rows = last ? (a.tail_load ? tail : 0) : kChunk;
+        mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
+        if (rows > 0) {
+          const CUtensorMap* m = last ? &kv_tail_map : &kv_map;
+          const int y = int((tile * 2 + (is_k ? 0 : 1)) * p.R + int64_t(c) * kChunk);
+          unsigned char* dst = ring + st * kStageBytes;
+          tma_load_2d(dst, m, 0, y, &fullb[st]);
+          tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
+        }
+      }
+    };
     bool ok = true;
+    int pre = 0;  // chunks of the first tile issued before the grid dependency wait
+    if (a.mode == kAttendViewsSettled && n_items > 0) {
+      // the views are complete: the first tile's chunks that fit the empty ring (the last
+      // chunk waits: it carries the caller's boundary row)
+      int b, lc, g;
+      tile_coords(item_tile(0), p, a.lcount, b, lc, g);
+      const int64_t tile = (int64_t(b) * p.L + (a.lb + lc)) * p.Hkv + g;
+      for (int c = c_first; c < nC - 1 && pre < nst; c = next_chunk(a.chunk_mask, c)) {
+        load_chunk(tile, c, pre);  // stage `pre`: the ring is empty at the start
+        ++pre;
+        ++issued;
+      }
+    }
+    if (is_k && a.mode == kAttendAfterCommit && n_items > 0) {
+      // Q is an input complete before the commit started; the boundary rows and the
+      // arena are state the commit writes
+      int b, lc, g;
+      tile_coords(item_tile(0), p, a.lcount, b, lc, g);
+      ok = load_q(0, b, lc, g);
+    }
+    if (!no_wait) grid_dependency_wait();
+    allow_dependent_launch();
     int k = 0;  // chunks of this CTA so far: ring stage and phase
     for (int i = 0; i < n_items && ok; ++i) {
       int b, lc, g;
       tile_coords(item_tile(i), p, a.lcount, b, lc, g);
       const int64_t tile = (int64_t(b) * p.L + (a.lb + lc)) * p.Hkv + g;
-      if (is_k) {  // Q of the item first
-        const int qb = i & 1;
-        if (!__all_sync(0xffffffffu, wait_or_abort(s, &s.q_empty[qb], ((i >> 1) & 1) ^ 1, p.err))) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&s.q_full[qb], kQBytes);
-          const int zrow = (b * a.lcount + lc) * p.B;
-          tma_load_3d(q_buf + qb * kQBytes, &q_map, 0, g * grp, zrow, &s.q_full[qb]);
-          tma_load_3d(q_buf + qb * kQBytes + kQBytes / 2, &q_map, 64, g * grp, zrow, &s.q_full[qb]);
-        }
-        // Q is an input; the boundary rows and the arena are state a preceding commit writes
-        if (i == 0) grid_dependency_wait();
+      if (is_k && !(i == 0 && a.mode == kAttendAfterCommit)) {  // Q of the item first
+        if (!load_q(i, b, lc, g)) break;
       }
       // the boundary row is loaded once the tile's first chunk is on its way (its latency
       // then overlaps the stream), or before a one-chunk tile's only chunk
@@ -296,9 +350,13 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
       uint4 brow = make_uint4(0, 0, 0, 0);
       for (int c = c_first; c < nC; c = next_chunk(a.chunk_mask, c), ++k) {
         const int st = k % nst;
+        const bool last = c == nC - 1;
+        if (k < pre) {  // issued before the wait
+          if (c == c_first && !last && lane < 16) brow = ld_nc_v4(bptr);
+          continue;
+        }
         if (!__all_sync(0xffffffffu, wait_or_abort(s, &emptyb[st], ((k / nst) & 1) ^ 1, p.err))) { ok = false; break; }
         unsigned char* dst = ring + st * kStageBytes;
-        const bool last = c == nC - 1;
         if (last) {  // the boundary row, row `tail` of the stage
           if (c == c_first && lane < 16) brow = ld_nc_v4(bptr);
           if (lane < 16)
@@ -307,16 +365,7 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
           fence_proxy_async_smem();
           __syncwarp();
         }
-        if (lane == 0) {
-          const int rows = last ? (a.tail_load ? tail : 0) : kChunk;
-          mbar_arrive_expect_tx(&fullb[st], uint32_t(rows * 256));
-          if (rows > 0) {
-            const CUtensorMap* m = last ? &kv_tail_map : &kv_map;
-            const int y = int((tile * 2 + (is_k ? 0 : 1)) * p.R + int64_t(c) * kChunk);
-            tma_load_2d(dst, m, 0, y, &fullb[st]);
-            tma_load_2d(dst + kStageBytes / 2, m, 64, y, &fullb[st]);
-          }
-        }
+        load_chunk(tile, c, st);
         if (c == c_first && !last && lane < 16) brow = ld_nc_v4(bptr);
         ++issued;
       }
@@ -513,10 +562,20 @@ attend_tc_kernel(const Dev p, const TcArgs a, const __grid_constant__ CUtensorMa
             view_mask(p, 64 * lane, len < p.W ? int(len) : p.W, sinfo, len > 0, a.views);
     };
     if (warp == 8) {
-      grid_dependency_wait();  // the counters are state a preceding commit writes
+      // the counters are state a commit before this kernel writes, unless the views are
+      // settled
+      const bool early = a.mode == kAttendViewsSettled || no_wait;
+      if (!early) {
+        grid_dependency_wait();
+        allow_dependent_launch();
+      }
       for (int i = 0; i < 2 && i < n_items; ++i) {
         fill_masks(i);
         mbar_arrive(&s.info_full[i]);
+      }
+      if (early) {
+        if (!no_wait) grid_dependency_wait();
+        allow_dependent_launch();
       }
     }
     for (int i = 0; i < n_items; ++i) {
@@ -640,7 +699,7 @@ int tc_prepare(const Dev& p, TcPlan* plan) {
 
 cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
                              const void* bk, const void* bv, int64_t bstride, float scale, int views,
-                             void* out, int sms, bool after_commit, cudaStream_t stream) {
+                             void* out, int sms, AttendLaunch mode, cudaStream_t stream) {
   // Q in, and a bf16 O out, are [b, lcount, B, Hq, D]: one tile is the box (64 columns,
   // the group's heads, the block's queries) at (0 or 64, g * group, first query)
   CUtensorMap qmap, omap;
@@ -660,6 +719,7 @@ cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcoun
   a.bstride = bstride;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = out;
+  a.mode = mode;
   // chunks holding rows of a view that takes part are streamed; the last chunk always is
   // (it carries the boundary row), its arena rows only when a view needs them
   a.views = views;
@@ -685,13 +745,12 @@ cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcoun
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
+  // scheduled once the kernel before it on `stream` triggers or completes (see AttendLaunch)
   cudaLaunchAttribute attr[1];
-  if (after_commit) {  // scheduled while the commit kernel just launched on `stream` runs
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   const CUtensorMap& kv = *reinterpret_cast<const CUtensorMap*>(plan.kv_map);
   const CUtensorMap& kv_tail = *reinterpret_cast<const CUtensorMap*>(plan.kv_tail_map);
   return p.out_f32 ? cudaLaunchKernelEx(&cfg, attend_tc_kernel<true>, p, a, kv, kv_tail, qmap, omap)

@@ -15,11 +15,24 @@ struct alignas(64) TcPlan {
 
 bool tc_supported(const Dev& p);
 int tc_prepare(const Dev& p, TcPlan* plan);
-// after_commit: launched right behind ls_commit_round's kernel on the same stream as its
-// programmatic dependent (the kernel waits on the device for the commit's writes).
+// The kernel is always launched as the programmatic dependent of the kernel before it on
+// `stream`: its threads wait on the device (griddepcontrol.wait) before they read what that
+// kernel may write, and trigger their own dependents right after that wait. What may be
+// read before the wait depends on what the caller knows about the kernel before it:
+enum AttendLaunch : int {
+  kAttendPlain = 0,        // nothing: every input after the wait
+  kAttendAfterCommit = 1,  // the first tile's Q before the wait: an input complete before
+                           // that kernel started (it is this state's commit kernel, or the
+                           // caller says so with LS_ATTEND_INPUTS_READY)
+  kAttendViewsSettled = 2, // no call has written the views since an attention launched on
+                           // this stream: the first K/V chunks of the views before the wait
+                           // (Q and the boundary rows after it)
+  kAttendFree = 3          // settled views, and the caller's inputs were complete before the
+                           // kernel before it started (LS_ATTEND_INPUTS_READY): no wait
+};
 // views: non-zero OR of LS_VIEW_* (the views that take part in the softmax).
 cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
                              const void* bk, const void* bv, int64_t bstride, float scale, int views,
-                             void* out, int sms, bool after_commit, cudaStream_t stream);
+                             void* out, int sms, AttendLaunch mode, cudaStream_t stream);
 
 }  // namespace ls

@@ -87,6 +87,14 @@ extern "C" {
 #define LS_VIEW_SUMMARY  0x4        /* the global context summary (segment means per
                                        scale, partial means, global mean)             */
 #define LS_VIEW_ALL      0x7
+/* Launch hint for ls_draft_attend_views, OR-ed into `views`: the call's queries and
+ * boundary rows were complete before the kernel launched just before this call on
+ * `stream` started, and that kernel neither reads nor writes d_out (e.g. the drafter's
+ * queries of every layer came from one earlier ls_draft_prologue, and the attention is
+ * called layer by layer). The attention may then read those inputs, and write d_out,
+ * while that kernel still runs, so consecutive per-layer calls overlap. A hint that
+ * does not hold gives wrong outputs (never a fault).                                  */
+#define LS_ATTEND_INPUTS_READY 0x100
 
 /* ---- dtypes and flags -------------------------------------------------------- */
 #define LS_F32  0
@@ -317,7 +325,13 @@ LS_API int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const v
  *                  with l the absolute layer; boundary_stride >= Hkv*D, multiple of 8.
  *   softmax_scale  logit multiplier, finite and > 0 (1/sqrt(D) for the usual attention).
  * Uses the tcgen05 tensor-core kernel when dtype is bf16, (Hq/Hkv)*B == 64, D == 128 and
- * kv_rows <= 768 (unless LS_FLAG_FORCE_SIMT), otherwise a CUDA-core kernel.          */
+ * kv_rows <= 768 (unless LS_FLAG_FORCE_SIMT), otherwise a CUDA-core kernel. The
+ * tensor-core kernel is launched as the programmatic dependent of the kernel before it
+ * on `stream`: it reads the inputs that kernel may write only once that kernel has
+ * completed. When no call has written this state's views since an attention was launched
+ * on the same stream (per-layer calls), it loads its first rows of the views before that,
+ * so one call's start overlaps the end of the call before it. Inside a stream capture it
+ * does not (the order of the graph's replays is not known when it is captured).       */
 LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count,
                     const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
                     int64_t boundary_stride, float softmax_scale, void* d_out,
@@ -329,8 +343,9 @@ LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t laye
  * no part in the softmax, and the kernels do not read them where whole 128-row chunks
  * (or the summary rows of the last chunk) belong to left-out views. A query row whose
  * remaining views hold no valid row (e.g. the window alone before the first commit)
- * gets an all-zero output. Other arguments and errors as ls_draft_attend;
- * LS_ERR_INVALID_ARG when `views` is 0 or has bits outside LS_VIEW_ALL.            */
+ * gets an all-zero output. `views` may also hold LS_ATTEND_INPUTS_READY. Other
+ * arguments and errors as ls_draft_attend; LS_ERR_INVALID_ARG when `views` names no
+ * view or has bits outside LS_VIEW_ALL | LS_ATTEND_INPUTS_READY.                    */
 LS_API int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer_count,
                                  const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
                                  int64_t boundary_stride, float softmax_scale, int32_t views,

@@ -145,3 +145,17 @@ def test_make_paged_kv_descriptor():
         F.make_paged_kv([0x10] * (F.LS_MAX_PAGED_LAYERS + 1), [0x10] * (F.LS_MAX_PAGED_LAYERS + 1), 0, 256, 1, 1, 1, 1)
     with pytest.raises(ValueError):
         F.make_paged_kv([0x10, 0x20], [0x10], 0, 256, 1, 1, 1, 1)
+
+
+def test_binding_constants_match_the_header():
+    """Every LS_* integer constant the binding defines has the header's value."""
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "include", "longspark.h")) as f:
+        text = f.read()
+    found = 0
+    for name, val in re.findall(r"^#define\s+(LS_[A-Z0-9_]+)\s+\(?(-?(?:0x[0-9a-fA-F]+|\d+))\)?", text, re.M):
+        if hasattr(F, name):
+            assert getattr(F, name) == int(val, 0), name
+            found += 1
+    assert found >= 20 and F.LS_ATTEND_INPUTS_READY == 0x100

@@ -207,6 +207,127 @@ def test_per_layer_calls_match_one_call():
         assert torch.equal(one[:, 0], full[:, l])
 
 
+def test_per_layer_calls_back_to_back_match_one_call():
+    """Per-layer calls issued back to back, with no synchronisation: nothing writes the
+    views between them, so each launch loads its first K/V chunks before the launch ahead
+    of it has completed. They give the bits of one call over all layers."""
+    wl = _mid(rounds=3)
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    inp = run.make_round_inputs()
+    for r in range(3):
+        run.commit(inp, r)
+    full = run.new_out()
+    run.attend(inp, 2, full)
+    torch.cuda.synchronize()
+    ones = [run.new_out(1) for _ in range(wl.n_layers)]
+    for rep in range(2):
+        for l in range(wl.n_layers):
+            ones[l].fill_(float("nan"))
+        for l in range(wl.n_layers):
+            run.attend(inp, 2, ones[l], layer_begin=l, layer_count=1)
+        torch.cuda.synchronize()
+        for l in range(wl.n_layers):
+            assert torch.equal(ones[l][:, 0], full[:, l]), (rep, l)
+    assert run.error() == (F.LS_OK, 0)
+
+
+def test_per_layer_calls_with_inputs_ready_hint():
+    """LS_ATTEND_INPUTS_READY (every layer's queries computed before the calls): the first
+    per-layer call right after a commit reads its queries before the commit has completed
+    (the views only after), the next ones do not wait for the call before them at all.
+    Same bits as one call over all layers on a twin state; repeated back to back."""
+    wl = _mid(rounds=3)
+    runs = [WL.DeviceRun(wl), WL.DeviceRun(wl)]
+    for run in runs:
+        run.prefill()
+    inp = runs[0].make_round_inputs()
+    for run in runs:
+        for r in range(3):
+            run.commit(inp, r)
+    full = runs[1].new_out()
+    runs[1].attend(inp, 2, full)
+    a = runs[0]
+    a.commit(inp, 2)  # (both states get a third commit of the same round: still equal)
+    runs[1].commit(inp, 2)
+    runs[1].attend(inp, 2, full)
+    torch.cuda.synchronize()
+    qs = [inp["q"][2][:, l:l + 1].contiguous() for l in range(wl.n_layers)]
+    ones = [a.new_out(1) for _ in range(wl.n_layers)]
+    hint = F.LS_VIEW_ALL | F.LS_ATTEND_INPUTS_READY
+    for rep in range(3):
+        for o in ones:
+            o.fill_(float("nan"))
+        if rep == 2:
+            a.commit(inp, 2)
+            runs[1].commit(inp, 2)
+            runs[1].attend(inp, 2, full)
+        for l in range(wl.n_layers):
+            F.ls_draft_attend_views(a.state, l, 1, qs[l], a.boundary_k, a.boundary_v, wl.hidden, a.softmax_scale,
+                                    hint, ones[l], a.stream)
+        torch.cuda.synchronize()
+        for l in range(wl.n_layers):
+            assert torch.equal(ones[l][:, 0], full[:, l]), (rep, l)
+    assert a.error() == (F.LS_OK, 0) and runs[1].error() == (F.LS_OK, 0)
+    with pytest.raises(F.LsError):  # the hint alone names no view
+        F.ls_draft_attend_views(a.state, 0, 1, qs[0], a.boundary_k, a.boundary_v, wl.hidden, a.softmax_scale,
+                                F.LS_ATTEND_INPUTS_READY, ones[0], a.stream)
+
+
+def test_attention_reads_the_previous_attentions_output():
+    """Two attentions back to back, the second taking the first's output as its queries:
+    the second launch may start before the first completes (its early loads are of the
+    unchanged views only), but its queries are read after the first has completed. Same
+    bits as the two calls with a synchronisation between them. Against the oracle with
+    those queries through a state with fp32 outputs: these queries concentrate the softmax
+    enough for outputs above 4, where a bf16 output's own rounding (up to 2^-5 / 2) would
+    exceed the 1e-2 bound by itself."""
+    wl = _mid(rounds=2)
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    inp = run.make_round_inputs()
+    for r in range(2):
+        run.commit(inp, r)
+    q = inp["q"][1]
+    L, H, D = wl.n_layers, wl.n_kv_heads, wl.head_dim
+    args = (run.boundary_k, run.boundary_v, wl.hidden, run.softmax_scale)
+    o1, o2 = run.new_out(), run.new_out()
+    F.ls_draft_attend(run.state, 0, L, q, *args, o1, run.stream)
+    F.ls_draft_attend(run.state, 0, L, o1, *args, o2, run.stream)
+    torch.cuda.synchronize()
+    r1, r2 = run.new_out(), run.new_out()
+    F.ls_draft_attend(run.state, 0, L, q, *args, r1, run.stream)
+    torch.cuda.synchronize()
+    q2 = r1.clone()
+    torch.cuda.synchronize()
+    F.ls_draft_attend(run.state, 0, L, q2, *args, r2, run.stream)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, r1) and torch.equal(o2, r2)
+    wl32 = _mid(rounds=2, flags=F.LS_FLAG_OUT_F32)
+    run32 = WL.DeviceRun(wl32)
+    run32.prefill()
+    for r in range(2):
+        run32.commit(inp, r)
+    o32 = run32.new_out()
+    F.ls_draft_attend(run32.state, 0, L, q2, run32.boundary_k, run32.boundary_v, wl.hidden, run32.softmax_scale,
+                      o32, run32.stream)
+    torch.cuda.synchronize()
+    st = run.read_state()
+    assert all(np.array_equal(st[k], v) for k, v in run32.read_state().items())
+    draft, target = run.draft.cpu().numpy(), run.target.cpu().numpy()
+    acc = OS.accepts_from_ids(draft[:2], target[:2])
+    q2h = O.to_f64(q2.view(torch.int16).cpu().numpy().view(np.uint16), "bf16")
+    for b, l, g in [(b, l, g) for b in range(wl.batch) for l in range(L) for g in range(H)]:
+        sh, views = OS.tile_views(wl, b, l, g, int(run.prefix_len[b]), acc[:, b], run.scale_host)
+        hv = O.to_f64(st["boundary"][b, l], "bf16")
+        bk = hv[g * D:(g + 1) * D].reshape(1, 1, D)
+        bv = hv[H * D + g * D:H * D + (g + 1) * D].reshape(1, 1, D)
+        qt = q2h[b, l].reshape(wl.block, wl.n_q_heads, D)[:, g * wl.group:(g + 1) * wl.group][None]
+        ref = O.draft_attend(sh, views, qt, bk, bv, 1.0 / np.sqrt(D))[0]
+        assert OS.attend_error_excess(_out_tile(o32, wl, b, l, g), ref) <= 0
+    assert run.error() == (F.LS_OK, 0) and run32.error() == (F.LS_OK, 0)
+
+
 def test_chunked_prefill_matches_oracle():
     wl = _mid(rounds=6, prefix=(700, 1337), flags=F.LS_FLAG_OUT_F32)
     run = WL.DeviceRun(wl, prefill_chunk=256)

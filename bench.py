@@ -1135,9 +1135,11 @@ def drafting_round_measure(WLM, wl, dev, flush, n, prefixes=None):
     scale = 1.0 / math.sqrt(D)
 
     def series(w, rounds):
-        run = WLM.DeviceRun(w, device=dev, rounds=rounds,
-                            prefill_chunk=32768 if int(np.max(w.prefix_lengths())) * w.batch > 4 * 1024 * 1024
-                            else None)
+        # prefill in 8192-row chunks: freeing one large prefix buffer (34 GB at 128K) right
+        # before the timed rounds took the launch overlap away from most rounds (a driver
+        # state after a large free, not the round's work: the same rounds with 40 GB freed
+        # just before were as slow at a 4K prefix, and as fast with it held)
+        run = WLM.DeviceRun(w, device=dev, rounds=rounds, prefill_chunk=8192)
         run.prefill()
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
@@ -1146,17 +1148,27 @@ def drafting_round_measure(WLM, wl, dev, flush, n, prefixes=None):
         st = run.stream
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(rounds)]
         a_seen = []
+
+        def one_round(r, e=None):
+            # events between the calls (the split) serialise them: the chained time is
+            # taken without them
+            F.ls_accept_sampled(run.state, draft, qp, pp, V, us_draws[r % n_u], acc, nxt, st)
+            if e is not None:
+                e[1].record(st)
+            F.ls_commit_accepted(run.state, acc, inp["vk"][r], inp["vv"][r], inp["vh"][r], st)
+            if e is not None:
+                e[2].record(st)
+            F.ls_draft_prologue(run.state, w_kv, w_q, x, bkv, qd, st)
+            if e is not None:
+                e[3].record(st)
+            F.ls_draft_attend(run.state, 0, L, qd, bkv, bkv[..., H * D:], 2 * H * D, scale, out, st)
+
+        half = rounds // 2
         for r in range(rounds):
             flush.zero_()
             e = evs[r]
             e[0].record(st)
-            F.ls_accept_sampled(run.state, draft, qp, pp, V, us_draws[r % n_u], acc, nxt, st)
-            e[1].record(st)
-            F.ls_commit_accepted(run.state, acc, inp["vk"][r], inp["vv"][r], inp["vh"][r], st)
-            e[2].record(st)
-            F.ls_draft_prologue(run.state, w_kv, w_q, x, bkv, qd, st)
-            e[3].record(st)
-            F.ls_draft_attend(run.state, 0, L, qd, bkv, bkv[..., H * D:], 2 * H * D, scale, out, st)
+            one_round(r, e if r >= half else None)
             e[4].record(st)
             if r < n_u:
                 a_seen.append(acc.clone())
@@ -1165,9 +1177,10 @@ def drafting_round_measure(WLM, wl, dev, flush, n, prefixes=None):
         if status != F.LS_OK:
             raise RuntimeError(f"device error word {word:#x} in the drafting round")
         warm = 3
-        tot = [e[0].elapsed_time(e[4]) for e in evs[warm:]]
-        parts = {k: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs[warm:]])) * 1e3
+        tot = [e[0].elapsed_time(e[4]) for e in evs[warm:half]]
+        parts = {k: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs[half:]])) * 1e3
                  for i, k in enumerate(("accept_sampled_us", "commit_accepted_us", "prologue_us", "attend_us"))}
+        parts["sum_us"] = sum(parts.values())
         a_all = torch.stack(a_seen).cpu().numpy()
         rows = float(np.mean(np.where(a_all < B, 2, 1).sum(axis=1)))  # probability rows the draw reads
         run.close()
@@ -1175,19 +1188,20 @@ def drafting_round_measure(WLM, wl, dev, flush, n, prefixes=None):
         torch.cuda.empty_cache()
         return tot, parts, float(a_all.mean()), rows
 
-    tot, parts, a_mean, rows = series(wl, n)
+    tot, parts, a_mean, rows = series(wl, max(2 * n, 32))
     nbytes = (int(b * 2 * B * 4 + b * (B + 1) * 4 + rows * V * 4)  # sampling: tests, draws, the drawn rows
               + commit_bytes(wl, a_mean + 1)
               + (w_kv.numel() + w_q.numel() + x.numel() + b * L * hid + bkv.numel() + qd.numel()) * 2
               + attend_bytes(wl))
     st = us_stats(tot)
     res = {"kernels": "ls_accept_sampled -> ls_commit_accepted -> ls_draft_prologue -> ls_draft_attend",
-           "vocab": V, "us_per_round": st, "rounds_per_s": 1e6 / st["mean"], "rounds": len(tot), "split": parts,
+           "vocab": V, "us_per_round": st, "rounds_per_s": 1e6 / st["mean"], "rounds": len(tot),
+           "split": dict(parts, note="other rounds, with an event between the calls (which serialises them)"),
            "accept_mean": a_mean, "bytes": nbytes, "frac": nbytes / st["mean"] / 1e3 / peak, "launches_per_round": 4}
     if prefixes:
         by_p, split_p = {}, {}
         for P in prefixes:
-            t, parts_p, _, _ = series(replace(wl, name=f"{wl.name}_p{P}", prefix=P), max(16, n // 4))
+            t, parts_p, _, _ = series(replace(wl, name=f"{wl.name}_p{P}", prefix=P), 32)
             by_p[str(P)] = float(np.median(t)) * 1e3
             split_p[str(P)] = parts_p
         v = list(by_p.values())

@@ -45,9 +45,10 @@ struct ls_state {
   int sms;
   int use_tc;
   ls::TcPlan tc;
-  // No call has written the views since a tensor-core attention was launched on
-  // settled_stream: an attention launched next on that stream may load its first K/V
-  // chunks before its grid dependency wait (ls::kAttendViewsSettled).
+  // No call has written the views since a launch on settled_stream after which every
+  // earlier writer has completed before the next kernel on that stream starts (see
+  // mark_settled): an attention launched next on that stream may load its first K/V chunks
+  // before its grid dependency wait (ls::kAttendViewsSettled).
   // (kept by the calls that only read the state too: mutable)
   mutable int views_settled;
   mutable cudaStream_t settled_stream;
@@ -63,6 +64,15 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 bool on_state_device(const ls_state* st) {
   int dev = -1;
   return cudaGetDevice(&dev) == cudaSuccess && dev == st->device;
+}
+
+// After a launch on `stream` that writes no views and lets the kernels behind it start only
+// once everything before it has completed (it triggers its dependents after its grid
+// dependency wait, or it is launched without programmatic serialization), every call that
+// wrote the views has completed by the time a kernel launched next on `stream` starts.
+void mark_settled(const ls_state* st, cudaStream_t stream) {
+  st->views_settled = 1;
+  st->settled_stream = stream;
 }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -226,6 +236,7 @@ int ls_init_state(const ls_config* cfg, void* d_arena, size_t arena_bytes, ls_st
   p.boundary = base + y.boundary;
   p.samp_count = reinterpret_cast<int32_t*>(base + y.sample);
   p.samp_part = reinterpret_cast<float*>(base + y.sample + int64_t(cfg->batch) * 4);
+  p.samp_seg = p.samp_part + int64_t(cfg->batch) * ls::kSampleMaxChunks;
   p.pro_part = reinterpret_cast<float*>(base + y.prologue);
   p.pro_count = reinterpret_cast<int32_t*>(base + y.prologue + int64_t(ls::kProMaxSlots) * ls::kProTileN *
                                                                        ls::prologue_boundary_rows(cfg->batch) * 4);
@@ -376,8 +387,10 @@ int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const float* d_d
   if (vocab < 4 || vocab % 4 != 0) return LS_ERR_SHAPE;
   if (vocab > ls::kSampleChunk * ls::kSampleMaxChunks) return LS_ERR_UNSUPPORTED;
   if (!aligned16(d_draft_probs) || !aligned16(d_target_probs)) return LS_ERR_INVALID_ARG;
-  return cuda_status(ls::launch_sample(st->dev, d_draft_ids, d_draft_probs, d_target_probs, vocab, d_uniforms,
-                                       d_accept_len, d_next_token, stream));
+  const int r = cuda_status(ls::launch_sample(st->dev, d_draft_ids, d_draft_probs, d_target_probs, vocab, d_uniforms,
+                                              d_accept_len, d_next_token, stream));
+  if (r == LS_OK) mark_settled(st, stream);
+  return r;
 }
 
 int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q, const void* d_x, void* d_bkv,
@@ -388,6 +401,7 @@ int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q,
   if (!aligned16(d_w_kv) || !aligned16(d_w_q) || !aligned16(d_x) || !aligned16(d_bkv) || !aligned16(d_q))
     return LS_ERR_INVALID_ARG;
   const cudaError_t e = ls::launch_prologue(st->dev, d_w_kv, d_w_q, d_x, d_bkv, d_q, st->sms, stream);
+  if (e == cudaSuccess) mark_settled(st, stream);
   return e == cudaErrorNotSupported ? LS_ERR_UNSUPPORTED : cuda_status(e);
 }
 
@@ -434,10 +448,7 @@ int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer
     const int r = cuda_status(ls::launch_attend_tc(st->dev, st->tc, layer_begin, layer_count, d_q, d_boundary_k,
                                                    d_boundary_v, boundary_stride, softmax_scale, views, d_out,
                                                    st->sms, mode, stream));
-    if (r == LS_OK) {
-      st->views_settled = 1;
-      st->settled_stream = stream;
-    }
+    if (r == LS_OK) mark_settled(st, stream);
     return r;
   }
   return cuda_status(ls::launch_attend_simt(st->dev, layer_begin, layer_count, d_q, d_boundary_k,
@@ -486,10 +497,7 @@ int round_attend(ls_state* st, const void* d_q, int64_t boundary_k_offset, int64
     const int r = cuda_status(ls::launch_attend_tc(st->dev, st->tc, 0, c.n_layers, d_q, bnd + boundary_k_offset * e,
                                                    bnd + boundary_v_offset * e, c.hidden, softmax_scale, LS_VIEW_ALL,
                                                    d_out, st->sms, ls::kAttendAfterCommit, stream));
-    if (r == LS_OK) {
-      st->views_settled = 1;
-      st->settled_stream = stream;
-    }
+    if (r == LS_OK) mark_settled(st, stream);
     return r;
   }
   return ls_draft_attend(st, 0, c.n_layers, d_q, bnd + boundary_k_offset * e, bnd + boundary_v_offset * e, c.hidden,
@@ -543,7 +551,9 @@ int ls_clear_error(ls_state* st, cudaStream_t stream) {
 int ls_check_wait_timeout(ls_state* st, uint32_t polls, cudaStream_t stream) {
   if (!st || polls == 0 || polls > ls::kWaitLimit) return LS_ERR_INVALID_ARG;
   if (!on_state_device(st)) return LS_ERR_INVALID_ARG;
-  return cuda_status(ls::launch_wait_timeout(st->dev, polls, stream));
+  const int r = cuda_status(ls::launch_wait_timeout(st->dev, polls, stream));
+  if (r == LS_OK) mark_settled(st, stream);
+  return r;
 }
 
 void ls_destroy_state(ls_state* st) { delete st; }

@@ -28,6 +28,7 @@ struct Dev {
   char* boundary;     // [b][L][hidden] elements
   int32_t* samp_count;  // [b] arrivals of a sequence's CTAs in ls_accept_sampled
   float* samp_part;     // [b][kSampleMaxChunks] vocabulary chunk sums of ls_accept_sampled
+  float* samp_seg;      // [b][kSampleMaxChunks][64] the chunks' segment sums (128 entries each)
   float* pro_part;      // [kProMaxSlots][128][boundary rows] split-tile partial sums of ls_draft_prologue
   int32_t* pro_count;   // [kProMaxGrid] arrivals of a split tile's pieces
 };
@@ -77,7 +78,7 @@ __host__ inline Layout make_layout(const ls_config& c) {
   y.part = off;     off = align256(off + tiles * c.n_scales * 2 * c.head_dim * 4);
   y.glob = off;     off = align256(off + tiles * 2 * c.head_dim * 4);
   y.boundary = off; off = align256(off + int64_t(c.batch) * c.n_layers * c.hidden * y.elem);
-  y.sample = off;   off = align256(off + int64_t(c.batch) * (1 + kSampleMaxChunks) * 4);
+  y.sample = off;   off = align256(off + int64_t(c.batch) * (1 + kSampleMaxChunks + kSampleMaxChunks * 64) * 4);
   y.prologue = off;
   if (prologue_shapes_ok(c.dtype, c.hidden, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block))
     off = align256(off + int64_t(kProMaxSlots) * kProTileN * prologue_boundary_rows(c.batch) * 4 + kProMaxGrid * 4);

@@ -21,6 +21,11 @@
 // tile leaves its fp32 partial sums in the state's scratch; the last piece of a tile to
 // arrive adds them up in piece order (the same sum whatever the arrival order) and stores
 // the tile.
+// Launched as the programmatic dependent of the kernel before it on the stream: the weights
+// (the drafter's parameters, nearly all of the bytes) stream from the start; the
+// activations (the block inputs and the boundary view, which that kernel may write: a
+// commit writes the boundary view) are read only after the grid dependency wait. Every
+// thread triggers this grid's dependents once it has passed that wait.
 // Every wait is bounded.
 #include "ls_tc.cuh"
 
@@ -191,10 +196,15 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   int issued = 0;  // producers: copies issued into their ring (for the drain after an abort)
+  if (warp != 0) {  // the weight producer waits once its first ring of weights is on its way
+    grid_dependency_wait();
+    allow_dependent_launch();
+  }
 
   if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------ TMA producers
     // warp 0: the weights (A) of every k-step; warp 6: the activations (B)
+    bool waited = warp != 0;
     if (lane == 0) {
       const bool is_a = warp == 0;
       const int nst = is_a ? kPAStages : kPBStages;
@@ -215,6 +225,11 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
         // every weight tile of the layer) out of L2
         for (int ks = it.k0; ks < it.k1; ++ks, ++k) {
           const int st = k % nst;
+          if (k == nst && !waited) {  // (the first ring's weights are in flight)
+            grid_dependency_wait();
+            allow_dependent_launch();
+            waited = true;
+          }
           if (!pwait(s, &emptyb[st], ((k / nst) & 1) ^ 1, a.err)) { ok = false; break; }
           mbar_arrive_expect_tx(&fullb[st], bytes);
           if (is_a)
@@ -228,6 +243,10 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
           ++issued;
         }
       }
+    }
+    if (!waited) {  // (every thread of the CTA passes the wait before it triggers)
+      grid_dependency_wait();
+      allow_dependent_launch();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -465,8 +484,17 @@ cudaError_t launch_prologue(const Dev& p, const void* w_kv, const void* w_q, con
   a.rem_steps = split ? rem * a.k_steps : 0;
   a.part = p.pro_part;
   a.count = p.pro_count;
-  prologue_kernel<<<grid, kPThreads, kPSmemBytes, stream>>>(a, mw0, mx0, mw1, mx1);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPThreads);
+  cfg.dynamicSmemBytes = kPSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prologue_kernel, a, mw0, mx0, mw1, mx1);
 }
 
 }  // namespace ls

@@ -8,12 +8,14 @@
 // order with the draw u_B. A row drawn from that has no mass sets LS_DEVERR_SAMPLE.
 //
 // Grid (vocabulary chunks of 8192, sequences), 256 threads. Every CTA of a sequence makes
-// the B acceptance tests itself (2 B gathers) and sums the draw's weights over its chunk
-// in a fixed order: sub-block m of 1024 entries, one float4 per thread, sub-blocks in
-// order, then a tree over the threads. The last CTA of the sequence to arrive (a counter
-// in the arena, reset by that CTA; nobody waits) adds the chunk sums in order, finds the
-// chunk, then the sub-block, thread and entry holding the draw. HBM traffic: the rows of
-// the draw (one, or two after a rejection) once, plus the drawn chunk again.
+// the B acceptance tests itself (2 B gathers) and sums the draw's weights over its chunk:
+// per segment of 128 entries (64 segments: sub-block m of 1024 entries, one float4 per
+// thread, warp w's 128 of them) a fixed tree, and the chunk's total a fixed tree over its
+// segments; it leaves both in the arena. The last CTA of the sequence to arrive (a counter
+// in the arena, reset by that CTA; nobody waits) scans the chunk totals in order for the
+// chunk holding u_B times the total, then that chunk's segment sums for the segment, and
+// one warp re-reads the segment's 128 entries from L2 for the entry. HBM traffic: the rows
+// of the draw (one, or two after a rejection) once.
 #include "ls_common.cuh"
 
 namespace ls {
@@ -51,52 +53,51 @@ __device__ inline float4 weights4(const float* prow, const float* qrow, int j, i
 }
 __device__ inline float sum4(const float4& w) { return (w.x + w.y) + (w.z + w.w); }
 
-// Sum over the CTA (warp trees, then the 8 warp sums in order); every thread gets it.
-__device__ inline float block_sum(float x, float* sh) {
+// Segment j = 8 m + w of a chunk: the 128 entries [1024 m + 128 w, +128) that warp w's
+// float4 loads of sub-block m cover. A chunk's 64 segment sums, in entry order, and its
+// total (a fixed tree over them) are what the chunk's CTA leaves for the sequence's last CTA.
+constexpr int kSegs = kSubs * (kSampleThreads / 32);  // 64
+static_assert(kSegs == 64, "the segment scan covers 64 entries with two warps");
+
+// The segment sums of chunk c into seg[64] (every thread calls it; ends with a barrier).
+__device__ inline void chunk_segments(const float* prow, const float* qrow, int c, int V, float* seg) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int base = c * kSampleChunk + 4 * threadIdx.x;
+  float r[kSubs];
 #pragma unroll
-  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = x;
-  __syncthreads();
-  float t = 0.f;
+  for (int m = 0; m < kSubs; ++m) r[m] = sum4(weights4(prow, qrow, base + m * kSub, V));
 #pragma unroll
-  for (int w = 0; w < kSampleThreads / 32; ++w) t += sh[w];
-  return t;
+  for (int m = 0; m < kSubs; ++m)
+#pragma unroll
+    for (int o = 16; o; o >>= 1) r[m] += __shfl_xor_sync(0xffffffffu, r[m], o);
+  if (lane == 0)
+#pragma unroll
+    for (int m = 0; m < kSubs; ++m) seg[m * (kSampleThreads / 32) + warp] = r[m];
+  __syncthreads();
 }
 
-// Exclusive prefix of x over the threads in order; *total gets the sum of all.
-__device__ inline float block_exclusive(float x, float* sh, float* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float inc = x;
+// The total of 64 segment sums: a fixed tree (pairs j, j + 32, then across the warp). Called
+// by one whole warp; every lane gets it.
+__device__ inline float segments_total(const float* seg) {
+  const int lane = threadIdx.x & 31;
+  float v = seg[lane] + seg[lane + 32];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const float y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
-  }
-  __syncthreads();
-  if (lane == 31) sh[warp] = inc;
-  __syncthreads();
-  float before = 0.f, all = 0.f;
-#pragma unroll
-  for (int w = 0; w < kSampleThreads / 32; ++w) {
-    if (w < warp) before += sh[w];
-    all += sh[w];
-  }
-  *total = all;
-  return before + inc - x;
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
-// The chunk holding the draw: the first chunk whose running sum (chunks in order) passes
-// t = u * total, or the last chunk with mass when rounding leaves none. The first two warps
-// scan the nchunks <= 64 sums in csum; *cstar gets the chunk (-1: no mass at all) and *rem
-// the part of t left inside it (infinity in the rounding case). Every thread calls it.
-__device__ inline void find_chunk(const float* csum, int nchunks, float u, float* sh, float* scratch, int* cstar_out,
-                                  float* rem_out) {
+// The first of n <= 64 sums (in order) whose running sum passes t: t = x * (their total)
+// when `fraction`, else t = x. When rounding leaves none (or t is infinite), the last with
+// mass, and *rem_out infinite; *idx_out -1 when none has mass. *rem_out otherwise gets t
+// minus the sums before the one found. The first two warps scan; every thread calls it
+// (ends with a barrier).
+__device__ inline void find_first(const float* vals, int n, float x, bool fraction, float* sh, float* scratch,
+                                  int* idx_out, float* rem_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp < 2) {
     const int k = threadIdx.x;
-    const float v = k < nchunks ? csum[k] : 0.f;
-    float inc = v;  // inclusive prefix within the warp, in chunk order
+    const float v = k < n ? vals[k] : 0.f;
+    float inc = v;  // inclusive prefix within the warp, in order
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float y = __shfl_up_sync(0xffffffffu, inc, o);
@@ -106,9 +107,9 @@ __device__ inline void find_chunk(const float* csum, int nchunks, float u, float
     asm volatile("bar.sync 1, 64;" ::: "memory");  // the two warps' totals
     if (warp == 1) inc += sh[0];
     const float z = sh[0] + sh[1];
-    const float t = u * z;
-    const unsigned hit = __ballot_sync(0xffffffffu, z > 0.f && k < nchunks && inc > t);
-    const unsigned mass = __ballot_sync(0xffffffffu, k < nchunks && v > 0.f);
+    const float t = fraction ? x * z : x;
+    const unsigned hit = __ballot_sync(0xffffffffu, z > 0.f && k < n && inc > t);
+    const unsigned mass = __ballot_sync(0xffffffffu, k < n && v > 0.f);
     if (lane == 0) {
       scratch[warp] = __int_as_float(int(hit));
       scratch[2 + warp] = __int_as_float(int(mass));
@@ -116,17 +117,17 @@ __device__ inline void find_chunk(const float* csum, int nchunks, float u, float
     asm volatile("bar.sync 1, 64;" ::: "memory");
     const unsigned h0 = __float_as_int(scratch[0]), h1 = __float_as_int(scratch[1]);
     const unsigned m0 = __float_as_int(scratch[2]), m1 = __float_as_int(scratch[3]);
-    int cstar = h0 ? __ffs(int(h0)) - 1 : (h1 ? 32 + __ffs(int(h1)) - 1 : -1);
+    int idx = h0 ? __ffs(int(h0)) - 1 : (h1 ? 32 + __ffs(int(h1)) - 1 : -1);
     bool force_last = false;
-    if (cstar < 0 && z > 0.f) {
-      cstar = m1 ? 63 - __clz(int(m1)) : 31 - __clz(int(m0));
+    if (idx < 0 && (m0 | m1)) {
+      idx = m1 ? 63 - __clz(int(m1)) : 31 - __clz(int(m0));
       force_last = true;
     }
-    if (k == cstar) {
-      *cstar_out = cstar;
+    if (k == idx) {
+      *idx_out = idx;
       *rem_out = force_last ? INFINITY : t - (inc - v);
     }
-    if (threadIdx.x == 0 && cstar < 0) *cstar_out = -1;
+    if (threadIdx.x == 0 && idx < 0) *idx_out = -1;
   }
   __syncthreads();
 }
@@ -135,11 +136,11 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
   const int c = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ float sh[kSampleThreads / 32];
-  __shared__ float sub_tot[kSubs];
-  __shared__ float sub_part[kSampleThreads / 32][kSubs];
+  __shared__ float scratch[4];
   __shared__ float csum_s[kSampleMaxChunks];
-  __shared__ int a_s, last_s, cstar_s, found_s, lastpos_s;
-  __shared__ float rem_s;
+  __shared__ float seg_s[kSegs];
+  __shared__ int a_s, last_s, cstar_s, sstar_s;
+  __shared__ float rem_s, rem2_s;
 
   // the accepted count: first position whose test fails (B <= 32: one warp)
   if (warp == 0) {
@@ -163,24 +164,22 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
   const float* prow = s.p + (int64_t(b) * (p.B + 1) + a) * s.V;
   const float* qrow = a < p.B ? s.q + (int64_t(b) * p.B + a) * s.V : nullptr;  // null: draw from p
 
-  // this chunk's share of the draw's mass
-  {
-    const int base = c * kSampleChunk + 4 * threadIdx.x;
-    float acc = 0.f;
-#pragma unroll
-    for (int m = 0; m < kSubs; ++m) acc += sum4(weights4(prow, qrow, base + m * kSub, s.V));
-    const float tot = block_sum(acc, sh);
-    if (threadIdx.x == 0) {
-      p.samp_part[b * kSampleMaxChunks + c] = tot;
-      __threadfence();
-      last_s = atomicAdd(p.samp_count + b, 1) == s.nchunks - 1;
-    }
-    __syncthreads();
-    if (!last_s) return;
+  // this chunk's share of the draw's mass: its 64 segment sums and their total
+  float* seg_g = p.samp_seg + (int64_t(b) * kSampleMaxChunks + c) * kSegs;
+  chunk_segments(prow, qrow, c, s.V, seg_s);
+  if (threadIdx.x < kSegs) seg_g[threadIdx.x] = seg_s[threadIdx.x];
+  if (warp == 0) {
+    const float tot = segments_total(seg_s);
+    if (lane == 0) p.samp_part[b * kSampleMaxChunks + c] = tot;
   }
+  __threadfence();  // (the segment sums and the total are visible before the arrival)
+  __syncthreads();
+  if (threadIdx.x == 0) last_s = atomicAdd(p.samp_count + b, 1) == s.nchunks - 1;
+  __syncthreads();
+  if (!last_s) return;
 
-  // the sequence's last CTA: the chunk sums (loaded at once, chunk k by thread k), then
-  // the chunk holding u_B * total
+  // The sequence's last CTA: the chunk holding u_B times the total, then its segment, then
+  // the entry (one warp re-reads the segment's 128 entries from L2).
   __threadfence();
   if (threadIdx.x < kSampleMaxChunks)
     csum_s[threadIdx.x] =
@@ -188,22 +187,23 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
   if (threadIdx.x == 0) p.samp_count[b] = 0;  // zero again for the next call
   __syncthreads();
   const float ub = s.u[b * (p.B + 1) + p.B];
-  find_chunk(csum_s, s.nchunks, ub, sh, sub_tot, &cstar_s, &rem_s);
+  find_first(csum_s, s.nchunks, ub, true, sh, scratch, &cstar_s, &rem_s);
+  bool local = false;  // the chosen chunk's segment sums are computed here, not loaded
   if (cstar_s < 0 && qrow != nullptr) {
     // The residual has no mass (p_a <= q_a everywhere: equal rows up to rounding, or a
     // draft neither row gives mass): the token is drawn from the target's row p_a itself,
     // whose chunk sums this CTA makes in the order the chunk CTAs use.
     qrow = nullptr;
+    local = true;
     for (int c2 = 0; c2 < s.nchunks; ++c2) {
-      const int base = c2 * kSampleChunk + 4 * threadIdx.x;
-      float acc = 0.f;
-#pragma unroll
-      for (int m = 0; m < kSubs; ++m) acc += sum4(weights4(prow, nullptr, base + m * kSub, s.V));
-      const float tot = block_sum(acc, sh);
-      if (threadIdx.x == 0) csum_s[c2] = tot;
+      chunk_segments(prow, nullptr, c2, s.V, seg_s);
+      if (warp == 0) {
+        const float tot = segments_total(seg_s);
+        if (lane == 0) csum_s[c2] = tot;
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    find_chunk(csum_s, s.nchunks, ub, sh, sub_tot, &cstar_s, &rem_s);
+    find_first(csum_s, s.nchunks, ub, true, sh, scratch, &cstar_s, &rem_s);
   }
   if (cstar_s < 0) {  // the row drawn from has no mass: not a distribution
     if (threadIdx.x == 0) {
@@ -213,84 +213,53 @@ __global__ void __launch_bounds__(kSampleThreads) sample_kernel(const Dev p, con
     }
     return;
   }
-
-  // sub-block and entry: the first entry whose running sum in the chunk passes rem
-  const int cbase = cstar_s * kSampleChunk;
-  float4 w[kSubs];
-  float ws[kSubs];
-#pragma unroll
-  for (int m = 0; m < kSubs; ++m) {
-    w[m] = weights4(prow, qrow, cbase + m * kSub + 4 * threadIdx.x, s.V);
-    ws[m] = sum4(w[m]);
-  }
-  {
-    // the 8 sub-block sums in one round: warp trees, then the warps' partials in order
-    float r[kSubs];
-#pragma unroll
-    for (int m = 0; m < kSubs; ++m) {
-      r[m] = ws[m];
-#pragma unroll
-      for (int o = 16; o; o >>= 1) r[m] += __shfl_xor_sync(0xffffffffu, r[m], o);
-    }
-    if (lane == 0)
-#pragma unroll
-      for (int m = 0; m < kSubs; ++m) sub_part[warp][m] = r[m];
-    if (threadIdx.x == 0) {
-      found_s = 0x7fffffff;
-      lastpos_s = -1;
-    }
-    __syncthreads();
-    if (threadIdx.x < kSubs) {
-      float t = 0.f;
-#pragma unroll
-      for (int w2 = 0; w2 < kSampleThreads / 32; ++w2) t += sub_part[w2][threadIdx.x];
-      sub_tot[threadIdx.x] = t;
-    }
+  const int cs = cstar_s;
+  if (local) {
+    chunk_segments(prow, nullptr, cs, s.V, seg_s);
+  } else {
+    if (threadIdx.x < kSegs)
+      seg_s[threadIdx.x] = __ldcg(p.samp_seg + (int64_t(b) * kSampleMaxChunks + cs) * kSegs + threadIdx.x);
     __syncthreads();
   }
-  float rem = rem_s;
-  int mstar = -1;
-  for (int m = 0; m < kSubs && mstar < 0; ++m) {
-    if (sub_tot[m] > rem) mstar = m;
-    else rem -= sub_tot[m];
-  }
-  if (mstar < 0) {  // rounding: the last sub-block with mass, its last entry with mass
-    for (int m = kSubs - 1; m >= 0 && mstar < 0; --m)
-      if (sub_tot[m] > 0.f) mstar = m;
-    if (mstar < 0) mstar = 0;  // (the chunk had mass in the first pass: not reached)
-    rem = INFINITY;
-  }
-  float4 wm = w[0];
-  float wsm = ws[0];
+  find_first(seg_s, kSegs, rem_s, false, sh, scratch, &sstar_s, &rem2_s);
+  if (warp == 0) {
+    // (the chunk has mass, so some segment has: sstar_s >= 0)
+    const int sg = sstar_s < 0 ? 0 : sstar_s;
+    const int j0 = cs * kSampleChunk + (sg / (kSampleThreads / 32)) * kSub + (sg % (kSampleThreads / 32)) * 128;
+    const int pos = j0 + 4 * lane;
+    const float4 w = weights4(prow, qrow, pos, s.V);
+    const float ls = sum4(w);
+    float inc = ls;  // running sum over the lanes, in order
 #pragma unroll
-  for (int m = 1; m < kSubs; ++m)
-    if (m == mstar) { wm = w[m]; wsm = ws[m]; }
-  float total;
-  const float excl = block_exclusive(wsm, sh, &total);
-  const int pos0 = cbase + mstar * kSub + 4 * threadIdx.x;
-  const float e4[4] = {wm.x, wm.y, wm.z, wm.w};
-  if (excl <= rem && rem < excl + wsm) {  // this thread's four entries hold the draw
-    float run = excl;
-    int pick = -1;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      run += e4[e];
-      if (pick < 0 && run > rem && e4[e] > 0.f) pick = e;
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
     }
-    if (pick < 0)  // rounding inside the four: their last entry with mass (wsm > 0 here)
-      for (int e = 3; e >= 0 && pick < 0; --e)
-        if (e4[e] > 0.f) pick = e;
-    atomicMin(&found_s, pos0 + pick);
-  }
-  // fallback for rounding at the end of the sub-block: its last entry with mass
+    float excl = __shfl_up_sync(0xffffffffu, inc, 1);
+    if (lane == 0) excl = 0.f;
+    float rem = rem2_s;
+    const unsigned hit = __ballot_sync(0xffffffffu, inc > rem);
+    const unsigned mass = __ballot_sync(0xffffffffu, ls > 0.f);
+    int ln = hit ? __ffs(int(hit)) - 1 : -1;
+    if (ln < 0) {  // rounding: the last lane with mass
+      ln = mass ? 31 - __clz(int(mass)) : 0;
+      rem = INFINITY;
+    }
+    if (lane == ln) {
+      const float e4[4] = {w.x, w.y, w.z, w.w};
+      float run = excl;
+      int pick = -1;
 #pragma unroll
-  for (int e = 3; e >= 0; --e)
-    if (e4[e] > 0.f) { atomicMax(&lastpos_s, pos0 + e); break; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    s.accept_len[b] = a;
-    const int tok = found_s != 0x7fffffff ? found_s : lastpos_s;
-    s.next_token[b] = tok >= 0 ? tok : 0;
+      for (int e = 0; e < 4; ++e) {
+        run += e4[e];
+        if (pick < 0 && run > rem && e4[e] > 0.f) pick = e;
+      }
+      if (pick < 0)  // rounding inside the four: their last entry with mass
+        for (int e = 3; e >= 0 && pick < 0; --e)
+          if (e4[e] > 0.f) pick = e;
+      s.accept_len[b] = a;
+      s.next_token[b] = pos + (pick < 0 ? 0 : pick);
+    }
   }
 }
 

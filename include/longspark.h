@@ -306,7 +306,11 @@ LS_API int ls_accept_sampled(ls_state* st, const int32_t* d_draft_ids, const flo
  * pointers 16-byte aligned. Boundary tiles left over after whole waves of CTAs are split
  * along the hidden size; their fp32 partial sums use the state's prologue scratch
  * (ls_layout.off_prologue), so two calls on one state must not overlap on the GPU (order
- * them on one stream). Repeated calls give the same bits.                               */
+ * them on one stream). Repeated calls give the same bits. The kernel is launched as the
+ * programmatic dependent of the kernel before it on `stream` and streams the weights
+ * before that kernel has completed (the block inputs and the boundary view only after):
+ * d_w_kv and d_w_q, the drafter's parameters, must not be written by the kernel launched
+ * just before this call on the stream.                                                  */
 LS_API int ls_draft_prologue(const ls_state* st, const void* d_w_kv, const void* d_w_q, const void* d_x,
                              void* d_bkv, void* d_q, cudaStream_t stream);
 
@@ -328,10 +332,11 @@ LS_API int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const v
  * kv_rows <= 768 (unless LS_FLAG_FORCE_SIMT), otherwise a CUDA-core kernel. The
  * tensor-core kernel is launched as the programmatic dependent of the kernel before it
  * on `stream`: it reads the inputs that kernel may write only once that kernel has
- * completed. When no call has written this state's views since an attention was launched
- * on the same stream (per-layer calls), it loads its first rows of the views before that,
- * so one call's start overlaps the end of the call before it. Inside a stream capture it
- * does not (the order of the graph's replays is not known when it is captured).       */
+ * completed. When no commit or prefill has written this state's views since another call
+ * on the state was launched on the same stream (per-layer calls, or the call after
+ * ls_draft_prologue), it loads its first rows of the views before that, so its start
+ * overlaps the end of the kernel before it. Inside a stream capture it does not (the
+ * order of the graph's replays is not known when it is captured).                     */
 LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count,
                     const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
                     int64_t boundary_stride, float softmax_scale, void* d_out,

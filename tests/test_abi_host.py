@@ -76,9 +76,9 @@ def test_view_state_bytes():
         assert F.ls_view_state_bytes(c, views) == n, views
     everything = F.ls_view_state_bytes(c, F.LS_VIEW_ALL)
     # the arena adds the error word, the commit's arrival counts, the sampler's scratch
-    # (counts + 64 chunk sums per sequence), the projections' scratch and the 256-byte
-    # alignment of its 11 regions
-    extra = 16 + b * L * 4 + b * 65 * 4 + 320 * 128 * 16 * 4 + 160 * 4
+    # (counts, 64 chunk sums and 64 x 64 segment sums per sequence), the projections'
+    # scratch and the 256-byte alignment of its 11 regions
+    extra = 16 + b * L * 4 + b * (1 + 64 + 64 * 64) * 4 + 320 * 128 * 16 * 4 + 160 * 4
     assert everything + extra <= F.ls_state_bytes(c) < everything + extra + 11 * 256
     assert F.ls_view_state_bytes(c, 8) == 0 and F.ls_view_state_bytes(_cfg(batch=0), 1) == 0
 

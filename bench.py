@@ -1058,8 +1058,7 @@ def sweep_grid(WLM, dev, flush, rounds, flags=0):
     """The prefix x concurrency x accept-mean sweep (Qwen3-8B shapes): per point the
     per-round time (median over the rounds after 3 untimed ones, an L2 flush before each)
     and the drafter state bytes; flatness of the per-round time over the prefixes for
-    every (batch, accept mean). Prefixes of more than 4M rows in total run the chunked
-    prefill (32K rows per call)."""
+    every (batch, accept mean). The prefill runs in chunks of 8192 rows."""
     import torch
     import fixed_cost_drafter_b200 as F
     from dataclasses import replace
@@ -1071,8 +1070,9 @@ def sweep_grid(WLM, dev, flush, rounds, flags=0):
             for P in WLM.SWEEP_PREFIXES:
                 wl = WLM.sweep_point(P, b, m)
                 wl = replace(wl, flags=wl.flags | flags)
-                chunk = 32768 if P * b > 4 * 1024 * 1024 else None
-                run = WLM.DeviceRun(wl, device=dev, rounds=rounds, prefill_chunk=chunk)
+                # 8192-row prefill chunks: no large buffer is freed right before the timed
+                # rounds (see drafting_round_measure)
+                run = WLM.DeviceRun(wl, device=dev, rounds=rounds, prefill_chunk=8192)
                 run.prefill()
                 torch.cuda.synchronize()
                 torch.cuda.empty_cache()

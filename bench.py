@@ -79,6 +79,13 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def job_rate(units_per_rank: int, seconds_max: float, world: int, strong: bool) -> float:
+    """Units per second of the whole job over the slowest rank's time: weak scaling (every
+    rank its own batch) counts every rank's units, strong scaling (ranks share one batch's
+    KV heads) counts the batch's once."""
+    return (1 if strong else world) * units_per_rank / seconds_max
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -647,7 +654,7 @@ def run_gpu(args):
     configs = None
     if not args.no_configs and rank == 0 and not strong:
         configs = {name: config_record(WLM, name, dev, flush, 0, wl.flags & F.LS_FLAG_OUT_F32)
-                   for name in ("qwen3_4b_32k", "qwen3_8b_128k_ragged")}
+                   for name in ("tiny", "qwen3_4b_32k", "qwen3_8b_128k_ragged")}
 
     # the prefix x concurrency x accept-mean sweep; flatness over the prefixes
     grid, flat = None, None
@@ -671,7 +678,7 @@ def run_gpu(args):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": (1 if strong else world) * K / total_max, "unit": "rounds/s",
+            "metric": METRIC, "value": job_rate(K, total_max, world, strong), "unit": "rounds/s",
             "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": total_max * 1e3 / K, "higher_is_better": True,
             "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(full_wl),
@@ -713,6 +720,10 @@ def run_gpu(args):
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget)
+            if configs:  # the oracle on the other configurations' rounds, a shorter sample each
+                for name in configs:
+                    cwl = WLM.CONFIGS[name]
+                    configs[name]["cpu_oracle"] = cpu_record(cwl, *oracle_timing(name, 1, budget_s=args.cpu_budget / 3))
         print(json.dumps(line))
     run.close()
     if world > 1:
@@ -947,7 +958,7 @@ def e2e_measure(run, wl, dev, flush, steps, world, inp, strong=False):
     e1.record(cout)
     e1.synchronize()
     tot = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
-    return {"value": (1 if strong else world) * steps / tot, "unit": "rounds/s", "h2d_bytes_per_step": int(h2d),
+    return {"value": job_rate(steps, tot, world, strong), "unit": "rounds/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps, "pipelined": "2 buffer slots, copy streams in and out"}
 
 

@@ -35,7 +35,10 @@ def _worker(rank, world, port, q):
     heads = bench.kv_head_range(r, w, 8)
     t = bench.max_over_ranks(1.0 + r, w, torch.device("cpu"))
     bench.barrier(w)
-    q.put((r, off, heads, t))
+    # the job's rate: 20 rounds per rank, rank r's timed region 0.5 (r + 1) s
+    tr = bench.max_over_ranks(0.5 * (r + 1), w, torch.device("cpu"))
+    rates = (bench.job_rate(20, tr, w, False), bench.job_rate(20, tr, w, True))
+    q.put((r, off, heads, t, rates))
     dist.destroy_process_group()
 
 
@@ -50,9 +53,11 @@ def test_two_ranks_shard_and_max():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert [o for _, o, _, _ in res] == [0, 16]            # disjoint sequence ranges
-    assert [h for _, _, h, _ in res] == [(0, 4), (4, 8)]   # or disjoint KV-head ranges covering all
-    assert all(t == 2.0 for _, _, _, t in res)              # every rank sees the slowest rank's time
+    assert [o for _, o, _, _, _ in res] == [0, 16]            # disjoint sequence ranges
+    assert [h for _, _, h, _, _ in res] == [(0, 4), (4, 8)]   # or disjoint KV-head ranges covering all
+    assert all(t == 2.0 for _, _, _, t, _ in res)              # every rank sees the slowest rank's time
+    # weak scaling: both ranks' 20 rounds over the slowest rank's 1.0 s; strong: the batch's 20
+    assert all(rt == (40.0, 20.0) for _, _, _, _, rt in res)
 
 
 def test_kv_head_ranges():

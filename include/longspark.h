@@ -336,7 +336,10 @@ LS_API int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const v
  * on the state was launched on the same stream (per-layer calls, or the call after
  * ls_draft_prologue), it loads its first rows of the views before that, so its start
  * overlaps the end of the kernel before it. Inside a stream capture it does not (the
- * order of the graph's replays is not known when it is captured).                     */
+ * order of the graph's replays is not known when it is captured). A caller that writes
+ * the arena itself (a checkpoint restored into it) does so with a copy, or a kernel that
+ * does not trigger programmatic dependents before it completes (any kernel launched
+ * without that trigger, as a plain copy kernel is).                                     */
 LS_API int ls_draft_attend(const ls_state* st, int32_t layer_begin, int32_t layer_count,
                     const void* d_q, const void* d_boundary_k, const void* d_boundary_v,
                     int64_t boundary_stride, float softmax_scale, void* d_out,

@@ -42,6 +42,7 @@ sys.path.insert(0, ROOT)
 METRIC = "draft rounds/s at batch 16 (Qwen3-8B shapes), 32K-128K prefix; % HBM roofline"
 WORKLOAD = "qwen3_8b_64k"
 FALLBACK_HBM_GBS = 6650.0
+LOADED_W = 300.0  # power draw above which a clock sample counts as under load (idle: about 200 W)
 
 
 # ---------------------------------------------------------------------------------------
@@ -198,15 +199,15 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, path: str):
-        self.path, self.proc, self.gpu = path, None, gpu_index
+    def __init__(self, gpu_index: int, path: str, period_ms: int = 100):
+        self.path, self.proc, self.gpu, self.period = path, None, gpu_index, period_ms
 
     def __enter__(self):
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", str(self.period)], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
         return self
@@ -220,7 +221,9 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
-    def summary(self):
+    def summary(self, min_power_w: float = 0.0):
+        """Median SM clock, max clock and the throttle reasons seen, over the samples drawn
+        at min_power_w or more (the GPU under load)."""
         if self.proc is None:
             return None
         rows = []
@@ -230,10 +233,12 @@ class ClockSampler:
                 if len(parts) < 9:
                     continue
                 try:
-                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                    if float(parts[3]) >= min_power_w:
+                        rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
                 except ValueError:
                     continue
-        rows = rows[1:] if len(rows) > 1 else rows  # the first sample may precede the load
+        if not min_power_w:
+            rows = rows[1:] if len(rows) > 1 else rows  # the first sample may precede the load
         if not rows:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -490,6 +495,12 @@ def run_gpu(args):
     clock_path = (args.clock_log or os.path.join(ROOT, "_build", "clocks_rank{rank}.csv")).format(rank=rank)
     os.makedirs(os.path.dirname(clock_path), exist_ok=True)
     overlapped = F.ls_round_overlaps(run.state)
+    # clocks over the whole GPU part of the run (20 ms samples; the timed rounds last a few
+    # ms only), and over the warm-up and timed rounds alone
+    run_clk = ClockSampler(local, clock_path.replace(".csv", "_run.csv"), period_ms=20)
+    run_clk.__enter__()
+    import atexit
+    atexit.register(run_clk.__exit__)  # (also on an error before the end)
     # the sampler starts with the warm-up rounds so that its samples cover a loaded GPU
     with ClockSampler(local, clock_path) as clk:
         for r in range(W):
@@ -665,6 +676,7 @@ def run_gpu(args):
         flat = {"us_per_round": b16, "flatness": grid["flatness"]["batch16_mean4.0"], "batch": 16,
                 "accept_mean": 4.0, "rounds": grid["rounds_per_point"]}
 
+    run_clk.__exit__()
     peak, peak_kind = hbm_peak()
     a_bytes = attend_bytes(wl)
     deltas = run.accept_host[[(W + i) % n_rounds for i in range(K)]] + 1
@@ -716,7 +728,10 @@ def run_gpu(args):
             "drafting_round": drafting,
             "gpu_launches": 2 * K,
             "e2e": e2e,
-            "clocks": clk.summary(),
+            "clocks": dict(run_clk.summary(min_power_w=LOADED_W) or {},
+                           window=f"the run's GPU work, {run_clk.period} ms samples at {LOADED_W:.0f} W or more "
+                                  "(the timed rounds included)"),
+            "clocks_timed_region": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget)

@@ -447,7 +447,7 @@ int ls_draft_attend_views(const ls_state* st, int32_t layer_begin, int32_t layer
                                           : (inputs_ready ? ls::kAttendAfterCommit : ls::kAttendPlain);
     const int r = cuda_status(ls::launch_attend_tc(st->dev, st->tc, layer_begin, layer_count, d_q, d_boundary_k,
                                                    d_boundary_v, boundary_stride, softmax_scale, views, d_out,
-                                                   st->sms, mode, stream));
+                                                   st->sms, mode, inputs_ready, stream));
     if (r == LS_OK) mark_settled(st, stream);
     return r;
   }
@@ -496,7 +496,7 @@ int round_attend(ls_state* st, const void* d_q, int64_t boundary_k_offset, int64
   if (st->use_tc) {  // the attention kernel is scheduled while the commit runs
     const int r = cuda_status(ls::launch_attend_tc(st->dev, st->tc, 0, c.n_layers, d_q, bnd + boundary_k_offset * e,
                                                    bnd + boundary_v_offset * e, c.hidden, softmax_scale, LS_VIEW_ALL,
-                                                   d_out, st->sms, ls::kAttendAfterCommit, stream));
+                                                   d_out, st->sms, ls::kAttendAfterCommit, false, stream));
     if (r == LS_OK) mark_settled(st, stream);
     return r;
   }

@@ -31,8 +31,11 @@ enum AttendLaunch : int {
                            // kernel before it started (LS_ATTEND_INPUTS_READY): no wait
 };
 // views: non-zero OR of LS_VIEW_* (the views that take part in the softmax).
+// side_by_side: the caller chains launches that need not wait for one another
+// (LS_ATTEND_INPUTS_READY): a launch of at most one wave of tiles then takes at most half
+// of the SMs, so that the next launch's CTAs stream beside it.
 cudaError_t launch_attend_tc(const Dev& p, const TcPlan& plan, int lb, int lcount, const void* q,
                              const void* bk, const void* bv, int64_t bstride, float scale, int views,
-                             void* out, int sms, AttendLaunch mode, cudaStream_t stream);
+                             void* out, int sms, AttendLaunch mode, bool side_by_side, cudaStream_t stream);
 
 }  // namespace ls

@@ -115,6 +115,27 @@ def test_full_config_view_ablations():
         _sampled_check(run, wl, out, TILES, view_set)
 
 
+def test_full_config_per_layer_calls():
+    """The bench workload's attention as per-layer calls (128 tiles each), with and without
+    LS_ATTEND_INPUTS_READY (with it, each call runs on half of the SMs, two tiles per CTA,
+    beside the next call), back to back: the bits of one call over the four layers."""
+    wl = WL.CONFIGS["qwen3_8b_64k"]
+    run, out, _ = _run_full(wl, rounds=8)
+    inp = run.make_round_inputs(run.rounds - 1, 1)
+    r = run.rounds - 1
+    qs = [inp["q"][0][:, l:l + 1].contiguous() for l in range(wl.n_layers)]
+    for views in (F.LS_VIEW_ALL | F.LS_ATTEND_INPUTS_READY, F.LS_VIEW_ALL):
+        ones = [run.new_out(1).fill_(float("nan")) for _ in range(wl.n_layers)]
+        for rep in range(2):
+            for l in range(wl.n_layers):
+                F.ls_draft_attend_views(run.state, l, 1, qs[l], run.boundary_k, run.boundary_v, wl.hidden,
+                                        run.softmax_scale, views, ones[l], run.stream)
+        torch.cuda.synchronize()
+        for l in range(wl.n_layers):
+            assert torch.equal(ones[l][:, 0], out[:, l]), (views, l)
+    assert run.error() == (F.LS_OK, 0) and r >= 0
+
+
 @pytest.mark.parametrize("prefix,batch,mean", [(4096, 1, 2.5), (16384, 4, 4.0), (131072, 64, 6.0)])
 def test_sweep_points(prefix, batch, mean):
     wl = WL.sweep_point(prefix, batch, mean)

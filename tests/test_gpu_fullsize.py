@@ -133,6 +133,18 @@ def test_full_config_per_layer_calls():
         torch.cuda.synchronize()
         for l in range(wl.n_layers):
             assert torch.equal(ones[l][:, 0], out[:, l]), (views, l)
+    # a view subset with the hint: the same bits as one call over that subset
+    sub = F.LS_VIEW_WINDOW | F.LS_VIEW_SUMMARY
+    full_sub = run.new_out()
+    F.ls_draft_attend_views(run.state, 0, wl.n_layers, inp["q"][0], run.boundary_k, run.boundary_v, wl.hidden,
+                            run.softmax_scale, sub, full_sub, run.stream)
+    ones = [run.new_out(1).fill_(float("nan")) for _ in range(wl.n_layers)]
+    for l in range(wl.n_layers):
+        F.ls_draft_attend_views(run.state, l, 1, qs[l], run.boundary_k, run.boundary_v, wl.hidden,
+                                run.softmax_scale, sub | F.LS_ATTEND_INPUTS_READY, ones[l], run.stream)
+    torch.cuda.synchronize()
+    for l in range(wl.n_layers):
+        assert torch.equal(ones[l][:, 0], full_sub[:, l]), ("subset", l)
     assert run.error() == (F.LS_OK, 0) and r >= 0
 
 

@@ -274,6 +274,29 @@ def test_per_layer_calls_with_inputs_ready_hint():
                                 F.LS_ATTEND_INPUTS_READY, ones[0], a.stream)
 
 
+def test_inputs_ready_hint_on_the_cuda_core_path():
+    """The tiny fp32 config (CUDA-core attention, which launches no programmatic
+    dependents): per-layer calls with LS_ATTEND_INPUTS_READY equal one call bit for bit."""
+    wl = WL.CONFIGS["tiny"]
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    inp = run.make_round_inputs()
+    for r in range(3):
+        run.commit(inp, r)
+    assert not F.ls_attend_uses_tensor_cores(run.state)
+    full = run.new_out()
+    run.attend(inp, 2, full)
+    ones = [run.new_out(1) for _ in range(wl.n_layers)]
+    for l in range(wl.n_layers):
+        F.ls_draft_attend_views(run.state, l, 1, inp["q"][2][:, l:l + 1].contiguous(), run.boundary_k,
+                                run.boundary_v, wl.hidden, run.softmax_scale,
+                                F.LS_VIEW_ALL | F.LS_ATTEND_INPUTS_READY, ones[l], run.stream)
+    torch.cuda.synchronize()
+    for l in range(wl.n_layers):
+        assert torch.equal(ones[l][:, 0], full[:, l])
+    assert run.error() == (F.LS_OK, 0)
+
+
 def test_attention_reads_the_previous_attentions_output():
     """Two attentions back to back, the second taking the first's output as its queries:
     the second launch may start before the first completes (its early loads are of the

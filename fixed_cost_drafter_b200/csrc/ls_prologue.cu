@@ -478,8 +478,13 @@ cudaError_t launch_prologue(const Dev& p, const void* w_kv, const void* w_q, con
   if (a.n_units < grid) grid = a.n_units;
   // units left over after whole waves: split their k-steps over every CTA when they are all
   // boundary tiles (their partial sums fit the state's scratch: 128 x K.act_rows fp32 each)
+  // and there are at least as many k-steps as CTAs (then every CTA's range is non-empty, so
+  // a tile's pieces are those of the CTAs from the one holding its first k-step to the one
+  // holding its last; with fewer, the CTAs between could hold none and the tile's arrival
+  // count would never be reached)
   const int rem = a.n_units % grid;
-  const bool split = rem > 0 && rem <= K.n_units && K.act_rows == prologue_boundary_rows(p.b);
+  const bool split = rem > 0 && rem <= K.n_units && K.act_rows == prologue_boundary_rows(p.b) &&
+                     int64_t(rem) * a.k_steps >= grid;
   a.n_full = split ? a.n_units - rem : a.n_units;
   a.rem_steps = split ? rem * a.k_steps : 0;
   a.part = p.pro_part;

@@ -194,6 +194,31 @@ def test_prologue_split_tiles_match_the_oracle():
     assert run.error() == (F.LS_OK, 0)
 
 
+def test_prologue_leftover_tiles_with_few_k_steps():
+    """Hidden 128 (2 k-steps per tile) at Qwen3-8B head counts: 192 tiles on 148 CTAs leave
+    44 boundary tiles, only 88 k-steps, fewer than the CTAs. Split over every CTA, some CTAs'
+    ranges would be empty and a tile's pieces fewer than the CTAs its first and last k-steps
+    span, so its sum would never be stored; such leftovers run whole instead. Every output
+    against the oracle."""
+    wl = _wl(batch=16, n_layers=4, n_kv_heads=8, n_q_heads=32, hidden=128, prefix=(300, 300))
+    run = WL.DeviceRun(wl)
+    run.prefill()
+    dev = run.dev
+    L, H, Hq, D, hid, B = wl.n_layers, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.hidden, wl.block
+    w_kv = _gen((L, 2 * H * D, hid), 51, dev, hid ** -0.5)
+    w_q = _gen((L, Hq * D, hid), 52, dev, hid ** -0.5)
+    x = _gen((wl.batch, L, B, hid), 53, dev, 1.0)
+    bkv, q = _run_prologue(run, wl, w_kv, w_q, x)
+    h = O.to_f64(run.read_state()["boundary"], "bf16")
+    Wkv, Wq, X = _f64(w_kv), _f64(w_q), _f64(x)
+    ref_bkv, ref_q = O.draft_prologue(Wkv, Wq, h, X)
+    for l in range(L):
+        _check(_f64(bkv)[:, l], ref_bkv[:, l], _bound_terms(Wkv[l], h[:, l], hid))
+        _check(_f64(q)[:, l].reshape(-1, Hq * D), ref_q[:, l].reshape(-1, Hq * D),
+               _bound_terms(Wq[l], X[:, l].reshape(-1, hid), hid))
+    assert run.error() == (F.LS_OK, 0)
+
+
 def test_prologue_split_tiles_selection_exact():
     """The split boundary tiles with selection weights: every partial sum is exact, so the
     keys/values equal the boundary slices bit for bit however the pieces are cut."""

@@ -70,8 +70,13 @@ bool on_state_device(const ls_state* st) {
 // once everything before it has completed (it triggers its dependents after its grid
 // dependency wait, or it is launched without programmatic serialization), every call that
 // wrote the views has completed by the time a kernel launched next on `stream` starts.
+// A launch captured into a graph runs only when the graph is launched, in an order the host
+// does not see: it settles nothing for the launches made on the stream after the capture
+// (which follow whatever was launched before it), so the state is left unsettled.
 void mark_settled(const ls_state* st, cudaStream_t stream) {
-  st->views_settled = 1;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const bool captured = cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone;
+  st->views_settled = captured ? 0 : 1;
   st->settled_stream = stream;
 }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }

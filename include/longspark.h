@@ -336,7 +336,9 @@ LS_API int ls_commit_accepted(ls_state* st, const int32_t* d_accept_len, const v
  * on the state was launched on the same stream (per-layer calls, or the call after
  * ls_draft_prologue), it loads its first rows of the views before that, so its start
  * overlaps the end of the kernel before it. Inside a stream capture it does not (the
- * order of the graph's replays is not known when it is captured). A caller that writes
+ * order of the graph's replays is not known when it is captured), and a call captured
+ * into a graph counts as no such earlier call for the calls launched directly after the
+ * capture (they follow whatever was launched on the stream before it). A caller that writes
  * the arena itself (a checkpoint restored into it) does so with a copy, or a kernel that
  * does not trigger programmatic dependents before it completes (any kernel launched
  * without that trigger, as a plain copy kernel is).                                     */

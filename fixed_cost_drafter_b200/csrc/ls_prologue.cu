@@ -11,7 +11,13 @@
 // Persistent kernel, 7 warps: warp 0 TMA producer of the weights (a ring of 6 stages of 64
 // hidden entries of the unit's 128 weight rows, from HBM), warp 6 TMA producer of the
 // activations (3 stages of up to 256 rows, mostly from L2), both 128-byte swizzled; warp 1
-// TMEM allocator and MMA issuer (double-buffered accumulator, 2 x 256 columns); warps 2-5
+// TMEM allocator and MMA issuer (double-buffered accumulator, 2 x 256 columns). The one
+// MMA-issuing thread bounds the k-step rate (its waits, MMA issues and commits take tens of
+// nanoseconds each), so a k-step costs it one wait and one commit: both producers' copies
+// of k-step k complete on the weight ring's barrier of k (two arrivals), and the release of
+// that barrier's stage also frees the activation stage of k (the activation ring, 3 deep,
+// is refilled for k-step k once k - 3 is released, which the weight ring's barrier of
+// k - 3 tells). Warps 2-5
 // epilogue (one TMEM subpartition each: a thread owns one weight row, its outputs go
 // through a shared-memory tile so that whole 256-byte output rows leave as 16-byte
 // stores). Units: (problem, layer, 128-row weight tile, activation tile), queries first.
@@ -71,8 +77,8 @@ struct PArgs {
 };
 
 struct PBars {
-  uint64_t afull[kPAStages], aempty[kPAStages];
-  uint64_t bfull[kPBStages], bempty[kPBStages];
+  uint64_t afull[kPAStages], aempty[kPAStages];  // per k-step k: stage k mod kPAStages of
+                                                 // both rings full (2 arrivals) / released
   uint64_t acc_full[2], acc_empty[2];
   uint64_t out_full, out_free;  // epilogue pass: staged by all 128 threads / copied out
   uint64_t drain;               // after an abort: the MMAs issued so far have completed
@@ -80,6 +86,7 @@ struct PBars {
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t last;                // the epilogue's piece was its tile's last to arrive
+  int32_t issued[2];            // k-steps each producer arrived for (weights, activations)
 };
 
 struct PUnit {
@@ -150,6 +157,9 @@ __device__ inline PItem item_of(const PArgs& a, const PWork& w, int i) {
   return it;
 }
 
+// uses of stage st among the first n k-steps of a ring of nst stages
+__device__ inline int stage_uses(int n, int st, int nst) { return n > st ? (n - 1 - st) / nst + 1 : 0; }
+
 __device__ inline bool pwait(PBars& s, uint64_t* bar, uint32_t parity, int32_t* err) {
 #pragma unroll 1
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
@@ -175,14 +185,14 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   const PWork w = work_of(a);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPAStages; ++i) { mbar_init(&s.afull[i], 1); mbar_init(&s.aempty[i], 1); }
-    for (int i = 0; i < kPBStages; ++i) { mbar_init(&s.bfull[i], 1); mbar_init(&s.bempty[i], 1); }
+    for (int i = 0; i < kPAStages; ++i) { mbar_init(&s.afull[i], 2); mbar_init(&s.aempty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&s.acc_full[i], 1); mbar_init(&s.acc_empty[i], 128); }
     mbar_init(&s.out_full, 128);
     mbar_init(&s.out_free, 128);
     mbar_init(&s.drain, 1);
     mbar_init(&s.epi, 128);
     s.abort = 0;
+    s.issued[0] = s.issued[1] = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -195,7 +205,6 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  int issued = 0;  // producers: copies issued into their ring (for the drain after an abort)
   if (warp != 0) {  // the weight producer waits once its first ring of weights is on its way
     grid_dependency_wait();
     allow_dependent_launch();
@@ -208,8 +217,6 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
     if (lane == 0) {
       const bool is_a = warp == 0;
       const int nst = is_a ? kPAStages : kPBStages;
-      uint64_t* fullb = is_a ? s.afull : s.bfull;
-      uint64_t* emptyb = is_a ? s.aempty : s.bempty;
       prefetch_map(is_a ? &w0 : &x0);
       prefetch_map(is_a ? &w1 : &x1);
       const uint64_t pol = is_a ? l2_evict_first() : l2_evict_last();
@@ -224,25 +231,31 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
         // the weights are read once: they must not push the activations (read again by
         // every weight tile of the layer) out of L2
         for (int ks = it.k0; ks < it.k1; ++ks, ++k) {
-          const int st = k % nst;
+          const int st = k % nst;          // this ring's stage
+          uint64_t* full = &s.afull[k % kPAStages];  // the k-step's barrier
           if (k == nst && !waited) {  // (the first ring's weights are in flight)
             grid_dependency_wait();
             allow_dependent_launch();
             waited = true;
           }
-          if (!pwait(s, &emptyb[st], ((k / nst) & 1) ^ 1, a.err)) { ok = false; break; }
-          mbar_arrive_expect_tx(&fullb[st], bytes);
+          // the stage is free once the MMAs of the k-step that used it before have completed
+          // (k - nst); the MMAs of a k-step complete in order, and the one wait before for
+          // the same barrier covered its previous phase, so the parity names this phase
+          const int prev = k - nst;
+          if (prev >= 0 && !pwait(s, &s.aempty[prev % kPAStages], uint32_t(prev / kPAStages) & 1, a.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full, bytes);
           if (is_a)
-            tma_load_2d_hint(a_ring + st * kPABytes, m, ks * kPKStep, u.l * P.n_out + u.nt * kPTileN, &fullb[st],
-                             pol);
+            tma_load_2d_hint(a_ring + st * kPABytes, m, ks * kPKStep, u.l * P.n_out + u.nt * kPTileN, full, pol);
           else if (P.is_4d)
-            tma_load_4d_hint(b_ring + st * kPBBytes, m, ks * kPKStep, 0, u.l, u.mt * P.seq_per_unit, &fullb[st],
-                             pol);
+            tma_load_4d_hint(b_ring + st * kPBBytes, m, ks * kPKStep, 0, u.l, u.mt * P.seq_per_unit, full, pol);
           else
-            tma_load_3d_hint(b_ring + st * kPBBytes, m, ks * kPKStep, u.l, u.mt * P.seq_per_unit, &fullb[st], pol);
-          ++issued;
+            tma_load_3d_hint(b_ring + st * kPBBytes, m, ks * kPKStep, u.l, u.mt * P.seq_per_unit, full, pol);
         }
       }
+      s.issued[is_a ? 0 : 1] = k;
     }
     if (!waited) {  // (every thread of the CTA passes the wait before it triggers)
       grid_dependency_wait();
@@ -265,15 +278,13 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
         for (int ks = it.k0; ks < it.k1; ++ks, ++k) {
           const int sa = k % kPAStages, sb = k % kPBStages;
           if (!pwait(s, &s.afull[sa], (k / kPAStages) & 1, a.err)) { ok = false; break; }
-          if (!pwait(s, &s.bfull[sb], (k / kPBStages) & 1, a.err)) { ok = false; break; }
           tc_fence_after();
           const uint64_t da = sdesc(smem_u32(a_ring + sa * kPABytes), 16, 1024);
           const uint64_t db = sdesc(smem_u32(b_ring + sb * kPBBytes), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kPKStep / 16; ++kk)  // K = 16 per MMA: 32 bytes along the row
             mma_bf16(d, da + uint32_t(kk * 2), db + uint32_t(kk * 2), id, (ks > it.k0 || kk > 0) ? 1u : 0u);
-          mma_commit(&s.aempty[sa]);
-          mma_commit(&s.bempty[sb]);
+          mma_commit(&s.aempty[sa]);  // frees both stages of the k-step
         }
         if (ok) mma_commit(&s.acc_full[ab]);
       }
@@ -379,12 +390,17 @@ prologue_kernel(const PArgs a, const __grid_constant__ CUtensorMap w0, const __g
   }
 
   __syncthreads();
-  if ((warp == 0 || warp == 6) && lane == 0 && s.abort) {
-    // let the copies still in flight land before the shared memory is released
-    const int nst = warp == 0 ? kPAStages : kPBStages;
-    uint64_t* fullb = warp == 0 ? s.afull : s.bfull;
-    for (int n = issued > nst ? issued - nst : 0; n < issued; ++n)
-      mbar_wait_bounded(&fullb[n % nst], (n / nst) & 1, kWaitLimit);
+  if (warp == 0 && lane == 0 && s.abort) {
+    // let the copies still in flight land before the shared memory is released: a k-step
+    // barrier that only one producer arrived for (the other gave up first; the producers
+    // are at most a ring apart, so by one use of a barrier) gets the other's arrival, then
+    // each barrier's last phase completes once its copies have landed
+    for (int st = 0; st < kPAStages; ++st) {
+      const int na = stage_uses(s.issued[0], st, kPAStages), nb = stage_uses(s.issued[1], st, kPAStages);
+      if (na != nb) mbar_arrive(&s.afull[st]);
+      const int n = na > nb ? na : nb;
+      if (n > 0) mbar_wait_bounded(&s.afull[st], uint32_t(n - 1) & 1, kWaitLimit);
+    }
   }
   if (warp == 1 && lane == 0 && s.abort) {
     // and the MMAs issued so far, before TMEM is released

@@ -11,13 +11,12 @@
 // Persistent kernel, 7 warps: warp 0 TMA producer of the weights (a ring of 6 stages of 64
 // hidden entries of the unit's 128 weight rows, from HBM), warp 6 TMA producer of the
 // activations (3 stages of up to 256 rows, mostly from L2), both 128-byte swizzled; warp 1
-// TMEM allocator and MMA issuer (double-buffered accumulator, 2 x 256 columns). The one
-// MMA-issuing thread bounds the k-step rate (its waits, MMA issues and commits take tens of
-// nanoseconds each), so a k-step costs it one wait and one commit: both producers' copies
-// of k-step k complete on the weight ring's barrier of k (two arrivals), and the release of
-// that barrier's stage also frees the activation stage of k (the activation ring, 3 deep,
-// is refilled for k-step k once k - 3 is released, which the weight ring's barrier of
-// k - 3 tells). Warps 2-5
+// TMEM allocator and MMA issuer (double-buffered accumulator, 2 x 256 columns). Every wait,
+// MMA issue and commit of the one MMA-issuing thread takes tens of nanoseconds, so a k-step
+// costs it one wait and one commit: both producers' copies of k-step k complete on the
+// weight ring's barrier of k (two arrivals), and the release of that barrier's stage also
+// frees the activation stage of k (the activation ring, 3 deep, is refilled for k-step k
+// once k - 3 is released, which the weight ring's barrier of k - 3 tells). Warps 2-5
 // epilogue (one TMEM subpartition each: a thread owns one weight row, its outputs go
 // through a shared-memory tile so that whole 256-byte output rows leave as 16-byte
 // stores). Units: (problem, layer, 128-row weight tile, activation tile), queries first.

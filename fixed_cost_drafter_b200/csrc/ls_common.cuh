@@ -219,33 +219,48 @@ __device__ inline uint4 ld_nc_v4(const void* p) {
 }
 
 // ---- paged KV cache ---------------------------------------------------------------
-// Byte address of the row (all KV heads) at position `pos` of sequence b in the layer
-// whose pages start at `base`: page block_table[b][pos / page_size], offset
+// paged_row: byte address of the row (all KV heads) at position `pos` of sequence b in the
+// layer whose pages start at `base`: page block_table[b][pos / page_size], offset
 // pos mod page_size. A position past the block table or a page id outside
 // [0, num_pages) sets LS_DEVERR_PAGE and gives the same offset in page 0, so no access
-// leaves the caller's pages.
-__device__ inline const char* paged_row(const ls_paged_kv& kv, const char* base, int b, int64_t pos, int elem,
-                                        int32_t* err) {
-  int64_t pi;
-  int off;
+// leaves the caller's pages. Its three steps, for callers that look pages up ahead:
+// Page index and in-page offset of position `pos`.
+__device__ inline int64_t paged_index(const ls_paged_kv& kv, int64_t pos, int& off) {
   const int ps = kv.page_size;
   if ((ps & (ps - 1)) == 0) {  // the usual page sizes: shift and mask
-    pi = pos >> (__ffs(ps) - 1);
     off = int(pos & (ps - 1));
-  } else if (pos < (int64_t(1) << 32)) {
-    const uint32_t q = uint32_t(pos) / uint32_t(ps);
-    pi = q;
-    off = int(uint32_t(pos) - q * uint32_t(ps));
-  } else {
-    pi = pos / ps;
-    off = int(pos - pi * ps);
+    return pos >> (__ffs(ps) - 1);
   }
-  int64_t page = pi < kv.max_blocks ? int64_t(__ldg(kv.block_table + int64_t(b) * kv.max_blocks + pi)) : -1;
+  if (pos < (int64_t(1) << 32)) {
+    const uint32_t q = uint32_t(pos) / uint32_t(ps);
+    off = int(uint32_t(pos) - q * uint32_t(ps));
+    return q;
+  }
+  const int64_t pi = pos / ps;
+  off = int(pos - pi * ps);
+  return pi;
+}
+// The block table's entry for page index pi of sequence b (-1 past the table). The load is
+// issued here; a caller that uses the value later overlaps its latency with other work.
+__device__ inline int32_t paged_entry(const ls_paged_kv& kv, int b, int64_t pi) {
+  return pi < kv.max_blocks ? __ldg(kv.block_table + int64_t(b) * kv.max_blocks + pi) : -1;
+}
+// Byte address of offset `off` in page `entry` of the layer at `base`; an entry outside
+// [0, num_pages) sets LS_DEVERR_PAGE and gives the same offset in page 0.
+__device__ inline const char* paged_at(const ls_paged_kv& kv, const char* base, int32_t entry, int off, int elem,
+                                       int32_t* err) {
+  int64_t page = entry;
   if (page < 0 || page >= kv.num_pages) {
     set_err(err, LS_DEVERR_PAGE);
     page = 0;
   }
   return base + (page * kv.page_stride + int64_t(off) * kv.slot_stride) * elem;
+}
+__device__ inline const char* paged_row(const ls_paged_kv& kv, const char* base, int b, int64_t pos, int elem,
+                                        int32_t* err) {
+  int off;
+  const int64_t pi = paged_index(kv, pos, off);
+  return paged_at(kv, base, paged_entry(kv, b, pi), off, elem, err);
 }
 
 // Byte address of slot `slot` (page * page_size + offset) in the layer at `base`; a slot

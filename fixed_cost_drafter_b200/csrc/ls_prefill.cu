@@ -99,13 +99,21 @@ __device__ inline void issue_prefix_rows(const Dev&, const PrefillArgs& a, const
 }
 
 // Paged: one copy per run of rows inside a page (per row when the slots are not packed).
-// The runs (their page lookups included) are planned before the producer waits for a free
-// stage, so the lookups' latency overlaps that wait instead of delaying the refill.
-struct PrefixPlan {
+// The producer loads a stage's block-table entries one stage ahead (PrefixLookup: the loads
+// are issued, their values used an iteration later) and turns them into the copies' source
+// addresses (PrefixPlan) before it waits for the stage's buffer, so the entries' latency
+// overlaps the stage before instead of delaying the refill.
+struct PrefixLookup {
   static constexpr int kMaxRuns = 2;  // a stage of G rows spans at most 2 pages when page_size >= G
+  int32_t entry[kMaxRuns];  // the runs' block-table entries (loads in flight)
+  int off[kMaxRuns], r0[kMaxRuns], n[kMaxRuns], nrun;
+  bool ok;  // false: the stage needs more runs, issue_prefix_rows looks it up after the wait
+};
+struct PrefixPlan {
+  static constexpr int kMaxRuns = PrefixLookup::kMaxRuns;
   const char* src[2][kMaxRuns];
-  int r0[2][kMaxRuns], n[2][kMaxRuns], nrun[2];
-  bool ok;  // false: the stage needs more runs, issue_prefix_rows plans it after the wait
+  int r0[kMaxRuns], n[kMaxRuns], nrun;
+  bool ok;
 };
 
 __device__ inline int page_offset(int64_t pos, int ps) {
@@ -115,36 +123,55 @@ __device__ inline int page_offset(int64_t pos, int ps) {
 }
 
 template <typename T>
-__device__ inline void plan_prefix_rows(const Dev&, const DensePrefix&, int, int64_t, int, PrefixPlan& pl) {
-  pl.ok = false;  // dense: addresses are plain arithmetic, nothing to plan
+__device__ inline void lookup_prefix_rows(const Dev&, const DensePrefix&, int, int64_t, int, PrefixLookup& lk) {
+  lk.ok = false;  // dense: addresses are plain arithmetic, nothing to look up
 }
 
 template <typename T>
-__device__ inline void plan_prefix_rows(const Dev& p, const ls_paged_kv& kv, int bl, int64_t g0, int nrows,
-                                        PrefixPlan& pl) {
-  const int b = bl / p.L, l = bl - b * p.L;
-  pl.ok = true;
-  // (fixed trip counts: the plan stays in registers)
+__device__ inline void lookup_prefix_rows(const Dev& p, const ls_paged_kv& kv, int bl, int64_t g0, int nrows,
+                                          PrefixLookup& lk) {
+  const int b = bl / p.L;
+  int r = 0;
+  lk.nrun = 0;
+  // (fixed trip count: the lookup stays in registers)
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const char* base = static_cast<const char*>(t == 0 ? kv.k_layers[l] : kv.v_layers[l]);
-    int r = 0;
-    pl.nrun[t] = 0;
-#pragma unroll
-    for (int k = 0; k < PrefixPlan::kMaxRuns; ++k) {
-      pl.src[t][k] = nullptr;
-      pl.r0[t][k] = r;
-      pl.n[t][k] = 0;
-      if (r < nrows) {
-        const int64_t pos = g0 + r;
-        const int run = min(nrows - r, kv.page_size - page_offset(pos, kv.page_size));
-        pl.src[t][k] = paged_row(kv, base, b, pos, int(sizeof(T)), p.err);
-        pl.n[t][k] = run;
-        pl.nrun[t] = k + 1;
-        r += run;
-      }
+  for (int k = 0; k < PrefixLookup::kMaxRuns; ++k) {
+    lk.entry[k] = -1;
+    lk.off[k] = 0;
+    lk.r0[k] = r;
+    lk.n[k] = 0;
+    if (r < nrows) {
+      const int64_t pos = g0 + r;
+      const int64_t pi = paged_index(kv, pos, lk.off[k]);
+      lk.entry[k] = paged_entry(kv, b, pi);
+      lk.n[k] = min(nrows - r, kv.page_size - lk.off[k]);
+      lk.nrun = k + 1;
+      r += lk.n[k];
     }
-    if (r < nrows) pl.ok = false;
+  }
+  lk.ok = r >= nrows;
+}
+
+template <typename T>
+__device__ inline void plan_prefix_rows(const Dev&, const DensePrefix&, int, const PrefixLookup&, PrefixPlan& pl) {
+  pl.ok = false;
+}
+
+template <typename T>
+__device__ inline void plan_prefix_rows(const Dev& p, const ls_paged_kv& kv, int bl, const PrefixLookup& lk,
+                                        PrefixPlan& pl) {
+  const int l = bl - (bl / p.L) * p.L;
+  pl.ok = lk.ok;
+  pl.nrun = lk.nrun;
+#pragma unroll
+  for (int k = 0; k < PrefixPlan::kMaxRuns; ++k) {
+    pl.r0[k] = lk.r0[k];
+    pl.n[k] = lk.n[k];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const char* base = static_cast<const char*>(t == 0 ? kv.k_layers[l] : kv.v_layers[l]);
+      pl.src[t][k] = k < lk.nrun ? paged_at(kv, base, lk.entry[k], lk.off[k], int(sizeof(T)), p.err) : nullptr;
+    }
   }
 }
 
@@ -154,12 +181,12 @@ __device__ inline void issue_plan(const ls_paged_kv& kv, const PrefixPlan& pl, i
   const bool packed = kv.slot_stride * int64_t(sizeof(T)) == rowBytes;
 #pragma unroll
   for (int k = 0; k < PrefixPlan::kMaxRuns; ++k) {
-    if (k >= pl.nrun[t]) break;
+    if (k >= pl.nrun) break;
     if (packed) {
-      bulk_g2s(dst + pl.r0[t][k] * rowBytes, pl.src[t][k], uint32_t(pl.n[t][k] * rowBytes), bar);
+      bulk_g2s(dst + pl.r0[k] * rowBytes, pl.src[t][k], uint32_t(pl.n[k] * rowBytes), bar);
     } else {
-      for (int i = 0; i < pl.n[t][k]; ++i)
-        bulk_g2s(dst + (pl.r0[t][k] + i) * rowBytes, pl.src[t][k] + int64_t(i) * kv.slot_stride * int64_t(sizeof(T)),
+      for (int i = 0; i < pl.n[k]; ++i)
+        bulk_g2s(dst + (pl.r0[k] + i) * rowBytes, pl.src[t][k] + int64_t(i) * kv.slot_stride * int64_t(sizeof(T)),
                  uint32_t(rowBytes), bar);
     }
   }
@@ -233,16 +260,37 @@ prefill_units_kernel(Dev p, PrefillArgs a, const Src src) {
       int n = 0;
       int last_issue[kPrefillStages];
       for (int s = 0; s < kPrefillStages; ++s) last_issue[s] = -1;
+      // the rows of the stage at cursor c
+      auto stage_rows = [&](const Cursor& c, int& bl, int64_t& g0, int& nrows) {
+        const int it = blockIdx.x + c.j * gridDim.x;
+        int u; int64_t r0, r1;
+        item_rows(a, p, it, bl, u, r0, r1);
+        g0 = r0 + int64_t(c.grp) * a.G;
+        nrows = int(min(int64_t(a.G), r1 - g0));
+      };
+      int bl = 0, nrows = 0;
+      int64_t g0 = 0;
+      PrefixLookup look;
+      if (prod.valid) {
+        stage_rows(prod, bl, g0, nrows);
+        lookup_prefix_rows<T>(p, src, bl, g0, nrows, look);
+      }
       for (; prod.valid; ++n) {
         const int buf = n % kPrefillStages;
-        // the stage's rows (and, paged, their page lookups) before waiting for the buffer
-        const int it = blockIdx.x + prod.j * gridDim.x;
-        int bl, u; int64_t r0, r1;
-        item_rows(a, p, it, bl, u, r0, r1);
-        const int64_t g0 = r0 + int64_t(prod.grp) * a.G;
-        const int nrows = int(min(int64_t(a.G), r1 - g0));
+        // the next stage's page lookups go out now; this stage's (loaded one stage ago)
+        // become its copies' addresses before waiting for the buffer
+        Cursor nx = prod;
+        cursor_next(a, p, nx);
+        int nbl = 0, nnrows = 0;
+        int64_t ng0 = 0;
+        PrefixLookup nlook;
+        nlook.ok = false;
+        if (nx.valid) {
+          stage_rows(nx, nbl, ng0, nnrows);
+          lookup_prefix_rows<T>(p, src, nbl, ng0, nnrows, nlook);
+        }
         PrefixPlan plan;
-        plan_prefix_rows<T>(p, src, bl, g0, nrows, plan);
+        plan_prefix_rows<T>(p, src, bl, look, plan);
         if (!wait(&empty[buf], ((n / kPrefillStages) & 1) ^ 1)) break;
         fence_proxy_async_smem();  // the consumers' reads of the buffer come before its refill
         char* dst = smem + buf * stageBytes;
@@ -255,7 +303,11 @@ prefill_units_kernel(Dev p, PrefillArgs a, const Src src) {
             issue_prefix_rows<T>(p, a, src, t, bl, g0, nrows, dst + t * a.G * rowBytes, rowBytes, &full[buf]);
         }
         last_issue[buf] = n;
-        cursor_next(a, p, prod);
+        prod = nx;
+        bl = nbl;
+        g0 = ng0;
+        nrows = nnrows;
+        look = nlook;
       }
       if (*reinterpret_cast<volatile uint32_t*>(&abort_flag)) {
         // let every copy still in flight land before the CTA's shared memory goes away

@@ -903,6 +903,21 @@ class L2Flush:
         self.r.sum()
 
 
+def pack_layout(ts):
+    """Byte offsets of tensors ``ts`` packed back to back in one buffer, each starting on a
+    256-byte boundary, and the buffer's size."""
+    offs, off = [], 0
+    for t in ts:
+        offs.append(off)
+        off += (t.numel() * t.element_size() + 255) // 256 * 256
+    return offs, off
+
+
+def pack_views(buf, ts, offs):
+    """Views of the uint8 buffer ``buf`` with the dtypes and shapes of ``ts`` at ``offs``."""
+    return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for t, o in zip(ts, offs)]
+
+
 def e2e_measure(run, wl, dev, flush, steps, world, inp, strong=False):
     """Rounds/s through the public entry point with every step's inputs in pinned host memory
     and its results read back to pinned host memory, inside one timed region.
@@ -921,16 +936,7 @@ def e2e_measure(run, wl, dev, flush, steps, world, inp, strong=False):
     # (256-byte aligned pieces, viewed as the call's tensors), and its results come back as
     # one block: one copy each way per step, as a streaming caller would pack them.
     keys = ("vk", "vv", "vh", "q", "draft", "target")
-
-    def layout(ts):
-        offs, off = [], 0
-        for t in ts:
-            offs.append(off)
-            off += (t.numel() * t.element_size() + 255) // 256 * 256
-        return offs, off
-
-    def views(buf, ts, offs):
-        return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for t, o in zip(ts, offs)]
+    layout, views = pack_layout, pack_views
 
     proto = [inp[k][0] for k in keys[:4]] + [run.draft[0], run.target[0]]
     in_offs, in_bytes = layout(proto)
